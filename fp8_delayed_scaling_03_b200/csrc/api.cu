@@ -1,0 +1,486 @@
+// api.cu -- the extern "C" boundary of libfp8lin (see include/fp8lin.h).
+//
+// Validation happens before anything is enqueued; the library allocates no
+// memory and never synchronizes the host (fp8_get_device_status excepted).
+// TMA tensor maps are encoded on the host per call (cuTensorMapEncodeTiled,
+// fetched through the runtime's driver entry point so the shared object loads
+// on machines without a GPU driver) and passed as __grid_constant__ kernel
+// parameters.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "device.cuh"
+#include "fp8lin.h"
+#include "internal.h"
+
+namespace fp8lin {
+
+__device__ int g_device_status;
+
+namespace {
+
+thread_local char g_err[256] = "";
+
+int cuda_fail(cudaError_t e) {
+  snprintf(g_err, sizeof(g_err), "CUDA error %d: %s", static_cast<int>(e), cudaGetErrorString(e));
+  return FP8_ERR_CUDA;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+int g_sms[64] = {};
+int* g_status_ptr[64] = {};
+
+EncodeTiledFn encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+
+int* status_ptr(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) == cudaSuccess) g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool is_fmt(int f) { return f == FP8_E4M3 || f == FP8_E5M2; }
+bool is_wide(int dt) { return dt == FP8_DT_BF16 || dt == FP8_DT_FP16 || dt == FP8_DT_FP32; }
+bool is_fp8(int dt) { return dt == FP8_DT_E4M3 || dt == FP8_DT_E5M2; }
+int esize(int dt) { return dt == FP8_DT_FP32 ? 4 : (is_fp8(dt) ? 1 : 2); }
+float fp8_max(int fmt) { return fmt == FP8_E4M3 ? 448.0f : 57344.0f; }
+bool ring_len_ok(int H) { return H >= 1 && H <= 4096; }
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+int check_fp8_matrix(const void* p, int64_t ld, int64_t cols) {
+  if (!p) return FP8_ERR_INVALID_ARG;
+  if (ld < cols) return FP8_ERR_INVALID_ARG;
+  if (ld % 16 != 0 || !aligned(p, 16)) return FP8_ERR_MISALIGNED;
+  return FP8_OK;
+}
+
+// 2-D uint8 tensor map, 128-byte swizzle, zero fill out of bounds.
+int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld_bytes,
+             uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) {
+    snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled unavailable");
+    return FP8_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return FP8_ERR_CUDA;
+  }
+  return FP8_OK;
+}
+
+struct MmCall {
+  int64_t m, n, k;
+  const uint8_t* a; int fmt_a; int a_major; int64_t lda;
+  const uint8_t* b; int fmt_b; int b_major; int64_t ldb;
+  const float* scale_a; const float* scale_b;
+  const void* bias; int bias_dtype; const float* bias_scale;
+  void* d; int64_t ldd;
+};
+
+int validate_mm(const MmCall& c) {
+  if (c.m < 0 || c.n < 0 || c.k < 0 || c.m > kMaxDim || c.n > kMaxDim || c.k > kMaxDim) return FP8_ERR_INVALID_ARG;
+  if (!is_fmt(c.fmt_a) || !is_fmt(c.fmt_b)) return FP8_ERR_INVALID_ARG;
+  if ((c.a_major != FP8_K_MAJOR && c.a_major != FP8_MN_MAJOR) ||
+      (c.b_major != FP8_K_MAJOR && c.b_major != FP8_MN_MAJOR))
+    return FP8_ERR_INVALID_ARG;
+  if (!c.scale_a || !c.scale_b || !c.d) return FP8_ERR_INVALID_ARG;
+  int s = check_fp8_matrix(c.a, c.lda, c.a_major == FP8_K_MAJOR ? c.k : c.m);
+  if (s) return s;
+  s = check_fp8_matrix(c.b, c.ldb, c.b_major == FP8_K_MAJOR ? c.k : c.n);
+  if (s) return s;
+  if (c.ldd < c.n || !aligned(c.d, 2)) return FP8_ERR_INVALID_ARG;
+  if (c.bias) {
+    if (c.bias_dtype != FP8_DT_BF16 && !is_fp8(c.bias_dtype)) return FP8_ERR_INVALID_ARG;
+    if (is_fp8(c.bias_dtype) && !c.bias_scale) return FP8_ERR_INVALID_ARG;
+    if (c.bias_dtype == FP8_DT_BF16 && !aligned(c.bias, 2)) return FP8_ERR_INVALID_ARG;
+  }
+  return FP8_OK;
+}
+
+// Output tile width: the candidate with the smallest (waves x tile width),
+// preferring the wider tile on ties (fewer operand re-reads per flop).
+int pick_bn(int64_t m, int64_t n, int sms) {
+  const int64_t tm = (m + 127) / 128;
+  int best = 256;
+  int64_t best_cost = -1;
+  for (int bn : {256, 128}) {
+    const int64_t tiles = tm * ((n + bn - 1) / bn);
+    const int64_t waves = (tiles + sms - 1) / sms;
+    const int64_t cost = waves * bn;
+    if (best_cost < 0 || cost < best_cost) { best = bn; best_cost = cost; }
+  }
+  return best;
+}
+
+// Enqueue one GEMM (validated already).  side: writes folded into the launch.
+int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int sms = num_sms(dev);
+  if (sms <= 0) return cuda_fail(cudaGetLastError());
+  const int bn = pick_bn(c.m, c.n, sms);
+  CUtensorMap ta, tb;
+  std::memset(&ta, 0, sizeof(ta));
+  std::memset(&tb, 0, sizeof(tb));
+  if (c.k > 0) {
+    int s = c.a_major == FP8_K_MAJOR ? make_map(&ta, c.a, c.k, c.m, c.lda, 128, 128)
+                                     : make_map(&ta, c.a, c.m, c.k, c.lda, 128, 128);
+    if (s) return s;
+    s = c.b_major == FP8_K_MAJOR ? make_map(&tb, c.b, c.k, c.n, c.ldb, 128, bn)
+                                 : make_map(&tb, c.b, c.n, c.k, c.ldb, 128, 128);
+    if (s) return s;
+  }
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.m = static_cast<int>(c.m);
+  p.n = static_cast<int>(c.n);
+  p.k = static_cast<int>(c.k);
+  p.tiles_m = static_cast<int>((c.m + 127) / 128);
+  p.tiles_n = static_cast<int>((c.n + bn - 1) / bn);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.k_blocks = static_cast<int>((c.k + 127) / 128);
+  p.raster_group = 8;
+  p.idesc = idesc_f8(c.fmt_a, c.fmt_b, c.a_major, c.b_major, 128, bn);
+  p.a_major = c.a_major;
+  p.b_major = c.b_major;
+  p.scale_a = c.scale_a;
+  p.scale_b = c.scale_b;
+  p.bias = c.bias;
+  p.bias_kind = !c.bias ? 0 : (c.bias_dtype == FP8_DT_BF16 ? 1 : (c.bias_dtype == FP8_DT_E4M3 ? 2 : 3));
+  p.bias_scale = c.bias_scale;
+  p.d = c.d;
+  p.ldd = c.ldd;
+  p.vec_store = aligned(c.d, 16) && ((c.ldd * 2) % 16 == 0);
+  p.status = status_ptr(dev);
+  if (side) p.side = *side;
+  e = launch_gemm(ta, tb, p, bn, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FP8_OK;
+}
+
+int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt, void* ring,
+                 int H, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out, cudaStream_t st) {
+  QuantizeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.in = in;
+  p.out = out;
+  p.ring = static_cast<float*>(ring);
+  p.H = H;
+  p.fp8_max = fp8_max(fmt);
+  p.amax_out = amax_out;
+  p.scale_out = scale_out;
+  const int es = esize(in_dtype);
+  if (ld_in == cols && ld_out == cols) {  // contiguous: one long row
+    p.rows = 1;
+    p.cols = rows * cols;
+    p.ld_in = p.cols;
+    p.ld_out = p.cols;
+  } else {
+    p.rows = rows;
+    p.cols = cols;
+    p.ld_in = ld_in;
+    p.ld_out = ld_out;
+  }
+  p.chunks_per_row = (p.cols + 15) / 16;
+  p.total_chunks = p.rows * p.chunks_per_row;
+  p.vec_ok = aligned(in, 16) && ((p.ld_in * es) % 16 == 0);
+  cudaError_t e = launch_quantize(in_dtype, fmt, p, st);
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
+int validate_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt,
+                      void* ring, int H, uint8_t* out, int64_t ld_out) {
+  if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
+  if (!is_wide(in_dtype) || !is_fmt(fmt)) return FP8_ERR_INVALID_ARG;
+  if (!ring_len_ok(H)) return FP8_ERR_INVALID_ARG;
+  if (!in || !ring || !out) return FP8_ERR_INVALID_ARG;
+  if (!aligned(ring, 4) || !aligned(in, esize(in_dtype))) return FP8_ERR_INVALID_ARG;
+  if (ld_in < cols) return FP8_ERR_INVALID_ARG;
+  return check_fp8_matrix(out, ld_out, cols);
+}
+
+}  // namespace
+
+int num_sms(int dev) {
+  if (dev < 0 || dev >= 64) return 0;
+  if (!g_sms[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    g_sms[dev] = v;
+  }
+  return g_sms[dev];
+}
+
+}  // namespace fp8lin
+
+using namespace fp8lin;
+
+extern "C" {
+
+size_t fp8_ring_bytes(int hist_len) {
+  return ring_len_ok(hist_len) ? static_cast<size_t>(hist_len + 4) * 4u : 0u;
+}
+
+int fp8_ring_init(void* ring, int hist_len, fp8_stream_t stream) {
+  if (!ring || !ring_len_ok(hist_len) || !aligned(ring, 4)) return FP8_ERR_INVALID_ARG;
+  cudaError_t e = launch_ring_set(static_cast<float*>(ring), hist_len, 1.0f, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
+int fp8_ring_seed(void* ring, int hist_len, int fmt, float amax, fp8_stream_t stream) {
+  if (!ring || !ring_len_ok(hist_len) || !aligned(ring, 4) || !is_fmt(fmt)) return FP8_ERR_INVALID_ARG;
+  float s = 1.0f;
+  if (amax > 0.0f && std::isfinite(amax)) {
+    volatile float q = fp8_max(fmt) / amax;
+    if (std::isfinite(q)) s = q;
+  }
+  cudaError_t e = launch_ring_set(static_cast<float*>(ring), hist_len, s, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
+int fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt, void* ring,
+                 int hist_len, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out,
+                 fp8_stream_t stream) {
+  int s = validate_quantize(in, in_dtype, rows, cols, ld_in, fmt, ring, hist_len, out, ld_out);
+  if (s) return s;
+  if (rows == 0 || cols == 0) return FP8_OK;
+  return run_quantize(in, in_dtype, rows, cols, ld_in, fmt, ring, hist_len, out, ld_out, amax_out, scale_out,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fp8_mm(const fp8_mm_args* a, fp8_stream_t stream) {
+  if (!a) return FP8_ERR_INVALID_ARG;
+  MmCall c{a->m, a->n, a->k, a->a, a->fmt_a, a->a_major, a->lda, a->b, a->fmt_b, a->b_major, a->ldb,
+           a->scale_a, a->scale_b, a->bias, a->bias_dtype, a->bias_scale, a->d, a->ldd};
+  int s = validate_mm(c);
+  if (s) return s;
+  if (c.m == 0 || c.n == 0 || c.k == 0) return FP8_OK;
+  return run_mm(c, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fp8_dbias_workspace_bytes(int64_t M, int64_t N) {
+  if (M <= 0 || N <= 0) return 0;
+  int R;
+  int64_t rps;
+  dbias_geometry(M, N, &R, &rps);
+  const int64_t tiles = (N + kDbiasColsPerTile - 1) / kDbiasColsPerTile;
+  const size_t part = (static_cast<size_t>(R) * static_cast<size_t>(N) * 4u + 15u) & ~size_t(15);
+  return part + ((static_cast<size_t>(tiles) * 4u + 15u) & ~size_t(15));
+}
+
+int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg, const float* g_scale, void* dbias,
+              void* workspace, size_t workspace_bytes, fp8_stream_t stream) {
+  if (M < 0 || N < 0 || M > kMaxDim || N > kMaxDim) return FP8_ERR_INVALID_ARG;
+  if (!is_wide(g_dtype) && !is_fp8(g_dtype)) return FP8_ERR_INVALID_ARG;
+  if (!g || !dbias || ldg < N || !aligned(g, esize(g_dtype)) || !aligned(dbias, 2)) return FP8_ERR_INVALID_ARG;
+  if (is_fp8(g_dtype) && !g_scale) return FP8_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP8_OK;
+  const size_t need = fp8_dbias_workspace_bytes(M, N);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return FP8_ERR_WORKSPACE;
+  DbiasParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.g = g;
+  p.dtype = g_dtype;
+  p.M = M;
+  p.N = N;
+  p.ldg = ldg;
+  p.g_scale = g_scale;
+  p.dbias = dbias;
+  dbias_geometry(M, N, &p.R, &p.rows_per_split);
+  p.partial = static_cast<float*>(workspace);
+  const size_t part = (static_cast<size_t>(p.R) * static_cast<size_t>(N) * 4u + 15u) & ~size_t(15);
+  p.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + part);
+  const int es = esize(g_dtype);
+  p.vec_ok = is_fp8(g_dtype) ? (aligned(g, 8) && (ldg % 8 == 0)) : (aligned(g, 16) && ((ldg * es) % 16 == 0));
+  cudaError_t e = launch_dbias(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
+size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)K;
+  return fp8_dbias_workspace_bytes(M, N);
+}
+
+int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
+  if (!a) return FP8_ERR_INVALID_ARG;
+  const int64_t M = a->M, N = a->N, K = a->K;
+  if (M < 0 || N < 0 || K < 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8_ERR_INVALID_ARG;
+  if (!is_fmt(a->fmt_x) || !is_fmt(a->fmt_w)) return FP8_ERR_INVALID_ARG;
+  if (!a->x || !a->w || !a->y || !a->sx_out || !a->sw_out) return FP8_ERR_INVALID_ARG;
+  const bool xq = is_fp8(a->x_dtype), wq = is_fp8(a->w_dtype);
+  if (!xq && !is_wide(a->x_dtype)) return FP8_ERR_INVALID_ARG;
+  if (!wq && !is_wide(a->w_dtype)) return FP8_ERR_INVALID_ARG;
+  int s;
+  if (xq) {
+    if (a->x_dtype - FP8_DT_E4M3 != a->fmt_x || !a->x_scale_in) return FP8_ERR_INVALID_ARG;
+    if ((s = check_fp8_matrix(a->x, a->ldx, K))) return s;
+  } else if ((s = validate_quantize(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8,
+                                    a->ldx8))) {
+    return s;
+  }
+  if (wq) {
+    if (a->w_dtype - FP8_DT_E4M3 != a->fmt_w || !a->w_scale_in) return FP8_ERR_INVALID_ARG;
+    if ((s = check_fp8_matrix(a->w, a->ldw, K))) return s;
+  } else if ((s = validate_quantize(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8,
+                                    a->ldw8))) {
+    return s;
+  }
+  if (!xq && !wq && a->ring_x == a->ring_w) return FP8_ERR_INVALID_ARG;
+  const uint8_t* x8 = xq ? static_cast<const uint8_t*>(a->x) : a->x8;
+  const uint8_t* w8 = wq ? static_cast<const uint8_t*>(a->w) : a->w8;
+  MmCall c{M, N, K, x8, a->fmt_x, FP8_K_MAJOR, xq ? a->ldx : a->ldx8, w8, a->fmt_w, FP8_K_MAJOR,
+           wq ? a->ldw : a->ldw8, xq ? a->x_scale_in : a->sx_out, wq ? a->w_scale_in : a->sw_out,
+           a->bias, a->bias_dtype, a->bias_scale, a->y, a->ldy};
+  if ((s = validate_mm(c))) return s;
+  if (M == 0 || N == 0 || K == 0) return FP8_OK;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  SideWrites side;
+  std::memset(&side, 0, sizeof(side));
+  if (xq) {
+    side.copy_src[0] = a->x_scale_in; side.copy_dst[0] = a->sx_out; side.zero_dst[0] = a->amax_x_out;
+  } else if ((s = run_quantize(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8, a->ldx8,
+                               a->amax_x_out, a->sx_out, st))) {
+    return s;
+  }
+  if (wq) {
+    side.copy_src[1] = a->w_scale_in; side.copy_dst[1] = a->sw_out; side.zero_dst[1] = a->amax_w_out;
+  } else if ((s = run_quantize(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8, a->ldw8,
+                               a->amax_w_out, a->sw_out, st))) {
+    return s;
+  }
+  return run_mm(c, &side, st);
+}
+
+int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
+  if (!a) return FP8_ERR_INVALID_ARG;
+  const int64_t M = a->M, N = a->N, K = a->K;
+  if (M < 0 || N < 0 || K < 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8_ERR_INVALID_ARG;
+  if (!is_fmt(a->fmt_g) || !is_fmt(a->fmt_x) || !is_fmt(a->fmt_w)) return FP8_ERR_INVALID_ARG;
+  if (!a->g || !a->sg_out) return FP8_ERR_INVALID_ARG;
+  const bool gq = is_fp8(a->g_dtype);
+  if (!gq && !is_wide(a->g_dtype)) return FP8_ERR_INVALID_ARG;
+  int s;
+  if (gq) {
+    if (a->g_dtype - FP8_DT_E4M3 != a->fmt_g || !a->g_scale_in) return FP8_ERR_INVALID_ARG;
+    if ((s = check_fp8_matrix(a->g, a->ldg, N))) return s;
+  } else if ((s = validate_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8,
+                                    a->ldg8))) {
+    return s;
+  }
+  const uint8_t* g8 = gq ? static_cast<const uint8_t*>(a->g) : a->g8;
+  const int64_t ldg8 = gq ? a->ldg : a->ldg8;
+  const float* sg = gq ? a->g_scale_in : a->sg_out;
+  // dX[M,K] = G8[M,N] . W8[N,K]: A = G8 K-major, B(j=k, n) = W8[n, k] MN-major.
+  MmCall cdx{M, K, N, g8, a->fmt_g, FP8_K_MAJOR, ldg8, a->w8, a->fmt_w, FP8_MN_MAJOR, a->ldw8,
+             sg, a->sw, nullptr, 0, nullptr, a->dx, a->lddx};
+  // dW[N,K] = G8^T . X8: A(i=n, m) = G8[m, n] MN-major, B(j=k, m) = X8[m, k] MN-major.
+  MmCall cdw{N, K, M, g8, a->fmt_g, FP8_MN_MAJOR, ldg8, a->x8, a->fmt_x, FP8_MN_MAJOR, a->ldx8,
+             sg, a->sx, nullptr, 0, nullptr, a->dw, a->lddw};
+  if (a->need_dx && (s = validate_mm(cdx))) return s;
+  if (a->need_dw && (s = validate_mm(cdw))) return s;
+  const size_t ws_need = a->need_dbias ? fp8_dbias_workspace_bytes(M, N) : 0;
+  if (a->need_dbias) {
+    if (!a->dbias || !aligned(a->dbias, 2)) return FP8_ERR_INVALID_ARG;
+    if (ws_need && (!a->workspace || a->workspace_bytes < ws_need || !aligned(a->workspace, 16)))
+      return FP8_ERR_WORKSPACE;
+  }
+  if (M == 0 || N == 0 || K == 0) return FP8_OK;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  SideWrites side;
+  std::memset(&side, 0, sizeof(side));
+  bool side_pending = false;
+  if (gq) {
+    side.copy_src[0] = a->g_scale_in; side.copy_dst[0] = a->sg_out; side.zero_dst[0] = a->amax_g_out;
+    side_pending = true;
+  } else if ((s = run_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
+                               a->amax_g_out, a->sg_out, st))) {
+    return s;
+  }
+  if (a->need_dx) {
+    if ((s = run_mm(cdx, side_pending ? &side : nullptr, st))) return s;
+    side_pending = false;
+  }
+  if (a->need_dw) {
+    if ((s = run_mm(cdw, side_pending ? &side : nullptr, st))) return s;
+    side_pending = false;
+  }
+  if (side_pending) {
+    cudaError_t e = launch_side_writes(side, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (a->need_dbias) {
+    if ((s = fp8_dbias(a->g, a->g_dtype, M, N, a->ldg, a->g_scale_in, a->dbias, a->workspace, a->workspace_bytes,
+                       stream)))
+      return s;
+  }
+  return FP8_OK;
+}
+
+int fp8_get_device_status(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8_ERR_CUDA;
+  int* p = status_ptr(dev);
+  if (!p) return cuda_fail(cudaGetLastError());
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return v;
+}
+
+const char* fp8_status_string(int status) {
+  switch (status) {
+    case FP8_OK: return "ok";
+    case FP8_ERR_INVALID_ARG: return "invalid argument";
+    case FP8_ERR_UNSUPPORTED: return "unsupported";
+    case FP8_ERR_MISALIGNED: return "fp8 matrix misaligned (ld % 16 != 0 or base not 16-byte aligned)";
+    case FP8_ERR_CUDA: return g_err[0] ? g_err : "CUDA error";
+    case FP8_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case FP8_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+  }
+}
+
+const char* fp8_version(void) { return "fp8lin 0.1 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,167 @@
+// dbias.cu -- bias gradient: dbias[n] = bf16( sum_m g[m, n] ), fp32 sums.
+//
+// Computed only when the bias needs a gradient (AstrAI commit log, astrai
+// @4019dda, bullet on the unconditional column sum).  A pre-quantized g is
+// dequantized element by element before the sum (astrai/extension/ops
+// @057c0d3, grad dtype bullet).
+//
+// HBM-bound: one read of g.  Grid (column tiles of 256, R row splits); a
+// block of 8 x 32 threads streams rows of its split with 16-byte loads (8
+// columns per thread), reduces its 8 row lanes in shared memory in a fixed
+// order and writes 256 fp32 partials.  The block that draws the last ticket
+// of its column tile sums the R partials in split order, so the result does
+// not depend on block scheduling, and rezeroes the tile's counter.
+#include "device.cuh"
+#include "internal.h"
+
+namespace fp8lin {
+namespace {
+
+constexpr int kCols = kDbiasColsPerTile;  // 256 = 32 lanes x 8 columns
+constexpr int kRowLanes = 8;
+
+template <int DT>
+__device__ __forceinline__ void load8(const DbiasParams& p, int64_t r, int64_t c, float inv, float (&v)[8]) {
+  const int64_t idx = r * p.ldg + c;
+  const bool full = c + 8 <= p.N;
+  if constexpr (DT == kBF16) {
+    const uint16_t* g = static_cast<const uint16_t*>(p.g);
+    if (p.vec_ok && full) {
+      uint4 q = __ldg(reinterpret_cast<const uint4*>(g + idx));
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&q);
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    } else {
+      #pragma unroll
+      for (int j = 0; j < 8; ++j)
+        v[j] = (c + j < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(g + idx + j)) << 16) : 0.0f;
+    }
+  } else if constexpr (DT == kFP16) {
+    const __half* g = static_cast<const __half*>(p.g);
+    if (p.vec_ok && full) {
+      uint4 q = __ldg(reinterpret_cast<const uint4*>(g + idx));
+      const __half2* h = reinterpret_cast<const __half2*>(&q);
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 f = __half22float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+      }
+    } else {
+      #pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = (c + j < p.N) ? __half2float(g[idx + j]) : 0.0f;
+    }
+  } else if constexpr (DT == kFP32) {
+    const float* g = static_cast<const float*>(p.g);
+    if (p.vec_ok && full) {
+      float4 a = __ldg(reinterpret_cast<const float4*>(g + idx));
+      float4 b = __ldg(reinterpret_cast<const float4*>(g + idx) + 1);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+      #pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = (c + j < p.N) ? __ldg(g + idx + j) : 0.0f;
+    }
+  } else {
+    const uint8_t* g = static_cast<const uint8_t*>(p.g);
+    uint32_t w[2];
+    if (p.vec_ok && full) {
+      uint2 q = __ldg(reinterpret_cast<const uint2*>(g + idx));
+      w[0] = q.x;
+      w[1] = q.y;
+    } else {
+      w[0] = w[1] = 0;
+      #pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (c + j < p.N) w[j >> 2] |= static_cast<uint32_t>(__ldg(g + idx + j)) << (8 * (j & 3));
+    }
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint16_t pair = static_cast<uint16_t>(w[i >> 1] >> (16 * (i & 1)));
+      const float2 f = DT == kDtE4M3 ? dec_e4m3x2(pair) : dec_e5m2x2(pair);
+      v[2 * i] = f.x * inv;
+      v[2 * i + 1] = f.y * inv;
+    }
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kRowLanes * 32) dbias_kernel(const DbiasParams p) {
+  __shared__ float red[kRowLanes][kCols];
+  __shared__ int last;
+  const int tx = threadIdx.x & 31;
+  const int ty = threadIdx.x >> 5;
+  const int64_t c_base = static_cast<int64_t>(blockIdx.x) * kCols;
+  const int64_t c = c_base + tx * 8;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * p.rows_per_split;
+  const int64_t r1 = min(p.M, r0 + p.rows_per_split);
+  const float inv = (DT == kDtE4M3 || DT == kDtE5M2) ? 1.0f / *p.g_scale : 1.0f;
+
+  float acc[8];
+  #pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+  if (c < p.N) {
+    #pragma unroll 2
+    for (int64_t r = r0 + ty; r < r1; r += kRowLanes) {
+      float v[8];
+      load8<DT>(p, r, c, inv, v);
+      #pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += v[j];
+    }
+  }
+  #pragma unroll
+  for (int j = 0; j < 8; ++j) red[ty][tx * 8 + j] = acc[j];
+  __syncthreads();
+
+  const int64_t col = c_base + threadIdx.x;
+  float s = 0.0f;
+  #pragma unroll
+  for (int y = 0; y < kRowLanes; ++y) s += red[y][threadIdx.x];
+  if (col < p.N) p.partial[static_cast<int64_t>(blockIdx.y) * p.N + col] = s;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&p.counters[blockIdx.x], 1u) == static_cast<unsigned>(p.R - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  if (col < p.N) {
+    float tot = 0.0f;
+    for (int r = 0; r < p.R; ++r) tot += __ldcg(p.partial + static_cast<int64_t>(r) * p.N + col);
+    static_cast<__nv_bfloat16*>(p.dbias)[col] = __float2bfloat16_rn(tot);
+  }
+  if (threadIdx.x == 0) atomicExch(&p.counters[blockIdx.x], 0u);
+}
+
+}  // namespace
+
+void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
+  const int64_t col_tiles = (N + kCols - 1) / kCols;
+  int64_t r = (1184 + col_tiles - 1) / (col_tiles > 0 ? col_tiles : 1);
+  const int64_t rmax = (M + 31) / 32;
+  if (r > rmax) r = rmax;
+  if (r < 1) r = 1;
+  int64_t rps = (M + r - 1) / r;
+  if (rps < 1) rps = 1;
+  r = (M + rps - 1) / rps;
+  if (r < 1) r = 1;
+  *R = static_cast<int>(r);
+  *rows_per_split = rps;
+}
+
+cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>((p.N + kCols - 1) / kCols), static_cast<unsigned>(p.R));
+  const int threads = kRowLanes * 32;
+  switch (p.dtype) {
+    case kBF16: dbias_kernel<kBF16><<<grid, threads, 0, s>>>(p); break;
+    case kFP16: dbias_kernel<kFP16><<<grid, threads, 0, s>>>(p); break;
+    case kFP32: dbias_kernel<kFP32><<<grid, threads, 0, s>>>(p); break;
+    case kDtE4M3: dbias_kernel<kDtE4M3><<<grid, threads, 0, s>>>(p); break;
+    default: dbias_kernel<kDtE5M2><<<grid, threads, 0, s>>>(p); break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fp8lin

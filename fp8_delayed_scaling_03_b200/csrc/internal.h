@@ -1,0 +1,87 @@
+// internal.h -- launchers shared between the translation units of libfp8lin.
+// Host-side only types; no CUDA device code.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fp8lin {
+
+enum : int { kE4M3 = 0, kE5M2 = 1 };
+enum : int { kBF16 = 0, kFP16 = 1, kFP32 = 2, kDtE4M3 = 3, kDtE5M2 = 4 };
+
+// Ring word offsets (in 32-bit words) for history length H.
+inline int ring_scale(int H) { return H; }
+inline int ring_ticket(int H) { return H + 1; }
+inline int ring_step(int H) { return H + 2; }
+inline int ring_scratch(int H) { return H + 3; }
+
+struct QuantizeParams {
+  const void* in;
+  int64_t rows, cols, ld_in;  // rows == 1 with cols = total for contiguous data
+  uint8_t* out;
+  int64_t ld_out;
+  int64_t chunks_per_row;     // ceil(cols / 16)
+  int64_t total_chunks;
+  float* ring;                // [hist | scale | ticket | step | scratch]
+  int H;
+  float fp8_max;
+  float* amax_out;
+  float* scale_out;
+  int vec_ok;                 // 16-byte vector loads are legal for full chunks
+};
+
+// Side writes a GEMM launch performs once (block 0), for operands that arrive
+// pre-quantized: dst = *src for the scale snapshot, zero for its amax.
+struct SideWrites {
+  const float* copy_src[2];
+  float* copy_dst[2];
+  float* zero_dst[2];
+};
+
+struct GemmParams {
+  int m, n, k;
+  int tiles_m, tiles_n, num_tiles, k_blocks;
+  int raster_group;           // M-tiles per raster group
+  uint32_t idesc;
+  int a_major, b_major;
+  const float* scale_a;
+  const float* scale_b;
+  const void* bias;
+  int bias_kind;              // 0 none, 1 bf16, 2 e4m3, 3 e5m2
+  const float* bias_scale;
+  void* d;
+  int64_t ldd;
+  int vec_store;              // 16-byte stores of bf16 rows are legal
+  int* status;
+  SideWrites side;
+};
+
+struct DbiasParams {
+  const void* g;
+  int dtype;
+  int64_t M, N, ldg;
+  const float* g_scale;
+  void* dbias;
+  float* partial;             // [R, N] fp32
+  unsigned* counters;         // [col_tiles]
+  int64_t rows_per_split;
+  int R;
+  int vec_ok;
+};
+
+int num_sms(int device);
+
+cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams& p, cudaStream_t s);
+cudaError_t launch_ring_set(float* ring, int H, float scale, cudaStream_t s);
+cudaError_t launch_side_writes(const SideWrites& w, cudaStream_t s);
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, int bn, cudaStream_t s);
+cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s);
+
+// dbias geometry shared by the size query and the launcher.
+constexpr int kDbiasColsPerTile = 256;
+void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split);
+
+}  // namespace fp8lin

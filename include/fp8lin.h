@@ -1,0 +1,225 @@
+/*
+ * fp8lin.h -- C ABI of the FP8 linear layer with delayed scaling (sm_100a).
+ *
+ * Sources: the AstrAI commit logs, cited by the path filter and commit of the
+ * page and by the bullet that states the behaviour:
+ *   [tests/extension@2eeac02]      ring finalize in the quantize kernel, bias
+ *                                  fusion, pre-quantized w8, autograd pair;
+ *   [csrc@2eeac02]                 FP8 GEMM kernel history, FP8Params bias;
+ *   [astrai/extension/ops@057c0d3] two-primitive API (quantize + mm_fp8),
+ *                                  scale snapshot, backward scale reuse;
+ *   [astrai@4019dda]               in-kernel fold, fused bias epilogue, dbias
+ *                                  only when requested;
+ *   [astrai/extension/fp8.py@3e57cc8] amax of raw values, E5M2 gradients.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless marked "host".  The caller allocates
+ *     and owns every buffer; the library allocates nothing and keeps no pointer
+ *     after a call returns.
+ *   - Work is enqueued on `stream` in stream order; no call synchronizes the
+ *     host.  A ring (and a workspace) must not be used by two launches that can
+ *     run concurrently.
+ *   - Arguments are validated before anything is enqueued.  A failed check
+ *     returns a negative fp8_status and enqueues nothing.  A launch failure
+ *     returns FP8_ERR_CUDA; fp8_status_string(FP8_ERR_CUDA) then names the CUDA
+ *     error.  Sizes of zero are accepted and do nothing (rings untouched).
+ *   - Matrices are row-major with an explicit row stride `ld` in ELEMENTS.
+ *     fp8 matrices (read or written) need ld % 16 == 0 and a 16-byte aligned
+ *     base (the GEMMs read them with TMA); bf16/fp16/fp32 inputs may have any
+ *     ld >= cols and any element-aligned base.  bf16 outputs need an even-byte
+ *     aligned base and ld >= cols.
+ */
+#ifndef FP8LIN_H
+#define FP8LIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8LIN_API __attribute__((visibility("default")))
+#else
+#define FP8LIN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fp8_stream_t;  /* = cudaStream_t; NULL = legacy default stream */
+
+typedef enum { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_fmt;
+
+typedef enum {
+  FP8_DT_BF16 = 0, FP8_DT_FP16 = 1, FP8_DT_FP32 = 2, FP8_DT_E4M3 = 3, FP8_DT_E5M2 = 4
+} fp8_dtype;
+
+typedef enum { FP8_K_MAJOR = 0, FP8_MN_MAJOR = 1 } fp8_major;
+
+typedef enum {
+  FP8_OK = 0,
+  FP8_ERR_INVALID_ARG = -1,    /* NULL required pointer, bad enum, ld < cols, ... */
+  FP8_ERR_UNSUPPORTED = -2,    /* valid request this build does not implement   */
+  FP8_ERR_MISALIGNED = -3,     /* fp8 ld % 16 != 0 or base not 16-byte aligned  */
+  FP8_ERR_CUDA = -4,           /* a CUDA call failed (see fp8_status_string)    */
+  FP8_ERR_DEVICE_TIMEOUT = -5, /* a kernel gave up on a bounded wait            */
+  FP8_ERR_WORKSPACE = -6       /* workspace missing or smaller than required    */
+} fp8_status;
+
+/* ------------------------------------------------------------------ rings
+ * A scale ring is the delayed-scaling state of one tensor, one device buffer
+ * of fp8_ring_bytes(H) bytes, 4-byte aligned, laid out as 32-bit words:
+ *   [0, H)   hist    fp32 amax history (slot step % H holds the newest)
+ *   H        scale   fp32 scale the next quantize multiplies by
+ *   H+1      ticket  u32 block counter of the in-kernel finalize (0 at rest)
+ *   H+2      step    u32 number of quantizes folded so far
+ *   H+3      scratch u32 bits of the running amax of a launch (0 at rest)
+ * [tests/extension@2eeac02]: the ring packs history, scale and counter in one
+ * buffer; the quantize kernel's last block folds the amax in and publishes
+ * the next scale, so a step costs no extra launch.  Checkpointing a ring is
+ * copying its bytes between launches.  1 <= H <= 4096. */
+FP8LIN_API size_t fp8_ring_bytes(int hist_len);
+
+/* hist = 0, scale = 1.0, ticket = step = scratch = 0.  One tiny kernel. */
+FP8LIN_API int fp8_ring_init(void* ring, int hist_len, fp8_stream_t stream);
+
+/* fp8_ring_init, then scale = fp8_max(fmt) / amax when amax (host value) is
+ * positive and finite and the quotient is finite; otherwise scale stays 1.0.
+ * The history is left at zero ([astrai@4019dda] names seed() on the ring). */
+FP8LIN_API int fp8_ring_seed(void* ring, int hist_len, int fmt, float amax, fp8_stream_t stream);
+
+/* ------------------------------------------------------------------ quantize
+ * out[r, c] = cast_sat_rne_fmt( fp32(in[r, c]) * s ), s = the ring's scale at
+ * launch, for r < rows, c < cols; bytes c in [cols, ld_out) are written 0.
+ * In the same launch: amax = max |fp32(in)| over non-NaN elements of the RAW
+ * input ([astrai/extension/fp8.py@3e57cc8]: the quantized max pinned the scale
+ * at 1); the last block to finish then writes hist[step % H] = amax, takes
+ * m = max(hist), publishes scale = fp8_max / m (kept when m is 0 or inf or the
+ * quotient overflows), advances step, and rezeroes ticket and scratch.
+ *   in        bf16/fp16/fp32 [rows, ld_in]            (in_dtype FP8_DT_BF16/FP16/FP32)
+ *   fmt       FP8_E4M3 (max 448) or FP8_E5M2 (max 57344)
+ *   ring      required; fp8_ring_bytes(hist_len) bytes, initialized
+ *   out       fp8 codes [rows, ld_out], ld_out % 16 == 0, 16-byte aligned
+ *   amax_out  optional fp32: the amax of this launch
+ *   scale_out optional fp32: the scale this launch multiplied by (the snapshot
+ *             taken before the ring overwrites it, [astrai/extension/ops@057c0d3])
+ * NaN inputs give the NaN code and do not enter amax; +-inf saturate to +-max. */
+FP8LIN_API int fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in,
+                 int fmt, void* ring, int hist_len,
+                 uint8_t* out, int64_t ld_out,
+                 float* amax_out, float* scale_out, fp8_stream_t stream);
+
+/* ------------------------------------------------------------------ mm
+ * The GEMM primitive ([astrai/extension/ops@057c0d3] two-primitive API;
+ * [astrai@4019dda] fused bias):
+ *   D[i, j] = bf16_rne( (sum_k A(i,k) * B(j,k)) / (scale_a * scale_b) + bias[j] )
+ * products and sums in fp32 on the tensor cores (tcgen05, kind::f8f6f4), one
+ * rounding to bf16.  Operand storage:
+ *   a_major FP8_K_MAJOR : A(i,k) = a[i*lda + k]  (a is [m, lda], lda >= k)
+ *   a_major FP8_MN_MAJOR: A(i,k) = a[k*lda + i]  (a is [k, lda], lda >= m)
+ *   b_major FP8_K_MAJOR : B(j,k) = b[j*ldb + k]  (b is [n, ldb], ldb >= k)
+ *   b_major FP8_MN_MAJOR: B(j,k) = b[k*ldb + j]  (b is [k, ldb], ldb >= n)
+ * so the forward (X W^T: both K-major), dX (G W: A K-major, B MN-major) and
+ * dW (G^T X: both MN-major) run without transposed copies.
+ *   scale_a, scale_b  required device fp32 scalars (the quantize snapshots)
+ *   bias              optional [n]: bias_dtype FP8_DT_BF16 adds the bf16 value;
+ *                     FP8_DT_E4M3/E5M2 adds decode(bias[j]) / *bias_scale
+ *                     ([csrc@2eeac02] FP8Params bias bullet: fp8 bias
+ *                     dequantized after the operand scaling)
+ *   d                 bf16 [m, ldd], ldd >= n
+ * Out-of-range rows/columns/k of partial tiles contribute nothing. */
+typedef struct fp8_mm_args {
+  int64_t m, n, k;
+  const uint8_t* a; int fmt_a; int a_major; int64_t lda;
+  const uint8_t* b; int fmt_b; int b_major; int64_t ldb;
+  const float* scale_a; const float* scale_b;
+  const void* bias; int bias_dtype; const float* bias_scale;
+  void* d; int64_t ldd;
+} fp8_mm_args;
+FP8LIN_API int fp8_mm(const fp8_mm_args* args, fp8_stream_t stream);
+
+/* ------------------------------------------------------------------ dbias
+ * dbias[n] = bf16_rne( sum_m g(m, n) ), fp32 sums, for n < N.  g is bf16,
+ * fp16 or fp32 [M, ldg], or fp8 (E4M3/E5M2) [M, ldg] with g_scale required:
+ * then each element is dequantized, decode(g8) / *g_scale, before the sum
+ * ([astrai/extension/ops@057c0d3]: a pre-quantized g dequantizes before the
+ * bias sum).  The result is deterministic for a given (M, N) (fixed partial
+ * order).  workspace: >= fp8_dbias_workspace_bytes(M, N) bytes, 16-byte
+ * aligned, ZERO-FILLED before its first use; every call leaves it ready for
+ * the next (its counters back at zero). */
+FP8LIN_API size_t fp8_dbias_workspace_bytes(int64_t M, int64_t N);
+FP8LIN_API int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg,
+              const float* g_scale, void* dbias,
+              void* workspace, size_t workspace_bytes, fp8_stream_t stream);
+
+/* ------------------------------------------------------------------ linear
+ * Forward of the FP8 linear ([tests/extension@2eeac02], [astrai/extension/ops@057c0d3]):
+ *   x [M, K] and w [N, K] (PyTorch out x in) are each either bf16/fp16/fp32,
+ *   quantized here with their own ring (x with fmt_x into x8, w with fmt_w into
+ *   w8), or already fp8 in the matching format, in which case the quantize is
+ *   skipped, the operand is used in place, its scale is *x_scale_in /
+ *   *w_scale_in and its amax output is 0 ([tests/extension@2eeac02], w8 bullet).
+ *   Then y = bf16( X8 W8^T / (sx sw) + bias ), as fp8_mm.
+ * Outputs: y (bf16 [M, ldy]); x8/w8 (fp8, kept by the caller for the
+ * backward; unused when that operand arrives fp8); sx_out/sw_out (required:
+ * the scales the GEMM dequantized with); amax_x_out/amax_w_out (optional).
+ * 2 to 3 launches.  hist_len is the H of both rings. */
+typedef struct fp8_linear_fwd_args {
+  int64_t M, N, K;
+  const void* x; int x_dtype; int64_t ldx; const float* x_scale_in;
+  const void* w; int w_dtype; int64_t ldw; const float* w_scale_in;
+  const void* bias; int bias_dtype; const float* bias_scale;
+  int fmt_x, fmt_w, hist_len;
+  void* ring_x; void* ring_w;
+  uint8_t* x8; int64_t ldx8;
+  uint8_t* w8; int64_t ldw8;
+  float* sx_out; float* sw_out; float* amax_x_out; float* amax_w_out;
+  void* y; int64_t ldy;
+} fp8_linear_fwd_args;
+FP8LIN_API int fp8_linear_forward(const fp8_linear_fwd_args* args, fp8_stream_t stream);
+
+/* Backward of the FP8 linear ([astrai/extension/ops@057c0d3]):
+ *   g [M, N] is bf16/fp16/fp32, quantized with ring_g (fmt_g, normally E5M2)
+ *   into g8, or already fp8 (then *g_scale_in is its scale, amax_g_out = 0).
+ *   dx = bf16( G8 W8 / (sg sw) )    [M, K]  when need_dx
+ *   dw = bf16( G8^T X8 / (sg sx) )  [N, K]  when need_dw
+ *   dbias = bf16( sum_m g )         [N]     when need_dbias ([astrai@4019dda]:
+ *                                           only when the bias needs a grad)
+ * sx, sw, x8, w8 are the FORWARD's snapshots and quantized operands: the
+ * backward reuses the forward's scales.  Outputs are bf16 whatever the input
+ * dtypes.  workspace: as fp8_dbias, needed only when need_dbias (size from
+ * fp8_linear_workspace_bytes).  Up to 4 launches. */
+typedef struct fp8_linear_bwd_args {
+  int64_t M, N, K;
+  const void* g; int g_dtype; int64_t ldg; const float* g_scale_in;
+  int fmt_g, hist_len; void* ring_g;
+  uint8_t* g8; int64_t ldg8;
+  float* sg_out; float* amax_g_out;
+  const uint8_t* x8; int64_t ldx8; const float* sx; int fmt_x;
+  const uint8_t* w8; int64_t ldw8; const float* sw; int fmt_w;
+  int need_dx, need_dw, need_dbias;
+  void* dx; int64_t lddx;
+  void* dw; int64_t lddw;
+  void* dbias;
+  void* workspace; size_t workspace_bytes;
+} fp8_linear_bwd_args;
+FP8LIN_API int fp8_linear_backward(const fp8_linear_bwd_args* args, fp8_stream_t stream);
+
+FP8LIN_API size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* ------------------------------------------------------------------ status
+ * Kernels never wait without a bound: a wait that runs out records
+ * FP8_ERR_DEVICE_TIMEOUT in a device word and the kernel returns.  This call
+ * reads that word (synchronizing the device) and clears it; FP8_OK if clear. */
+FP8LIN_API int fp8_get_device_status(void);
+
+/* Static description of a status code (for FP8_ERR_CUDA: the last CUDA error
+ * this library saw, on the calling host thread). */
+FP8LIN_API const char* fp8_status_string(int status);
+
+/* Library version string, e.g. "fp8lin 0.1 sm_100a". */
+FP8LIN_API const char* fp8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8LIN_H */

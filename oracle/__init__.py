@@ -185,7 +185,8 @@ class Ring:
         a = np.float32(amax_value)
         s = np.float32(1.0)
         if np.isfinite(a) and a > 0:
-            q = np.float32(FP8_MAX[fmt]) / a
+            with np.errstate(over="ignore"):
+                q = np.float32(FP8_MAX[fmt]) / a
             if np.isfinite(q):
                 s = np.float32(q)
         self.scale = s

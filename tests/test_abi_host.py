@@ -1,0 +1,165 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/fp8lin.h, and rejects bad arguments before enqueuing any
+work (so no CUDA call is reached here).  Pointers passed are fake aligned
+addresses; validation never dereferences them."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    from fp8_delayed_scaling_03_b200 import build as b
+    b.build()
+    import fp8_delayed_scaling_03_b200 as m
+    return m
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "fp8lin.h")).read()
+    return re.findall(r"FP8LIN_API\s+[\w\s\*]+?\b(fp8_\w+)\s*\(", src)
+
+
+def test_exports_every_header_symbol(fp8):
+    names = header_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(fp8._lib, n), n
+        assert n in fp8.EXPORTED, n
+    assert set(fp8.EXPORTED) == set(names)
+
+
+def test_version_and_status_strings(fp8):
+    assert "sm_100a" in fp8.fp8_version()
+    for s in (0, -1, -2, -3, -5, -6):
+        assert fp8.fp8_status_string(s)
+    assert fp8.fp8_status_string(12345) == "unknown status"
+
+
+def test_ring_bytes(fp8):
+    assert fp8.fp8_ring_bytes(16) == 80
+    assert fp8.fp8_ring_bytes(1) == 20
+    assert fp8.fp8_ring_bytes(0) == 0
+    assert fp8.fp8_ring_bytes(4097) == 0
+
+
+A = 0x100000  # a fake 16-byte aligned device address
+
+
+def q(fp8, **kw):
+    a = dict(inp=A, dt=fp8.FP8_DT_BF16, rows=4, cols=32, ld_in=32, fmt=0, ring=A + 0x1000, H=16,
+             out=A + 0x2000, ld_out=32)
+    a.update(kw)
+    return fp8._lib.fp8_quantize(a["inp"], a["dt"], a["rows"], a["cols"], a["ld_in"], a["fmt"], a["ring"], a["H"],
+                                 a["out"], a["ld_out"], None, None, None)
+
+
+def test_quantize_validation(fp8):
+    E = fp8
+    assert q(fp8, inp=None) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, ring=None) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, out=None) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, dt=E.FP8_DT_E4M3) == E.FP8_ERR_INVALID_ARG       # fp8 input is not quantized again
+    assert q(fp8, dt=9) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, fmt=2) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, H=0) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, ld_in=31) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, ld_out=40) == E.FP8_ERR_MISALIGNED
+    assert q(fp8, out=A + 8) == E.FP8_ERR_MISALIGNED
+    assert q(fp8, ring=A + 2) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, inp=A + 1) == E.FP8_ERR_INVALID_ARG            # bf16 must be 2-byte aligned
+    assert q(fp8, rows=-1) == E.FP8_ERR_INVALID_ARG
+    # zero sizes: accepted, nothing enqueued
+    assert q(fp8, rows=0) == E.FP8_OK
+    assert q(fp8, cols=0, ld_in=0, ld_out=0) == E.FP8_OK
+
+
+def mm(fp8, **kw):
+    a = dict(m=128, n=128, k=128, a=A, fmt_a=0, a_major=0, lda=128, b=A + 0x10000, fmt_b=0, b_major=0, ldb=128,
+             scale_a=A + 0x20000, scale_b=A + 0x20010, bias=None, bias_dtype=0, bias_scale=None, d=A + 0x30000,
+             ldd=128)
+    a.update(kw)
+    args = fp8.MmArgs(**a)
+    return fp8._lib.fp8_mm(ctypes.byref(args), None)
+
+
+def test_mm_validation(fp8):
+    E = fp8
+    assert mm(fp8, scale_a=None) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, d=None) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, a_major=2) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, fmt_b=3) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, lda=136 - 4) == E.FP8_ERR_MISALIGNED
+    assert mm(fp8, lda=112) == E.FP8_ERR_INVALID_ARG                  # lda < k
+    assert mm(fp8, a_major=1, m=300, lda=288) == E.FP8_ERR_INVALID_ARG   # MN-major: lda >= m
+    assert mm(fp8, b=A + 4) == E.FP8_ERR_MISALIGNED
+    assert mm(fp8, ldd=100) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, bias=A, bias_dtype=E.FP8_DT_E4M3) == E.FP8_ERR_INVALID_ARG  # fp8 bias needs a scale
+    assert mm(fp8, bias=A, bias_dtype=E.FP8_DT_FP32) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, m=0) == E.FP8_OK
+    assert mm(fp8, k=0) == E.FP8_OK
+    assert fp8._lib.fp8_mm(None, None) == E.FP8_ERR_INVALID_ARG
+
+
+def test_dbias_workspace_rules(fp8):
+    E = fp8
+    assert fp8.fp8_dbias_workspace_bytes(0, 10) == 0
+    need = fp8.fp8_dbias_workspace_bytes(2048, 1024)
+    assert need > 0 and need % 16 == 0
+    assert fp8.fp8_linear_workspace_bytes(2048, 1024, 4096) == need
+    f = fp8._lib.fp8_dbias
+    assert f(A, E.FP8_DT_BF16, 2048, 1024, 1024, None, A + 0x100, None, 0, None) == E.FP8_ERR_WORKSPACE
+    assert f(A, E.FP8_DT_BF16, 2048, 1024, 1024, None, A + 0x100, A, need - 16, None) == E.FP8_ERR_WORKSPACE
+    assert f(A, E.FP8_DT_E5M2, 2048, 1024, 1024, None, A + 0x100, A, need, None) == E.FP8_ERR_INVALID_ARG
+    assert f(A, E.FP8_DT_BF16, 2048, 1024, 1000, None, A + 0x100, A, need, None) == E.FP8_ERR_INVALID_ARG
+    assert f(A, E.FP8_DT_BF16, 0, 1024, 1024, None, A + 0x100, None, 0, None) == E.FP8_OK
+
+
+def fwd(fp8, **kw):
+    a = dict(M=64, N=192, K=128, x=A, x_dtype=0, ldx=128, x_scale_in=None, w=A + 0x10000, w_dtype=0, ldw=128,
+             w_scale_in=None, bias=None, bias_dtype=0, bias_scale=None, fmt_x=0, fmt_w=0, hist_len=16,
+             ring_x=A + 0x20000, ring_w=A + 0x20100, x8=A + 0x30000, ldx8=128, w8=A + 0x40000, ldw8=128,
+             sx_out=A + 0x50000, sw_out=A + 0x50010, amax_x_out=None, amax_w_out=None, y=A + 0x60000, ldy=192)
+    a.update(kw)
+    return fp8._lib.fp8_linear_forward(ctypes.byref(fp8.LinearFwdArgs(**a)), None)
+
+
+def test_linear_forward_validation(fp8):
+    E = fp8
+    assert fwd(fp8, ring_w=A + 0x20000) == E.FP8_ERR_INVALID_ARG           # one ring for two tensors
+    assert fwd(fp8, sx_out=None) == E.FP8_ERR_INVALID_ARG
+    assert fwd(fp8, x_dtype=E.FP8_DT_E5M2, x_scale_in=A) == E.FP8_ERR_INVALID_ARG  # fmt mismatch
+    assert fwd(fp8, w_dtype=E.FP8_DT_E4M3) == E.FP8_ERR_INVALID_ARG        # pre-quantized needs its scale
+    assert fwd(fp8, w_dtype=E.FP8_DT_E4M3, w_scale_in=A, ldw=136) == E.FP8_ERR_MISALIGNED
+    assert fwd(fp8, ldx8=136) == E.FP8_ERR_MISALIGNED
+    assert fwd(fp8, ldx8=120) == E.FP8_ERR_INVALID_ARG
+    assert fwd(fp8, ldy=100) == E.FP8_ERR_INVALID_ARG
+    assert fwd(fp8, hist_len=0) == E.FP8_ERR_INVALID_ARG
+    assert fwd(fp8, M=0) == E.FP8_OK
+    assert fp8._lib.fp8_linear_forward(None, None) == E.FP8_ERR_INVALID_ARG
+
+
+def bwd(fp8, **kw):
+    a = dict(M=64, N=192, K=128, g=A, g_dtype=0, ldg=192, g_scale_in=None, fmt_g=1, hist_len=16,
+             ring_g=A + 0x20000, g8=A + 0x30000, ldg8=192, sg_out=A + 0x50000, amax_g_out=None,
+             x8=A + 0x40000, ldx8=128, sx=A + 0x50010, fmt_x=0, w8=A + 0x70000, ldw8=128, sw=A + 0x50020, fmt_w=0,
+             need_dx=1, need_dw=1, need_dbias=0, dx=A + 0x80000, lddx=128, dw=A + 0x90000, lddw=128, dbias=None,
+             workspace=None, workspace_bytes=0)
+    a.update(kw)
+    return fp8._lib.fp8_linear_backward(ctypes.byref(fp8.LinearBwdArgs(**a)), None)
+
+
+def test_linear_backward_validation(fp8):
+    E = fp8
+    assert bwd(fp8, need_dbias=1, dbias=A) == E.FP8_ERR_WORKSPACE
+    assert bwd(fp8, need_dbias=1, dbias=None) == E.FP8_ERR_INVALID_ARG
+    assert bwd(fp8, sw=None) == E.FP8_ERR_INVALID_ARG
+    assert bwd(fp8, ldw8=136) == E.FP8_ERR_MISALIGNED
+    assert bwd(fp8, ldx8=136, need_dw=1) == E.FP8_ERR_MISALIGNED
+    assert bwd(fp8, g_dtype=E.FP8_DT_E5M2) == E.FP8_ERR_INVALID_ARG         # pre-quantized g needs its scale
+    assert bwd(fp8, sg_out=None) == E.FP8_ERR_INVALID_ARG
+    assert bwd(fp8, N=0) == E.FP8_OK

@@ -1,0 +1,172 @@
+"""GPU parity of the FP8 GEMM primitive (fp8_mm) against the oracle, for all
+four operand layouts (the forward's K-major x K-major, dX's K-major x MN-major,
+dW's MN-major x MN-major, and MN-major x K-major), ragged and multi-tile
+shapes, both fp8 formats and the bias variants.  Tolerance per element:
+max(1 bf16 ulp of the oracle value, 2e-6 sum_k |a_k b_k| / (sa sb))."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_gemm_close, sample_points
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fp8_delayed_scaling_03_b200 as m
+    return m
+
+
+def codes_like_tensor(rng, fmt, shape, std):
+    """fp8 codes of a normal tensor scaled into the format's range (oracle cast)."""
+    v = (rng.standard_normal(shape) * std).astype(np.float32)
+    return oracle.encode(fmt, v)
+
+
+def store(codes_logical, major, pad):
+    """Logical [I, Kc] operand -> storage array with row stride ld: K-major
+    [I, ld >= Kc], MN-major [Kc, ld >= I].  Padding bytes hold junk (0x77)."""
+    mat = codes_logical if major == 0 else np.ascontiguousarray(codes_logical.T)
+    rows, cols = mat.shape
+    ld = (cols + 15) // 16 * 16 + pad
+    buf = np.full((rows, ld), 0x77, np.uint8)
+    buf[:, :cols] = mat
+    return buf, ld
+
+
+def strides(major, ld):
+    return (ld, 1) if major == 0 else (1, ld)
+
+
+def run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=0, fmt_b=0, sa=1.0, sb=1.0, bias_kind=None,
+             pad=0, ldd_extra=0, full=True, a_codes=None, b_codes=None):
+    A = a_codes if a_codes is not None else codes_like_tensor(rng, fmt_a, (m, k), 60.0 if fmt_a == 0 else 3000.0)
+    B = b_codes if b_codes is not None else codes_like_tensor(rng, fmt_b, (n, k), 60.0 if fmt_b == 0 else 3000.0)
+    a_st, lda = store(A, a_major, pad)
+    b_st, ldb = store(B, b_major, pad)
+    dev_a = torch.from_numpy(a_st).cuda()
+    dev_b = torch.from_numpy(b_st).cuda()
+    scales = torch.tensor([sa, sb], dtype=torch.float32, device="cuda")
+    ldd = n + ldd_extra
+    d = torch.full((m, ldd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    bias = bias_dev = bias_scale = None
+    bias_dtype = fp8.FP8_DT_BF16
+    bsc = 1.0
+    if bias_kind == "bf16":
+        bias = torch.from_numpy((rng.standard_normal(n) * 5).astype(np.float32)).to(torch.bfloat16)
+        bias_dev = bias.cuda()
+        bias_np = bias.view(torch.int16).numpy().view(np.uint16)
+        odt = oracle.DT_BF16
+    elif bias_kind in ("e4m3", "e5m2"):
+        bf = 0 if bias_kind == "e4m3" else 1
+        bias_np = codes_like_tensor(rng, bf, (n,), 100.0)
+        bias_dev = torch.from_numpy(bias_np).cuda()
+        bsc = 7.25
+        bias_scale = torch.tensor([bsc], dtype=torch.float32, device="cuda")
+        bias_dtype = fp8.FP8_DT_E4M3 + bf
+        odt = oracle.DT_E4M3 + bf
+    fp8.fp8_mm(m, n, k, dev_a, fmt_a, a_major, lda, dev_b, fmt_b, b_major, ldb, scales[0:1], scales[1:2], d, ldd,
+               bias=bias_dev, bias_dtype=bias_dtype, bias_scale=bias_scale)
+    torch.cuda.synchronize()
+    y = d.cpu().view(torch.int16).numpy().view(np.uint16)
+    if ldd_extra:
+        assert np.all(y[:, n:] == 0x7FC0), "bytes past n must stay untouched"
+        y = y[:, :n]
+    a_si, a_sk = strides(a_major, lda)
+    b_sj, b_sk = strides(b_major, ldb)
+    if full:
+        acc, _, sab = oracle.gemm_acc(a_st, fmt_a, a_si, a_sk, b_st, fmt_b, b_sj, b_sk, m, n, k)
+        want, _ = oracle.epilogue(acc, sa, sb, bias_np if bias_kind else None,
+                                  odt if bias_kind else 0, bsc)
+        return assert_gemm_close(y, want, sab, sa, sb, f"mm {m}x{n}x{k} {a_major}{b_major}"), y, want
+    pi, pj = sample_points(rng, m, n)
+    acc, sab = oracle.gemm_acc_points(pi, pj, a_st, fmt_a, a_si, a_sk, b_st, fmt_b, b_sj, b_sk, k)
+    want, _ = oracle.epilogue(acc, sa, sb, bias_np if bias_kind else None, odt if bias_kind else 0, bsc,
+                              col_idx=pj)
+    return assert_gemm_close(y[pi, pj], want, sab, sa, sb, f"mm {m}x{n}x{k} {a_major}{b_major} sampled"), y, None
+
+
+LAYOUTS = [(0, 0), (0, 1), (1, 1), (1, 0)]
+
+
+@pytest.mark.parametrize("a_major,b_major", LAYOUTS)
+@pytest.mark.parametrize("m,n,k", [(64, 192, 128), (128, 256, 256), (200, 300, 333), (3, 100, 7),
+                                   (1000, 700, 1040), (130, 129, 2000)])
+def test_mm_layouts_full(fp8, a_major, b_major, m, n, k):
+    rng = np.random.default_rng(m * 7 + n * 3 + k + 10 * a_major + b_major)
+    run_case(fp8, rng, m, n, k, a_major, b_major, sa=448.0 / 300, sb=0.75, pad=16 if m == 200 else 0)
+
+
+@pytest.mark.parametrize("fmt_a,fmt_b", [(1, 0), (1, 1), (0, 1)])
+@pytest.mark.parametrize("a_major,b_major", LAYOUTS)
+def test_mm_formats(fp8, fmt_a, fmt_b, a_major, b_major):
+    rng = np.random.default_rng(99 + fmt_a * 2 + fmt_b)
+    run_case(fp8, rng, 257, 384, 640, a_major, b_major, fmt_a, fmt_b, sa=57344.0 / 9000, sb=448.0 / 200)
+
+
+@pytest.mark.parametrize("bias_kind", ["bf16", "e4m3", "e5m2"])
+def test_mm_bias(fp8, bias_kind):
+    rng = np.random.default_rng(5)
+    run_case(fp8, rng, 300, 500, 384, 0, 0, sa=2.0, sb=3.0, bias_kind=bias_kind)
+    run_case(fp8, rng, 64, 100, 96, 0, 0, sa=1.0, sb=1.0, bias_kind=bias_kind, ldd_extra=4)
+
+
+def test_mm_odd_ldd_untouched_columns(fp8):
+    rng = np.random.default_rng(6)
+    run_case(fp8, rng, 129, 100, 128, 0, 1, ldd_extra=3)
+    run_case(fp8, rng, 77, 264, 300, 1, 1, ldd_extra=8)
+
+
+@pytest.mark.parametrize("a_major,b_major", LAYOUTS)
+def test_mm_small_integers_exact(fp8, a_major, b_major):
+    """Small-integer fp8 values with unit scales: every partial sum is an integer
+    below 2^24, so the GPU must equal the oracle (and the integer matmul) bit
+    for bit."""
+    rng = np.random.default_rng(7)
+    t = oracle.decode_table(0)
+    ints = np.array([c for c in range(256) if np.isfinite(t[c]) and t[c] == np.round(t[c]) and abs(t[c]) <= 4],
+                    np.uint8)
+    m, n, k = 300, 520, 1000
+    A = rng.choice(ints, size=(m, k))
+    B = rng.choice(ints, size=(n, k))
+    _, y, want = run_case(fp8, rng, m, n, k, a_major, b_major, a_codes=A, b_codes=B)
+    ref = (t[A].astype(np.int64) @ t[B].astype(np.int64).T).astype(np.float32)
+    assert np.array_equal(oracle.bf16_to_f32(y), oracle.bf16_to_f32(want))
+    assert np.array_equal(oracle.bf16_to_f32(y), oracle.bf16_to_f32(oracle.bf16_rne(ref)))
+
+
+def test_mm_identity_weight(fp8):
+    """W8 = identity: Y = bf16(decode(x8) / (sx sw)) (bf16 rounding of one product)."""
+    rng = np.random.default_rng(8)
+    K = 384
+    A = codes_like_tensor(rng, 0, (256, K), 100.0)
+    B = np.where(np.eye(K, dtype=bool), 0x38, 0x00).astype(np.uint8)
+    run_case(fp8, rng, 256, K, K, 0, 0, a_codes=A, b_codes=B, sa=0.5, sb=1.0)
+    run_case(fp8, rng, 256, K, K, 0, 1, a_codes=A, b_codes=B, sa=0.5, sb=1.0)
+
+
+@pytest.mark.parametrize("a_major,b_major", LAYOUTS)
+def test_mm_long_k_accumulation(fp8, a_major, b_major):
+    """K = 11008 (the longest contraction of the workloads): random signs and
+    all-positive operands.  The all-positive case bounds the accumulation error
+    of the tensor-core path against the exact dot."""
+    rng = np.random.default_rng(9)
+    run_case(fp8, rng, 256, 256, 11008, a_major, b_major, sa=448.0 / 200, sb=448.0 / 150)
+    pos = oracle.encode(0, np.abs(rng.standard_normal((128, 11008)) * 30).astype(np.float32) + 1.0)
+    posb = oracle.encode(0, np.abs(rng.standard_normal((256, 11008)) * 30).astype(np.float32) + 1.0)
+    run_case(fp8, rng, 128, 256, 11008, a_major, b_major, a_codes=pos, b_codes=posb)
+
+
+@pytest.mark.parametrize("m,n,k,a_major,b_major", [
+    (2048, 1024, 1024, 0, 0), (2048, 1024, 4096, 0, 1), (4096, 1024, 2048, 1, 1), (512, 6912, 1536, 0, 0),
+    (1536, 1536, 512, 1, 1), (640, 2304, 4096, 0, 0)])
+def test_mm_large_sampled(fp8, m, n, k, a_major, b_major):
+    rng = np.random.default_rng(m + n + k)
+    run_case(fp8, rng, m, n, k, a_major, b_major, sa=3.0, sb=0.25, full=False)
+
+
+def test_mm_no_device_timeouts(fp8):
+    torch.cuda.synchronize()
+    assert fp8.fp8_get_device_status() == 0

@@ -1,0 +1,139 @@
+"""GPU parity of the quantize + in-kernel ring finalize against the oracle.
+fp8 codes, amax, the scale snapshot and every ring word must match bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from helpers import (assert_codes_equal, bits, dt_code, fp8_buffer, host_rows, oracle_ring_words, padded,
+                     ring_words)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fp8_delayed_scaling_03_b200 as m
+    return m
+
+
+def gpu_quantize(fp8, x_dev, fmt, ring, ld_out=None):
+    rows, cols = x_dev.shape
+    out = fp8_buffer(rows, cols, ld_out)
+    amax = torch.full((1,), -1.0, device="cuda")
+    scale = torch.full((1,), -1.0, device="cuda")
+    fp8.fp8_quantize(x_dev, fmt, ring.buf, ring.H, out, amax, scale)
+    torch.cuda.synchronize()
+    return out, amax.item(), scale.item()
+
+
+def check_step(fp8, x_cpu, fmt, ring, oring, ld_in=None, ld_out=None):
+    rows, cols = x_cpu.shape
+    x_dev = padded(x_cpu, ld_in) if ld_in else x_cpu.cuda()
+    out, amax, scale = gpu_quantize(fp8, x_dev, fmt, ring, ld_out)
+    xb = bits(x_cpu)
+    q, a, s = oracle.quantize(xb, dt_code(x_cpu), fmt, oring)
+    assert np.float32(scale) == s, (scale, s)
+    assert np.float32(amax).view(np.uint32) == np.float32(a).view(np.uint32), (amax, a)
+    assert_codes_equal(host_rows(out), q, fmt)
+    ldo = out.stride(0)
+    if ldo > cols:
+        base = torch.as_strided(out, (rows, ldo), (ldo, 1))
+        pad = base[:, cols:].cpu()
+        assert bool((pad == 0).all()), "padding bytes must be written as zero"
+    assert np.array_equal(ring_words(ring), oracle_ring_words(oring)), (ring_words(ring), oracle_ring_words(oring))
+    return out
+
+
+def test_ring_evolution_c1(fp8):
+    """Config 1: x ~ N(0,1) 2^step, 4 delayed steps, H=16: codes, amax,
+    snapshot and ring words bit-exact at every step (the doubling amax makes
+    the delayed scale saturate the top values)."""
+    ring = fp8.ScaleRing(wl.HIST_LEN)
+    oring = oracle.Ring(wl.HIST_LEN)
+    M, K = wl.C1.M, wl.C1.K
+    for step in range(wl.C1_STEPS):
+        x = wl.normal((M, K), 2.0 ** step, wl.seed_for(1, step, wl.OP_X))
+        check_step(fp8, x, fp8.FP8_E4M3, ring, oring)
+    assert ring.step == wl.C1_STEPS
+
+
+@pytest.mark.parametrize("dtype", (torch.bfloat16, torch.float16, torch.float32))
+@pytest.mark.parametrize("fmt", (0, 1))
+@pytest.mark.parametrize("rows,cols,ld_in,ld_out", [
+    (37, 53, 61, 64), (1, 7, 7, 16), (2048, 7, 7, 16), (3, 1534, 1534, 1536), (300, 100, 104, 112),
+    (64, 128, 128, 128), (2048, 1024, 1024, 1024), (513, 4096, 4100, 4096)])
+def test_quantize_shapes(fp8, dtype, fmt, rows, cols, ld_in, ld_out):
+    """Ragged, strided, single-row, odd-K and contiguous tensors, three steps
+    each so the history and step counter move."""
+    ring = fp8.ScaleRing(16)
+    oring = oracle.Ring(16)
+    for step in range(3):
+        std = (1.0, 37.0, 0.01)[step] * (1000.0 if fmt == 1 else 1.0)
+        x = wl.normal((rows, cols), std, 777 + step + rows, dtype=dtype)
+        check_step(fp8, x, fmt, ring, oring, ld_in=ld_in if ld_in != cols else None, ld_out=ld_out)
+
+
+def test_quantize_special_values(fp8):
+    """NaN (ignored by amax, NaN code), +-inf (saturate; amax inf keeps the old
+    scale), -0, values that round to zero, exact ties after scaling."""
+    vals = np.array([np.nan, np.inf, -np.inf, -0.0, 0.0, 1e-30, -1e-30, 448.0, 449.0, 464.0, 1e6, -1e6,
+                     3.0, 0.5, 2.0 ** -10, 2.0 ** -9, 1.0625, 1.1875], np.float32)
+    x = torch.from_numpy(np.tile(vals, (5, 3)).astype(np.float32))
+    for fmt in (0, 1):
+        ring = fp8.ScaleRing(4)
+        oring = oracle.Ring(4)
+        check_step(fp8, x, fmt, ring, oring)           # amax inf -> scale kept at 1
+        check_step(fp8, x.to(torch.bfloat16), fmt, ring, oring)
+        xf = torch.nan_to_num(x, posinf=3.0e4, neginf=-2.0e4)
+        check_step(fp8, xf, fmt, ring, oring)
+        check_step(fp8, x, fmt, ring, oring)
+
+
+def test_quantize_large_many_blocks(fp8):
+    """c4 x with 0.1% outliers x50 (4096 x 4096) and c3 x (2048 x 6912): a grid
+    of hundreds of blocks, bit-exact codes and ring."""
+    ring = fp8.ScaleRing(16)
+    oring = oracle.Ring(16)
+    x = wl.normal_with_outliers((4096, 4096), 1.0, wl.seed_for(4, 0, wl.OP_X), wl.seed_for(4, 0, wl.OP_MASK))
+    check_step(fp8, x, 0, ring, oring)
+    x2 = wl.normal((2048, 6912), 1.0, wl.seed_for(3, 0, wl.OP_X))
+    check_step(fp8, x2, 0, ring, oring)
+    check_step(fp8, x, 0, ring, oring)
+
+
+def test_ring_init_seed(fp8):
+    for fmt, amax in ((0, 3.5), (1, 1e-3), (0, 0.0), (0, float("inf")), (1, 1e-42)):
+        ring = fp8.ScaleRing(16, seed_amax=amax, fmt=fmt)
+        oring = oracle.Ring(16)
+        oring.seed(amax, fmt)
+        torch.cuda.synchronize()
+        assert np.array_equal(ring_words(ring), oracle_ring_words(oring)), (fmt, amax)
+
+
+def test_ring_checkpoint_resume(fp8):
+    """Copying a ring's bytes between launches checkpoints it: resuming from the
+    copy gives the same scales as the uninterrupted run."""
+    ring = fp8.ScaleRing(8)
+    xs = [wl.normal((256, 256), 1.5 ** i, 4242 + i).cuda() for i in range(12)]
+    out = fp8_buffer(256, 256)
+    for x in xs[:5]:
+        fp8.fp8_quantize(x, 0, ring.buf, 8, out)
+    saved = ring.buf.clone()
+    for x in xs[5:]:
+        fp8.fp8_quantize(x, 0, ring.buf, 8, out)
+    ring.buf.copy_(saved)
+    for x in xs[5:]:
+        fp8.fp8_quantize(x, 0, ring.buf, 8, out)
+    a = ring.buf.clone()
+    ring2 = fp8.ScaleRing(8)
+    for x in xs:
+        fp8.fp8_quantize(x, 0, ring2.buf, 8, out)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int32), ring2.buf.view(torch.int32))
+
+
+def test_no_device_timeouts_recorded(fp8):
+    torch.cuda.synchronize()
+    assert fp8.fp8_get_device_status() == 0

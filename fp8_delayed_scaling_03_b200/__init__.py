@@ -226,9 +226,16 @@ class ScaleRing:
     """Delayed-scaling state of one tensor: a device buffer laid out as
     [hist (H fp32) | scale | ticket | step | scratch]."""
 
-    def __init__(self, hist_len: int = 16, device="cuda", seed_amax: float | None = None, fmt: int = FP8_E4M3):
+    def __init__(self, hist_len: int = 16, device="cuda", seed_amax: float | None = None, fmt: int = FP8_E4M3,
+                 buf: torch.Tensor | None = None):
         self.H = hist_len
-        self.buf = torch.empty(fp8_ring_bytes(hist_len) // 4, dtype=torch.float32, device=device)
+        words = fp8_ring_bytes(hist_len) // 4
+        if buf is not None:
+            if buf.dtype != torch.float32 or buf.numel() != words or not buf.is_contiguous():
+                raise ValueError(f"ring buffer must be {words} contiguous fp32 words")
+            self.buf = buf
+        else:
+            self.buf = torch.empty(words, dtype=torch.float32, device=device)
         if seed_amax is None:
             fp8_ring_init(self.buf, hist_len)
         else:

@@ -144,9 +144,11 @@ static float load_in(const void* p, int dtype, int64_t idx) {
 
 /* ------------------------------------------------------------ quantize */
 
-/* amax = max |x| over all non-NaN elements, taken on the raw input values. */
+/* amax = max |x| over all non-NaN elements, taken on the raw input values
+ * (a max is independent of evaluation order, so rows may run in parallel). */
 float orc_amax(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld) {
   float m = 0.0f;
+#pragma omp parallel for reduction(max : m) schedule(static)
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c) {
       float v = load_in(x, dtype, r * ld + c);

@@ -1,0 +1,266 @@
+"""GPU parity of the whole FP8 linear (fp8_linear_forward / fp8_linear_backward)
+against the oracle's forward/backward orchestration, on the five workload
+configurations: quantized operands, amaxes, scale snapshots and ring words
+bit-exact; y, dX, dW within max(1 bf16 ulp, 2e-6 sum|ab| / (sa sb)); dbias
+within max(1 bf16 ulp, 2e-6 sum|g|).  Large shapes compare sampled GEMM
+outputs (full rows, full columns, random points); quantize is always full."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from helpers import assert_codes_equal, assert_gemm_close, bits, host_rows, oracle_ring_words, ring_words, \
+    sample_points
+
+pytestmark = pytest.mark.gpu
+E4, E5 = oracle.E4M3, oracle.E5M2
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fp8_delayed_scaling_03_b200 as m
+    return m
+
+
+def gemm_check(y_gpu, a8, a_major_rows, fmt_a, b8, fmt_b, I, J, Kc, sa, sb, kind, full, rng, bias=None,
+               bias_dtype=0, bias_scale=1.0, what=""):
+    """kind: 'fwd' (A=X8 [I,Kc], B=W8 [J,Kc]), 'dx' (A=G8 [I,Kc], B=W8 [Kc,J]),
+    'dw' (A=G8 [Kc,I], B=X8 [Kc,J]).  Operands are contiguous numpy arrays."""
+    lda, ldb = a8.shape[1], b8.shape[1]
+    a_s = {"fwd": (lda, 1), "dx": (lda, 1), "dw": (1, lda)}[kind]
+    b_s = {"fwd": (ldb, 1), "dx": (1, ldb), "dw": (1, ldb)}[kind]
+    y = y_gpu.cpu().view(torch.int16).numpy().view(np.uint16)
+    if full:
+        acc, _, sab = oracle.gemm_acc(a8, fmt_a, *a_s, b8, fmt_b, *b_s, I, J, Kc)
+        want, _ = oracle.epilogue(acc, sa, sb, bias, bias_dtype, bias_scale)
+        return assert_gemm_close(y, want, sab, sa, sb, what)
+    pi, pj = sample_points(rng, I, J)
+    acc, sab = oracle.gemm_acc_points(pi, pj, a8, fmt_a, *a_s, b8, fmt_b, *b_s, Kc)
+    want, _ = oracle.epilogue(acc, sa, sb, bias, bias_dtype, bias_scale, col_idx=pj)
+    return assert_gemm_close(y[pi, pj], want, sab, sa, sb, what + " (sampled)")
+
+
+def dbias_check(got, g_bits, M, N):
+    want, _, sa = oracle.dbias(g_bits, oracle.DT_BF16, M, N)
+    g = oracle.bf16_to_f32(got.cpu().view(torch.int16).numpy().view(np.uint16)).astype(np.float64)
+    o = oracle.bf16_to_f32(want).astype(np.float64)
+    tol = np.maximum(oracle.bf16_ulp(o), 2e-6 * sa)
+    assert np.all(np.abs(g - o) <= tol), np.max(np.abs(g - o) / tol)
+
+
+def linear_step(fp8, x, w, g, rings, orings, full, rng, bias=None, bias8=None, bias_scale=None,
+                need_dbias=False, w_pre=None, what=""):
+    """One forward + backward on the GPU and in the oracle; compare everything.
+    w_pre: (w8 codes [N,K] numpy, scale) for the pre-quantized weight path."""
+    M, K = x.shape
+    N = w.shape[0] if w is not None else w_pre[0].shape[0]
+    rx, rw, rg = rings
+    orx, orw, org = orings
+    dev_bias, bias_np, bias_dt, bsc = None, None, oracle.DT_BF16, 1.0
+    dev_bsc = None
+    if bias is not None:
+        dev_bias, bias_np = bias.cuda(), bits(bias)
+    elif bias8 is not None:
+        dev_bias, bias_np, bias_dt, bsc = torch.from_numpy(bias8).cuda(), bias8, oracle.DT_E4M3, bias_scale
+        dev_bsc = torch.tensor([bias_scale], dtype=torch.float32, device="cuda")
+    if w_pre is not None:
+        w8_np, wsc = w_pre
+        wbuf = torch.zeros((N, (K + 15) // 16 * 16), dtype=torch.uint8)
+        wbuf[:, :K] = torch.from_numpy(w8_np[:, :K])
+        w_dev = wbuf.cuda()[:, :K]
+        w_scale_in = torch.tensor([wsc], dtype=torch.float32, device="cuda")
+        ring_w_words = ring_words(rw)
+    else:
+        w_dev, w_scale_in = w.cuda(), None
+    f = fp8.linear_forward(x.cuda(), w_dev, rx, None if w_pre is not None else rw, bias=dev_bias,
+                           bias_scale=dev_bsc, w_scale_in=w_scale_in, hist_len=rx.H)
+    b = fp8.linear_backward(g.cuda(), f, rg, need_dbias=need_dbias)
+    torch.cuda.synchronize()
+    assert fp8.fp8_get_device_status() == 0
+
+    # oracle quantize (always full) and the scale snapshots
+    x8o, ax, sx = oracle.quantize(bits(x), oracle.DT_BF16, E4, orx, ld_out=(K + 15) // 16 * 16)
+    if w_pre is not None:
+        w8o, aw, sw = np.ascontiguousarray(w8_np), np.float32(0.0), np.float32(w_pre[1])
+    else:
+        w8o, aw, sw = oracle.quantize(bits(w), oracle.DT_BF16, E4, orw, ld_out=(K + 15) // 16 * 16)
+    g8o, ag, sg = oracle.quantize(bits(g), oracle.DT_BF16, E5, org, ld_out=(N + 15) // 16 * 16)
+    assert f.sx.item() == sx and f.sw.item() == sw and b.sg.item() == sg, what
+    assert f.amax_x.item() == ax and f.amax_w.item() == aw and b.amax_g.item() == ag, what
+    assert_codes_equal(host_rows(f.x8), x8o[:, :K], E4)
+    if w_pre is None:
+        assert_codes_equal(host_rows(f.w8), w8o[:, :K], E4)
+    else:
+        assert np.array_equal(ring_words(rw), ring_w_words), "ring_w must stay untouched"
+    assert_codes_equal(host_rows(b.g8), g8o[:, :N], E5)
+    assert np.array_equal(ring_words(rx), oracle_ring_words(orx)), what
+    if w_pre is None:
+        assert np.array_equal(ring_words(rw), oracle_ring_words(orw)), what
+    assert np.array_equal(ring_words(rg), oracle_ring_words(org)), what
+    # GEMMs (operands: the oracle's own quantized bytes, equal to the GPU's)
+    gemm_check(f.y, x8o, 0, E4, w8o, E4, M, N, K, sx, sw, "fwd", full, rng, bias_np if dev_bias is not None else None,
+               bias_dt, bsc, what + " y")
+    gemm_check(b.dx, g8o, 0, E5, w8o, E4, M, K, N, sg, sw, "dx", full, rng, what=what + " dx")
+    gemm_check(b.dw, g8o, 0, E5, x8o, E4, N, K, M, sg, sx, "dw", full, rng, what=what + " dw")
+    if need_dbias:
+        dbias_check(b.dbias, bits(g), M, N)
+    return f, b
+
+
+def make_rings(fp8, H=16):
+    return (fp8.ScaleRing(H), fp8.ScaleRing(H), fp8.ScaleRing(H)), (oracle.Ring(H), oracle.Ring(H), oracle.Ring(H))
+
+
+def test_config1_four_steps(fp8):
+    """Config 1: 4 delayed steps, x ~ N(0,1) 2^step, w ~ N(0,0.02), bf16 bias
+    ~ N(0,0.01), g ~ N(0,1e-3); full oracle comparison incl. dbias."""
+    c = wl.C1
+    rings, orings = make_rings(fp8)
+    rng = np.random.default_rng(1)
+    w = wl.normal((c.N, c.K), 0.02, wl.seed_for(1, 0, wl.OP_W))
+    bias = wl.normal((c.N,), 0.01, wl.seed_for(1, 0, wl.OP_BIAS))
+    for step in range(wl.C1_STEPS):
+        x = wl.normal((c.M, c.K), 2.0 ** step, wl.seed_for(1, step, wl.OP_X))
+        g = wl.normal((c.M, c.N), 1e-3, wl.seed_for(1, step, wl.OP_G))
+        linear_step(fp8, x, w, g, rings, orings, True, rng, bias=bias, need_dbias=True, what=f"c1 step {step}")
+
+
+def test_config1_no_scale_ratio_leak(fp8):
+    """Two delayed steps with a doubling amax: Y at the later step stays within
+    fp8 noise of the float64 GEMM of the unquantized inputs."""
+    c = wl.C1
+    rings, _ = make_rings(fp8)
+    w = wl.normal((c.N, c.K), 0.02, wl.seed_for(1, 0, wl.OP_W))
+    for step in range(3):
+        x = wl.normal((c.M, c.K), 2.0 ** step, wl.seed_for(1, step, wl.OP_X))
+        f = fp8.linear_forward(x.cuda(), w.cuda(), rings[0], rings[1])
+        y = f.y.float().cpu().double().numpy()
+        ref = x.double().numpy() @ w.double().numpy().T
+        rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+        ratio = np.dot(y.ravel(), ref.ravel()) / np.dot(ref.ravel(), ref.ravel())
+        assert rel < 0.25 and 0.8 < ratio < 1.2, (step, rel, ratio)
+
+
+def test_prequantized_weight(fp8):
+    """A pre-quantized w8 skips its quantize: amax_w = 0, sw = w_scale_in,
+    ring_w untouched; config 1 shapes and config 4's path at a small size."""
+    c = wl.C1
+    rings, orings = make_rings(fp8)
+    rng = np.random.default_rng(2)
+    w = wl.normal((c.N, c.K), 0.02, wl.seed_for(1, 0, wl.OP_W))
+    wsc = np.float32(448.0) / oracle.amax(bits(w), oracle.DT_BF16)
+    w8 = oracle.quantize_codes(bits(w), oracle.DT_BF16, E4, wsc)
+    for step in range(2):
+        x = wl.normal((c.M, c.K), 1.0, wl.seed_for(1, step, wl.OP_X))
+        g = wl.normal((c.M, c.N), 1e-3, wl.seed_for(1, step, wl.OP_G))
+        linear_step(fp8, x, None, g, rings, orings, True, rng, w_pre=(w8, float(wsc)), what=f"w8 step {step}")
+
+
+@pytest.mark.parametrize("shape", wl.C2_SHAPES, ids=lambda s: s.name)
+def test_config2_shapes(fp8, shape):
+    rings, orings = make_rings(fp8)
+    rng = np.random.default_rng(3)
+    x = wl.normal((shape.M, shape.K), 1.0, wl.seed_for(2, 0, wl.OP_X))
+    w = wl.normal((shape.N, shape.K), wl.weight_std(shape.K), wl.seed_for(2, 0, wl.OP_W))
+    g = wl.normal((shape.M, shape.N), 1e-3, wl.seed_for(2, 0, wl.OP_G))
+    linear_step(fp8, x, w, g, rings, orings, False, rng, what=f"c2 {shape.name}")
+
+
+@pytest.mark.parametrize("shape", wl.C3_SHAPES, ids=lambda s: s.name)
+def test_config3_fp8_bias(fp8, shape):
+    """Production shapes with the bias stored as E4M3 with bias_scale =
+    448 / amax(bias), plus dbias."""
+    rings, orings = make_rings(fp8)
+    rng = np.random.default_rng(4)
+    x = wl.normal((shape.M, shape.K), 1.0, wl.seed_for(3, 0, wl.OP_X))
+    w = wl.normal((shape.N, shape.K), wl.weight_std(shape.K), wl.seed_for(3, 0, wl.OP_W))
+    g = wl.normal((shape.M, shape.N), 1e-3, wl.seed_for(3, 0, wl.OP_G))
+    b = wl.normal((1, shape.N), 0.01, wl.seed_for(3, 0, wl.OP_BIAS))
+    bsc = np.float32(448.0) / oracle.amax(bits(b), oracle.DT_BF16)
+    b8 = oracle.quantize_codes(bits(b), oracle.DT_BF16, E4, bsc)[0]
+    linear_step(fp8, x, w, g, rings, orings, False, rng, bias8=b8, bias_scale=float(bsc), need_dbias=True,
+                what=f"c3 {shape.name}")
+
+
+@pytest.mark.parametrize("shape", wl.C4_SHAPES, ids=lambda s: s.name)
+def test_config4_outliers_and_prequantized(fp8, shape):
+    rings, orings = make_rings(fp8)
+    rng = np.random.default_rng(5)
+    x = wl.normal_with_outliers((shape.M, shape.K), 1.0, wl.seed_for(4, 0, wl.OP_X), wl.seed_for(4, 0, wl.OP_MASK))
+    w = wl.normal((shape.N, shape.K), wl.weight_std(shape.K), wl.seed_for(4, 0, wl.OP_W))
+    g = wl.normal((shape.M, shape.N), 1e-3, wl.seed_for(4, 0, wl.OP_G))
+    linear_step(fp8, x, w, g, rings, orings, False, rng, what=f"c4 {shape.name}")
+    if shape is wl.C4_SHAPES[0]:
+        wsc = np.float32(448.0) / oracle.amax(bits(w), oracle.DT_BF16)
+        w8 = oracle.quantize_codes(bits(w), oracle.DT_BF16, E4, wsc)
+        linear_step(fp8, x, None, g, rings, orings, False, rng, w_pre=(w8, float(wsc)), what="c4 w8")
+
+
+@pytest.mark.parametrize("shape", wl.C5_EDGE, ids=lambda s: s.name)
+def test_config5_edge_shapes(fp8, shape):
+    """Odd K (7, 100, 1534), M in {3, 64, 2048}, N in {1024, 100} (N=100 gives
+    a bf16 output row of 200 bytes: the unaligned store path); bf16 bias and
+    dbias; two steps."""
+    rings, orings = make_rings(fp8)
+    rng = np.random.default_rng(6)
+    full = shape.M * shape.N * shape.K <= 64 * 1024 * 1534
+    w = wl.normal((shape.N, shape.K), wl.weight_std(shape.K), wl.seed_for(5, 0, wl.OP_W))
+    bias = wl.normal((shape.N,), 0.01, wl.seed_for(5, 0, wl.OP_BIAS))
+    for step in range(2):
+        x = wl.normal((shape.M, shape.K), 1.0 + step, wl.seed_for(5, step, wl.OP_X))
+        g = wl.normal((shape.M, shape.N), 1e-3, wl.seed_for(5, step, wl.OP_G))
+        linear_step(fp8, x, w, g, rings, orings, full, rng, bias=bias, need_dbias=True,
+                    what=f"c5 {shape.name} step {step}")
+
+
+def test_config5_twenty_step_sequence(fp8):
+    """Config 5: 20 steps over 12 layers x 6 linears (216 rings), M = 2048, input
+    std drifting log-uniformly in [0.5, 4] per step.  Every ring word matches
+    the oracle after every step; the backward's dX/dW use the forward's
+    snapshots (checked on sampled outputs of two linears at three steps)."""
+    H, M = wl.HIST_LEN, 2048
+    words = fp8.fp8_ring_bytes(H) // 4
+    nlin = wl.C5_LAYERS * len(wl.C5_LAYER)
+    allbuf = torch.empty((nlin * 3, words), dtype=torch.float32, device="cuda")
+    rings = [fp8.ScaleRing(H, buf=allbuf[i]) for i in range(nlin * 3)]
+    orings = [oracle.Ring(H) for _ in range(nlin * 3)]
+    rng = np.random.default_rng(7)
+    base_x = {s.K: wl.normal((M, s.K), 1.0, wl.seed_for(5, 0, wl.OP_X, s.K)) for s in wl.C5_LAYER}
+    base_g = {s.N: wl.normal((M, s.N), 1e-3, wl.seed_for(5, 0, wl.OP_G, s.N)) for s in wl.C5_LAYER}
+    ws = [wl.normal((s.N, s.K), wl.weight_std(s.K), wl.seed_for(5, 0, wl.OP_W, li)) for li, s in
+          enumerate(wl.C5_LAYER * wl.C5_LAYERS)]
+    ws_dev = [w.cuda() for w in ws]
+    w_bits = [bits(w) for w in ws]
+    amax_w = [oracle.amax(b, oracle.DT_BF16) for b in w_bits]
+    for step in range(wl.C5_STEPS):
+        sigma = wl.log_uniform(0.5, 4.0, wl.seed_for(5, step, wl.OP_STD))
+        xs = {K: (t.float() * sigma).to(torch.bfloat16) for K, t in base_x.items()}
+        gs = {N: (t.float() * (sigma / 2)).to(torch.bfloat16) for N, t in base_g.items()}
+        xs_dev = {K: t.cuda() for K, t in xs.items()}
+        gs_dev = {N: t.cuda() for N, t in gs.items()}
+        xa = {K: oracle.amax(bits(t), oracle.DT_BF16) for K, t in xs.items()}
+        ga = {N: oracle.amax(bits(t), oracle.DT_BF16) for N, t in gs.items()}
+        check_now = step in (0, 10, 19)
+        for li, s in enumerate(wl.C5_LAYER * wl.C5_LAYERS):
+            rx, rw, rg = rings[3 * li: 3 * li + 3]
+            f = fp8.linear_forward(xs_dev[s.K], ws_dev[li], rx, rw)
+            b = fp8.linear_backward(gs_dev[s.N], f, rg)
+            orx, orw, org = orings[3 * li: 3 * li + 3]
+            sx, sw, sg = orx.scale, orw.scale, org.scale
+            orx.advance(xa[s.K], E4)
+            orw.advance(amax_w[li], E4)
+            org.advance(ga[s.N], E5)
+            if check_now and li in (0, nlin - 1):
+                torch.cuda.synchronize()
+                assert (f.sx.item(), f.sw.item(), b.sg.item()) == (sx, sw, sg)
+                x8 = oracle.quantize_codes(bits(xs[s.K]), oracle.DT_BF16, E4, sx)
+                w8 = oracle.quantize_codes(w_bits[li], oracle.DT_BF16, E4, sw)
+                g8 = oracle.quantize_codes(bits(gs[s.N]), oracle.DT_BF16, E5, sg)
+                gemm_check(b.dx, g8, 0, E5, w8, E4, M, s.K, s.N, sg, sw, "dx", False, rng, what="c5 dx")
+                gemm_check(b.dw, g8, 0, E5, x8, E4, s.N, s.K, M, sg, sx, "dw", False, rng, what="c5 dw")
+        torch.cuda.synchronize()
+        got = allbuf.cpu().view(torch.int32).numpy().view(np.uint32)
+        want = np.stack([oracle_ring_words(r) for r in orings])
+        assert np.array_equal(got, want), f"ring words differ at step {step}"
+    assert fp8.fp8_get_device_status() == 0

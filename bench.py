@@ -1,0 +1,544 @@
+#!/usr/bin/env python
+"""Throughput of the FP8 linear layer with delayed scaling on B200.
+
+One step = forward + backward of every linear of the 12L/dim1024/B4xT512 model
+(12 layers x {q, k, v, o: 1024x1024; up: 1024x4096; down: 4096x1024}, M = 2048
+tokens): per linear, quantize x and w (E4M3, delayed scaling rings), the
+forward GEMM with fused dequant + bf16 bias, quantize g (E5M2), dX, dW and
+dbias -- 504 kernel launches, replayed as one CUDA graph of C-ABI calls.
+The value is TFLOP/s of the three GEMMs (6 M N K per linear) over the whole
+step.  Inputs are synthetic, seeded and resident in HBM; the step's working
+set (about 3 GB) is far larger than L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the step (weak
+scaling, no collective on the data path); the time is the max over ranks.
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+METRIC = "FP8 linear fwd/dX/dW TFLOP/s and % dense FP8 peak; quantize GB/s % HBM"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_PER_BF16 = 2.0          # nominal dense fp8 : bf16 tensor-core ratio (4.5 : 2.25 PFLOP/s)
+NOMINAL_FP8_TFLOPS = 4500.0
+REF_TOKENS = 128            # tokens of one layer per reference-arm step
+BASELINE_TOKENS = 1024      # tokens of one layer for the cpu_baseline sample
+
+
+# --------------------------------------------------------------------------- helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (the process group is already up)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread while
+    the timed region runs (reads only; changes no setting)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x100: "display_clock_setting", 0x10: "sync_boost"}
+
+    def __init__(self, device_index: int):
+        self.ok = False
+        self.samples, self.reasons = [], set()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = repr(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- workload
+
+class Linear:
+    """Device buffers and prebuilt C-ABI argument structs of one FP8 linear."""
+
+    def __init__(self, F, shape, seed_base, device, H=wl.HIST_LEN):
+        M, K, N = shape.M, shape.K, shape.N
+        self.shape = shape
+        ldk, ldn = (K + 15) // 16 * 16, (N + 15) // 16 * 16
+        self.x = wl.normal_device((M, K), 1.0, seed_base + wl.OP_X, device)
+        self.w = wl.normal_device((N, K), wl.weight_std(K), seed_base + wl.OP_W, device)
+        self.b = wl.normal_device((N,), wl.BENCH_BIAS_STD, seed_base + wl.OP_BIAS, device)
+        self.g = wl.normal_device((M, N), 1e-3, seed_base + wl.OP_G, device)
+        self.x8 = torch.zeros((M, ldk), dtype=torch.uint8, device=device)
+        self.w8 = torch.zeros((N, ldk), dtype=torch.uint8, device=device)
+        self.g8 = torch.zeros((M, ldn), dtype=torch.uint8, device=device)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.dx = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+        self.dw = torch.empty((N, K), dtype=torch.bfloat16, device=device)
+        self.db = torch.empty((N,), dtype=torch.bfloat16, device=device)
+        words = F.fp8_ring_bytes(H) // 4
+        self.rings = torch.empty((3, words), dtype=torch.float32, device=device)
+        for i in range(3):
+            F.fp8_ring_init(self.rings[i], H)
+        self.sc = torch.zeros(6, dtype=torch.float32, device=device)
+        self.ws = torch.zeros(max(16, F.fp8_linear_workspace_bytes(M, N, K)), dtype=torch.uint8, device=device)
+        p = lambda t: t.data_ptr()  # noqa: E731
+        sc = self.sc.data_ptr()
+        self.fwd = F.LinearFwdArgs(M, N, K, p(self.x), F.FP8_DT_BF16, K, None, p(self.w), F.FP8_DT_BF16, K, None,
+                                   p(self.b), F.FP8_DT_BF16, None, F.FP8_E4M3, F.FP8_E4M3, H,
+                                   p(self.rings[0]), p(self.rings[1]), p(self.x8), ldk, p(self.w8), ldk,
+                                   sc, sc + 4, sc + 12, sc + 16, p(self.y), N)
+        self.bwd = F.LinearBwdArgs(M, N, K, p(self.g), F.FP8_DT_BF16, N, None, F.FP8_E5M2, H, p(self.rings[2]),
+                                   p(self.g8), ldn, sc + 8, sc + 20, p(self.x8), ldk, sc, F.FP8_E4M3,
+                                   p(self.w8), ldk, sc + 4, F.FP8_E4M3, 1, 1, 1, p(self.dx), K, p(self.dw), K,
+                                   p(self.db), p(self.ws), self.ws.numel())
+
+    def inputs(self):
+        return [self.x, self.w, self.b, self.g]
+
+    def outputs(self):
+        return [self.y, self.dx, self.dw, self.db]
+
+
+def build_model(F, device, rank):
+    lins = []
+    for layer in range(wl.BENCH_LAYERS):
+        for j, s in enumerate(wl.BENCH_LAYER):
+            lins.append(Linear(F, s, wl.seed_for(2, 0, 0, extra=1 + rank * 1000 + layer * 10 + j) * 10, device))
+    return lins
+
+
+def run_step(F, lins, stream_handle):
+    """Forward over the layers in order, then backward in reverse, through the C ABI."""
+    fwd, bwd = F._lib.fp8_linear_forward, F._lib.fp8_linear_backward
+    for L in lins:
+        s = fwd(ctypes.byref(L.fwd), stream_handle)
+        if s:
+            raise F.Fp8Error(s, "fp8_linear_forward")
+    for L in reversed(lins):
+        s = bwd(ctypes.byref(L.bwd), stream_handle)
+        if s:
+            raise F.Fp8Error(s, "fp8_linear_backward")
+
+
+LAUNCHES_PER_LINEAR = 7  # quantize x, quantize w, fwd GEMM, quantize g, dX GEMM, dW GEMM, dbias
+
+
+# --------------------------------------------------------------------------- kernel-level timing
+
+def step_primitives(F, lins, h):
+    """The step's kernels as (class, algorithmic work, label, call) in launch
+    order: the same primitives the linear entry points launch."""
+    lib = F._lib
+    out = []
+    for L in lins:
+        M, K, N = L.shape.M, L.shape.K, L.shape.N
+        ldk, ldn = L.x8.shape[1], L.g8.shape[1]
+        sc = L.sc.data_ptr()
+        mm = lambda *a: (lambda args=F.MmArgs(*a): lib.fp8_mm(ctypes.byref(args), h))  # noqa: E731
+        out += [
+            ("quantize", M * K * 3, None, lambda L=L, M=M, K=K, ldk=ldk, sc=sc: lib.fp8_quantize(
+                L.x.data_ptr(), 0, M, K, K, 0, L.rings[0].data_ptr(), wl.HIST_LEN, L.x8.data_ptr(), ldk, sc + 12, sc, h)),
+            ("quantize", N * K * 3, None, lambda L=L, N=N, K=K, ldk=ldk, sc=sc: lib.fp8_quantize(
+                L.w.data_ptr(), 0, N, K, K, 0, L.rings[1].data_ptr(), wl.HIST_LEN, L.w8.data_ptr(), ldk, sc + 16, sc + 4, h)),
+            ("gemm", 2 * M * N * K, f"fwd {M}x{N}x{K}", mm(M, N, K, L.x8.data_ptr(), 0, 0, ldk, L.w8.data_ptr(), 0, 0, ldk,
+                                                         sc, sc + 4, L.b.data_ptr(), 0, None, L.y.data_ptr(), N)),
+        ]
+    for L in reversed(lins):
+        M, K, N = L.shape.M, L.shape.K, L.shape.N
+        ldk, ldn = L.x8.shape[1], L.g8.shape[1]
+        sc = L.sc.data_ptr()
+        mm = lambda *a: (lambda args=F.MmArgs(*a): lib.fp8_mm(ctypes.byref(args), h))  # noqa: E731
+        out += [
+            ("quantize", M * N * 3, None, lambda L=L, M=M, N=N, ldn=ldn, sc=sc: lib.fp8_quantize(
+                L.g.data_ptr(), 0, M, N, N, 1, L.rings[2].data_ptr(), wl.HIST_LEN, L.g8.data_ptr(), ldn, sc + 20, sc + 8, h)),
+            ("gemm", 2 * M * N * K, f"dX {M}x{K}x{N}", mm(M, K, N, L.g8.data_ptr(), 1, 0, ldn, L.w8.data_ptr(), 0, 1, ldk,
+                                                        sc + 8, sc + 4, None, 0, None, L.dx.data_ptr(), K)),
+            ("gemm", 2 * M * N * K, f"dW {N}x{K}x{M}", mm(N, K, M, L.g8.data_ptr(), 1, 1, ldn, L.x8.data_ptr(), 0, 1, ldk,
+                                                        sc + 8, sc, None, 0, None, L.dw.data_ptr(), K)),
+            ("dbias", M * N * 2 + N * 2, None, lambda L=L, M=M, N=N: lib.fp8_dbias(
+                L.g.data_ptr(), 0, M, N, N, None, L.db.data_ptr(), L.ws.data_ptr(), L.ws.numel(), h)),
+        ]
+    return out
+
+
+def time_kernels(F, lins, stream, reps=5):
+    """Device time of each kernel class of the step: the class's launches (in
+    step order, same buffers) captured as one CUDA graph and replayed between
+    CUDA events on the launching stream, so host launch gaps are excluded.
+    Returns (ms per step by class, work by class, launches by class, per-shape
+    GEMM times)."""
+    h = stream.cuda_stream
+    prims = step_primitives(F, lins, h)
+    res_ms, work, count = {}, {}, {}
+    for cls in ("gemm", "quantize", "dbias"):
+        calls = [c for c in prims if c[0] == cls]
+        work[cls] = sum(c[1] for c in calls)
+        count[cls] = len(calls)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _, _, _, fn in calls:
+                st = fn()
+                if st:
+                    raise F.Fp8Error(st, cls)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        res_ms[cls] = e0.elapsed_time(e1) / reps
+        del g
+    # per-shape GEMM times: one graph per distinct GEMM of a layer, 12 launches each
+    shapes = {}
+    layer = len(wl.BENCH_LAYER)
+    first_layer = [c for c in prims if c[0] == "gemm"]
+    seen = {}
+    for c in first_layer:
+        seen.setdefault(c[2], c)
+    for name, c in seen.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(12):
+                c[3]()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / 12
+        shapes[name] = {"us": us, "tflops": c[1] / us / 1e6, "note": "same operands back to back (warm L2)"}
+        del g
+    del layer
+    return res_ms, work, count, shapes
+
+
+# --------------------------------------------------------------------------- GEMM traffic (ncu summary)
+
+def gemm_source_sha():
+    src = os.path.join(ROOT, "fp8_delayed_scaling_03_b200", "csrc", "gemm.cu")
+    with open(src, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def gemm_traffic_per_launch():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when
+    the summary is missing or was taken on a different gemm.cu."""
+    p = os.path.join(ROOT, "profiles", "gemm_dram_traffic_dim1024_layer.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as fh:
+        for line in fh:
+            if "=" in line and not line.startswith("#"):
+                k, v = line.strip().split("=", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("gemm_cu_sha256_16") != gemm_source_sha():
+        return None
+    try:
+        return float(kv["dram_bytes_per_gemm_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_layer_sample(tokens: int, seed: int = 1234):
+    """The oracle's forward + backward of one dim1024 layer's six linears on
+    `tokens` tokens (quantize x/w/g with rings, fwd/dX/dW GEMMs, bias, dbias).
+    Returns (seconds, flops)."""
+    import numpy as np
+
+    import oracle
+    rng_seed = seed
+    flops = 0
+    prepared = []
+    for j, s in enumerate(wl.BENCH_LAYER):
+        x = wl.normal((tokens, s.K), 1.0, rng_seed + 10 * j)
+        w = wl.normal((s.N, s.K), wl.weight_std(s.K), rng_seed + 10 * j + 1)
+        b = wl.normal((s.N,), wl.BENCH_BIAS_STD, rng_seed + 10 * j + 2)
+        g = wl.normal((tokens, s.N), 1e-3, rng_seed + 10 * j + 3)
+        bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+        prepared.append((s, bits(x), bits(w), bits(b), bits(g)))
+        flops += 6 * tokens * s.N * s.K
+    t0 = time.perf_counter()
+    for s, x, w, b, g in prepared:
+        rx, rw, rg = oracle.Ring(wl.HIST_LEN), oracle.Ring(wl.HIST_LEN), oracle.Ring(wl.HIST_LEN)
+        f = oracle.linear_forward(tokens, s.N, s.K, x, oracle.DT_BF16, w, oracle.DT_BF16, rx, rw, bias=b,
+                                  sumabs=False)
+        oracle.linear_backward(tokens, s.N, s.K, g, oracle.DT_BF16, rg, f["x8"], oracle.E4M3, f["sx"], f["w8"],
+                               oracle.E4M3, f["sw"], need_dbias=True, sumabs=False)
+    return time.perf_counter() - t0, flops
+
+
+def oracle_threads():
+    import oracle
+    return oracle.num_threads()
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_layer_sample(REF_TOKENS)
+    secs, flops = [], 0
+    for i in range(args.steps):
+        s, flops = oracle_layer_sample(REF_TOKENS, seed=4321 + i)
+        secs.append(s)
+    total = sum(secs)
+    value = flops * len(secs) / total / 1e12
+    sample = (f"{REF_TOKENS} of 2048 tokens of one of the 12 dim1024 layers per step (6 linears: quantize x/w/g "
+              f"with rings, fwd+dX+dW GEMMs, bf16 bias, dbias)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(secs),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8 e4m3/e5m2 (fp32 accumulate)",
+            "data": "synthetic", "config": config_dict(),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict():
+    return {"workload": "12L/dim1024/B4xT512 linears: 12 layers x {q,k,v,o 1024x1024, up 1024x4096, "
+                        "down 4096x1024}, M=2048 tokens, fwd+dX+dW, E4M3 x/w, E5M2 g, delayed scaling H=16, "
+                        "bf16 bias + dbias",
+            "M": 2048, "layers": wl.BENCH_LAYERS, "linears_per_step": wl.BENCH_LAYERS * len(wl.BENCH_LAYER),
+            "hist_len": wl.HIST_LEN, "l2": "inputs larger than L2 (step working set ~3 GB, 126 MB L2)",
+            "timing": "CUDA graph of the step's C-ABI calls, CUDA events, max over ranks"}
+
+
+# --------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=wl.BENCH_LAYERS, help="layers per step (profiling runs only)")
+    ap.add_argument("--no-extras", action="store_true", help="skip e2e, kernel timing and cpu baseline")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import fp8_delayed_scaling_03_b200 as F
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    wl.BENCH_LAYERS = args.layers
+    lins = build_model(F, device, rank)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+    flops_step = wl.bench_flops_per_step(args.layers)
+
+    # eager warm-up (first-launch set-up happens outside the capture), then capture
+    with torch.cuda.stream(stream):
+        run_step(F, lins, stream.cuda_stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run_step(F, lins, stream.cuda_stream)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    max_ms = reduce_max(ms, world, device)
+    value = aggregate_throughput(flops_step * args.steps, world, max_ms / 1e3) / 1e12
+    status = F.fp8_get_device_status()
+    if status:
+        raise F.Fp8Error(status, "device status after timed region")
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8 e4m3/e5m2 (fp32 accumulate, bf16 out)", "data": "synthetic",
+            "config": config_dict(), "clocks": clk.report(),
+            "gpu_launches": LAUNCHES_PER_LINEAR * len(lins) * args.steps}
+
+    if not args.no_extras:
+        pk, pk_kind = peaks()
+        # ---- kernel-level timing and roofline of the dominant kernel
+        tot, work, count, shapes = time_kernels(F, lins, stream)
+        gemm_tflops = work["gemm"] / (tot["gemm"] / 1e3) / 1e12
+        fp8_peak = pk["bf16_tflops"] * FP8_PER_BF16
+        traffic = gemm_traffic_per_launch()
+        line["roofline"] = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                            "frac": gemm_tflops / fp8_peak, "traffic": traffic,
+                            "kernel": "fp8_gemm_kernel (the step's 216 fwd/dX/dW launches, replayed as one graph)",
+                            "peak_source": f"{pk_kind} bf16 burst x {FP8_PER_BF16} (nominal fp8:bf16)",
+                            "frac_of_nominal_4.5PF": gemm_tflops / NOMINAL_FP8_TFLOPS}
+        q_gbs = work["quantize"] / (tot["quantize"] / 1e3) / 1e9
+        d_gbs = work["dbias"] / (tot["dbias"] / 1e3) / 1e9
+        step_kernels_ms = sum(tot.values())
+        line["kernels"] = {
+            "share": {k: v / step_kernels_ms for k, v in tot.items()},
+            "ms_per_step": tot, "launches_per_step": count,
+            "step_ms_vs_sum_of_classes": (max_ms / args.steps) / step_kernels_ms,
+            "quantize": {"achieved_gbs": q_gbs, "peak_gbs": pk["hbm_gbs"], "frac": q_gbs / pk["hbm_gbs"],
+                         "bytes_per_elem": 3, "note": "bf16 in + fp8 out; class graph replay"},
+            "dbias": {"achieved_gbs": d_gbs, "frac": d_gbs / pk["hbm_gbs"], "bytes_per_elem": 2},
+            "gemm_by_shape": shapes}
+
+        # ---- end to end through the C ABI with host buffers
+        host_in = [[t.cpu().pin_memory() for t in L.inputs()] for L in lins]
+        host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in L.outputs()] for L in lins]
+        h2d = sum(t.numel() * t.element_size() for ts in host_in for t in ts)
+        d2h = sum(t.numel() * t.element_size() for ts in host_out for t in ts)
+
+        def e2e_step():
+            for L, hs in zip(lins, host_in):
+                for d, h in zip(L.inputs(), hs):
+                    d.copy_(h, non_blocking=True)
+            run_step(F, lins, stream.cuda_stream)
+            for L, hs in zip(lins, host_out):
+                for d, h in zip(L.outputs(), hs):
+                    h.copy_(d, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 10))
+        with torch.cuda.stream(stream):
+            e2e_step()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(e2e_steps):
+                e2e_step()
+            a1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(a0.elapsed_time(a1), world, device)
+        line["e2e"] = {"value": aggregate_throughput(flops_step * e2e_steps, world, e2e_ms / 1e3) / 1e12,
+                       "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps,
+                       "path": "pinned host -> device copies, fp8_linear_forward/backward per linear, device -> "
+                               "pinned host copies of y, dX, dW, dbias, one stream"}
+
+        # ---- CPU oracle baseline (rank 0, one GPU only)
+        if rank == 0 and world == 1:
+            secs, flops = oracle_layer_sample(BASELINE_TOKENS)
+            line["cpu_baseline"] = {
+                "value": flops / secs / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                "sample": f"{BASELINE_TOKENS} of 2048 tokens of one of the 12 dim1024 layers (6 linears: quantize "
+                          f"x/w/g with rings, fwd+dX+dW GEMMs with fp32 accumulation, bf16 bias, dbias), "
+                          f"{secs:.1f} s"}
+
+    if world > 1:
+        del graph
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -79,9 +79,9 @@ int check_fp8_matrix(const void* p, int64_t ld, int64_t cols) {
   return FP8_OK;
 }
 
-// 2-D uint8 tensor map, 128-byte swizzle, zero fill out of bounds.
-int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld_bytes,
-             uint32_t box_inner, uint32_t box_outer) {
+// 2-D tensor map with zero fill out of bounds (loads) / clipping (stores).
+int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+             uint64_t ld_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
   EncodeTiledFn enc = encoder();
   if (!enc) {
     snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled unavailable");
@@ -91,14 +91,18 @@ int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
   cuuint64_t strides[1] = {ld_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
     return FP8_ERR_CUDA;
   }
   return FP8_OK;
+}
+
+// fp8 operand map: 128-byte rows of a 128 x `rows` box, 128-byte swizzle.
+int make_fp8_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_rows) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, inner, outer, ld, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 struct MmCall {
@@ -153,15 +157,26 @@ int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st) {
   const int sms = num_sms(dev);
   if (sms <= 0) return cuda_fail(cudaGetLastError());
   const int bn = pick_bn(c.m, c.n, sms);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, td;
   std::memset(&ta, 0, sizeof(ta));
   std::memset(&tb, 0, sizeof(tb));
+  std::memset(&td, 0, sizeof(td));
   if (c.k > 0) {
-    int s = c.a_major == FP8_K_MAJOR ? make_map(&ta, c.a, c.k, c.m, c.lda, 128, 128)
-                                     : make_map(&ta, c.a, c.m, c.k, c.lda, 128, 128);
+    int s = c.a_major == FP8_K_MAJOR ? make_fp8_map(&ta, c.a, c.k, c.m, c.lda, 128)
+                                     : make_fp8_map(&ta, c.a, c.m, c.k, c.lda, 128);
     if (s) return s;
-    s = c.b_major == FP8_K_MAJOR ? make_map(&tb, c.b, c.k, c.n, c.ldb, 128, bn)
-                                 : make_map(&tb, c.b, c.n, c.k, c.ldb, 128, 128);
+    s = c.b_major == FP8_K_MAJOR ? make_fp8_map(&tb, c.b, c.k, c.n, c.ldb, bn)
+                                 : make_fp8_map(&tb, c.b, c.n, c.k, c.ldb, 128);
+    if (s) return s;
+  }
+  // bf16 output through TMA stores when the rows are 16-byte addressable and
+  // end on a 16-byte boundary (a B200 run showed the store clipping the row
+  // end at 16-byte granularity, writing up to 7 columns past n otherwise):
+  // 32 x 32 boxes, 64-byte swizzle (matches the epilogue's staging layout).
+  const bool tma_store = aligned(c.d, 16) && ((c.ldd * 2) % 16 == 0) && (c.n % 8 == 0);
+  if (tma_store) {
+    int s = make_map(&td, c.d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.n, c.m, c.ldd * 2, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
     if (s) return s;
   }
   GemmParams p;
@@ -184,16 +199,17 @@ int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st) {
   p.bias_scale = c.bias_scale;
   p.d = c.d;
   p.ldd = c.ldd;
-  p.vec_store = aligned(c.d, 16) && ((c.ldd * 2) % 16 == 0);
+  p.tma_store = tma_store ? 1 : 0;
   p.status = status_ptr(dev);
   if (side) p.side = *side;
-  e = launch_gemm(ta, tb, p, bn, st);
+  e = launch_gemm(ta, tb, td, p, bn, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return FP8_OK;
 }
 
-int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt, void* ring,
-                 int H, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out, cudaStream_t st) {
+QuantizeParams make_qparams(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt,
+                            void* ring, int H, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out,
+                            bool allow_flatten) {
   QuantizeParams p;
   std::memset(&p, 0, sizeof(p));
   p.in = in;
@@ -204,7 +220,7 @@ int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
   p.amax_out = amax_out;
   p.scale_out = scale_out;
   const int es = esize(in_dtype);
-  if (ld_in == cols && ld_out == cols) {  // contiguous: one long row
+  if (allow_flatten && ld_in == cols && ld_out == cols) {  // contiguous: one long row
     p.rows = 1;
     p.cols = rows * cols;
     p.ld_in = p.cols;
@@ -218,7 +234,14 @@ int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
   p.chunks_per_row = (p.cols + 15) / 16;
   p.total_chunks = p.rows * p.chunks_per_row;
   p.vec_ok = aligned(in, 16) && ((p.ld_in * es) % 16 == 0);
-  cudaError_t e = launch_quantize(in_dtype, fmt, p, st);
+  return p;
+}
+
+int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt, void* ring,
+                 int H, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out, cudaStream_t st) {
+  const QuantizeParams p =
+      make_qparams(in, in_dtype, rows, cols, ld_in, fmt, ring, H, out, ld_out, amax_out, scale_out, true);
+  cudaError_t e = launch_quantize(in_dtype, fmt, &p, nullptr, st);
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
 
@@ -371,17 +394,23 @@ int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   SideWrites side;
   std::memset(&side, 0, sizeof(side));
-  if (xq) {
-    side.copy_src[0] = a->x_scale_in; side.copy_dst[0] = a->sx_out; side.zero_dst[0] = a->amax_x_out;
-  } else if ((s = run_quantize(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8, a->ldx8,
-                               a->amax_x_out, a->sx_out, st))) {
-    return s;
-  }
-  if (wq) {
-    side.copy_src[1] = a->w_scale_in; side.copy_dst[1] = a->sw_out; side.zero_dst[1] = a->amax_w_out;
-  } else if ((s = run_quantize(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8, a->ldw8,
-                               a->amax_w_out, a->sw_out, st))) {
-    return s;
+  if (xq) { side.copy_src[0] = a->x_scale_in; side.copy_dst[0] = a->sx_out; side.zero_dst[0] = a->amax_x_out; }
+  if (wq) { side.copy_src[1] = a->w_scale_in; side.copy_dst[1] = a->sw_out; side.zero_dst[1] = a->amax_w_out; }
+  if (!xq && !wq && a->x_dtype == a->w_dtype && a->fmt_x == a->fmt_w) {
+    // x and w in one launch (each with its own ring and finalize)
+    const QuantizeParams qx = make_qparams(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8,
+                                           a->ldx8, a->amax_x_out, a->sx_out, true);
+    const QuantizeParams qw = make_qparams(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8,
+                                           a->ldw8, a->amax_w_out, a->sw_out, true);
+    cudaError_t e = launch_quantize(a->x_dtype, a->fmt_x, &qx, &qw, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  } else {
+    if (!xq && (s = run_quantize(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8, a->ldx8,
+                                 a->amax_x_out, a->sx_out, st)))
+      return s;
+    if (!wq && (s = run_quantize(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8, a->ldw8,
+                                 a->amax_w_out, a->sw_out, st)))
+      return s;
   }
   return run_mm(c, &side, st);
 }
@@ -425,9 +454,24 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   SideWrites side;
   std::memset(&side, 0, sizeof(side));
   bool side_pending = false;
+  bool dbias_done = false;
   if (gq) {
     side.copy_src[0] = a->g_scale_in; side.copy_dst[0] = a->sg_out; side.zero_dst[0] = a->amax_g_out;
     side_pending = true;
+  } else if (a->need_dbias) {
+    // quantize g and sum its columns in the same pass over g
+    ColsumParams cp;
+    std::memset(&cp, 0, sizeof(cp));
+    cp.q = make_qparams(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
+                        a->amax_g_out, a->sg_out, false);
+    dbias_geometry(M, N, &cp.R, &cp.rows_per_split);
+    cp.partial = static_cast<float*>(a->workspace);
+    const size_t part = (static_cast<size_t>(cp.R) * static_cast<size_t>(N) * 4u + 15u) & ~size_t(15);
+    cp.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(a->workspace) + part);
+    cp.dbias = a->dbias;
+    cudaError_t e = launch_quantize_colsum(a->g_dtype, a->fmt_g, cp, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    dbias_done = true;
   } else if ((s = run_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
                                a->amax_g_out, a->sg_out, st))) {
     return s;
@@ -444,7 +488,7 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
     cudaError_t e = launch_side_writes(side, st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
-  if (a->need_dbias) {
+  if (a->need_dbias && !dbias_done) {
     if ((s = fp8_dbias(a->g, a->g_dtype, M, N, a->ldg, a->g_scale_in, a->dbias, a->workspace, a->workspace_bytes,
                        stream)))
       return s;

@@ -9,10 +9,11 @@
 // block of 8 x 32 threads streams rows of its split with 16-byte loads (8
 // columns per thread), reduces its 8 row lanes in shared memory in a fixed
 // order and writes 256 fp32 partials.  The block that draws the last ticket
-// of its column tile sums the R partials in split order, so the result does
+// of its column tile sums the R partials in a fixed order, so the result does
 // not depend on block scheduling, and rezeroes the tile's counter.
 #include "device.cuh"
 #include "internal.h"
+#include "launch.h"
 
 namespace fp8lin {
 namespace {
@@ -92,6 +93,8 @@ template <int DT>
 __global__ void __launch_bounds__(kRowLanes * 32) dbias_kernel(const DbiasParams p) {
   __shared__ float red[kRowLanes][kCols];
   __shared__ int last;
+  pdl_wait();
+  pdl_trigger();
   const int tx = threadIdx.x & 31;
   const int ty = threadIdx.x >> 5;
   const int64_t c_base = static_cast<int64_t>(blockIdx.x) * kCols;
@@ -128,8 +131,20 @@ __global__ void __launch_bounds__(kRowLanes * 32) dbias_kernel(const DbiasParams
   if (!last) return;
   __threadfence();
   if (col < p.N) {
-    float tot = 0.0f;
-    for (int r = 0; r < p.R; ++r) tot += __ldcg(p.partial + static_cast<int64_t>(r) * p.N + col);
+    // Four interleaved partial sums (split r goes to sum r % 4), combined as
+    // (s0 + s1) + (s2 + s3): a fixed order, with four loads in flight.
+    float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const float* pc = p.partial + col;
+    int r = 0;
+    for (; r + 4 <= p.R; r += 4) {
+      float t[4];
+      #pragma unroll
+      for (int u = 0; u < 4; ++u) t[u] = __ldcg(pc + static_cast<int64_t>(r + u) * p.N);
+      #pragma unroll
+      for (int u = 0; u < 4; ++u) s4[u] += t[u];
+    }
+    for (; r < p.R; ++r) s4[r & 3] += __ldcg(pc + static_cast<int64_t>(r) * p.N);
+    const float tot = (s4[0] + s4[1]) + (s4[2] + s4[3]);
     static_cast<__nv_bfloat16*>(p.dbias)[col] = __float2bfloat16_rn(tot);
   }
   if (threadIdx.x == 0) atomicExch(&p.counters[blockIdx.x], 0u);
@@ -138,9 +153,10 @@ __global__ void __launch_bounds__(kRowLanes * 32) dbias_kernel(const DbiasParams
 }  // namespace
 
 void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
+  // About 296 blocks (two per SM of a B200) in total, at least 64 rows each.
   const int64_t col_tiles = (N + kCols - 1) / kCols;
-  int64_t r = (1184 + col_tiles - 1) / (col_tiles > 0 ? col_tiles : 1);
-  const int64_t rmax = (M + 31) / 32;
+  int64_t r = (296 + col_tiles - 1) / (col_tiles > 0 ? col_tiles : 1);
+  const int64_t rmax = (M + 63) / 64;
   if (r > rmax) r = rmax;
   if (r < 1) r = 1;
   int64_t rps = (M + r - 1) / r;
@@ -155,13 +171,12 @@ cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>((p.N + kCols - 1) / kCols), static_cast<unsigned>(p.R));
   const int threads = kRowLanes * 32;
   switch (p.dtype) {
-    case kBF16: dbias_kernel<kBF16><<<grid, threads, 0, s>>>(p); break;
-    case kFP16: dbias_kernel<kFP16><<<grid, threads, 0, s>>>(p); break;
-    case kFP32: dbias_kernel<kFP32><<<grid, threads, 0, s>>>(p); break;
-    case kDtE4M3: dbias_kernel<kDtE4M3><<<grid, threads, 0, s>>>(p); break;
-    default: dbias_kernel<kDtE5M2><<<grid, threads, 0, s>>>(p); break;
+    case kBF16: return launch_pdl(dbias_kernel<kBF16>, grid, dim3(threads), 0, s, p);
+    case kFP16: return launch_pdl(dbias_kernel<kFP16>, grid, dim3(threads), 0, s, p);
+    case kFP32: return launch_pdl(dbias_kernel<kFP32>, grid, dim3(threads), 0, s, p);
+    case kDtE4M3: return launch_pdl(dbias_kernel<kDtE4M3>, grid, dim3(threads), 0, s, p);
+    default: return launch_pdl(dbias_kernel<kDtE5M2>, grid, dim3(threads), 0, s, p);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace fp8lin

@@ -17,13 +17,23 @@
 //   * the transposed ("crosswise") operands of dX and dW are read in place:
 //     the smem descriptor and instruction descriptor mark them MN-major, which
 //     tcgen05 supports for E4M3/E5M2 -- no transpose pass, no copy;
-//   * warps 2-5: epilogue.  tcgen05.ld 32 lanes x 16 columns, multiply by the
-//     dequant factor, add bias in fp32 (bf16, or fp8 / bias_scale), one RNE
-//     rounding to bf16, 16-byte stores (astrai @4019dda fused-bias bullet).
+//   * warps 2-9: epilogue, two warps per TMEM lane quadrant splitting the
+//     tile's columns.  Per 32-column step: tcgen05.ld 32 lanes x 32 columns,
+//     multiply by the dequant factor, add the bias in fp32 (bf16, or fp8 /
+//     bias_scale; one load per lane, broadcast by shuffle), one RNE rounding
+//     to bf16 (astrai @4019dda fused-bias bullet), then the 32x32 bf16 block is
+//     staged in a 64-byte-swizzled shared slab and written by a TMA store
+//     (coalesced, asynchronous, clipped at the matrix edge) -- the pages'
+//     kernel also staged its epilogue through shared memory for write
+//     efficiency (astrai @4019dda, epilogue bullet).  The accumulator is handed
+//     back to the MMA warp right after its last TMEM read.  Output strides that
+//     TMA cannot address (row pitch not a multiple of 16 bytes) take guarded
+//     per-element stores instead.
 // Every mbarrier wait is bounded (see device.cuh); a timeout records
 // FP8_ERR_DEVICE_TIMEOUT and the CTA winds down instead of hanging.
 #include "device.cuh"
 #include "internal.h"
+#include "launch.h"
 
 namespace fp8lin {
 namespace {
@@ -31,7 +41,10 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 128;  // fp8 elements (= bytes) of k per stage
 constexpr int kUmmaK = 32;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;       // 10 warps: TMA, MMA, 8 epilogue
+constexpr int kEpiWarps = 8;
+constexpr int kEpiCols = 32;        // columns per epilogue step
+constexpr int kEpiSlab = 32 * kEpiCols * 2;  // one 32x32 bf16 staging slab
 
 template <int BN>
 struct Cfg {
@@ -40,8 +53,9 @@ struct Cfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = BN == 256 ? 4 : 6;
   static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiSlab;  // two slabs per epilogue warp
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
+  static constexpr int kSmem = kStages * kStageBytes + kEpiBytes + kBarBytes + 1024;
   static_assert(BN == 128 || BN == 256, "BN");
 };
 
@@ -71,13 +85,14 @@ __device__ __forceinline__ float bias_value(const GemmParams& p, int j, float bi
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tma_d, const GemmParams p) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * C::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+  uint8_t* sEpi = sB + C::kStages * C::kBBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::kEpiBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
@@ -94,17 +109,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], kEpiWarps);
     }
     *abort_flag = 0;
     fence_mbar_init();
-    prefetch_tmap(&tma_a);
-    prefetch_tmap(&tma_b);
+    if (p.k_blocks > 0) {
+      prefetch_tmap(&tma_a);
+      prefetch_tmap(&tma_b);
+    }
+    if (p.tma_store) prefetch_tmap(&tma_d);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
+  // Everything above overlaps the previous kernel on the stream; from here on
+  // its results (operands, scales) are read.
+  pdl_wait();
+  pdl_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 64) {
     for (int i = 0; i < 2; ++i) {
       if (p.side.copy_dst[i]) *p.side.copy_dst[i] = *p.side.copy_src[i];
@@ -179,57 +201,80 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int ew = warp - 2;                 // 0..7
+    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+    const int half = ew >> 2;                // which half of the tile's columns
     const int row_in_tile = q * 32 + lane;
     const float inv = 1.0f / (*p.scale_a * *p.scale_b);
     const float binv = (p.bias_kind >= 2) ? 1.0f / *p.bias_scale : 1.0f;
     const bool have_k = p.k_blocks > 0;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    uint8_t* slabs = sEpi + ew * 2 * kEpiSlab;
+    int slab = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     __nv_bfloat16* D = static_cast<__nv_bfloat16*>(p.d);
+    constexpr int kSteps = BN / 2 / kEpiCols;
     for (int t = blockIdx.x; t < p.num_tiles && !*abort_flag; t += gridDim.x) {
       int tm, tn;
       tile_coords(p, t, tm, tn);
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag)) break;
       tc_fence_after();
       const int row = tm * kBM + row_in_tile;
-      const bool row_ok = row < p.m;
-      __nv_bfloat16* drow = D + static_cast<int64_t>(row) * p.ldd;
+      const int col_half = tn * BN + half * (BN / 2);
+      const int live_steps = min(kSteps, max(0, (p.n - col_half + kEpiCols - 1) / kEpiCols));
       #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        const int col0 = tn * BN + c0;
-        if (col0 >= p.n) break;  // warp-uniform
-        __syncwarp();            // tcgen05.ld is .sync.aligned
-        uint32_t r[16];
-        tmem_ld16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c0), r);
-        tmem_ld_wait();
-        float v[16];
-        #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v[j] = (have_k ? __uint_as_float(r[j]) : 0.0f) * inv;
-          if (p.bias_kind && col0 + j < p.n) v[j] += bias_value(p, col0 + j, binv);
+      for (int st = 0; st < kSteps; ++st) {
+        const int col0 = col_half + st * kEpiCols;
+        uint32_t r[32];
+        if (st < live_steps) {
+          __syncwarp();  // tcgen05.ld is .sync.aligned
+          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + half * (BN / 2) + st * kEpiCols), r);
+          tmem_ld_wait();
         }
-        if (row_ok) {
-          if (p.vec_store && col0 + 16 <= p.n) {
-            uint4 o0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                  pack_bf16x2(v[6], v[7]));
-            uint4 o1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                                  pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
-            uint4* dst = reinterpret_cast<uint4*>(drow + col0);
-            dst[0] = o0;
-            dst[1] = o1;
-          } else {
-            #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (col0 + j < p.n) drow[col0 + j] = __float2bfloat16_rn(v[j]);
+        if (st == kSteps - 1) {  // last TMEM read of this accumulator: hand it back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        if (st >= live_steps) continue;
+        float bl = 0.0f;
+        if (p.bias_kind && col0 + lane < p.n) bl = bias_value(p, col0 + lane, binv);
+        float v[32];
+        #pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          v[j] = (have_k ? __uint_as_float(r[j]) : 0.0f) * inv;
+          if (p.bias_kind) v[j] += __shfl_sync(0xFFFFFFFFu, bl, j);
+        }
+        if (p.tma_store) {
+          uint8_t* buf = slabs + slab * kEpiSlab;
+          if (lane == 0) bulk_wait_read<1>();  // the store that last read this slab is done
+          __syncwarp();
+          // row `lane` of the 32x32 block, 4 chunks of 16 bytes, 64-byte swizzle
+          #pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint4 o = make_uint4(pack_bf16x2(v[8 * c + 0], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                 pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+            const int phys = c ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4*>(buf + lane * 64 + phys * 16) = o;
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_d, buf, col0, tm * kBM + q * 32);
+            bulk_commit();
+          }
+          slab ^= 1;
+        } else if (row < p.m) {
+          __nv_bfloat16* drow = D + static_cast<int64_t>(row) * p.ldd;
+          #pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < p.n) drow[col0 + j] = __float2bfloat16_rn(v[j]);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (p.tma_store && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -242,7 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t s) {
+cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const GemmParams& p,
+                      cudaStream_t s) {
   using C = Cfg<BN>;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -254,15 +300,15 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPa
   }
   const int sms = num_sms(dev);
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  fp8_gemm_kernel<BN><<<grid, kThreads, C::kSmem, s>>>(ta, tb, p);
-  return cudaGetLastError();
+  return launch_pdl(fp8_gemm_kernel<BN>, dim3(grid), dim3(kThreads), C::kSmem, s, ta, tb, td, p);
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, int bn, cudaStream_t s) {
-  if (bn == 256) return launch_bn<256>(ta, tb, p, s);
-  return launch_bn<128>(ta, tb, p, s);
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, GemmParams p, int bn,
+                        cudaStream_t s) {
+  if (bn == 256) return launch_bn<256>(ta, tb, td, p, s);
+  return launch_bn<128>(ta, tb, td, p, s);
 }
 
 }  // namespace fp8lin

@@ -33,6 +33,25 @@ struct QuantizeParams {
   int vec_ok;                 // 16-byte vector loads are legal for full chunks
 };
 
+// One or two tensors quantized by one launch: blocks [0, blocks0) work on
+// t[0], the rest on t[1] (each with its own ring and last-block finalize).
+struct QuantizePair {
+  QuantizeParams t[2];
+  int blocks0;
+};
+
+// Quantize of a [rows, cols] tensor (not flattened) that also produces its
+// column sums: grid (ceil(cols / 256), R), partial [R, cols] fp32 and one
+// counter per column tile in a caller workspace.
+struct ColsumParams {
+  QuantizeParams q;
+  float* partial;
+  unsigned* counters;
+  void* dbias;                // bf16 [cols]
+  int64_t rows_per_split;
+  int R;
+};
+
 // Side writes a GEMM launch performs once (block 0), for operands that arrive
 // pre-quantized: dst = *src for the scale snapshot, zero for its amax.
 struct SideWrites {
@@ -54,7 +73,7 @@ struct GemmParams {
   const float* bias_scale;
   void* d;
   int64_t ldd;
-  int vec_store;              // 16-byte stores of bf16 rows are legal
+  int tma_store;              // D is addressable by TMA (16-byte aligned base and row pitch)
   int* status;
   SideWrites side;
 };
@@ -74,10 +93,13 @@ struct DbiasParams {
 
 int num_sms(int device);
 
-cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams& p, cudaStream_t s);
+// b may be NULL (one tensor); both tensors share in_dtype and fmt.
+cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, const QuantizeParams* b, cudaStream_t s);
+cudaError_t launch_quantize_colsum(int in_dtype, int fmt, const ColsumParams& cp, cudaStream_t s);
 cudaError_t launch_ring_set(float* ring, int H, float scale, cudaStream_t s);
 cudaError_t launch_side_writes(const SideWrites& w, cudaStream_t s);
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, int bn, cudaStream_t s);
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, GemmParams p, int bn,
+                        cudaStream_t s);
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s);
 
 // dbias geometry shared by the size query and the launcher.

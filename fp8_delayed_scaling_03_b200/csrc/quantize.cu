@@ -1,114 +1,114 @@
 // quantize.cu -- HBM-bound fp8 quantize with in-kernel delayed-scaling finalize.
 //
-// One launch per tensor (AstrAI commit log, tests/extension @2eeac02, bullets
-// on finalizing scale rings inside the quantize kernels):
-//   1. every thread reads the ring's current scale s (block 0 also stores it to
-//      scale_out: the snapshot the GEMM dequantizes with, astrai/extension/ops
-//      @057c0d3 snapshot bullet);
-//   2. a grid-stride loop over 16-element chunks loads the input with 16-byte
-//      vector loads, keeps a running max of |x| over the RAW values (NaN
-//      ignored), multiplies by s in fp32 and casts pairs with
+// One launch per tensor, or per pair of tensors (AstrAI commit log,
+// tests/extension @2eeac02, bullets on finalizing scale rings inside the
+// quantize kernels; astrai @4019dda, quantize_dual bullet):
+//   1. every thread reads its ring's current scale s (the first block of the
+//      tensor also stores it to scale_out: the snapshot the GEMM dequantizes
+//      with, astrai/extension/ops @057c0d3 snapshot bullet);
+//   2. a grid-stride loop over 16-element chunks streams the input with
+//      16-byte loads (the next iteration's loads are issued before the
+//      current chunks are converted), keeps a running max of |x| over the RAW
+//      values (NaN ignored), multiplies by s in fp32 and casts pairs with
 //      cvt.rn.satfinite.{e4m3,e5m2}x2, storing 16 fp8 codes per 16-byte store;
-//   3. warp max (redux.sync) -> block max -> one atomicMax on the ring's
+//   3. warp max (redux.sync) -> block max -> one relaxed red.max on the ring's
 //      scratch word (non-negative floats order like their bit patterns);
-//   4. threadfence + atomicAdd ticket: the block that draws the last ticket
-//      folds the launch's amax into hist[step % H], reduces the window, and
-//      publishes fp8_max / max as the next scale (kept when the max is 0 or
-//      inf or the quotient overflows), then rezeroes ticket and scratch.
+//   4. an acquire-release fetch-add on the ring's ticket: the block that draws
+//      the tensor's last ticket sees every block's max, folds the launch's
+//      amax into hist[step % H], reduces the window, and publishes
+//      fp8_max / max as the next scale (kept when the max is 0 or inf or the
+//      quotient overflows), then rezeroes ticket and scratch.  History and
+//      step are prefetched into shared memory at kernel start, so this tail is
+//      two dependent global round trips.
+// The column-sum variant (quantize of g with the bias gradient) walks 2-D
+// tiles of 256 columns instead, so each thread also accumulates the column
+// sums of its 16 columns; per-tile partials meet in a workspace and the last
+// block of each column tile (its own ticket) sums them in a fixed order
+// (astrai @4019dda: the column sum runs only when the bias needs a gradient).
 // No block ever waits on another, so nothing here can hang.
+#include <type_traits>
+
 #include "device.cuh"
 #include "internal.h"
+#include "launch.h"
 
 namespace fp8lin {
 namespace {
 
 constexpr int kThreads = 256;
 constexpr int kChunk = 16;
+constexpr int kHistCache = 64;  // ring histories up to this length are prefetched
+
+// ---------------------------------------------------------------- raw chunks
+
+// 16 consecutive input elements, kept as raw bits until converted.
+template <typename T>
+struct Raw {
+  static constexpr int kWords = static_cast<int>(sizeof(T)) * kChunk / 16;
+  uint4 w[kWords];
+};
 
 template <typename T>
-struct Src;
+__device__ __forceinline__ uint32_t elem_bits(const void* base, int64_t idx) {
+  if constexpr (sizeof(T) == 2) return static_cast<uint32_t>(__ldg(static_cast<const unsigned short*>(base) + idx));
+  else return __float_as_uint(__ldg(static_cast<const float*>(base) + idx));
+}
 
-template <>
-struct Src<__nv_bfloat16> {
-  static constexpr int kBytes = 2;
-  static __device__ __forceinline__ void vec(const void* base, int64_t idx, float (&v)[16]) {
-    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + idx);
-    uint4 q[2] = {__ldg(p), __ldg(p + 1)};
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(q);
+// Load the chunk starting at (r, col): 16-byte loads when the whole chunk is
+// inside the row and the rows are 16-byte aligned, else element loads with
+// zeros past the row end.
+template <typename T>
+__device__ __forceinline__ void load_raw(const QuantizeParams& p, int64_t r, int64_t col, Raw<T>& raw) {
+  const int64_t base = r * p.ld_in + col;
+  if (p.vec_ok && col + kChunk <= p.cols) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(p.in) + base);
+    #pragma unroll
+    for (int i = 0; i < Raw<T>::kWords; ++i) raw.w[i] = __ldg(src + i);
+  } else {
+    const int64_t left = p.cols - col;
+    uint32_t b[kChunk];
+    #pragma unroll
+    for (int j = 0; j < kChunk; ++j) b[j] = (j < left) ? elem_bits<T>(p.in, base + j) : 0u;
+    #pragma unroll
+    for (int i = 0; i < Raw<T>::kWords; ++i) {
+      if constexpr (sizeof(T) == 2)
+        raw.w[i] = make_uint4(b[8 * i] | (b[8 * i + 1] << 16), b[8 * i + 2] | (b[8 * i + 3] << 16),
+                              b[8 * i + 4] | (b[8 * i + 5] << 16), b[8 * i + 6] | (b[8 * i + 7] << 16));
+      else
+        raw.w[i] = make_uint4(b[4 * i], b[4 * i + 1], b[4 * i + 2], b[4 * i + 3]);
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void to_floats(const Raw<T>& raw, float (&v)[16]) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(raw.w);
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
     #pragma unroll
     for (int i = 0; i < 8; ++i) {
       v[2 * i] = __uint_as_float(w[i] << 16);
       v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
-  }
-  static __device__ __forceinline__ float one(const void* base, int64_t idx) {
-    return __uint_as_float(static_cast<uint32_t>(__ldg(static_cast<const unsigned short*>(base) + idx)) << 16);
-  }
-};
-
-template <>
-struct Src<__half> {
-  static constexpr int kBytes = 2;
-  static __device__ __forceinline__ void vec(const void* base, int64_t idx, float (&v)[16]) {
-    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const __half*>(base) + idx);
-    uint4 q[2] = {__ldg(p), __ldg(p + 1)};
-    const __half2* h = reinterpret_cast<const __half2*>(q);
+  } else if constexpr (std::is_same<T, __half>::value) {
     #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float2 f = __half22float2(h[i]);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
       v[2 * i] = f.x;
       v[2 * i + 1] = f.y;
     }
-  }
-  static __device__ __forceinline__ float one(const void* base, int64_t idx) {
-    return __half2float(static_cast<const __half*>(base)[idx]);
-  }
-};
-
-template <>
-struct Src<float> {
-  static constexpr int kBytes = 4;
-  static __device__ __forceinline__ void vec(const void* base, int64_t idx, float (&v)[16]) {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+  } else {
     #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 f = __ldg(p + i);
-      v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
-    }
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(w[i]);
   }
-  static __device__ __forceinline__ float one(const void* base, int64_t idx) {
-    return __ldg(static_cast<const float*>(base) + idx);
-  }
-};
+}
 
 template <int FMT>
 __device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
   return FMT == kE4M3 ? cvt_e4m3x2(lo, hi) : cvt_e5m2x2(lo, hi);
 }
 
-// Chunk c -> (row, first column).
-__device__ __forceinline__ void chunk_pos(const QuantizeParams& p, int64_t c, int64_t& r, int64_t& col) {
-  if (p.rows == 1) {
-    r = 0;
-    col = c * kChunk;
-  } else {
-    r = c / p.chunks_per_row;
-    col = (c - r * p.chunks_per_row) * kChunk;
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ void load_chunk(const QuantizeParams& p, int64_t r, int64_t col, float (&v)[16]) {
-  const int64_t base = r * p.ld_in + col;
-  if (p.vec_ok && col + kChunk <= p.cols) {
-    Src<T>::vec(p.in, base, v);
-  } else {
-    const int64_t left = p.cols - col;
-    #pragma unroll
-    for (int j = 0; j < kChunk; ++j) v[j] = (j < left) ? Src<T>::one(p.in, base + j) : 0.0f;
-  }
-}
-
+// amax, scale, cast and one 16-byte store of the chunk at (r, col); bytes past
+// cols (row padding up to ld_out) are written as zero.
 template <int FMT>
 __device__ __forceinline__ void cast_store(const QuantizeParams& p, int64_t r, int64_t col, const float (&v)[16],
                                            float s, float& amax) {
@@ -122,78 +122,236 @@ __device__ __forceinline__ void cast_store(const QuantizeParams& p, int64_t r, i
     else w[i >> 1] = h;
   }
   const int64_t left = p.cols - col;
-  if (left < kChunk) {  // bytes past cols are padding: write zeros
+  if (left < kChunk) {
     #pragma unroll
     for (int j = 0; j < kChunk; ++j)
       if (j >= left) w[j >> 2] &= ~(0xFFu << (8 * (j & 3)));
   }
-  uint4* dst = reinterpret_cast<uint4*>(p.out + r * p.ld_out + col);
-  *dst = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(p.out + r * p.ld_out + col) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-template <typename T, int FMT>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantizeParams p) {
-  __shared__ uint32_t warp_max[kThreads / 32];
-  const float s = p.ring[p.H];
-  if (blockIdx.x == 0 && threadIdx.x == 0 && p.scale_out) *p.scale_out = s;
-
-  float amax = 0.0f;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  #pragma unroll 1
-  for (int64_t c = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; c < p.total_chunks;
-       c += 2 * stride) {
-    const int64_t c2 = c + stride;
-    const bool two = c2 < p.total_chunks;
-    int64_t r1, col1, r2 = 0, col2 = 0;
-    float v1[16], v2[16];
-    chunk_pos(p, c, r1, col1);
-    load_chunk<T>(p, r1, col1, v1);
-    if (two) {
-      chunk_pos(p, c2, r2, col2);
-      load_chunk<T>(p, r2, col2, v2);
-    }
-    cast_store<FMT>(p, r1, col1, v1, s, amax);
-    if (two) cast_store<FMT>(p, r2, col2, v2, s, amax);
+__device__ __forceinline__ void chunk_pos(const QuantizeParams& p, int64_t c, int64_t& r, int64_t& col) {
+  if (p.rows == 1) {
+    r = 0;
+    col = c * kChunk;
+  } else {
+    r = c / p.chunks_per_row;
+    col = (c - r * p.chunks_per_row) * kChunk;
   }
+}
 
-  // amax: |x| >= 0 and never NaN here, so uint order == float order.
-  uint32_t bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
-  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = bits;
-  __syncthreads();
-  if (threadIdx.x != 0) return;
-  #pragma unroll
-  for (int w = 1; w < kThreads / 32; ++w) bits = max(bits, warp_max[w]);
-  bits = max(bits, warp_max[0]);
+// ---------------------------------------------------------------- ring finalize
 
+// Thread 0: the block's max goes to the ring; the tensor's last block folds
+// the launch amax into the ring and publishes the next scale.
+__device__ __forceinline__ void ring_finalize(const QuantizeParams& p, uint32_t bits, uint32_t nblocks, float s,
+                                              uint32_t step, const float* hist_s) {
   uint32_t* words = reinterpret_cast<uint32_t*>(p.ring);
   uint32_t* ticket = words + p.H + 1;
-  uint32_t* stepw = words + p.H + 2;
   uint32_t* scratch = words + p.H + 3;
-  if (bits) atomicMax(scratch, bits);
-  __threadfence();
-  const uint32_t t = atomicAdd(ticket, 1u);
-  if (t != gridDim.x - 1) return;
-
-  // Last block: every other block's atomicMax is visible (fence + ticket).
-  __threadfence();
+  if (bits) red_max_u32(scratch, bits);
+  // The release orders the red above before the ticket; the block that draws
+  // the last ticket acquires every earlier block's red.
+  if (atom_add_acq_rel(ticket, 1u) != nblocks - 1) return;
   const float a = __uint_as_float(atomicExch(scratch, 0u));
-  const uint32_t step = *reinterpret_cast<volatile uint32_t*>(stepw);
-  float* hist = p.ring;
-  hist[step % static_cast<uint32_t>(p.H)] = a;
-  float m = 0.0f;
-  for (int i = 0; i < p.H; ++i) m = fmaxf(m, hist[i]);
+  const uint32_t slot = step % static_cast<uint32_t>(p.H);
+  float m = a;
+  if (p.H <= kHistCache) {
+    for (int i = 0; i < p.H; ++i)
+      if (static_cast<uint32_t>(i) != slot) m = fmaxf(m, hist_s[i]);
+  } else {
+    for (int i = 0; i < p.H; ++i)
+      if (static_cast<uint32_t>(i) != slot) m = fmaxf(m, p.ring[i]);
+  }
   float snew = s;
   if (m > 0.0f && !isinf(m)) {
-    const float q = __fdiv_rn(p.fp8_max, m);
-    if (!isinf(q)) snew = q;
+    const float qv = __fdiv_rn(p.fp8_max, m);
+    if (!isinf(qv)) snew = qv;
   }
+  p.ring[slot] = a;
   p.ring[p.H] = snew;
-  *stepw = step + 1;
+  words[p.H + 2] = step + 1;
   atomicExch(ticket, 0u);
   if (p.amax_out) *p.amax_out = a;
 }
 
+__device__ __forceinline__ uint32_t block_max_bits(float amax, uint32_t* warp_max) {
+  uint32_t bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = bits;
+  __syncthreads();
+  #pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) bits = max(bits, warp_max[w]);
+  return bits;
+}
+
+// ---------------------------------------------------------------- flat kernel
+
+constexpr int unroll_for(int bytes) { return bytes == 2 ? 4 : 2; }
+
+template <typename T, int FMT>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const __grid_constant__ QuantizePair pair) {
+  __shared__ uint32_t warp_max[kThreads / 32];
+  __shared__ float hist_s[kHistCache];
+  constexpr int U = unroll_for(sizeof(T));
+  pdl_wait();
+  pdl_trigger();
+  const bool second = blockIdx.x >= pair.blocks0;
+  const QuantizeParams& p = second ? pair.t[1] : pair.t[0];
+  const uint32_t bid = second ? blockIdx.x - pair.blocks0 : blockIdx.x;
+  const uint32_t nblocks = second ? gridDim.x - pair.blocks0 : pair.blocks0;
+
+  const float s = p.ring[p.H];
+  uint32_t step = 0;
+  if (threadIdx.x == 0) {
+    step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
+    if (bid == 0 && p.scale_out) *p.scale_out = s;
+  }
+  // Only the tensor's last block writes its ring, after every block read it.
+  if (p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
+
+  float amax = 0.0f;
+  const int64_t stride = static_cast<int64_t>(nblocks) * kThreads;
+  int64_t c = static_cast<int64_t>(bid) * kThreads + threadIdx.x;
+  Raw<T> cur[U];
+  #pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t cu = c + u * stride;
+    if (cu < p.total_chunks) {
+      int64_t r, col;
+      chunk_pos(p, cu, r, col);
+      load_raw<T>(p, r, col, cur[u]);
+    }
+  }
+  #pragma unroll 1
+  while (c < p.total_chunks) {
+    const int64_t cn = c + U * stride;
+    Raw<T> nxt[U];
+    #pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t cu = cn + u * stride;
+      if (cu < p.total_chunks) {
+        int64_t r, col;
+        chunk_pos(p, cu, r, col);
+        load_raw<T>(p, r, col, nxt[u]);
+      }
+    }
+    #pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t cu = c + u * stride;
+      if (cu < p.total_chunks) {
+        int64_t r, col;
+        chunk_pos(p, cu, r, col);
+        float v[16];
+        to_floats<T>(cur[u], v);
+        cast_store<FMT>(p, r, col, v, s, amax);
+      }
+    }
+    #pragma unroll
+    for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+    c = cn;
+  }
+
+  const uint32_t bits = block_max_bits(amax, warp_max);
+  if (threadIdx.x == 0) ring_finalize(p, bits, nblocks, s, step, hist_s);
+}
+
+// ---------------------------------------------------------------- column-sum kernel
+
+constexpr int kColTile = kDbiasColsPerTile;        // 256 columns = 16 chunk lanes
+constexpr int kChunkLanes = kColTile / kChunk;     // 16
+constexpr int kRowLanes = kThreads / kChunkLanes;  // 16
+constexpr int kRowUnroll = 4;
+
+template <typename T, int FMT>
+__global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_constant__ ColsumParams cp) {
+  __shared__ uint32_t warp_max[kThreads / 32];
+  __shared__ float hist_s[kHistCache];
+  __shared__ __align__(16) float red[kRowLanes][kColTile];
+  __shared__ int last_tile;
+  pdl_wait();
+  pdl_trigger();
+  const QuantizeParams& p = cp.q;
+  const uint32_t nblocks = gridDim.x * gridDim.y;
+  const uint32_t bid = blockIdx.y * gridDim.x + blockIdx.x;
+  const float s = p.ring[p.H];
+  uint32_t step = 0;
+  if (threadIdx.x == 0) {
+    step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
+    if (bid == 0 && p.scale_out) *p.scale_out = s;
+  }
+  if (p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
+
+  const int cl = threadIdx.x % kChunkLanes;
+  const int rl = threadIdx.x / kChunkLanes;
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * kColTile + cl * kChunk;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * cp.rows_per_split;
+  const int64_t r1 = min(p.rows, r0 + cp.rows_per_split);
+  float amax = 0.0f;
+  float csum[16];
+  #pragma unroll
+  for (int j = 0; j < 16; ++j) csum[j] = 0.0f;
+  if (col < p.cols) {
+    #pragma unroll 1
+    for (int64_t r = r0 + rl; r < r1; r += kRowLanes * kRowUnroll) {
+      Raw<T> raw[kRowUnroll];
+      #pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u)
+        if (r + u * kRowLanes < r1) load_raw<T>(p, r + u * kRowLanes, col, raw[u]);
+      #pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u) {
+        if (r + u * kRowLanes < r1) {
+          float v[16];
+          to_floats<T>(raw[u], v);
+          #pragma unroll
+          for (int j = 0; j < 16; ++j) csum[j] += v[j];
+          cast_store<FMT>(p, r + u * kRowLanes, col, v, s, amax);
+        }
+      }
+    }
+  }
+  // column partials of this block: row lanes summed in lane order
+  #pragma unroll
+  for (int j = 0; j < 16; j += 4)
+    *reinterpret_cast<float4*>(&red[rl][cl * kChunk + j]) = make_float4(csum[j], csum[j + 1], csum[j + 2], csum[j + 3]);
+  const uint32_t bits = block_max_bits(amax, warp_max);  // includes __syncthreads
+  const int64_t ccol = static_cast<int64_t>(blockIdx.x) * kColTile + threadIdx.x;
+  float part = 0.0f;
+  #pragma unroll
+  for (int y = 0; y < kRowLanes; ++y) part += red[y][threadIdx.x];
+  if (ccol < p.cols) cp.partial[static_cast<int64_t>(blockIdx.y) * p.cols + ccol] = part;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ring_finalize(p, bits, nblocks, s, step, hist_s);
+    last_tile = atomicAdd(&cp.counters[blockIdx.x], 1u) == gridDim.y - 1;
+  }
+  __syncthreads();
+  if (!last_tile) return;
+  __threadfence();
+  if (ccol < p.cols) {
+    // four interleaved sums (split r -> sum r % 4), combined (s0+s1)+(s2+s3)
+    float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const float* pc = cp.partial + ccol;
+    const int R = static_cast<int>(gridDim.y);
+    int r = 0;
+    for (; r + 4 <= R; r += 4) {
+      float t[4];
+      #pragma unroll
+      for (int u = 0; u < 4; ++u) t[u] = __ldcg(pc + static_cast<int64_t>(r + u) * p.cols);
+      #pragma unroll
+      for (int u = 0; u < 4; ++u) s4[u] += t[u];
+    }
+    for (; r < R; ++r) s4[r & 3] += __ldcg(pc + static_cast<int64_t>(r) * p.cols);
+    static_cast<__nv_bfloat16*>(cp.dbias)[ccol] = __float2bfloat16_rn((s4[0] + s4[1]) + (s4[2] + s4[3]));
+  }
+  if (threadIdx.x == 0) atomicExch(&cp.counters[blockIdx.x], 0u);
+}
+
+// ---------------------------------------------------------------- small kernels
+
 __global__ void ring_set_kernel(float* ring, int H, float scale) {
+  pdl_wait();
+  pdl_trigger();
   for (int i = threadIdx.x; i < H; i += blockDim.x) ring[i] = 0.0f;
   if (threadIdx.x == 0) {
     uint32_t* w = reinterpret_cast<uint32_t*>(ring);
@@ -205,6 +363,8 @@ __global__ void ring_set_kernel(float* ring, int H, float scale) {
 }
 
 __global__ void side_writes_kernel(const SideWrites w) {
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x != 0) return;
   for (int i = 0; i < 2; ++i) {
     if (w.copy_dst[i]) *w.copy_dst[i] = *w.copy_src[i];
@@ -212,38 +372,69 @@ __global__ void side_writes_kernel(const SideWrites w) {
   }
 }
 
+// ---------------------------------------------------------------- launchers
+
+int64_t blocks_for(const QuantizeParams& p, int sms) {
+  // At most two blocks per SM: with U chunks per thread in flight plus the
+  // next iteration's loads that is plenty of bytes in flight, and few atomics
+  // on the ring's two words at the end.
+  const int64_t want = (p.total_chunks + kThreads - 1) / kThreads;
+  const int64_t cap = static_cast<int64_t>(sms) * 2;
+  return want < 1 ? 1 : (want > cap ? cap : want);
+}
+
 template <typename T, int FMT>
-cudaError_t launch_q(const QuantizeParams& p, cudaStream_t s) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const int64_t want = (p.total_chunks + 2 * kThreads - 1) / (2 * kThreads);
-  const int64_t cap = static_cast<int64_t>(num_sms(dev)) * 8;
-  const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  quantize_kernel<T, FMT><<<grid, kThreads, 0, s>>>(p);
-  return cudaGetLastError();
+cudaError_t launch_q(const QuantizePair& pair, int grid, cudaStream_t s) {
+  return launch_pdl(quantize_kernel<T, FMT>, dim3(grid), dim3(kThreads), 0, s, pair);
+}
+
+template <typename T, int FMT>
+cudaError_t launch_cs(const ColsumParams& cp, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>((cp.q.cols + kColTile - 1) / kColTile), static_cast<unsigned>(cp.R));
+  return launch_pdl(quantize_colsum_kernel<T, FMT>, grid, dim3(kThreads), 0, s, cp);
 }
 
 }  // namespace
 
-cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams& p, cudaStream_t s) {
+cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, const QuantizeParams* b,
+                            cudaStream_t s) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int sms = num_sms(dev);
+  QuantizePair pair;
+  pair.t[0] = *a;
+  pair.t[1] = b ? *b : *a;
+  const int64_t g0 = blocks_for(*a, sms);
+  const int64_t g1 = b ? blocks_for(*b, sms) : 0;
+  pair.blocks0 = static_cast<int>(g0);
+  const int grid = static_cast<int>(g0 + g1);
   if (fmt == kE4M3) {
-    if (in_dtype == kBF16) return launch_q<__nv_bfloat16, kE4M3>(p, s);
-    if (in_dtype == kFP16) return launch_q<__half, kE4M3>(p, s);
-    return launch_q<float, kE4M3>(p, s);
+    if (in_dtype == kBF16) return launch_q<__nv_bfloat16, kE4M3>(pair, grid, s);
+    if (in_dtype == kFP16) return launch_q<__half, kE4M3>(pair, grid, s);
+    return launch_q<float, kE4M3>(pair, grid, s);
   }
-  if (in_dtype == kBF16) return launch_q<__nv_bfloat16, kE5M2>(p, s);
-  if (in_dtype == kFP16) return launch_q<__half, kE5M2>(p, s);
-  return launch_q<float, kE5M2>(p, s);
+  if (in_dtype == kBF16) return launch_q<__nv_bfloat16, kE5M2>(pair, grid, s);
+  if (in_dtype == kFP16) return launch_q<__half, kE5M2>(pair, grid, s);
+  return launch_q<float, kE5M2>(pair, grid, s);
+}
+
+cudaError_t launch_quantize_colsum(int in_dtype, int fmt, const ColsumParams& cp, cudaStream_t s) {
+  if (fmt == kE4M3) {
+    if (in_dtype == kBF16) return launch_cs<__nv_bfloat16, kE4M3>(cp, s);
+    if (in_dtype == kFP16) return launch_cs<__half, kE4M3>(cp, s);
+    return launch_cs<float, kE4M3>(cp, s);
+  }
+  if (in_dtype == kBF16) return launch_cs<__nv_bfloat16, kE5M2>(cp, s);
+  if (in_dtype == kFP16) return launch_cs<__half, kE5M2>(cp, s);
+  return launch_cs<float, kE5M2>(cp, s);
 }
 
 cudaError_t launch_ring_set(float* ring, int H, float scale, cudaStream_t s) {
-  ring_set_kernel<<<1, 128, 0, s>>>(ring, H, scale);
-  return cudaGetLastError();
+  return launch_pdl(ring_set_kernel, dim3(1), dim3(128), 0, s, ring, H, scale);
 }
 
 cudaError_t launch_side_writes(const SideWrites& w, cudaStream_t s) {
-  side_writes_kernel<<<1, 32, 0, s>>>(w);
-  return cudaGetLastError();
+  return launch_pdl(side_writes_kernel, dim3(1), dim3(32), 0, s, w);
 }
 
 }  // namespace fp8lin

@@ -264,3 +264,82 @@ def test_config5_twenty_step_sequence(fp8):
         want = np.stack([oracle_ring_words(r) for r in orings])
         assert np.array_equal(got, want), f"ring words differ at step {step}"
     assert fp8.fp8_get_device_status() == 0
+
+
+@pytest.mark.parametrize("dtype", (torch.float16, torch.float32))
+@pytest.mark.parametrize("M,N,K", [(300, 100, 64), (1000, 1000, 128), (2048, 1536, 256)])
+def test_backward_fused_colsum_dtypes(fp8, dtype, M, N, K):
+    """g in fp16/fp32 (odd N, ragged row splits): the quantize-with-column-sum
+    launch gives bit-exact g8/ring and dbias within max(1 ulp, 2e-6 sum|g|)."""
+    rng = np.random.default_rng(M + N)
+    rx, rw, rg = fp8.ScaleRing(16), fp8.ScaleRing(16), fp8.ScaleRing(16)
+    org = oracle.Ring(16)
+    x = wl.normal((M, K), 1.0, 11, dtype=torch.bfloat16)
+    w = wl.normal((N, K), 0.05, 12, dtype=torch.bfloat16)
+    f = fp8.linear_forward(x.cuda(), w.cuda(), rx, rw)
+    for step in range(2):
+        g = wl.normal((M, N), 1e-3 * (1 + step), 13 + step, dtype=dtype)
+        b = fp8.linear_backward(g.cuda(), f, rg, need_dx=False, need_dw=False, need_dbias=True)
+        torch.cuda.synchronize()
+        gb = bits(g)
+        dt = oracle.DT_FP16 if dtype == torch.float16 else oracle.DT_FP32
+        g8o, ag, sg = oracle.quantize(gb, dt, E5, org, ld_out=(N + 15) // 16 * 16)
+        assert b.sg.item() == sg and b.amax_g.item() == ag
+        assert_codes_equal(host_rows(b.g8), g8o[:, :N], E5)
+        assert np.array_equal(ring_words(rg), oracle_ring_words(org))
+        want, _, sa = oracle.dbias(gb, dt, M, N)
+        gv = oracle.bf16_to_f32(b.dbias.cpu().view(torch.int16).numpy().view(np.uint16)).astype(np.float64)
+        ov = oracle.bf16_to_f32(want).astype(np.float64)
+        assert np.all(np.abs(gv - ov) <= np.maximum(oracle.bf16_ulp(ov), 2e-6 * sa))
+    assert fp8.fp8_get_device_status() == 0
+
+
+def test_backward_prequantized_g_dbias(fp8):
+    """A pre-quantized g (E5M2 codes with its scale) skips its quantize
+    (sg = g_scale_in, amax_g = 0, ring untouched) and dbias dequantizes each
+    element before the sum."""
+    rng = np.random.default_rng(21)
+    M, N, K = 512, 384, 256
+    rx, rw, rg = fp8.ScaleRing(16), fp8.ScaleRing(16), fp8.ScaleRing(16)
+    x = wl.normal((M, K), 1.0, 31)
+    w = wl.normal((N, K), 0.05, 32)
+    f = fp8.linear_forward(x.cuda(), w.cuda(), rx, rw)
+    g = wl.normal((M, N), 1e-3, 33)
+    sg = np.float32(57344.0) / oracle.amax(bits(g), oracle.DT_BF16)
+    g8 = oracle.quantize_codes(bits(g), oracle.DT_BF16, E5, sg)
+    before = ring_words(rg)
+    gdev = torch.from_numpy(g8).cuda()
+    sgd = torch.tensor([float(sg)], device="cuda")
+    b = fp8.linear_backward(gdev, f, rg, need_dbias=True, g_scale_in=sgd)
+    torch.cuda.synchronize()
+    assert b.sg.item() == sg and b.amax_g.item() == 0.0
+    assert np.array_equal(ring_words(rg), before)
+    want, _, sa = oracle.dbias(g8, oracle.DT_E5M2, M, N, sg)
+    gv = oracle.bf16_to_f32(b.dbias.cpu().view(torch.int16).numpy().view(np.uint16)).astype(np.float64)
+    ov = oracle.bf16_to_f32(want).astype(np.float64)
+    assert np.all(np.abs(gv - ov) <= np.maximum(oracle.bf16_ulp(ov), 2e-6 * sa))
+    torch.cuda.synchronize()
+    x8 = host_rows(f.x8)
+    w8 = host_rows(f.w8)
+    gemm_check(b.dx, g8, 0, E5, w8, E4, M, K, N, sg, f.sw.item(), "dx", True, rng, what="pre-g dx")
+    gemm_check(b.dw, g8, 0, E5, x8, E4, N, K, M, sg, f.sx.item(), "dw", True, rng, what="pre-g dw")
+
+
+def test_forward_mixed_input_dtypes(fp8):
+    """x fp32 and w bf16 (no shared launch): two quantize launches, same results
+    as the oracle."""
+    rng = np.random.default_rng(22)
+    M, N, K = 256, 320, 192
+    rx, rw = fp8.ScaleRing(16), fp8.ScaleRing(16)
+    orx, orw = oracle.Ring(16), oracle.Ring(16)
+    for step in range(2):
+        x = wl.normal((M, K), 1.0 + step, 41 + step, dtype=torch.float32)
+        w = wl.normal((N, K), 0.05, 43)
+        f = fp8.linear_forward(x.cuda(), w.cuda(), rx, rw)
+        torch.cuda.synchronize()
+        x8o, ax, sx = oracle.quantize(bits(x), oracle.DT_FP32, E4, orx)
+        w8o, aw, sw = oracle.quantize(bits(w), oracle.DT_BF16, E4, orw)
+        assert (f.sx.item(), f.sw.item(), f.amax_x.item(), f.amax_w.item()) == (sx, sw, ax, aw)
+        assert_codes_equal(host_rows(f.x8), x8o, E4)
+        assert np.array_equal(ring_words(rx), oracle_ring_words(orx))
+        gemm_check(f.y, x8o, 0, E4, w8o, E4, M, N, K, sx, sw, "fwd", True, rng, what="mixed y")

@@ -95,3 +95,22 @@ HIST_LEN = 16
 def weight_std(K: int) -> float:
     """w ~ N(0, 1/sqrt(K)): the std is 1/sqrt(K)."""
     return 1.0 / math.sqrt(K)
+
+
+def normal_device(shape, std: float, seed: int, device, dtype=torch.bfloat16) -> torch.Tensor:
+    """N(0, std^2) drawn in fp32 by a seeded generator on `device`, cast to dtype
+    (for large benchmark inputs; the tests use the CPU generator above)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    return (torch.randn(*shape, generator=g, dtype=torch.float32, device=device) * std).to(dtype)
+
+
+# Benchmark workload: the linears of the pages' 12L/dim1024/B4xT512 model
+# (configuration 2), forward and backward, with a bf16 bias and its gradient.
+BENCH_LAYERS = 12
+BENCH_LAYER = C2_LAYER
+BENCH_BIAS_STD = 0.01
+
+
+def bench_flops_per_step(layers: int = BENCH_LAYERS) -> int:
+    """fwd + dX + dW: 3 GEMMs of 2*M*N*K flops per linear."""
+    return layers * sum(6 * s.M * s.N * s.K for s in BENCH_LAYER)

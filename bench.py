@@ -199,45 +199,52 @@ def run_step(F, lins, stream_handle):
             raise F.Fp8Error(s, "fp8_linear_backward")
 
 
-LAUNCHES_PER_LINEAR = 7  # quantize x, quantize w, fwd GEMM, quantize g, dX GEMM, dW GEMM, dbias
+LAUNCHES_PER_LINEAR = 4  # quantize x+w, fwd GEMM, quantize g + dbias, dX+dW GEMMs
 
 
 # --------------------------------------------------------------------------- kernel-level timing
 
 def step_primitives(F, lins, h):
-    """The step's kernels as (class, algorithmic work, label, call) in launch
-    order: the same primitives the linear entry points launch."""
+    """The step's kernel launches as (class, algorithmic work, label, call) in
+    launch order, through the same fused entry points fp8_linear_forward /
+    fp8_linear_backward use: quantize x+w, forward GEMM (+bias); then in
+    reverse, quantize g (+dbias), dX+dW GEMMs."""
     lib = F._lib
     out = []
+    keep = []  # ctypes argument structs must outlive the calls and the graphs
+
+    def call(fn, *structs):
+        keep.append(structs)
+        return lambda: fn(*[ctypes.byref(s_) for s_ in structs], h)
     for L in lins:
         M, K, N = L.shape.M, L.shape.K, L.shape.N
-        ldk, ldn = L.x8.shape[1], L.g8.shape[1]
+        ldk = L.x8.shape[1]
         sc = L.sc.data_ptr()
-        mm = lambda *a: (lambda args=F.MmArgs(*a): lib.fp8_mm(ctypes.byref(args), h))  # noqa: E731
-        out += [
-            ("quantize", M * K * 3, None, lambda L=L, M=M, K=K, ldk=ldk, sc=sc: lib.fp8_quantize(
-                L.x.data_ptr(), 0, M, K, K, 0, L.rings[0].data_ptr(), wl.HIST_LEN, L.x8.data_ptr(), ldk, sc + 12, sc, h)),
-            ("quantize", N * K * 3, None, lambda L=L, N=N, K=K, ldk=ldk, sc=sc: lib.fp8_quantize(
-                L.w.data_ptr(), 0, N, K, K, 0, L.rings[1].data_ptr(), wl.HIST_LEN, L.w8.data_ptr(), ldk, sc + 16, sc + 4, h)),
-            ("gemm", 2 * M * N * K, f"fwd {M}x{N}x{K}", mm(M, N, K, L.x8.data_ptr(), 0, 0, ldk, L.w8.data_ptr(), 0, 0, ldk,
-                                                         sc, sc + 4, L.b.data_ptr(), 0, None, L.y.data_ptr(), N)),
-        ]
+        qx = F.QuantizeArgs(L.x.data_ptr(), 0, M, K, K, 0, L.rings[0].data_ptr(), wl.HIST_LEN, L.x8.data_ptr(), ldk,
+                            sc + 12, sc)
+        qw = F.QuantizeArgs(L.w.data_ptr(), 0, N, K, K, 0, L.rings[1].data_ptr(), wl.HIST_LEN, L.w8.data_ptr(), ldk,
+                            sc + 16, sc + 4)
+        fwd = F.MmArgs(M, N, K, L.x8.data_ptr(), 0, 0, ldk, L.w8.data_ptr(), 0, 0, ldk, sc, sc + 4,
+                       L.b.data_ptr(), 0, None, L.y.data_ptr(), N, 0)
+        out.append(("quantize", (M * K + N * K) * 3, None, call(lib.fp8_quantize_dual, qx, qw)))
+        out.append(("gemm", 2 * M * N * K, f"fwd {M}x{N}x{K}", call(lib.fp8_mm, fwd)))
     for L in reversed(lins):
         M, K, N = L.shape.M, L.shape.K, L.shape.N
         ldk, ldn = L.x8.shape[1], L.g8.shape[1]
         sc = L.sc.data_ptr()
-        mm = lambda *a: (lambda args=F.MmArgs(*a): lib.fp8_mm(ctypes.byref(args), h))  # noqa: E731
-        out += [
-            ("quantize", M * N * 3, None, lambda L=L, M=M, N=N, ldn=ldn, sc=sc: lib.fp8_quantize(
-                L.g.data_ptr(), 0, M, N, N, 1, L.rings[2].data_ptr(), wl.HIST_LEN, L.g8.data_ptr(), ldn, sc + 20, sc + 8, h)),
-            ("gemm", 2 * M * N * K, f"dX {M}x{K}x{N}", mm(M, K, N, L.g8.data_ptr(), 1, 0, ldn, L.w8.data_ptr(), 0, 1, ldk,
-                                                        sc + 8, sc + 4, None, 0, None, L.dx.data_ptr(), K)),
-            ("gemm", 2 * M * N * K, f"dW {N}x{K}x{M}", mm(N, K, M, L.g8.data_ptr(), 1, 1, ldn, L.x8.data_ptr(), 0, 1, ldk,
-                                                        sc + 8, sc, None, 0, None, L.dw.data_ptr(), K)),
-            ("dbias", M * N * 2 + N * 2, None, lambda L=L, M=M, N=N: lib.fp8_dbias(
-                L.g.data_ptr(), 0, M, N, N, None, L.db.data_ptr(), L.ws.data_ptr(), L.ws.numel(), h)),
-        ]
-    return out
+        qg = F.QuantizeArgs(L.g.data_ptr(), 0, M, N, N, 1, L.rings[2].data_ptr(), wl.HIST_LEN, L.g8.data_ptr(), ldn,
+                            sc + 20, sc + 8)
+        dx = F.MmArgs(M, K, N, L.g8.data_ptr(), 1, 0, ldn, L.w8.data_ptr(), 0, 1, ldk, sc + 8, sc + 4,
+                      None, 0, None, L.dx.data_ptr(), K, 0)
+        dw = F.MmArgs(N, K, M, L.g8.data_ptr(), 1, 1, ldn, L.x8.data_ptr(), 0, 1, ldk, sc + 8, sc,
+                      None, 0, None, L.dw.data_ptr(), K, 0)
+        ws = L.ws
+        out.append(("quantize", M * N * 3, None,
+                    (lambda qg=qg, L=L, ws=ws: lib.fp8_quantize_dbias(ctypes.byref(qg), L.db.data_ptr(), ws.data_ptr(),
+                                                                      ws.numel(), h))))
+        keep.append((qg,))
+        out.append(("gemm", 4 * M * N * K, f"dX+dW {M}x{N}x{K}", call(lib.fp8_mm_pair, dx, dw)))
+    return out, keep
 
 
 def time_kernels(F, lins, stream, reps=5):
@@ -247,9 +254,9 @@ def time_kernels(F, lins, stream, reps=5):
     Returns (ms per step by class, work by class, launches by class, per-shape
     GEMM times)."""
     h = stream.cuda_stream
-    prims = step_primitives(F, lins, h)
+    prims, keep = step_primitives(F, lins, h)
     res_ms, work, count = {}, {}, {}
-    for cls in ("gemm", "quantize", "dbias"):
+    for cls in ("gemm", "quantize"):
         calls = [c for c in prims if c[0] == cls]
         work[cls] = sum(c[1] for c in calls)
         count[cls] = len(calls)
@@ -293,7 +300,7 @@ def time_kernels(F, lins, stream, reps=5):
         us = e0.elapsed_time(e1) * 1e3 / 12
         shapes[name] = {"us": us, "tflops": c[1] / us / 1e6, "note": "same operands back to back (warm L2)"}
         del g
-    del layer
+    del layer, keep
     return res_ms, work, count, shapes
 
 
@@ -474,19 +481,20 @@ def main(argv=None):
         traffic = gemm_traffic_per_launch()
         line["roofline"] = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                             "frac": gemm_tflops / fp8_peak, "traffic": traffic,
-                            "kernel": "fp8_gemm_kernel (the step's 216 fwd/dX/dW launches, replayed as one graph)",
+                            "kernel": "fp8_gemm_kernel (the step's 144 launches: 72 forward, 72 dX+dW pairs, "
+                                      "replayed as one graph)",
                             "peak_source": f"{pk_kind} bf16 burst x {FP8_PER_BF16} (nominal fp8:bf16)",
                             "frac_of_nominal_4.5PF": gemm_tflops / NOMINAL_FP8_TFLOPS}
         q_gbs = work["quantize"] / (tot["quantize"] / 1e3) / 1e9
-        d_gbs = work["dbias"] / (tot["dbias"] / 1e3) / 1e9
         step_kernels_ms = sum(tot.values())
         line["kernels"] = {
             "share": {k: v / step_kernels_ms for k, v in tot.items()},
             "ms_per_step": tot, "launches_per_step": count,
             "step_ms_vs_sum_of_classes": (max_ms / args.steps) / step_kernels_ms,
             "quantize": {"achieved_gbs": q_gbs, "peak_gbs": pk["hbm_gbs"], "frac": q_gbs / pk["hbm_gbs"],
-                         "bytes_per_elem": 3, "note": "bf16 in + fp8 out; class graph replay"},
-            "dbias": {"achieved_gbs": d_gbs, "frac": d_gbs / pk["hbm_gbs"], "bytes_per_elem": 2},
+                         "bytes_per_elem": 3,
+                         "note": "bf16 in + fp8 out; x+w in one launch, g with its bias gradient in one launch; "
+                                 "class graph replay"},
             "gemm_by_shape": shapes}
 
         # ---- end to end through the C ABI with host buffers

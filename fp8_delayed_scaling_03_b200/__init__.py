@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "libfp8lin.so")
 FP8_E4M3, FP8_E5M2 = 0, 1
 FP8_DT_BF16, FP8_DT_FP16, FP8_DT_FP32, FP8_DT_E4M3, FP8_DT_E5M2 = 0, 1, 2, 3, 4
 FP8_K_MAJOR, FP8_MN_MAJOR = 0, 1
+FP8_TILE_AUTO, FP8_TILE_128x128, FP8_TILE_128x256, FP8_TILE_PAIR_256x256 = 0, 1, 2, 3
 FP8_OK = 0
 FP8_ERR_INVALID_ARG, FP8_ERR_UNSUPPORTED, FP8_ERR_MISALIGNED = -1, -2, -3
 FP8_ERR_CUDA, FP8_ERR_DEVICE_TIMEOUT, FP8_ERR_WORKSPACE = -4, -5, -6
@@ -50,7 +51,15 @@ class MmArgs(ctypes.Structure):
                 ("b", _P), ("fmt_b", _I), ("b_major", _I), ("ldb", _I64),
                 ("scale_a", _P), ("scale_b", _P),
                 ("bias", _P), ("bias_dtype", _I), ("bias_scale", _P),
-                ("d", _P), ("ldd", _I64)]
+                ("d", _P), ("ldd", _I64),
+                ("tile_cfg", _I)]
+
+
+class QuantizeArgs(ctypes.Structure):
+    _fields_ = [("in_", _P), ("in_dtype", _I), ("rows", _I64), ("cols", _I64), ("ld_in", _I64),
+                ("fmt", _I), ("ring", _P), ("hist_len", _I),
+                ("out", _P), ("ld_out", _I64),
+                ("amax_out", _P), ("scale_out", _P)]
 
 
 class LinearFwdArgs(ctypes.Structure):
@@ -86,7 +95,10 @@ _SIGS = {
     "fp8_ring_init": (_I, [_P, _I, _P]),
     "fp8_ring_seed": (_I, [_P, _I, _I, _F, _P]),
     "fp8_quantize": (_I, [_P, _I, _I64, _I64, _I64, _I, _P, _I, _P, _I64, _P, _P, _P]),
+    "fp8_quantize_dual": (_I, [ctypes.POINTER(QuantizeArgs), ctypes.POINTER(QuantizeArgs), _P]),
+    "fp8_quantize_dbias": (_I, [ctypes.POINTER(QuantizeArgs), _P, _P, _SZ, _P]),
     "fp8_mm": (_I, [ctypes.POINTER(MmArgs), _P]),
+    "fp8_mm_pair": (_I, [ctypes.POINTER(MmArgs), ctypes.POINTER(MmArgs), _P]),
     "fp8_dbias_workspace_bytes": (_SZ, [_I64, _I64]),
     "fp8_dbias": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "fp8_linear_forward": (_I, [ctypes.POINTER(LinearFwdArgs), _P]),
@@ -176,10 +188,31 @@ def fp8_quantize(x: torch.Tensor, fmt: int, ring: torch.Tensor, hist_len: int, o
            "fp8_quantize")
 
 
+def quantize_args(x: torch.Tensor, fmt: int, ring: torch.Tensor, hist_len: int, out: torch.Tensor,
+                  amax_out: torch.Tensor | None = None, scale_out: torch.Tensor | None = None) -> QuantizeArgs:
+    rows, cols = x.shape
+    return QuantizeArgs(_ptr(x), _dtype_code(x), rows, cols, _ld(x), fmt, _ptr(ring), hist_len, _ptr(out), _ld(out),
+                        _ptr(amax_out), _ptr(scale_out))
+
+
+def fp8_quantize_dual(a: QuantizeArgs, b: QuantizeArgs, device=None) -> None:
+    _check(_lib.fp8_quantize_dual(ctypes.byref(a), ctypes.byref(b), _stream(device)), "fp8_quantize_dual")
+
+
+def fp8_quantize_dbias(g: QuantizeArgs, dbias: torch.Tensor, workspace: torch.Tensor) -> None:
+    _check(_lib.fp8_quantize_dbias(ctypes.byref(g), _ptr(dbias), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(dbias.device)),
+           "fp8_quantize_dbias")
+
+
+def fp8_mm_pair(a: MmArgs, b: MmArgs, device=None) -> None:
+    _check(_lib.fp8_mm_pair(ctypes.byref(a), ctypes.byref(b), _stream(device)), "fp8_mm_pair")
+
+
 def fp8_mm(m, n, k, a, fmt_a, a_major, lda, b, fmt_b, b_major, ldb, scale_a, scale_b, d, ldd,
-           bias=None, bias_dtype=FP8_DT_BF16, bias_scale=None, stream=None) -> None:
+           bias=None, bias_dtype=FP8_DT_BF16, bias_scale=None, stream=None, tile_cfg=FP8_TILE_AUTO) -> None:
     args = MmArgs(m, n, k, _ptr(a), fmt_a, a_major, lda, _ptr(b), fmt_b, b_major, ldb,
-                  _ptr(scale_a), _ptr(scale_b), _ptr(bias), bias_dtype, _ptr(bias_scale), _ptr(d), ldd)
+                  _ptr(scale_a), _ptr(scale_b), _ptr(bias), bias_dtype, _ptr(bias_scale), _ptr(d), ldd, tile_cfg)
     s = stream if stream is not None else _stream(d.device if isinstance(d, torch.Tensor) else None)
     _check(_lib.fp8_mm(ctypes.byref(args), s), "fp8_mm")
 

@@ -112,6 +112,7 @@ struct MmCall {
   const float* scale_a; const float* scale_b;
   const void* bias; int bias_dtype; const float* bias_scale;
   void* d; int64_t ldd;
+  int tile_cfg;
 };
 
 int validate_mm(const MmCall& c) {
@@ -126,6 +127,7 @@ int validate_mm(const MmCall& c) {
   s = check_fp8_matrix(c.b, c.ldb, c.b_major == FP8_K_MAJOR ? c.k : c.n);
   if (s) return s;
   if (c.ldd < c.n || !aligned(c.d, 2)) return FP8_ERR_INVALID_ARG;
+  if (c.tile_cfg < FP8_TILE_AUTO || c.tile_cfg > FP8_TILE_PAIR_256x256) return FP8_ERR_INVALID_ARG;
   if (c.bias) {
     if (c.bias_dtype != FP8_DT_BF16 && !is_fp8(c.bias_dtype)) return FP8_ERR_INVALID_ARG;
     if (is_fp8(c.bias_dtype) && !c.bias_scale) return FP8_ERR_INVALID_ARG;
@@ -134,39 +136,46 @@ int validate_mm(const MmCall& c) {
   return FP8_OK;
 }
 
-// Output tile width: the candidate with the smallest (waves x tile width),
-// preferring the wider tile on ties (fewer operand re-reads per flop).
-int pick_bn(int64_t m, int64_t n, int sms) {
-  const int64_t tm = (m + 127) / 128;
-  int best = 256;
-  int64_t best_cost = -1;
-  for (int bn : {256, 128}) {
-    const int64_t tiles = tm * ((n + bn - 1) / bn);
-    const int64_t waves = (tiles + sms - 1) / sms;
-    const int64_t cost = waves * bn;
-    if (best_cost < 0 || cost < best_cost) { best = bn; best_cost = cost; }
+// Tile configuration with the smallest modelled time for a launch of one or
+// two problems: waves of tiles over the SMs (pairs of SMs for 2-SM tiles)
+// times the tile's mainloop at the k-block time measured on a B200 for that
+// tile shape, plus a fixed fill/drain cost.  Measured: 0.34 us per 128x128x128
+// k-block on one SM, 0.45 us per 128x256x128 on one SM and per 256x256x128 on
+// an SM pair; ~4-5 us fill + epilogue + launch.
+int pick_tile(const MmCall* calls, int n, int sms) {
+  struct Opt { int cfg; int64_t tm, tn, units; double t_kb, fixed; };
+  const Opt opts[3] = {{kGemm128, 128, 128, sms, 0.34, 4.0}, {kGemm256, 128, 256, sms, 0.45, 4.0},
+                       {kGemmPair256, 256, 256, sms / 2, 0.45, 5.0}};
+  int best = kGemm128;
+  double best_t = -1.0;
+  for (const Opt& o : opts) {
+    int64_t tiles = 0;
+    double work = 0.0;
+    for (int i = 0; i < n; ++i) {
+      const int64_t ti = ((calls[i].m + o.tm - 1) / o.tm) * ((calls[i].n + o.tn - 1) / o.tn);
+      tiles += ti;
+      work += static_cast<double>(ti) * static_cast<double>((calls[i].k + 127) / 128);
+    }
+    const double avg_kb = tiles ? work / static_cast<double>(tiles) : 0.0;
+    const int64_t waves = (tiles + o.units - 1) / o.units;
+    const double t = static_cast<double>(waves) * avg_kb * o.t_kb + o.fixed;
+    if (best_t < 0 || t < best_t) { best = o.cfg; best_t = t; }
   }
   return best;
 }
 
-// Enqueue one GEMM (validated already).  side: writes folded into the launch.
-int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  const int sms = num_sms(dev);
-  if (sms <= 0) return cuda_fail(cudaGetLastError());
-  const int bn = pick_bn(c.m, c.n, sms);
-  CUtensorMap ta, tb, td;
-  std::memset(&ta, 0, sizeof(ta));
-  std::memset(&tb, 0, sizeof(tb));
-  std::memset(&td, 0, sizeof(td));
+// Problem description and tensor maps of one GEMM for tile configuration cfg.
+int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) {
+  const int bn = cfg == kGemm128 ? 128 : 256;
+  const int tile_m = cfg == kGemmPair256 ? 256 : 128;
+  const int b_box_rows = cfg == kGemm256 ? 256 : 128;   // rows of B one CTA loads
+  std::memset(maps, 0, 3 * sizeof(CUtensorMap));
   if (c.k > 0) {
-    int s = c.a_major == FP8_K_MAJOR ? make_fp8_map(&ta, c.a, c.k, c.m, c.lda, 128)
-                                     : make_fp8_map(&ta, c.a, c.m, c.k, c.lda, 128);
+    int s = c.a_major == FP8_K_MAJOR ? make_fp8_map(&maps[0], c.a, c.k, c.m, c.lda, 128)
+                                     : make_fp8_map(&maps[0], c.a, c.m, c.k, c.lda, 128);
     if (s) return s;
-    s = c.b_major == FP8_K_MAJOR ? make_fp8_map(&tb, c.b, c.k, c.n, c.ldb, bn)
-                                 : make_fp8_map(&tb, c.b, c.n, c.k, c.ldb, 128);
+    s = c.b_major == FP8_K_MAJOR ? make_fp8_map(&maps[1], c.b, c.k, c.n, c.ldb, b_box_rows)
+                                 : make_fp8_map(&maps[1], c.b, c.n, c.k, c.ldb, 128);
     if (s) return s;
   }
   // bf16 output through TMA stores when the rows are 16-byte addressable and
@@ -175,37 +184,62 @@ int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st) {
   // 32 x 32 boxes, 64-byte swizzle (matches the epilogue's staging layout).
   const bool tma_store = aligned(c.d, 16) && ((c.ldd * 2) % 16 == 0) && (c.n % 8 == 0);
   if (tma_store) {
-    int s = make_map(&td, c.d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.n, c.m, c.ldd * 2, 32, 32,
+    int s = make_map(&maps[2], c.d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.n, c.m, c.ldd * 2, 32, 32,
                      CU_TENSOR_MAP_SWIZZLE_64B);
     if (s) return s;
   }
+  std::memset(pr, 0, sizeof(*pr));
+  pr->m = static_cast<int>(c.m);
+  pr->n = static_cast<int>(c.n);
+  pr->k = static_cast<int>(c.k);
+  pr->tiles_m = static_cast<int>((c.m + tile_m - 1) / tile_m);
+  pr->tiles_n = static_cast<int>((c.n + bn - 1) / bn);
+  pr->num_tiles = pr->tiles_m * pr->tiles_n;
+  pr->k_blocks = static_cast<int>((c.k + 127) / 128);
+  pr->raster_group = 8;
+  pr->idesc = idesc_f8(c.fmt_a, c.fmt_b, c.a_major, c.b_major, tile_m, bn);
+  pr->a_major = c.a_major;
+  pr->b_major = c.b_major;
+  pr->scale_a = c.scale_a;
+  pr->scale_b = c.scale_b;
+  pr->bias = c.bias;
+  pr->bias_kind = !c.bias ? 0 : (c.bias_dtype == FP8_DT_BF16 ? 1 : (c.bias_dtype == FP8_DT_E4M3 ? 2 : 3));
+  pr->bias_scale = c.bias_scale;
+  pr->d = c.d;
+  pr->ldd = c.ldd;
+  pr->tma_store = tma_store ? 1 : 0;
+  return FP8_OK;
+}
+
+// Enqueue one launch running n (1 or 2) validated GEMMs over one persistent
+// tile schedule.  side: writes folded into the launch.
+int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int sms = num_sms(dev);
+  if (sms <= 0) return cuda_fail(cudaGetLastError());
+  const int cfg = calls[0].tile_cfg != FP8_TILE_AUTO ? calls[0].tile_cfg : pick_tile(calls, n, sms);
+  CUtensorMap maps[6];
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
-  p.m = static_cast<int>(c.m);
-  p.n = static_cast<int>(c.n);
-  p.k = static_cast<int>(c.k);
-  p.tiles_m = static_cast<int>((c.m + 127) / 128);
-  p.tiles_n = static_cast<int>((c.n + bn - 1) / bn);
-  p.num_tiles = p.tiles_m * p.tiles_n;
-  p.k_blocks = static_cast<int>((c.k + 127) / 128);
-  p.raster_group = 8;
-  p.idesc = idesc_f8(c.fmt_a, c.fmt_b, c.a_major, c.b_major, 128, bn);
-  p.a_major = c.a_major;
-  p.b_major = c.b_major;
-  p.scale_a = c.scale_a;
-  p.scale_b = c.scale_b;
-  p.bias = c.bias;
-  p.bias_kind = !c.bias ? 0 : (c.bias_dtype == FP8_DT_BF16 ? 1 : (c.bias_dtype == FP8_DT_E4M3 ? 2 : 3));
-  p.bias_scale = c.bias_scale;
-  p.d = c.d;
-  p.ldd = c.ldd;
-  p.tma_store = tma_store ? 1 : 0;
+  std::memset(maps, 0, sizeof(maps));
+  for (int i = 0; i < n; ++i) {
+    int s = build_problem(calls[i], cfg, &p.pr[i], &maps[3 * i]);
+    if (s) return s;
+    p.any_tma_store |= p.pr[i].tma_store;
+  }
+  p.nprob = n;
+  p.tiles0 = p.pr[0].num_tiles;
+  p.total_tiles = p.pr[0].num_tiles + (n > 1 ? p.pr[1].num_tiles : 0);
   p.status = status_ptr(dev);
   if (side) p.side = *side;
-  e = launch_gemm(ta, tb, td, p, bn, st);
+  e = launch_gemm(maps, p, cfg, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return FP8_OK;
 }
+
+int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st) { return run_mm_group(&c, 1, side, st); }
 
 QuantizeParams make_qparams(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt,
                             void* ring, int H, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out,
@@ -242,6 +276,20 @@ int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
   const QuantizeParams p =
       make_qparams(in, in_dtype, rows, cols, ld_in, fmt, ring, H, out, ld_out, amax_out, scale_out, true);
   cudaError_t e = launch_quantize(in_dtype, fmt, &p, nullptr, st);
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
+int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace, cudaStream_t st) {
+  ColsumParams cp;
+  std::memset(&cp, 0, sizeof(cp));
+  cp.q = make_qparams(g.in, g.in_dtype, g.rows, g.cols, g.ld_in, g.fmt, g.ring, g.hist_len, g.out, g.ld_out,
+                      g.amax_out, g.scale_out, false);
+  dbias_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
+  cp.partial = static_cast<float*>(workspace);
+  const size_t part = (static_cast<size_t>(cp.R) * static_cast<size_t>(g.cols) * 4u + 15u) & ~size_t(15);
+  cp.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + part);
+  cp.dbias = dbias;
+  cudaError_t e = launch_quantize_colsum(g.in_dtype, g.fmt, cp, st);
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
 
@@ -305,10 +353,66 @@ int fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
+int fp8_quantize_dual(const fp8_quantize_args* a, const fp8_quantize_args* b, fp8_stream_t stream) {
+  if (!a || !b) return FP8_ERR_INVALID_ARG;
+  int s = validate_quantize(a->in, a->in_dtype, a->rows, a->cols, a->ld_in, a->fmt, a->ring, a->hist_len, a->out,
+                            a->ld_out);
+  if (s) return s;
+  s = validate_quantize(b->in, b->in_dtype, b->rows, b->cols, b->ld_in, b->fmt, b->ring, b->hist_len, b->out,
+                        b->ld_out);
+  if (s) return s;
+  if (a->in_dtype != b->in_dtype || a->fmt != b->fmt || a->ring == b->ring) return FP8_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool ea = a->rows == 0 || a->cols == 0, eb = b->rows == 0 || b->cols == 0;
+  if (ea && eb) return FP8_OK;
+  if (ea || eb) {
+    const fp8_quantize_args* o = ea ? b : a;
+    return run_quantize(o->in, o->in_dtype, o->rows, o->cols, o->ld_in, o->fmt, o->ring, o->hist_len, o->out,
+                        o->ld_out, o->amax_out, o->scale_out, st);
+  }
+  const QuantizeParams qa = make_qparams(a->in, a->in_dtype, a->rows, a->cols, a->ld_in, a->fmt, a->ring, a->hist_len,
+                                         a->out, a->ld_out, a->amax_out, a->scale_out, true);
+  const QuantizeParams qb = make_qparams(b->in, b->in_dtype, b->rows, b->cols, b->ld_in, b->fmt, b->ring, b->hist_len,
+                                         b->out, b->ld_out, b->amax_out, b->scale_out, true);
+  cudaError_t e = launch_quantize(a->in_dtype, a->fmt, &qa, &qb, st);
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
+int fp8_quantize_dbias(const fp8_quantize_args* g, void* dbias, void* workspace, size_t workspace_bytes,
+                       fp8_stream_t stream) {
+  if (!g) return FP8_ERR_INVALID_ARG;
+  int s = validate_quantize(g->in, g->in_dtype, g->rows, g->cols, g->ld_in, g->fmt, g->ring, g->hist_len, g->out,
+                            g->ld_out);
+  if (s) return s;
+  if (g->rows > kMaxDim || g->cols > kMaxDim) return FP8_ERR_INVALID_ARG;
+  if (!dbias || !aligned(dbias, 2)) return FP8_ERR_INVALID_ARG;
+  if (g->rows == 0 || g->cols == 0) return FP8_OK;
+  const size_t need = fp8_dbias_workspace_bytes(g->rows, g->cols);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return FP8_ERR_WORKSPACE;
+  return run_quantize_dbias(*g, dbias, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fp8_mm_pair(const fp8_mm_args* a, const fp8_mm_args* b, fp8_stream_t stream) {
+  if (!a || !b) return FP8_ERR_INVALID_ARG;
+  const MmCall c[2] = {
+      {a->m, a->n, a->k, a->a, a->fmt_a, a->a_major, a->lda, a->b, a->fmt_b, a->b_major, a->ldb, a->scale_a,
+       a->scale_b, a->bias, a->bias_dtype, a->bias_scale, a->d, a->ldd, a->tile_cfg},
+      {b->m, b->n, b->k, b->a, b->fmt_a, b->a_major, b->lda, b->b, b->fmt_b, b->b_major, b->ldb, b->scale_a,
+       b->scale_b, b->bias, b->bias_dtype, b->bias_scale, b->d, b->ldd, a->tile_cfg}};
+  int s = validate_mm(c[0]);
+  if (s) return s;
+  if ((s = validate_mm(c[1]))) return s;
+  const bool ea = c[0].m == 0 || c[0].n == 0 || c[0].k == 0, eb = c[1].m == 0 || c[1].n == 0 || c[1].k == 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (ea && eb) return FP8_OK;
+  if (ea || eb) return run_mm(ea ? c[1] : c[0], nullptr, st);
+  return run_mm_group(c, 2, nullptr, st);
+}
+
 int fp8_mm(const fp8_mm_args* a, fp8_stream_t stream) {
   if (!a) return FP8_ERR_INVALID_ARG;
   MmCall c{a->m, a->n, a->k, a->a, a->fmt_a, a->a_major, a->lda, a->b, a->fmt_b, a->b_major, a->ldb,
-           a->scale_a, a->scale_b, a->bias, a->bias_dtype, a->bias_scale, a->d, a->ldd};
+           a->scale_a, a->scale_b, a->bias, a->bias_dtype, a->bias_scale, a->d, a->ldd, a->tile_cfg};
   int s = validate_mm(c);
   if (s) return s;
   if (c.m == 0 || c.n == 0 || c.k == 0) return FP8_OK;
@@ -387,7 +491,7 @@ int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
   const uint8_t* w8 = wq ? static_cast<const uint8_t*>(a->w) : a->w8;
   MmCall c{M, N, K, x8, a->fmt_x, FP8_K_MAJOR, xq ? a->ldx : a->ldx8, w8, a->fmt_w, FP8_K_MAJOR,
            wq ? a->ldw : a->ldw8, xq ? a->x_scale_in : a->sx_out, wq ? a->w_scale_in : a->sw_out,
-           a->bias, a->bias_dtype, a->bias_scale, a->y, a->ldy};
+           a->bias, a->bias_dtype, a->bias_scale, a->y, a->ldy, FP8_TILE_AUTO};
   if ((s = validate_mm(c))) return s;
   if (M == 0 || N == 0 || K == 0) return FP8_OK;
 
@@ -436,10 +540,10 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   const float* sg = gq ? a->g_scale_in : a->sg_out;
   // dX[M,K] = G8[M,N] . W8[N,K]: A = G8 K-major, B(j=k, n) = W8[n, k] MN-major.
   MmCall cdx{M, K, N, g8, a->fmt_g, FP8_K_MAJOR, ldg8, a->w8, a->fmt_w, FP8_MN_MAJOR, a->ldw8,
-             sg, a->sw, nullptr, 0, nullptr, a->dx, a->lddx};
+             sg, a->sw, nullptr, 0, nullptr, a->dx, a->lddx, FP8_TILE_AUTO};
   // dW[N,K] = G8^T . X8: A(i=n, m) = G8[m, n] MN-major, B(j=k, m) = X8[m, k] MN-major.
   MmCall cdw{N, K, M, g8, a->fmt_g, FP8_MN_MAJOR, ldg8, a->x8, a->fmt_x, FP8_MN_MAJOR, a->ldx8,
-             sg, a->sx, nullptr, 0, nullptr, a->dw, a->lddw};
+             sg, a->sx, nullptr, 0, nullptr, a->dw, a->lddw, FP8_TILE_AUTO};
   if (a->need_dx && (s = validate_mm(cdx))) return s;
   if (a->need_dw && (s = validate_mm(cdw))) return s;
   const size_t ws_need = a->need_dbias ? fp8_dbias_workspace_bytes(M, N) : 0;
@@ -460,28 +564,20 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
     side_pending = true;
   } else if (a->need_dbias) {
     // quantize g and sum its columns in the same pass over g
-    ColsumParams cp;
-    std::memset(&cp, 0, sizeof(cp));
-    cp.q = make_qparams(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
-                        a->amax_g_out, a->sg_out, false);
-    dbias_geometry(M, N, &cp.R, &cp.rows_per_split);
-    cp.partial = static_cast<float*>(a->workspace);
-    const size_t part = (static_cast<size_t>(cp.R) * static_cast<size_t>(N) * 4u + 15u) & ~size_t(15);
-    cp.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(a->workspace) + part);
-    cp.dbias = a->dbias;
-    cudaError_t e = launch_quantize_colsum(a->g_dtype, a->fmt_g, cp, st);
-    if (e != cudaSuccess) return cuda_fail(e);
+    const fp8_quantize_args qg = {a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len,
+                                  a->g8, a->ldg8, a->amax_g_out, a->sg_out};
+    if ((s = run_quantize_dbias(qg, a->dbias, a->workspace, st))) return s;
     dbias_done = true;
   } else if ((s = run_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
                                a->amax_g_out, a->sg_out, st))) {
     return s;
   }
-  if (a->need_dx) {
-    if ((s = run_mm(cdx, side_pending ? &side : nullptr, st))) return s;
+  if (a->need_dx && a->need_dw) {  // one launch for both (they share the G8 operand)
+    const MmCall both[2] = {cdx, cdw};
+    if ((s = run_mm_group(both, 2, side_pending ? &side : nullptr, st))) return s;
     side_pending = false;
-  }
-  if (a->need_dw) {
-    if ((s = run_mm(cdw, side_pending ? &side : nullptr, st))) return s;
+  } else if (a->need_dx || a->need_dw) {
+    if ((s = run_mm(a->need_dx ? cdx : cdw, side_pending ? &side : nullptr, st))) return s;
     side_pending = false;
   }
   if (side_pending) {

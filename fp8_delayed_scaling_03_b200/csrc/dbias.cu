@@ -9,11 +9,13 @@
 // block of 8 x 32 threads streams rows of its split with 16-byte loads (8
 // columns per thread), reduces its 8 row lanes in shared memory in a fixed
 // order and writes 256 fp32 partials.  The block that draws the last ticket
-// of its column tile sums the R partials in a fixed order, so the result does
-// not depend on block scheduling, and rezeroes the tile's counter.
+// of its column tile sums the R partials in a fixed order (partials.cuh), so
+// the result does not depend on block scheduling, and rezeroes the tile's
+// counter.
 #include "device.cuh"
 #include "internal.h"
 #include "launch.h"
+#include "partials.cuh"
 
 namespace fp8lin {
 namespace {
@@ -124,29 +126,17 @@ __global__ void __launch_bounds__(kRowLanes * 32) dbias_kernel(const DbiasParams
   #pragma unroll
   for (int y = 0; y < kRowLanes; ++y) s += red[y][threadIdx.x];
   if (col < p.N) p.partial[static_cast<int64_t>(blockIdx.y) * p.N + col] = s;
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(&p.counters[blockIdx.x], 1u) == static_cast<unsigned>(p.R - 1);
+  if (threadIdx.x == 0) {
+    // the barrier above ordered every thread's partial before this fence
+    __threadfence();
+    last = atomicAdd(&p.counters[blockIdx.x], 1u) == static_cast<unsigned>(p.R - 1);
+    if (last) __threadfence();
+  }
   __syncthreads();
   if (!last) return;
-  __threadfence();
-  if (col < p.N) {
-    // Four interleaved partial sums (split r goes to sum r % 4), combined as
-    // (s0 + s1) + (s2 + s3): a fixed order, with four loads in flight.
-    float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const float* pc = p.partial + col;
-    int r = 0;
-    for (; r + 4 <= p.R; r += 4) {
-      float t[4];
-      #pragma unroll
-      for (int u = 0; u < 4; ++u) t[u] = __ldcg(pc + static_cast<int64_t>(r + u) * p.N);
-      #pragma unroll
-      for (int u = 0; u < 4; ++u) s4[u] += t[u];
-    }
-    for (; r < p.R; ++r) s4[r & 3] += __ldcg(pc + static_cast<int64_t>(r) * p.N);
-    const float tot = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-    static_cast<__nv_bfloat16*>(p.dbias)[col] = __float2bfloat16_rn(tot);
-  }
+  if (col < p.N)
+    static_cast<__nv_bfloat16*>(p.dbias)[col] = __float2bfloat16_rn(sum_partials(p.partial + col, p.N, p.R));
   if (threadIdx.x == 0) atomicExch(&p.counters[blockIdx.x], 0u);
 }
 

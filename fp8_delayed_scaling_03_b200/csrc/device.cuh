@@ -70,7 +70,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed.  Bounded: returns
 // false (and records a timeout in *status) after FP8LIN_WAIT_LIMIT_NS, or as
-// soon as *abort becomes nonzero (another role of the CTA gave up).
+// soon as *abort becomes nonzero (another role of the CTA gave up).  status and
+// abort may be NULL.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
                                           volatile int* abort) {
   const uint32_t a = smem_u32(bar);
@@ -83,10 +84,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(a, parity)) return true;
-    if (*abort) return false;
+    if (abort && *abort) return false;
     if (globaltimer_ns() - t0 > FP8LIN_WAIT_LIMIT_NS) {
       if (status) atomicExch(status, kDevTimeout);
-      *abort = 1;
+      if (abort) *abort = 1;
       return false;
     }
   }
@@ -99,7 +100,7 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
 }
 
 // 2-D tiled bulk tensor load global -> shared (this CTA), completion counted
-// in bytes on `bar`.  No cluster multicast.
+// in bytes on `bar`.  Each load fills only the issuing CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t x,
                                             int32_t y) {
   asm volatile(
@@ -216,6 +217,70 @@ __host__ __device__ constexpr uint32_t idesc_f8(int fmt_a, int fmt_b, int major_
          | (static_cast<uint32_t>(major_b) << 16)    // B major
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// ---------------------------------------------------------------- CTA pairs
+// A cluster of two CTAs runs one 2-SM MMA tile (tcgen05 cta_group::2).  Every
+// CTA loads only its own operand halves into its own shared memory (no load is
+// shared between CTAs), and the MMA issuer signals each CTA's barriers one by
+// one.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared::cluster address of the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on an mbarrier of any CTA of the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// 2-SM MMA: M = 256 over the pair (each CTA's shared memory holds its 128 rows
+// of A and N/2 rows of B at the same offsets), accumulator rows in each CTA's
+// TMEM.  Issued by the pair's even CTA only.
+__device__ __forceinline__ void umma_f8f6f4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the mbarrier at `cluster_addr` (either CTA of the pair) when
+// all 2-SM MMAs issued so far by this thread are done.
+__device__ __forceinline__ void umma_commit_pair(uint32_t cluster_addr) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// Tiled load into this CTA's shared memory whose completion is counted on the
+// pair's even CTA's mbarrier (`bar_cluster_addr`).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster_addr, int32_t x,
+                                                 int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
 }
 
 // ---------------------------------------------------------------- gpu-scope atomics

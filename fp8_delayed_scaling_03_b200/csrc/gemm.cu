@@ -5,15 +5,21 @@
 // The pages' kernel (AstrAI commit log, csrc @2eeac02: 128x128 CTA of
 // mma.sync warps fed by cp.async, PRMT byte transposes for the "crosswise"
 // operands of dX/dW) is prior art for sm_89; this is the Blackwell design:
-//   * one persistent CTA per SM, tiles in a grouped raster so the CTAs working
-//     at the same time share operand stripes in L2 (astrai @4019dda and csrc
-//     @2eeac02 describe grouped rasterization for the same reason);
+//   * persistent CTAs (or CTA pairs), tiles in a grouped raster so the CTAs
+//     working at the same time share operand stripes in L2 (astrai @4019dda
+//     and csrc @2eeac02 describe grouped rasterization for the same reason);
 //   * warp 0 lane 0: TMA producer.  128x128-byte boxes with 128-byte swizzle
 //     land in a STAGES-deep shared-memory ring; out-of-range rows, columns and
 //     k come back as zeros, so no tail predication exists in the mainloop;
-//   * warp 1 lane 0: tcgen05.mma.cta_group::1.kind::f8f6f4 issuer, M=128,
-//     N=BN, K=32 per instruction, fp32 accumulator in TMEM (two accumulators
-//     of BN columns, so the epilogue of tile t overlaps the mainloop of t+1);
+//   * warp 1 lane 0: tcgen05.mma kind::f8f6f4 issuer, K=32 per instruction,
+//     fp32 accumulators in TMEM (two of them, so the epilogue of tile t
+//     overlaps the mainloop of t+1);
+//   * single-CTA tiles are 128 x BN.  Pair tiles (kPair) are 256 x 256 over a
+//     cluster of two CTAs: each CTA loads its 128 rows of A and 128 rows of B,
+//     the even CTA issues 2-SM MMAs (cta_group::2, M=256) that read both CTAs'
+//     shared memory, and each CTA's TMEM holds its 128 x 256 accumulator
+//     slice.  Per MMA cycle a CTA then moves 2/3 of the operand bytes of a
+//     128x256 single-CTA tile through shared memory and L2;
 //   * the transposed ("crosswise") operands of dX and dW are read in place:
 //     the smem descriptor and instruction descriptor mark them MN-major, which
 //     tcgen05 supports for E4M3/E5M2 -- no transpose pass, no copy;
@@ -26,8 +32,8 @@
 //     (coalesced, asynchronous, clipped at the matrix edge) -- the pages'
 //     kernel also staged its epilogue through shared memory for write
 //     efficiency (astrai @4019dda, epilogue bullet).  The accumulator is handed
-//     back to the MMA warp right after its last TMEM read.  Output strides that
-//     TMA cannot address (row pitch not a multiple of 16 bytes) take guarded
+//     back to the MMA warp right after its last TMEM read.  Output rows that
+//     TMA cannot address (row pitch or row end not on 16 bytes) take guarded
 //     per-element stores instead.
 // Every mbarrier wait is bounded (see device.cuh); a timeout records
 // FP8_ERR_DEVICE_TIMEOUT and the CTA winds down instead of hanging.
@@ -38,35 +44,47 @@
 namespace fp8lin {
 namespace {
 
-constexpr int kBM = 128;
-constexpr int kBK = 128;  // fp8 elements (= bytes) of k per stage
+constexpr int kBM = 128;              // accumulator rows per CTA
+constexpr int kBK = 128;              // fp8 elements (= bytes) of k per stage
 constexpr int kUmmaK = 32;
-constexpr int kThreads = 320;       // 10 warps: TMA, MMA, 8 epilogue
+constexpr int kThreads = 320;         // 10 warps: TMA, MMA, 8 epilogue
 constexpr int kEpiWarps = 8;
-constexpr int kEpiCols = 32;        // columns per epilogue step
+constexpr int kEpiCols = 32;          // columns per epilogue step
 constexpr int kEpiSlab = 32 * kEpiCols * 2;  // one 32x32 bf16 staging slab
+constexpr int kRingBytes = 192 * 1024;       // operand stages
 
-template <int BN>
+template <int BN, bool kPair>
 struct Cfg {
+  static constexpr int kTileM = kPair ? 2 * kBM : kBM;    // rows of a (pair) tile
+  static constexpr int kBRows = kPair ? BN / 2 : BN;      // rows of B this CTA loads
   static constexpr int kABytes = kBM * kBK;
-  static constexpr int kBBytes = BN * kBK;
+  static constexpr int kBBytes = kBRows * kBK;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kStages = kRingBytes / kStageBytes;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiSlab;  // two slabs per epilogue warp
   static constexpr int kBarBytes = 256;
   static constexpr int kSmem = kStages * kStageBytes + kEpiBytes + kBarBytes + 1024;
+  static constexpr int kTempty = kPair ? 2 * kEpiWarps : kEpiWarps;
   static_assert(BN == 128 || BN == 256, "BN");
+  static_assert(!kPair || BN == 256, "pair tiles are 256 x 256");
 };
 
-__device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& tm, int& tn) {
-  const int per_group = p.raster_group * p.tiles_n;
+// Global tile index -> (problem, tile row, tile column).  Problem 0's tiles
+// come first; within a problem the tiles go in groups of raster_group tile
+// rows, column by column.
+__device__ __forceinline__ int tile_coords(const GemmParams& p, int t, int& tm, int& tn) {
+  const int pi = t >= p.tiles0 ? 1 : 0;
+  const GemmProblem& q = p.pr[pi];
+  if (pi) t -= p.tiles0;
+  const int per_group = q.raster_group * q.tiles_n;
   const int g = t / per_group;
-  const int first_m = g * p.raster_group;
-  const int gm = min(p.raster_group, p.tiles_m - first_m);
+  const int first_m = g * q.raster_group;
+  const int gm = min(q.raster_group, q.tiles_m - first_m);
   const int r = t - g * per_group;
   tm = first_m + r % gm;
   tn = r / gm;
+  return pi;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -74,7 +92,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ float bias_value(const GemmParams& p, int j, float binv) {
+__device__ __forceinline__ float bias_value(const GemmProblem& p, int j, float binv) {
   if (p.bias_kind == 1)
     return __uint_as_float(static_cast<uint32_t>(__ldg(static_cast<const unsigned short*>(p.bias) + j)) << 16);
   const uint16_t b = __ldg(static_cast<const uint8_t*>(p.bias) + j);
@@ -82,11 +100,13 @@ __device__ __forceinline__ float bias_value(const GemmParams& p, int j, float bi
   return f.x * binv;
 }
 
-template <int BN>
+template <int BN, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
-    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                    const __grid_constant__ CUtensorMap tma_d, const GemmParams p) {
-  using C = Cfg<BN>;
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
+                    const __grid_constant__ CUtensorMap td0, const __grid_constant__ CUtensorMap ta1,
+                    const __grid_constant__ CUtensorMap tb1, const __grid_constant__ CUtensorMap td1,
+                    const __grid_constant__ GemmParams p) {
+  using C = Cfg<BN, kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -96,11 +116,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = kPair ? cluster_rank() : 0u;   // 0 = the pair's MMA issuer
+  const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -109,20 +133,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiWarps);
+      mbar_init(&tempty[a], C::kTempty);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    if (p.k_blocks > 0) {
-      prefetch_tmap(&tma_a);
-      prefetch_tmap(&tma_b);
+    for (int i = 0; i < p.nprob; ++i) {
+      if (p.pr[i].k_blocks > 0) {
+        prefetch_tmap(i ? &ta1 : &ta0);
+        prefetch_tmap(i ? &tb1 : &tb0);
+      }
+      if (p.pr[i].tma_store) prefetch_tmap(i ? &td1 : &td0);
     }
-    if (p.tma_store) prefetch_tmap(&tma_d);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
+  tc_fence_before();
+  if constexpr (kPair) cluster_sync();  // both CTAs' barriers exist before either signals the other
+  else __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
   // Everything above overlaps the previous kernel on the stream; from here on
   // its results (operands, scales) are read.
   pdl_wait();
@@ -133,32 +170,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.side.zero_dst[i]) *p.side.zero_dst[i] = 0.0f;
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int t = blockIdx.x; t < p.num_tiles && !*abort_flag; t += gridDim.x) {
+      const int a_row0 = static_cast<int>(rank) * kBM;      // this CTA's rows within the tile
+      const int b_row0 = static_cast<int>(rank) * C::kBRows;
+      for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
         int tm, tn;
-        tile_coords(p, t, tm, tn);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        const int pi = tile_coords(p, t, tm, tn);
+        const GemmProblem& q = p.pr[pi];
+        const CUtensorMap* tma_a = pi ? &ta1 : &ta0;
+        const CUtensorMap* tma_b = pi ? &tb1 : &tb0;
+        const int am = tm * C::kTileM + a_row0;
+        const int bn0 = tn * BN + b_row0;
+        for (int kb = 0; kb < q.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) break;
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
           uint8_t* a_dst = sA + stage * C::kABytes;
           uint8_t* b_dst = sB + stage * C::kBBytes;
-          if (p.a_major == 0) tma_load_2d(a_dst, &tma_a, &full[stage], kb * kBK, tm * kBM);
-          else                tma_load_2d(a_dst, &tma_a, &full[stage], tm * kBM, kb * kBK);
-          if (p.b_major == 0) {
-            tma_load_2d(b_dst, &tma_b, &full[stage], kb * kBK, tn * BN);
+          if constexpr (kPair) {
+            // both CTAs' bytes are counted on the even CTA's full barrier
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+            if (q.a_major == 0) tma_load_2d_pair(a_dst, tma_a, bar, kb * kBK, am);
+            else                tma_load_2d_pair(a_dst, tma_a, bar, am, kb * kBK);
+            if (q.b_major == 0) tma_load_2d_pair(b_dst, tma_b, bar, kb * kBK, bn0);
+            else                tma_load_2d_pair(b_dst, tma_b, bar, bn0, kb * kBK);
           } else {
-            #pragma unroll
-            for (int h = 0; h < BN / 128; ++h)
-              tma_load_2d(b_dst + h * 128 * kBK, &tma_b, &full[stage], tn * BN + h * 128, kb * kBK);
+            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+            if (q.a_major == 0) tma_load_2d(a_dst, tma_a, &full[stage], kb * kBK, am);
+            else                tma_load_2d(a_dst, tma_a, &full[stage], am, kb * kBK);
+            if (q.b_major == 0) {
+              tma_load_2d(b_dst, tma_b, &full[stage], kb * kBK, bn0);
+            } else {
+              #pragma unroll
+              for (int h = 0; h < C::kBRows / 128; ++h)
+                tma_load_2d(b_dst + h * 128 * kBK, tma_b, &full[stage], bn0 + h * 128, kb * kBK);
+            }
           }
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
@@ -166,16 +216,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int t = blockIdx.x; t < p.num_tiles && !*abort_flag; t += gridDim.x) {
+      for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
+        const GemmProblem& q = p.pr[t >= p.tiles0 ? 1 : 0];
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = 0; kb < q.k_blocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) break;
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + stage * C::kABytes);
@@ -183,46 +234,73 @@ __global__ void __launch_bounds__(kThreads, 1)
           #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
             // K-major: advance 32 bytes along the swizzled 128-byte row.
-            // MN-major: advance 32 k-rows of 128 bytes (4 swizzle atoms).
-            const uint64_t ad = p.a_major == 0
+            // MN-major: advance 32 k-rows of 128 bytes (4 swizzle atoms); the
+            // leading offset steps between 128-element MN chunks of B.
+            const uint64_t ad = q.a_major == 0
                                     ? smem_desc_sw128(a_base + kk * kUmmaK, 16, 1024)
                                     : smem_desc_sw128(a_base + kk * kUmmaK * 128, 128 * kBK, 1024);
-            const uint64_t bd = p.b_major == 0
+            const uint64_t bd = q.b_major == 0
                                     ? smem_desc_sw128(b_base + kk * kUmmaK, 16, 1024)
                                     : smem_desc_sw128(b_base + kk * kUmmaK * 128, 128 * kBK, 1024);
-            umma_f8f6f4(d_tmem, ad, bd, p.idesc, (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (kPair) umma_f8f6f4_pair(d_tmem, ad, bd, q.idesc, (kb | kk) != 0 ? 1u : 0u);
+            else                 umma_f8f6f4(d_tmem, ad, bd, q.idesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
+          if constexpr (kPair) {
+            const uint32_t e = smem_u32(&empty[stage]);
+            umma_commit_pair(e);
+            umma_commit_pair(mapa_shared(e, 1));
+          } else {
+            umma_commit(&empty[stage]);
+          }
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
-        umma_commit(&tfull[acc]);
+        if constexpr (kPair) {
+          const uint32_t f = smem_u32(&tfull[acc]);
+          umma_commit_pair(f);
+          umma_commit_pair(mapa_shared(f, 1));
+        } else {
+          umma_commit(&tfull[acc]);
+        }
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
+      // Whatever path led here (a bounded wait may have given up), no MMA may
+      // still read shared memory or TMEM when the CTAs tear down.
+      if constexpr (kPair) umma_commit_pair(smem_u32(drain));
+      else umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, nullptr);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;                 // 0..7
-    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+    const int qd = warp & 3;                 // TMEM lane quadrant this warp may access
     const int half = ew >> 2;                // which half of the tile's columns
-    const int row_in_tile = q * 32 + lane;
-    const float inv = 1.0f / (*p.scale_a * *p.scale_b);
-    const float binv = (p.bias_kind >= 2) ? 1.0f / *p.bias_scale : 1.0f;
-    const bool have_k = p.k_blocks > 0;
-    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const int row_in_tile = static_cast<int>(rank) * kBM + qd * 32 + lane;
+    const float inv0 = 1.0f / (*p.pr[0].scale_a * *p.pr[0].scale_b);
+    const float binv0 = (p.pr[0].bias_kind >= 2) ? 1.0f / *p.pr[0].bias_scale : 1.0f;
+    float inv1 = 1.0f, binv1 = 1.0f;
+    if (p.nprob > 1) {
+      inv1 = 1.0f / (*p.pr[1].scale_a * *p.pr[1].scale_b);
+      binv1 = (p.pr[1].bias_kind >= 2) ? 1.0f / *p.pr[1].bias_scale : 1.0f;
+    }
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
     uint8_t* slabs = sEpi + ew * 2 * kEpiSlab;
     int slab = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(p.d);
     constexpr int kSteps = BN / 2 / kEpiCols;
-    for (int t = blockIdx.x; t < p.num_tiles && !*abort_flag; t += gridDim.x) {
+    for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
       int tm, tn;
-      tile_coords(p, t, tm, tn);
+      const int pi = tile_coords(p, t, tm, tn);
+      const GemmProblem& q = p.pr[pi];
+      const CUtensorMap* tma_d = pi ? &td1 : &td0;
+      const float tinv = pi ? inv1 : inv0;
+      const float tbinv = pi ? binv1 : binv0;
+      const bool have_k = q.k_blocks > 0;
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag)) break;
       tc_fence_after();
-      const int row = tm * kBM + row_in_tile;
+      const int row = tm * C::kTileM + row_in_tile;
       const int col_half = tn * BN + half * (BN / 2);
-      const int live_steps = min(kSteps, max(0, (p.n - col_half + kEpiCols - 1) / kEpiCols));
+      const int live_steps = min(kSteps, max(0, (q.n - col_half + kEpiCols - 1) / kEpiCols));
       #pragma unroll 1
       for (int st = 0; st < kSteps; ++st) {
         const int col0 = col_half + st * kEpiCols;
@@ -235,18 +313,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (st == kSteps - 1) {  // last TMEM read of this accumulator: hand it back
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
+          if (lane == 0) {
+            if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+            else mbar_arrive(&tempty[acc]);
+          }
         }
         if (st >= live_steps) continue;
         float bl = 0.0f;
-        if (p.bias_kind && col0 + lane < p.n) bl = bias_value(p, col0 + lane, binv);
+        if (q.bias_kind && col0 + lane < q.n) bl = bias_value(q, col0 + lane, tbinv);
         float v[32];
         #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          v[j] = (have_k ? __uint_as_float(r[j]) : 0.0f) * inv;
-          if (p.bias_kind) v[j] += __shfl_sync(0xFFFFFFFFu, bl, j);
+          v[j] = (have_k ? __uint_as_float(r[j]) : 0.0f) * tinv;
+          if (q.bias_kind) v[j] += __shfl_sync(0xFFFFFFFFu, bl, j);
         }
-        if (p.tma_store) {
+        if (q.tma_store) {
           uint8_t* buf = slabs + slab * kEpiSlab;
           if (lane == 0) bulk_wait_read<1>();  // the store that last read this slab is done
           __syncwarp();
@@ -261,54 +342,87 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tma_d, buf, col0, tm * kBM + q * 32);
+            tma_store_2d(tma_d, buf, col0, tm * C::kTileM + static_cast<int>(rank) * kBM + qd * 32);
             bulk_commit();
           }
           slab ^= 1;
-        } else if (row < p.m) {
-          __nv_bfloat16* drow = D + static_cast<int64_t>(row) * p.ldd;
+        } else if (row < q.m) {
+          __nv_bfloat16* drow = static_cast<__nv_bfloat16*>(q.d) + static_cast<int64_t>(row) * q.ldd;
           #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (col0 + j < p.n) drow[col0 + j] = __float2bfloat16_rn(v[j]);
+            if (col0 + j < q.n) drow[col0 + j] = __float2bfloat16_rn(v[j]);
         }
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
-    if (p.tma_store && lane == 0) bulk_wait_all();
+    // The stores' global writes complete on their own; the CTA only has to
+    // outlive their reads of its shared memory.
+    if (p.any_tma_store && lane == 0) bulk_wait_read<0>();
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair) cluster_sync();  // no CTA leaves while its pair still signals or reads it
+  else __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (kPair) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
-template <int BN>
-cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const GemmParams& p,
-                      cudaStream_t s) {
-  using C = Cfg<BN>;
+template <int BN, bool kPair>
+cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t s) {
+  using C = Cfg<BN, kPair>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool configured[64] = {};
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaError_t e =
+        cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int sms = num_sms(dev);
-  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  return launch_pdl(fp8_gemm_kernel<BN>, dim3(grid), dim3(kThreads), C::kSmem, s, ta, tb, td, p);
+  if (!kPair) {
+    const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+    return launch_pdl(fp8_gemm_kernel<BN, kPair>, dim3(grid), dim3(kThreads), C::kSmem, s, mp[0], mp[1], mp[2], mp[3],
+                      mp[4], mp[5], p);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  // persistent grid: no more pairs than can be resident at once
+  static int max_pairs[64] = {};
+  if (dev < 64 && max_pairs[dev] == 0) {
+    cfg.gridDim = dim3(2 * (sms / 2));
+    int clusters = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<BN, kPair>, &cfg);
+    if (e != cudaSuccess) return e;
+    max_pairs[dev] = clusters > 0 ? clusters : 1;
+  }
+  const int cap = dev < 64 ? max_pairs[dev] : 1;
+  const int pairs = p.total_tiles < cap ? p.total_tiles : cap;
+  cfg.gridDim = dim3(2 * pairs);
+  return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BN, kPair>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, GemmParams p, int bn,
-                        cudaStream_t s) {
-  if (bn == 256) return launch_bn<256>(ta, tb, td, p, s);
-  return launch_bn<128>(ta, tb, td, p, s);
+cudaError_t launch_gemm(const CUtensorMap* maps, const GemmParams& p, int cfg, cudaStream_t s) {
+  if (cfg == kGemmPair256) return launch_cfg<256, true>(maps, p, s);
+  if (cfg == kGemm256) return launch_cfg<256, false>(maps, p, s);
+  return launch_cfg<128, false>(maps, p, s);
 }
 
 }  // namespace fp8lin

@@ -60,7 +60,9 @@ struct SideWrites {
   float* zero_dst[2];
 };
 
-struct GemmParams {
+// One GEMM problem of a launch (a launch runs one or two of them over one
+// persistent tile schedule: the backward's dX and dW share a launch).
+struct GemmProblem {
   int m, n, k;
   int tiles_m, tiles_n, num_tiles, k_blocks;
   int raster_group;           // M-tiles per raster group
@@ -73,7 +75,15 @@ struct GemmParams {
   const float* bias_scale;
   void* d;
   int64_t ldd;
-  int tma_store;              // D is addressable by TMA (16-byte aligned base and row pitch)
+  int tma_store;              // D is addressable by TMA (16-byte aligned base, pitch and row end)
+};
+
+struct GemmParams {
+  GemmProblem pr[2];
+  int nprob;
+  int tiles0;                 // tiles of pr[0]; tile t >= tiles0 belongs to pr[1]
+  int total_tiles;
+  int any_tma_store;
   int* status;
   SideWrites side;
 };
@@ -98,8 +108,11 @@ cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, cons
 cudaError_t launch_quantize_colsum(int in_dtype, int fmt, const ColsumParams& cp, cudaStream_t s);
 cudaError_t launch_ring_set(float* ring, int H, float scale, cudaStream_t s);
 cudaError_t launch_side_writes(const SideWrites& w, cudaStream_t s);
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, GemmParams p, int bn,
-                        cudaStream_t s);
+// GEMM tile configurations: 128x128 and 128x256 on one CTA, 256x256 on a pair
+// of CTAs (2-SM MMA).
+enum : int { kGemm128 = 1, kGemm256 = 2, kGemmPair256 = 3 };
+// maps[0..2]: A, B, D of pr[0]; maps[3..5]: those of pr[1] (zeroed if unused).
+cudaError_t launch_gemm(const CUtensorMap* maps, const GemmParams& p, int cfg, cudaStream_t s);
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s);
 
 // dbias geometry shared by the size query and the launcher.

@@ -31,6 +31,7 @@
 #include "device.cuh"
 #include "internal.h"
 #include "launch.h"
+#include "partials.cuh"
 
 namespace fp8lin {
 namespace {
@@ -186,10 +187,11 @@ __device__ __forceinline__ uint32_t block_max_bits(float amax, uint32_t* warp_ma
 
 // ---------------------------------------------------------------- flat kernel
 
-constexpr int unroll_for(int bytes) { return bytes == 2 ? 4 : 2; }
+// chunks per thread per iteration (plus as many prefetched): 64 bytes of input
+constexpr int unroll_for(int bytes) { return bytes == 2 ? 2 : 1; }
 
 template <typename T, int FMT>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(const __grid_constant__ QuantizePair pair) {
+__global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_constant__ QuantizePair pair) {
   __shared__ uint32_t warp_max[kThreads / 32];
   __shared__ float hist_s[kHistCache];
   constexpr int U = unroll_for(sizeof(T));
@@ -257,6 +259,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const __grid_constan
 
 // ---------------------------------------------------------------- column-sum kernel
 
+
 constexpr int kColTile = kDbiasColsPerTile;        // 256 columns = 16 chunk lanes
 constexpr int kChunkLanes = kColTile / kChunk;     // 16
 constexpr int kRowLanes = kThreads / kChunkLanes;  // 16
@@ -319,31 +322,21 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   #pragma unroll
   for (int y = 0; y < kRowLanes; ++y) part += red[y][threadIdx.x];
   if (ccol < p.cols) cp.partial[static_cast<int64_t>(blockIdx.y) * p.cols + ccol] = part;
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    ring_finalize(p, bits, nblocks, s, step, hist_s);
+  // Two independent tails run side by side: thread 0 the ring's, thread 32
+  // the column tile's ticket.
+  if (threadIdx.x == 0) ring_finalize(p, bits, nblocks, s, step, hist_s);
+  if (threadIdx.x == 32) {
+    // the barrier above ordered every thread's partial before this fence
+    __threadfence();
     last_tile = atomicAdd(&cp.counters[blockIdx.x], 1u) == gridDim.y - 1;
+    if (last_tile) __threadfence();
   }
   __syncthreads();
   if (!last_tile) return;
-  __threadfence();
-  if (ccol < p.cols) {
-    // four interleaved sums (split r -> sum r % 4), combined (s0+s1)+(s2+s3)
-    float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const float* pc = cp.partial + ccol;
-    const int R = static_cast<int>(gridDim.y);
-    int r = 0;
-    for (; r + 4 <= R; r += 4) {
-      float t[4];
-      #pragma unroll
-      for (int u = 0; u < 4; ++u) t[u] = __ldcg(pc + static_cast<int64_t>(r + u) * p.cols);
-      #pragma unroll
-      for (int u = 0; u < 4; ++u) s4[u] += t[u];
-    }
-    for (; r < R; ++r) s4[r & 3] += __ldcg(pc + static_cast<int64_t>(r) * p.cols);
-    static_cast<__nv_bfloat16*>(cp.dbias)[ccol] = __float2bfloat16_rn((s4[0] + s4[1]) + (s4[2] + s4[3]));
-  }
+  if (ccol < p.cols)
+    static_cast<__nv_bfloat16*>(cp.dbias)[ccol] =
+        __float2bfloat16_rn(sum_partials(cp.partial + ccol, p.cols, static_cast<int>(gridDim.y)));
   if (threadIdx.x == 0) atomicExch(&cp.counters[blockIdx.x], 0u);
 }
 
@@ -374,12 +367,14 @@ __global__ void side_writes_kernel(const SideWrites w) {
 
 // ---------------------------------------------------------------- launchers
 
+// Resident blocks per SM (registers allow four); measured on a B200, four
+// blocks of 2 chunks (plus the next 2 in flight) per thread stream ~18% faster
+// than two blocks of 4.
+constexpr int kBlocksPerSm = 4;
+
 int64_t blocks_for(const QuantizeParams& p, int sms) {
-  // At most two blocks per SM: with U chunks per thread in flight plus the
-  // next iteration's loads that is plenty of bytes in flight, and few atomics
-  // on the ring's two words at the end.
   const int64_t want = (p.total_chunks + kThreads - 1) / kThreads;
-  const int64_t cap = static_cast<int64_t>(sms) * 2;
+  const int64_t cap = static_cast<int64_t>(sms) * kBlocksPerSm;
   return want < 1 ? 1 : (want > cap ? cap : want);
 }
 
@@ -404,8 +399,15 @@ cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, cons
   QuantizePair pair;
   pair.t[0] = *a;
   pair.t[1] = b ? *b : *a;
-  const int64_t g0 = blocks_for(*a, sms);
-  const int64_t g1 = b ? blocks_for(*b, sms) : 0;
+  int64_t g0 = blocks_for(*a, sms);
+  int64_t g1 = b ? blocks_for(*b, sms) : 0;
+  const int64_t cap = static_cast<int64_t>(sms) * kBlocksPerSm;  // one resident wave
+  if (g0 + g1 > cap) {  // share the wave in proportion to the chunks
+    const double f = static_cast<double>(a->total_chunks) / static_cast<double>(a->total_chunks + b->total_chunks);
+    g0 = static_cast<int64_t>(f * static_cast<double>(cap) + 0.5);
+    g0 = g0 < 1 ? 1 : (g0 > cap - 1 ? cap - 1 : g0);
+    g1 = cap - g0;
+  }
   pair.blocks0 = static_cast<int>(g0);
   const int grid = static_cast<int>(g0 + g1);
   if (fmt == kE4M3) {

@@ -55,6 +55,11 @@ typedef enum {
 
 typedef enum { FP8_K_MAJOR = 0, FP8_MN_MAJOR = 1 } fp8_major;
 
+/* GEMM output tiles: 128x128 or 128x256 per CTA, or 256x256 per pair of CTAs
+ * (2-SM MMA, cluster of 2).  Results do not depend on the choice beyond the
+ * fp32 summation order inside the tensor cores. */
+typedef enum { FP8_TILE_AUTO = 0, FP8_TILE_128x128 = 1, FP8_TILE_128x256 = 2, FP8_TILE_PAIR_256x256 = 3 } fp8_tile_cfg;
+
 typedef enum {
   FP8_OK = 0,
   FP8_ERR_INVALID_ARG = -1,    /* NULL required pointer, bad enum, ld < cols, ... */
@@ -108,6 +113,27 @@ FP8LIN_API int fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t 
                  uint8_t* out, int64_t ld_out,
                  float* amax_out, float* scale_out, fp8_stream_t stream);
 
+/* One quantize operand (the fields of fp8_quantize, as a struct). */
+typedef struct fp8_quantize_args {
+  const void* in; int in_dtype; int64_t rows, cols, ld_in;
+  int fmt; void* ring; int hist_len;
+  uint8_t* out; int64_t ld_out;
+  float* amax_out; float* scale_out;
+} fp8_quantize_args;
+
+/* Two quantizes in ONE launch ([astrai@4019dda] quantize_dual: x and w of a
+ * forward).  Each tensor keeps its own ring and last-block finalize, exactly
+ * as two fp8_quantize calls would.  Both must share in_dtype and fmt, and use
+ * different rings. */
+FP8LIN_API int fp8_quantize_dual(const fp8_quantize_args* a, const fp8_quantize_args* b, fp8_stream_t stream);
+
+/* fp8_quantize of g [rows, cols] plus, in the same pass over g, its column
+ * sums: dbias[c] = bf16( sum_r g[r, c] ) as fp8_dbias computes them (fp32
+ * sums in a fixed order).  workspace as fp8_dbias (size from
+ * fp8_dbias_workspace_bytes(rows, cols), zero-filled before first use). */
+FP8LIN_API int fp8_quantize_dbias(const fp8_quantize_args* g, void* dbias, void* workspace, size_t workspace_bytes,
+                                  fp8_stream_t stream);
+
 /* ------------------------------------------------------------------ mm
  * The GEMM primitive ([astrai/extension/ops@057c0d3] two-primitive API;
  * [astrai@4019dda] fused bias):
@@ -134,8 +160,14 @@ typedef struct fp8_mm_args {
   const float* scale_a; const float* scale_b;
   const void* bias; int bias_dtype; const float* bias_scale;
   void* d; int64_t ldd;
+  int tile_cfg;   /* FP8_TILE_AUTO (0, chosen per shape) or one of fp8_tile_cfg */
 } fp8_mm_args;
 FP8LIN_API int fp8_mm(const fp8_mm_args* args, fp8_stream_t stream);
+
+/* Two independent GEMMs in ONE launch over one persistent tile schedule (the
+ * backward's dX and dW).  Same results as two fp8_mm calls; the tile
+ * configuration (a->tile_cfg, or chosen for the pair when AUTO) is shared. */
+FP8LIN_API int fp8_mm_pair(const fp8_mm_args* a, const fp8_mm_args* b, fp8_stream_t stream);
 
 /* ------------------------------------------------------------------ dbias
  * dbias[n] = bf16_rne( sum_m g(m, n) ), fp32 sums, for n < N.  g is bf16,

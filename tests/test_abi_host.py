@@ -26,7 +26,7 @@ def header_functions():
 
 def test_exports_every_header_symbol(fp8):
     names = header_functions()
-    assert len(names) >= 13
+    assert len(names) >= 16
     for n in names:
         assert hasattr(fp8._lib, n), n
         assert n in fp8.EXPORTED, n
@@ -100,6 +100,8 @@ def test_mm_validation(fp8):
     assert mm(fp8, ldd=100) == E.FP8_ERR_INVALID_ARG
     assert mm(fp8, bias=A, bias_dtype=E.FP8_DT_E4M3) == E.FP8_ERR_INVALID_ARG  # fp8 bias needs a scale
     assert mm(fp8, bias=A, bias_dtype=E.FP8_DT_FP32) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, tile_cfg=4) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, tile_cfg=-1) == E.FP8_ERR_INVALID_ARG
     assert mm(fp8, m=0) == E.FP8_OK
     assert mm(fp8, k=0) == E.FP8_OK
     assert fp8._lib.fp8_mm(None, None) == E.FP8_ERR_INVALID_ARG
@@ -163,3 +165,30 @@ def test_linear_backward_validation(fp8):
     assert bwd(fp8, g_dtype=E.FP8_DT_E5M2) == E.FP8_ERR_INVALID_ARG         # pre-quantized g needs its scale
     assert bwd(fp8, sg_out=None) == E.FP8_ERR_INVALID_ARG
     assert bwd(fp8, N=0) == E.FP8_OK
+
+
+def test_fused_entry_points_validation(fp8):
+    E = fp8
+    qa = fp8.QuantizeArgs(A, 0, 4, 32, 32, 0, A + 0x1000, 16, A + 0x2000, 32, None, None)
+    qb = fp8.QuantizeArgs(A + 0x3000, 0, 8, 32, 32, 0, A + 0x4000, 16, A + 0x5000, 32, None, None)
+    same_ring = fp8.QuantizeArgs(A + 0x3000, 0, 8, 32, 32, 0, A + 0x1000, 16, A + 0x5000, 32, None, None)
+    other_fmt = fp8.QuantizeArgs(A + 0x3000, 0, 8, 32, 32, 1, A + 0x4000, 16, A + 0x5000, 32, None, None)
+    f = fp8._lib
+    assert f.fp8_quantize_dual(ctypes.byref(qa), ctypes.byref(same_ring), None) == E.FP8_ERR_INVALID_ARG
+    assert f.fp8_quantize_dual(ctypes.byref(qa), ctypes.byref(other_fmt), None) == E.FP8_ERR_INVALID_ARG
+    assert f.fp8_quantize_dual(None, ctypes.byref(qb), None) == E.FP8_ERR_INVALID_ARG
+    empty = fp8.QuantizeArgs(A, 0, 0, 32, 32, 0, A + 0x1000, 16, A + 0x2000, 32, None, None)
+    empty2 = fp8.QuantizeArgs(A, 0, 0, 32, 32, 0, A + 0x4000, 16, A + 0x2000, 32, None, None)
+    assert f.fp8_quantize_dual(ctypes.byref(empty), ctypes.byref(empty2), None) == E.FP8_OK
+    assert f.fp8_quantize_dbias(ctypes.byref(qa), A + 0x9000, None, 0, None) == E.FP8_ERR_WORKSPACE
+    assert f.fp8_quantize_dbias(ctypes.byref(qa), None, A, 1 << 20, None) == E.FP8_ERR_INVALID_ARG
+    assert f.fp8_quantize_dbias(ctypes.byref(empty), A + 0x9000, None, 0, None) == E.FP8_OK
+    good = fp8.MmArgs(m=128, n=128, k=128, a=A, lda=128, b=A + 0x10000, ldb=128, scale_a=A + 0x20000,
+                      scale_b=A + 0x20010, d=A + 0x30000, ldd=128)
+    bad = fp8.MmArgs(m=128, n=128, k=128, a=A, lda=120, b=A + 0x10000, ldb=128, scale_a=A + 0x20000,
+                     scale_b=A + 0x20010, d=A + 0x30000, ldd=128)
+    assert f.fp8_mm_pair(ctypes.byref(good), ctypes.byref(bad), None) == E.FP8_ERR_INVALID_ARG
+    assert f.fp8_mm_pair(None, ctypes.byref(good), None) == E.FP8_ERR_INVALID_ARG
+    zero = fp8.MmArgs(m=0, n=128, k=128, a=A, lda=128, b=A + 0x10000, ldb=128, scale_a=A + 0x20000,
+                      scale_b=A + 0x20010, d=A + 0x30000, ldd=128)
+    assert f.fp8_mm_pair(ctypes.byref(zero), ctypes.byref(zero), None) == E.FP8_OK

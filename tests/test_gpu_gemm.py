@@ -3,6 +3,8 @@ four operand layouts (the forward's K-major x K-major, dX's K-major x MN-major,
 dW's MN-major x MN-major, and MN-major x K-major), ragged and multi-tile
 shapes, both fp8 formats and the bias variants.  Tolerance per element:
 max(1 bf16 ulp of the oracle value, 2e-6 sum_k |a_k b_k| / (sa sb))."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -41,7 +43,7 @@ def strides(major, ld):
 
 
 def run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=0, fmt_b=0, sa=1.0, sb=1.0, bias_kind=None,
-             pad=0, ldd_extra=0, full=True, a_codes=None, b_codes=None):
+             pad=0, ldd_extra=0, full=True, a_codes=None, b_codes=None, tile=0):
     A = a_codes if a_codes is not None else codes_like_tensor(rng, fmt_a, (m, k), 60.0 if fmt_a == 0 else 3000.0)
     B = b_codes if b_codes is not None else codes_like_tensor(rng, fmt_b, (n, k), 60.0 if fmt_b == 0 else 3000.0)
     a_st, lda = store(A, a_major, pad)
@@ -68,8 +70,9 @@ def run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=0, fmt_b=0, sa=1.0, sb=1
         bias_dtype = fp8.FP8_DT_E4M3 + bf
         odt = oracle.DT_E4M3 + bf
     fp8.fp8_mm(m, n, k, dev_a, fmt_a, a_major, lda, dev_b, fmt_b, b_major, ldb, scales[0:1], scales[1:2], d, ldd,
-               bias=bias_dev, bias_dtype=bias_dtype, bias_scale=bias_scale)
+               bias=bias_dev, bias_dtype=bias_dtype, bias_scale=bias_scale, tile_cfg=tile)
     torch.cuda.synchronize()
+    assert fp8.fp8_get_device_status() == 0
     y = d.cpu().view(torch.int16).numpy().view(np.uint16)
     if ldd_extra:
         assert np.all(y[:, n:] == 0x7FC0), "bytes past n must stay untouched"
@@ -89,38 +92,45 @@ def run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=0, fmt_b=0, sa=1.0, sb=1
 
 
 LAYOUTS = [(0, 0), (0, 1), (1, 1), (1, 0)]
+TILES = [1, 2, 3]   # 128x128, 128x256 (one CTA), 256x256 (CTA pair, 2-SM MMA)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("a_major,b_major", LAYOUTS)
 @pytest.mark.parametrize("m,n,k", [(64, 192, 128), (128, 256, 256), (200, 300, 333), (3, 100, 7),
-                                   (1000, 700, 1040), (130, 129, 2000)])
-def test_mm_layouts_full(fp8, a_major, b_major, m, n, k):
+                                   (1000, 700, 1040), (130, 129, 2000), (600, 520, 384)])
+def test_mm_layouts_full(fp8, a_major, b_major, m, n, k, tile):
     rng = np.random.default_rng(m * 7 + n * 3 + k + 10 * a_major + b_major)
-    run_case(fp8, rng, m, n, k, a_major, b_major, sa=448.0 / 300, sb=0.75, pad=16 if m == 200 else 0)
+    run_case(fp8, rng, m, n, k, a_major, b_major, sa=448.0 / 300, sb=0.75, pad=16 if m == 200 else 0, tile=tile)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("fmt_a,fmt_b", [(1, 0), (1, 1), (0, 1)])
 @pytest.mark.parametrize("a_major,b_major", LAYOUTS)
-def test_mm_formats(fp8, fmt_a, fmt_b, a_major, b_major):
+def test_mm_formats(fp8, fmt_a, fmt_b, a_major, b_major, tile):
     rng = np.random.default_rng(99 + fmt_a * 2 + fmt_b)
-    run_case(fp8, rng, 257, 384, 640, a_major, b_major, fmt_a, fmt_b, sa=57344.0 / 9000, sb=448.0 / 200)
+    run_case(fp8, rng, 257, 384, 640, a_major, b_major, fmt_a, fmt_b, sa=57344.0 / 9000, sb=448.0 / 200, tile=tile)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("bias_kind", ["bf16", "e4m3", "e5m2"])
-def test_mm_bias(fp8, bias_kind):
+def test_mm_bias(fp8, bias_kind, tile):
     rng = np.random.default_rng(5)
-    run_case(fp8, rng, 300, 500, 384, 0, 0, sa=2.0, sb=3.0, bias_kind=bias_kind)
-    run_case(fp8, rng, 64, 100, 96, 0, 0, sa=1.0, sb=1.0, bias_kind=bias_kind, ldd_extra=4)
+    run_case(fp8, rng, 300, 500, 384, 0, 0, sa=2.0, sb=3.0, bias_kind=bias_kind, tile=tile)
+    run_case(fp8, rng, 64, 100, 96, 0, 0, sa=1.0, sb=1.0, bias_kind=bias_kind, ldd_extra=4, tile=tile)
 
 
-def test_mm_odd_ldd_untouched_columns(fp8):
+@pytest.mark.parametrize("tile", TILES)
+def test_mm_odd_ldd_untouched_columns(fp8, tile):
     rng = np.random.default_rng(6)
-    run_case(fp8, rng, 129, 100, 128, 0, 1, ldd_extra=3)
-    run_case(fp8, rng, 77, 264, 300, 1, 1, ldd_extra=8)
+    run_case(fp8, rng, 129, 100, 128, 0, 1, ldd_extra=3, tile=tile)
+    run_case(fp8, rng, 77, 264, 300, 1, 1, ldd_extra=8, tile=tile)
+    run_case(fp8, rng, 300, 264, 300, 0, 0, ldd_extra=8, tile=tile)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("a_major,b_major", LAYOUTS)
-def test_mm_small_integers_exact(fp8, a_major, b_major):
+def test_mm_small_integers_exact(fp8, a_major, b_major, tile):
     """Small-integer fp8 values with unit scales: every partial sum is an integer
     below 2^24, so the GPU must equal the oracle (and the integer matmul) bit
     for bit."""
@@ -131,7 +141,7 @@ def test_mm_small_integers_exact(fp8, a_major, b_major):
     m, n, k = 300, 520, 1000
     A = rng.choice(ints, size=(m, k))
     B = rng.choice(ints, size=(n, k))
-    _, y, want = run_case(fp8, rng, m, n, k, a_major, b_major, a_codes=A, b_codes=B)
+    _, y, want = run_case(fp8, rng, m, n, k, a_major, b_major, a_codes=A, b_codes=B, tile=tile)
     ref = (t[A].astype(np.int64) @ t[B].astype(np.int64).T).astype(np.float32)
     assert np.array_equal(oracle.bf16_to_f32(y), oracle.bf16_to_f32(want))
     assert np.array_equal(oracle.bf16_to_f32(y), oracle.bf16_to_f32(oracle.bf16_rne(ref)))
@@ -147,26 +157,74 @@ def test_mm_identity_weight(fp8):
     run_case(fp8, rng, 256, K, K, 0, 1, a_codes=A, b_codes=B, sa=0.5, sb=1.0)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("a_major,b_major", LAYOUTS)
-def test_mm_long_k_accumulation(fp8, a_major, b_major):
+def test_mm_long_k_accumulation(fp8, a_major, b_major, tile):
     """K = 11008 (the longest contraction of the workloads): random signs and
     all-positive operands.  The all-positive case bounds the accumulation error
     of the tensor-core path against the exact dot."""
     rng = np.random.default_rng(9)
-    run_case(fp8, rng, 256, 256, 11008, a_major, b_major, sa=448.0 / 200, sb=448.0 / 150)
+    run_case(fp8, rng, 256, 256, 11008, a_major, b_major, sa=448.0 / 200, sb=448.0 / 150, tile=tile)
     pos = oracle.encode(0, np.abs(rng.standard_normal((128, 11008)) * 30).astype(np.float32) + 1.0)
     posb = oracle.encode(0, np.abs(rng.standard_normal((256, 11008)) * 30).astype(np.float32) + 1.0)
-    run_case(fp8, rng, 128, 256, 11008, a_major, b_major, a_codes=pos, b_codes=posb)
+    run_case(fp8, rng, 128, 256, 11008, a_major, b_major, a_codes=pos, b_codes=posb, tile=tile)
 
 
+@pytest.mark.parametrize("tile", [0] + TILES)
 @pytest.mark.parametrize("m,n,k,a_major,b_major", [
     (2048, 1024, 1024, 0, 0), (2048, 1024, 4096, 0, 1), (4096, 1024, 2048, 1, 1), (512, 6912, 1536, 0, 0),
-    (1536, 1536, 512, 1, 1), (640, 2304, 4096, 0, 0)])
-def test_mm_large_sampled(fp8, m, n, k, a_major, b_major):
+    (1536, 1536, 512, 1, 1), (640, 2304, 4096, 0, 0), (4096, 11008, 512, 0, 0)])
+def test_mm_large_sampled(fp8, m, n, k, a_major, b_major, tile):
     rng = np.random.default_rng(m + n + k)
-    run_case(fp8, rng, m, n, k, a_major, b_major, sa=3.0, sb=0.25, full=False)
+    run_case(fp8, rng, m, n, k, a_major, b_major, sa=3.0, sb=0.25, full=False, tile=tile)
 
 
 def test_mm_no_device_timeouts(fp8):
     torch.cuda.synchronize()
+    assert fp8.fp8_get_device_status() == 0
+
+
+@pytest.mark.parametrize("tile", [0] + TILES)
+def test_mm_pair_matches_two_calls(fp8, tile):
+    """fp8_mm_pair runs dX-like (K x MN-major) and dW-like (MN x MN-major) GEMMs
+    of different shapes in one launch; each output equals its own fp8_mm call
+    with the same tile configuration bit for bit."""
+    rng = np.random.default_rng(31)
+    M, N, K = 700, 520, 300
+    g8 = codes_like_tensor(rng, 1, (M, N), 3000.0)
+    w8 = codes_like_tensor(rng, 0, (N, K), 60.0)
+    x8 = codes_like_tensor(rng, 0, (M, K), 60.0)
+    gs, ldg = store(g8, 0, 0)
+    ws, ldw = store(w8, 0, 0)
+    xs, ldx = store(x8, 0, 0)
+    G, W, X = (torch.from_numpy(t).cuda() for t in (gs, ws, xs))
+    sc = torch.tensor([3.0, 0.5, 0.25], device="cuda")
+    dx1 = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dw1 = torch.empty(N, K, dtype=torch.bfloat16, device="cuda")
+    dx2, dw2 = torch.empty_like(dx1), torch.empty_like(dw1)
+    p = lambda t: t.data_ptr()  # noqa: E731
+    s4 = sc.data_ptr()
+
+    def args(dx, dw, cfg):
+        a = fp8.MmArgs(M, K, N, p(G), 1, 0, ldg, p(W), 0, 1, ldw, s4, s4 + 4, None, 0, None, p(dx), K, cfg)
+        b = fp8.MmArgs(N, K, M, p(G), 1, 1, ldg, p(X), 0, 1, ldx, s4, s4 + 8, None, 0, None, p(dw), K, cfg)
+        return a, b
+    a, b = args(dx1, dw1, tile)
+    fp8.fp8_mm_pair(a, b)
+    torch.cuda.synchronize()
+    if tile == 0:
+        # auto picks one config for the pair; check against the oracle instead
+        gemm_dx, _, sab = oracle.gemm_acc(gs, 1, ldg, 1, ws, 0, 1, ldw, M, K, N)
+        want, _ = oracle.epilogue(gemm_dx, 3.0, 0.5)
+        assert_gemm_close(dx1.cpu().view(torch.int16).numpy().view(np.uint16), want, sab, 3.0, 0.5, "pair dx")
+        gemm_dw, _, sab = oracle.gemm_acc(gs, 1, 1, ldg, xs, 0, 1, ldx, N, K, M)
+        want, _ = oracle.epilogue(gemm_dw, 3.0, 0.25)
+        assert_gemm_close(dw1.cpu().view(torch.int16).numpy().view(np.uint16), want, sab, 3.0, 0.25, "pair dw")
+    else:
+        a2, b2 = args(dx2, dw2, tile)
+        fp8._lib.fp8_mm(ctypes.byref(a2), torch.cuda.current_stream().cuda_stream)
+        fp8._lib.fp8_mm(ctypes.byref(b2), torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        assert torch.equal(dx1.view(torch.int16), dx2.view(torch.int16))
+        assert torch.equal(dw1.view(torch.int16), dw2.view(torch.int16))
     assert fp8.fp8_get_device_status() == 0

@@ -137,3 +137,53 @@ def test_ring_checkpoint_resume(fp8):
 def test_no_device_timeouts_recorded(fp8):
     torch.cuda.synchronize()
     assert fp8.fp8_get_device_status() == 0
+
+
+@pytest.mark.parametrize("dtype", (torch.bfloat16, torch.float32))
+def test_quantize_dual_matches_two_launches(fp8, dtype):
+    """fp8_quantize_dual on (x, w) = two fp8_quantize calls: same codes, amax,
+    snapshots and ring words, for several steps."""
+    H = 16
+    r1, r2 = fp8.ScaleRing(H), fp8.ScaleRing(H)
+    o1, o2 = oracle.Ring(H), oracle.Ring(H)
+    for step in range(3):
+        x = wl.normal((2048, 1024), 1.0 + step, 900 + step, dtype=dtype)
+        w = wl.normal((1000, 1024), 0.03 * (3 - step), 950 + step, dtype=dtype)
+        xd, wd = x.cuda(), w.cuda()
+        x8, w8 = fp8_buffer(2048, 1024), fp8_buffer(1000, 1024)
+        sc = torch.zeros(4, device="cuda")
+        a = fp8.quantize_args(xd, 0, r1.buf, H, x8, sc[0:1], sc[1:2])
+        b = fp8.quantize_args(wd, 0, r2.buf, H, w8, sc[2:3], sc[3:4])
+        fp8.fp8_quantize_dual(a, b)
+        torch.cuda.synchronize()
+        qx, ax, sx = oracle.quantize(bits(x), dt_code(x), 0, o1)
+        qw, aw, sw = oracle.quantize(bits(w), dt_code(w), 0, o2)
+        assert sc.tolist() == [ax, sx, aw, sw]
+        assert_codes_equal(host_rows(x8), qx, 0)
+        assert_codes_equal(host_rows(w8), qw, 0)
+        assert np.array_equal(ring_words(r1), oracle_ring_words(o1))
+        assert np.array_equal(ring_words(r2), oracle_ring_words(o2))
+
+
+@pytest.mark.parametrize("rows,cols", [(2048, 1024), (300, 100), (4096, 4096), (1, 7), (77, 1534)])
+def test_quantize_dbias_entry(fp8, rows, cols):
+    """fp8_quantize_dbias: codes and ring bit-exact, dbias within
+    max(1 bf16 ulp, 2e-6 sum|g|) of the oracle's column sums."""
+    H = 16
+    ring = fp8.ScaleRing(H)
+    orr = oracle.Ring(H)
+    ws = torch.zeros(max(16, fp8.fp8_dbias_workspace_bytes(rows, cols)), dtype=torch.uint8, device="cuda")
+    for step in range(2):
+        g = wl.normal((rows, cols), 1e-3 * (1 + 3 * step), 970 + step)
+        out = fp8_buffer(rows, cols)
+        db = torch.empty(cols, dtype=torch.bfloat16, device="cuda")
+        fp8.fp8_quantize_dbias(fp8.quantize_args(g.cuda(), 1, ring.buf, H, out), db, ws)
+        torch.cuda.synchronize()
+        q, a, s = oracle.quantize(bits(g), oracle.DT_BF16, 1, orr)
+        assert_codes_equal(host_rows(out), q, 1)
+        assert np.array_equal(ring_words(ring), oracle_ring_words(orr))
+        want, _, sa = oracle.dbias(bits(g), oracle.DT_BF16, rows, cols)
+        gv = oracle.bf16_to_f32(bits(db.cpu())).astype(np.float64)
+        ov = oracle.bf16_to_f32(want).astype(np.float64)
+        assert np.all(np.abs(gv - ov) <= np.maximum(oracle.bf16_ulp(ov), 2e-6 * sa))
+    assert fp8.fp8_get_device_status() == 0

@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP8_PER_BF16 = 2.0          # nominal dense fp8 : bf16 tensor-core ratio (4.5 : 2.25 PFLOP/s)
 NOMINAL_FP8_TFLOPS = 4500.0
 REF_TOKENS = 128            # tokens of one layer per reference-arm step
-BASELINE_TOKENS = 1024      # tokens of one layer for the cpu_baseline sample
+CPU_SAMPLE_TOKENS = 1024      # tokens of one layer for the cpu_baseline sample
 
 
 # --------------------------------------------------------------------------- helpers
@@ -533,10 +533,10 @@ def main(argv=None):
 
         # ---- CPU oracle baseline (rank 0, one GPU only)
         if rank == 0 and world == 1:
-            secs, flops = oracle_layer_sample(BASELINE_TOKENS)
+            secs, flops = oracle_layer_sample(CPU_SAMPLE_TOKENS)
             line["cpu_baseline"] = {
                 "value": flops / secs / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                "sample": f"{BASELINE_TOKENS} of 2048 tokens of one of the 12 dim1024 layers (6 linears: quantize "
+                "sample": f"{CPU_SAMPLE_TOKENS} of 2048 tokens of one of the 12 dim1024 layers (6 linears: quantize "
                           f"x/w/g with rings, fwd+dX+dW GEMMs with fp32 accumulation, bf16 bias, dbias), "
                           f"{secs:.1f} s"}
 

@@ -1,7 +1,7 @@
 """CPU oracle for the FP8 linear layer with delayed scaling.
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by the smoke check in
-``__graft_entry__`` and by the CPU-baseline leg of ``bench.py``; never by the
+the smoke check and by the CPU-baseline leg of ``bench.py``; never by the
 product package, which shares no code with it.
 
 The arithmetic lives in ``fp8_oracle.c`` (plain C, OpenMP over independent

@@ -1,8 +1,8 @@
 """CPU oracle for the FP8 linear layer with delayed scaling.
 
-TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by the smoke check in
-the smoke check and by the CPU-baseline leg of ``bench.py``; never by the
-product package, which shares no code with it.
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by the smoke check and by
+the CPU-baseline leg of ``bench.py``; never by the product package, which
+shares no code with it.
 
 The arithmetic lives in ``fp8_oracle.c`` (plain C, OpenMP over independent
 output rows); this module marshals numpy arrays and holds the orchestration of

@@ -28,6 +28,7 @@ FP8_TILE_AUTO, FP8_TILE_128x128, FP8_TILE_128x256, FP8_TILE_PAIR_256x256 = 0, 1,
 FP8_OK = 0
 FP8_ERR_INVALID_ARG, FP8_ERR_UNSUPPORTED, FP8_ERR_MISALIGNED = -1, -2, -3
 FP8_ERR_CUDA, FP8_ERR_DEVICE_TIMEOUT, FP8_ERR_WORKSPACE = -4, -5, -6
+FP8_ERR_TOO_LARGE = -7
 FP8_MAX = {FP8_E4M3: 448.0, FP8_E5M2: 57344.0}
 
 
@@ -101,6 +102,7 @@ _SIGS = {
     "fp8_mm_pair": (_I, [ctypes.POINTER(MmArgs), ctypes.POINTER(MmArgs), _P]),
     "fp8_dbias_workspace_bytes": (_SZ, [_I64, _I64]),
     "fp8_dbias": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    "fp8_dbias_noalloc": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_linear_forward": (_I, [ctypes.POINTER(LinearFwdArgs), _P]),
     "fp8_linear_backward": (_I, [ctypes.POINTER(LinearBwdArgs), _P]),
     "fp8_linear_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
@@ -227,6 +229,17 @@ def fp8_dbias(g: torch.Tensor, dbias: torch.Tensor, workspace: torch.Tensor,
     _check(_lib.fp8_dbias(_ptr(g), _dtype_code(g, g_fmt), M, N, _ld(g), _ptr(g_scale), _ptr(dbias),
                           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(g.device)),
            "fp8_dbias")
+
+
+def fp8_dbias_noalloc(g: torch.Tensor, dbias: torch.Tensor, g_scale: torch.Tensor | None = None,
+                      g_fmt: int | None = None) -> None:
+    """fp8_dbias without a workspace: for callers that cannot allocate device
+    memory; its scratch is a fixed 1 MiB array inside the library (calls that
+    overlap on the GPU race; the first call on a device should come before any
+    stream capture)."""
+    M, N = g.shape
+    _check(_lib.fp8_dbias_noalloc(_ptr(g), _dtype_code(g, g_fmt), M, N, _ld(g), _ptr(g_scale), _ptr(dbias),
+                                  _stream(g.device)), "fp8_dbias_noalloc")
 
 
 def fp8_linear_forward(args: LinearFwdArgs, device=None) -> None:

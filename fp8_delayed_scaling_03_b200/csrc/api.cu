@@ -617,6 +617,7 @@ const char* fp8_status_string(int status) {
     case FP8_ERR_CUDA: return g_err[0] ? g_err : "CUDA error";
     case FP8_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
     case FP8_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case FP8_ERR_TOO_LARGE: return "request exceeds the fixed scratch of a no-allocation entry point";
     default: return "unknown status";
   }
 }

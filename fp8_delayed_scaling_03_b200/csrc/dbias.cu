@@ -12,6 +12,8 @@
 // of its column tile sums the R partials in a fixed order (partials.cuh), so
 // the result does not depend on block scheduling, and rezeroes the tile's
 // counter.
+#include <cstring>
+
 #include "device.cuh"
 #include "internal.h"
 #include "launch.h"
@@ -170,3 +172,89 @@ cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s) {
 }
 
 }  // namespace fp8lin
+
+// ---------------------------------------------------------------- no-allocation variant
+//
+// fp8_dbias_noalloc: the same bias-gradient kernel with its scratch (the R x N
+// fp32 partials and the per-tile counters) in a fixed array compiled into this
+// library instead of a caller workspace.  For callers that cannot allocate
+// device memory themselves -- code running under a memory manager it does not
+// control (a plugin inside a serving runtime with a fixed device-memory
+// budget, a C caller with no access to the framework's caching allocator) --
+// and so have no workspace to pass.
+
+#include <mutex>
+
+#include "fp8lin.h"
+
+namespace fp8lin {
+namespace {
+
+// 1 MiB, held by every GPU that loads this library until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
+static __device__ __align__(256) unsigned char g_dbias_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+unsigned char* g_noalloc_ptr[64] = {};
+
+// Device address of g_dbias_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+cudaError_t noalloc_scratch(int dev, unsigned char** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_dbias_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace fp8lin
+
+extern "C" int fp8_dbias_noalloc(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg, const float* g_scale,
+                                 void* dbias, fp8_stream_t stream) {
+  using namespace fp8lin;
+  const bool fp8_in = g_dtype == FP8_DT_E4M3 || g_dtype == FP8_DT_E5M2;
+  const bool wide = g_dtype == FP8_DT_BF16 || g_dtype == FP8_DT_FP16 || g_dtype == FP8_DT_FP32;
+  const int64_t kMax = (int64_t(1) << 31) - 1;
+  if (M < 0 || N < 0 || M > kMax || N > kMax) return FP8_ERR_INVALID_ARG;
+  if (!fp8_in && !wide) return FP8_ERR_INVALID_ARG;
+  const size_t esz = g_dtype == FP8_DT_FP32 ? 4 : (fp8_in ? 1 : 2);
+  if (!g || !dbias || ldg < N || reinterpret_cast<uintptr_t>(g) % esz || reinterpret_cast<uintptr_t>(dbias) % 2)
+    return FP8_ERR_INVALID_ARG;
+  if (fp8_in && !g_scale) return FP8_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP8_OK;
+  const size_t need = fp8_dbias_workspace_bytes(M, N);
+  if (need > kNoAllocScratchBytes) return FP8_ERR_TOO_LARGE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8_ERR_CUDA;
+  unsigned char* scratch = nullptr;
+  if (noalloc_scratch(dev, &scratch) != cudaSuccess) return FP8_ERR_CUDA;
+  DbiasParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.g = g;
+  p.dtype = g_dtype;
+  p.M = M;
+  p.N = N;
+  p.ldg = ldg;
+  p.g_scale = g_scale;
+  p.dbias = dbias;
+  dbias_geometry(M, N, &p.R, &p.rows_per_split);
+  const size_t part = (static_cast<size_t>(p.R) * static_cast<size_t>(N) * 4u + 15u) & ~size_t(15);
+  p.partial = reinterpret_cast<float*>(scratch);
+  p.counters = reinterpret_cast<unsigned*>(scratch + part);
+  p.vec_ok = fp8_in ? (reinterpret_cast<uintptr_t>(g) % 8 == 0 && ldg % 8 == 0)
+                    : (reinterpret_cast<uintptr_t>(g) % 16 == 0 && (static_cast<size_t>(ldg) * esz) % 16 == 0);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: the tile counters must start
+  // at zero (the kernel also leaves them at zero when it completes).
+  const size_t tiles = static_cast<size_t>((N + kDbiasColsPerTile - 1) / kDbiasColsPerTile);
+  if (cudaMemsetAsync(p.counters, 0, tiles * sizeof(unsigned), st) != cudaSuccess) return FP8_ERR_CUDA;
+  if (launch_dbias(p, st) != cudaSuccess) return FP8_ERR_CUDA;
+  return FP8_OK;
+}

@@ -67,7 +67,8 @@ typedef enum {
   FP8_ERR_MISALIGNED = -3,     /* fp8 ld % 16 != 0 or base not 16-byte aligned  */
   FP8_ERR_CUDA = -4,           /* a CUDA call failed (see fp8_status_string)    */
   FP8_ERR_DEVICE_TIMEOUT = -5, /* a kernel gave up on a bounded wait            */
-  FP8_ERR_WORKSPACE = -6       /* workspace missing or smaller than required    */
+  FP8_ERR_WORKSPACE = -6,      /* workspace missing or smaller than required    */
+  FP8_ERR_TOO_LARGE = -7       /* beyond the fixed scratch of a no-allocation entry point */
 } fp8_status;
 
 /* ------------------------------------------------------------------ rings
@@ -182,6 +183,27 @@ FP8LIN_API size_t fp8_dbias_workspace_bytes(int64_t M, int64_t N);
 FP8LIN_API int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg,
               const float* g_scale, void* dbias,
               void* workspace, size_t workspace_bytes, fp8_stream_t stream);
+
+/* fp8_dbias without a workspace argument.  No page of the source describes
+ * this entry point; it exists for callers that cannot allocate device memory
+ * themselves (code running under a memory manager it does not control, such as
+ * a plugin inside a serving runtime with a fixed device-memory budget, or a C
+ * caller with no access to the framework's allocator) and therefore have no
+ * workspace to pass.  The same kernel and arguments as fp8_dbias; its scratch
+ * is a 1 MiB array compiled into the library, which every GPU that loads the
+ * library holds until the process exits.
+ *   - Requests needing more than 1 MiB of scratch (fp8_dbias_workspace_bytes(M,
+ *     N) > 1048576; every N <= 131072 fits, whatever M) return
+ *     FP8_ERR_TOO_LARGE and enqueue nothing.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, under a lock); make that first call before any stream
+ *     capture.
+ *   - All calls share the one array: calls that can overlap on the GPU (other
+ *     streams, other host threads) race and must be serialized by the caller.
+ *     Each call clears the tile counters it needs before its kernel. */
+FP8LIN_API int fp8_dbias_noalloc(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg,
+                      const float* g_scale, void* dbias, fp8_stream_t stream);
 
 /* ------------------------------------------------------------------ linear
  * Forward of the FP8 linear ([tests/extension@2eeac02], [astrai/extension/ops@057c0d3]):

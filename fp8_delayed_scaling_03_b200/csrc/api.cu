@@ -212,8 +212,10 @@ int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) 
 }
 
 // Enqueue one launch running n (1 or 2) validated GEMMs over one persistent
-// tile schedule.  side: writes folded into the launch.
-int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_t st) {
+// tile schedule.  side: writes folded into the launch; fin: rings whose
+// quantize deferred its finalize to this launch.
+int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_t st,
+                 const RingFinalize* fin = nullptr, int nfin = 0) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -234,12 +236,21 @@ int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_
   p.total_tiles = p.pr[0].num_tiles + (n > 1 ? p.pr[1].num_tiles : 0);
   p.status = status_ptr(dev);
   if (side) p.side = *side;
+  for (int i = 0; i < nfin; ++i) p.fin[i] = fin[i];
+  p.nfin = nfin;
   e = launch_gemm(maps, p, cfg, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return FP8_OK;
 }
 
-int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st) { return run_mm_group(&c, 1, side, st); }
+int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st, const RingFinalize* fin = nullptr,
+           int nfin = 0) {
+  return run_mm_group(&c, 1, side, st, fin, nfin);
+}
+
+RingFinalize ring_fin(void* ring, int H, int fmt, float* amax_out) {
+  return RingFinalize{static_cast<float*>(ring), H, fp8_max(fmt), amax_out};
+}
 
 QuantizeParams make_qparams(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt,
                             void* ring, int H, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out,
@@ -271,19 +282,25 @@ QuantizeParams make_qparams(const void* in, int in_dtype, int64_t rows, int64_t 
   return p;
 }
 
+// defer: leave the ring's finalize to the GEMM launch that follows (which
+// must then list the ring in its RingFinalize set).
 int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt, void* ring,
-                 int H, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out, cudaStream_t st) {
-  const QuantizeParams p =
+                 int H, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out, cudaStream_t st,
+                 bool defer = false) {
+  QuantizeParams p =
       make_qparams(in, in_dtype, rows, cols, ld_in, fmt, ring, H, out, ld_out, amax_out, scale_out, true);
+  p.defer_finalize = defer ? 1 : 0;
   cudaError_t e = launch_quantize(in_dtype, fmt, &p, nullptr, st);
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
 
-int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace, cudaStream_t st) {
+int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace, cudaStream_t st,
+                       bool defer = false) {
   ColsumParams cp;
   std::memset(&cp, 0, sizeof(cp));
   cp.q = make_qparams(g.in, g.in_dtype, g.rows, g.cols, g.ld_in, g.fmt, g.ring, g.hist_len, g.out, g.ld_out,
                       g.amax_out, g.scale_out, false);
+  cp.q.defer_finalize = defer ? 1 : 0;
   dbias_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
   cp.partial = static_cast<float*>(workspace);
   const size_t part = (static_cast<size_t>(cp.R) * static_cast<size_t>(g.cols) * 4u + 15u) & ~size_t(15);
@@ -500,23 +517,30 @@ int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
   std::memset(&side, 0, sizeof(side));
   if (xq) { side.copy_src[0] = a->x_scale_in; side.copy_dst[0] = a->sx_out; side.zero_dst[0] = a->amax_x_out; }
   if (wq) { side.copy_src[1] = a->w_scale_in; side.copy_dst[1] = a->sw_out; side.zero_dst[1] = a->amax_w_out; }
+  // The quantize launches only max-reduce into their rings; the GEMM, which
+  // waits for them to complete anyway, finishes both ring steps.
+  RingFinalize fin[2];
+  int nfin = 0;
+  if (!xq) fin[nfin++] = ring_fin(a->ring_x, a->hist_len, a->fmt_x, a->amax_x_out);
+  if (!wq) fin[nfin++] = ring_fin(a->ring_w, a->hist_len, a->fmt_w, a->amax_w_out);
   if (!xq && !wq && a->x_dtype == a->w_dtype && a->fmt_x == a->fmt_w) {
-    // x and w in one launch (each with its own ring and finalize)
-    const QuantizeParams qx = make_qparams(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8,
-                                           a->ldx8, a->amax_x_out, a->sx_out, true);
-    const QuantizeParams qw = make_qparams(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8,
-                                           a->ldw8, a->amax_w_out, a->sw_out, true);
+    // x and w in one launch
+    QuantizeParams qx = make_qparams(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8,
+                                     a->ldx8, a->amax_x_out, a->sx_out, true);
+    QuantizeParams qw = make_qparams(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8,
+                                     a->ldw8, a->amax_w_out, a->sw_out, true);
+    qx.defer_finalize = qw.defer_finalize = 1;
     cudaError_t e = launch_quantize(a->x_dtype, a->fmt_x, &qx, &qw, st);
     if (e != cudaSuccess) return cuda_fail(e);
   } else {
     if (!xq && (s = run_quantize(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8, a->ldx8,
-                                 a->amax_x_out, a->sx_out, st)))
+                                 a->amax_x_out, a->sx_out, st, true)))
       return s;
     if (!wq && (s = run_quantize(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8, a->ldw8,
-                                 a->amax_w_out, a->sw_out, st)))
+                                 a->amax_w_out, a->sw_out, st, true)))
       return s;
   }
-  return run_mm(c, &side, st);
+  return run_mm(c, &side, st, fin, nfin);
 }
 
 int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
@@ -559,6 +583,11 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   std::memset(&side, 0, sizeof(side));
   bool side_pending = false;
   bool dbias_done = false;
+  // With a GEMM to follow, the quantize of g leaves its ring step to it.
+  const bool gemm_follows = a->need_dx || a->need_dw;
+  RingFinalize fin[1];
+  int nfin = 0;
+  if (!gq && gemm_follows) fin[nfin++] = ring_fin(a->ring_g, a->hist_len, a->fmt_g, a->amax_g_out);
   if (gq) {
     side.copy_src[0] = a->g_scale_in; side.copy_dst[0] = a->sg_out; side.zero_dst[0] = a->amax_g_out;
     side_pending = true;
@@ -566,18 +595,18 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
     // quantize g and sum its columns in the same pass over g
     const fp8_quantize_args qg = {a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len,
                                   a->g8, a->ldg8, a->amax_g_out, a->sg_out};
-    if ((s = run_quantize_dbias(qg, a->dbias, a->workspace, st))) return s;
+    if ((s = run_quantize_dbias(qg, a->dbias, a->workspace, st, gemm_follows))) return s;
     dbias_done = true;
   } else if ((s = run_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
-                               a->amax_g_out, a->sg_out, st))) {
+                               a->amax_g_out, a->sg_out, st, gemm_follows))) {
     return s;
   }
   if (a->need_dx && a->need_dw) {  // one launch for both (they share the G8 operand)
     const MmCall both[2] = {cdx, cdw};
-    if ((s = run_mm_group(both, 2, side_pending ? &side : nullptr, st))) return s;
+    if ((s = run_mm_group(both, 2, side_pending ? &side : nullptr, st, fin, nfin))) return s;
     side_pending = false;
   } else if (a->need_dx || a->need_dw) {
-    if ((s = run_mm(a->need_dx ? cdx : cdw, side_pending ? &side : nullptr, st))) return s;
+    if ((s = run_mm(a->need_dx ? cdx : cdw, side_pending ? &side : nullptr, st, fin, nfin))) return s;
     side_pending = false;
   }
   if (side_pending) {

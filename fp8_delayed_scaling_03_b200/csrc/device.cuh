@@ -286,6 +286,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
 // ---------------------------------------------------------------- gpu-scope atomics
 
 // Relaxed max on a global word, no return value.
+// The delayed-scaling update rule: the next scale is fp8_max / m for the
+// window maximum m, and the current scale s is kept when m is 0 or infinite
+// or the quotient overflows.
+__device__ __forceinline__ float next_scale(float s, float m, float fp8_max) {
+  if (m > 0.0f && !isinf(m)) {
+    const float q = __fdiv_rn(fp8_max, m);
+    if (!isinf(q)) return q;
+  }
+  return s;
+}
+
 __device__ __forceinline__ void red_max_u32(uint32_t* p, uint32_t v) {
   asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }

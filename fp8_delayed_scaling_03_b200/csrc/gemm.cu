@@ -73,14 +73,18 @@ struct Cfg {
 // Global tile index -> (problem, tile row, tile column).  Problem 0's tiles
 // come first; within a problem the tiles go in groups of raster_group tile
 // rows, column by column.
+// Fields of the problem a tile belongs to are read as pi ? pr[1].f : pr[0].f:
+// two fixed-offset parameter reads instead of one at a run-time offset.
+#define FP8_PR(f) (pi ? p.pr[1].f : p.pr[0].f)
+
 __device__ __forceinline__ int tile_coords(const GemmParams& p, int t, int& tm, int& tn) {
   const int pi = t >= p.tiles0 ? 1 : 0;
-  const GemmProblem& q = p.pr[pi];
   if (pi) t -= p.tiles0;
-  const int per_group = q.raster_group * q.tiles_n;
+  const int raster_group = FP8_PR(raster_group);
+  const int per_group = raster_group * FP8_PR(tiles_n);
   const int g = t / per_group;
-  const int first_m = g * q.raster_group;
-  const int gm = min(q.raster_group, q.tiles_m - first_m);
+  const int first_m = g * raster_group;
+  const int gm = min(raster_group, FP8_PR(tiles_m) - first_m);
   const int r = t - g * per_group;
   tm = first_m + r % gm;
   tn = r / gm;
@@ -92,12 +96,49 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ float bias_value(const GemmProblem& p, int j, float binv) {
-  if (p.bias_kind == 1)
-    return __uint_as_float(static_cast<uint32_t>(__ldg(static_cast<const unsigned short*>(p.bias) + j)) << 16);
-  const uint16_t b = __ldg(static_cast<const uint8_t*>(p.bias) + j);
-  const float2 f = p.bias_kind == 2 ? dec_e4m3x2(b) : dec_e5m2x2(b);
+// a[i] for a register array and a run-time i, without indexing (which would
+// move the array to local memory).
+template <int N>
+__device__ __forceinline__ float pick(const float (&a)[N], int i) {
+  float r = a[0];
+  #pragma unroll
+  for (int k = 1; k < N; ++k) r = (i == k) ? a[k] : r;
+  return r;
+}
+
+__device__ __forceinline__ float bias_value(const void* bias, int bias_kind, int j, float binv) {
+  if (bias_kind == 1)
+    return __uint_as_float(static_cast<uint32_t>(__ldg(static_cast<const unsigned short*>(bias) + j)) << 16);
+  const uint16_t b = __ldg(static_cast<const uint8_t*>(bias) + j);
+  const float2 f = bias_kind == 2 ? dec_e4m3x2(b) : dec_e5m2x2(b);
   return f.x * binv;
+}
+
+// Completes a delayed-scaling step for a ring whose quantize deferred it (its
+// blocks only max-reduced into the scratch word).  Runs after
+// griddepcontrol.wait, so every block's reduction is visible and nothing else
+// touches the ring until this grid completes.  Same rule as the quantize's
+// own last-block finalize: hist[step % H] = amax, window max over the history
+// with the new amax in place of the overwritten slot, next scale, step + 1.
+__device__ __forceinline__ void ring_finalize_warp(const RingFinalize& f, int lane) {
+  uint32_t* words = reinterpret_cast<uint32_t*>(f.ring);
+  const int H = f.H;
+  const uint32_t step = words[H + 2];
+  const float a = __uint_as_float(words[H + 3]);
+  const float s = f.ring[H];
+  const uint32_t slot = step % static_cast<uint32_t>(H);
+  float m = a;
+  for (int i = lane; i < H; i += 32)
+    if (static_cast<uint32_t>(i) != slot) m = fmaxf(m, f.ring[i]);
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if (lane == 0) {
+    f.ring[slot] = a;
+    f.ring[H] = next_scale(s, m, f.fp8_max);
+    words[H + 2] = step + 1;
+    words[H + 3] = 0u;
+    if (f.amax_out) *f.amax_out = a;
+  }
 }
 
 template <int BN, bool kPair>
@@ -126,7 +167,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int units = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
-  if (threadIdx.x == 0) {
+  // Barrier set-up (warp 2), TMEM allocation (warp 1) and the producer's
+  // first tile coordinates (warp 0) proceed side by side.
+  int first_tm = 0, first_tn = 0, first_pi = 0;
+  if (threadIdx.x == 0 && unit < p.total_tiles) first_pi = tile_coords(p, unit, first_tm, first_tn);
+  if (threadIdx.x == 64) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -160,16 +205,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // Everything above overlaps the previous kernel on the stream; from here on
-  // its results (operands, scales) are read.
-  pdl_wait();
+  // The next kernel on the stream may start its own set-up now; it reads what
+  // this one writes only after its own griddepcontrol.wait, which waits for
+  // this grid to complete.  Each role below waits for the previous kernel
+  // (griddepcontrol.wait) only before it first touches global memory: the
+  // producer before its first TMA load, the epilogue before reading scales
+  // and writing D; the MMA warp reads shared memory and TMEM only.
   pdl_trigger();
-  if (blockIdx.x == 0 && threadIdx.x == 64) {
-    for (int i = 0; i < 2; ++i) {
-      if (p.side.copy_dst[i]) *p.side.copy_dst[i] = *p.side.copy_src[i];
-      if (p.side.zero_dst[i]) *p.side.zero_dst[i] = 0.0f;
-    }
-  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -178,31 +220,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       const int a_row0 = static_cast<int>(rank) * kBM;      // this CTA's rows within the tile
       const int b_row0 = static_cast<int>(rank) * C::kBRows;
+      bool dep_done = false;
+      int issued = 0;  // k-blocks loaded so far; the first kStages find their stage free
       for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
-        int tm, tn;
-        const int pi = tile_coords(p, t, tm, tn);
-        const GemmProblem& q = p.pr[pi];
+        int tm = first_tm, tn = first_tn;
+        const int pi = t == unit ? first_pi : tile_coords(p, t, tm, tn);
         const CUtensorMap* tma_a = pi ? &ta1 : &ta0;
         const CUtensorMap* tma_b = pi ? &tb1 : &tb0;
         const int am = tm * C::kTileM + a_row0;
         const int bn0 = tn * BN + b_row0;
-        for (int kb = 0; kb < q.k_blocks; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) break;
+        const int k_blocks = FP8_PR(k_blocks);
+        const bool a_mn = FP8_PR(a_major) != 0, b_mn = FP8_PR(b_major) != 0;
+        for (int kb = 0; kb < k_blocks; ++kb, ++issued) {
+          if (issued >= C::kStages && !mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) break;
+          if (!dep_done) {  // operands are the previous kernel's output
+            pdl_wait();
+            dep_done = true;
+          }
           uint8_t* a_dst = sA + stage * C::kABytes;
           uint8_t* b_dst = sB + stage * C::kBBytes;
           if constexpr (kPair) {
             // both CTAs' bytes are counted on the even CTA's full barrier
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
-            if (q.a_major == 0) tma_load_2d_pair(a_dst, tma_a, bar, kb * kBK, am);
-            else                tma_load_2d_pair(a_dst, tma_a, bar, am, kb * kBK);
-            if (q.b_major == 0) tma_load_2d_pair(b_dst, tma_b, bar, kb * kBK, bn0);
-            else                tma_load_2d_pair(b_dst, tma_b, bar, bn0, kb * kBK);
+            if (!a_mn) tma_load_2d_pair(a_dst, tma_a, bar, kb * kBK, am);
+            else       tma_load_2d_pair(a_dst, tma_a, bar, am, kb * kBK);
+            if (!b_mn) tma_load_2d_pair(b_dst, tma_b, bar, kb * kBK, bn0);
+            else       tma_load_2d_pair(b_dst, tma_b, bar, bn0, kb * kBK);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-            if (q.a_major == 0) tma_load_2d(a_dst, tma_a, &full[stage], kb * kBK, am);
-            else                tma_load_2d(a_dst, tma_a, &full[stage], am, kb * kBK);
-            if (q.b_major == 0) {
+            if (!a_mn) tma_load_2d(a_dst, tma_a, &full[stage], kb * kBK, am);
+            else       tma_load_2d(a_dst, tma_a, &full[stage], am, kb * kBK);
+            if (!b_mn) {
               tma_load_2d(b_dst, tma_b, &full[stage], kb * kBK, bn0);
             } else {
               #pragma unroll
@@ -222,11 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
-        const GemmProblem& q = p.pr[t >= p.tiles0 ? 1 : 0];
+        const int pi = t >= p.tiles0 ? 1 : 0;
+        const int k_blocks = FP8_PR(k_blocks);
+        const bool a_mn = FP8_PR(a_major) != 0, b_mn = FP8_PR(b_major) != 0;
+        const uint32_t idesc = FP8_PR(idesc);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < q.k_blocks; ++kb) {
+        for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) break;
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + stage * C::kABytes);
@@ -236,14 +288,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // K-major: advance 32 bytes along the swizzled 128-byte row.
             // MN-major: advance 32 k-rows of 128 bytes (4 swizzle atoms); the
             // leading offset steps between 128-element MN chunks of B.
-            const uint64_t ad = q.a_major == 0
-                                    ? smem_desc_sw128(a_base + kk * kUmmaK, 16, 1024)
-                                    : smem_desc_sw128(a_base + kk * kUmmaK * 128, 128 * kBK, 1024);
-            const uint64_t bd = q.b_major == 0
-                                    ? smem_desc_sw128(b_base + kk * kUmmaK, 16, 1024)
-                                    : smem_desc_sw128(b_base + kk * kUmmaK * 128, 128 * kBK, 1024);
-            if constexpr (kPair) umma_f8f6f4_pair(d_tmem, ad, bd, q.idesc, (kb | kk) != 0 ? 1u : 0u);
-            else                 umma_f8f6f4(d_tmem, ad, bd, q.idesc, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t ad = !a_mn ? smem_desc_sw128(a_base + kk * kUmmaK, 16, 1024)
+                                      : smem_desc_sw128(a_base + kk * kUmmaK * 128, 128 * kBK, 1024);
+            const uint64_t bd = !b_mn ? smem_desc_sw128(b_base + kk * kUmmaK, 16, 1024)
+                                      : smem_desc_sw128(b_base + kk * kUmmaK * 128, 128 * kBK, 1024);
+            if constexpr (kPair) umma_f8f6f4_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            else                 umma_f8f6f4(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           if constexpr (kPair) {
             const uint32_t e = smem_u32(&empty[stage]);
@@ -275,6 +325,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qd = warp & 3;                 // TMEM lane quadrant this warp may access
     const int half = ew >> 2;                // which half of the tile's columns
     const int row_in_tile = static_cast<int>(rank) * kBM + qd * 32 + lane;
+    pdl_wait();
+    if (blockIdx.x == 0 && threadIdx.x == 64) {
+      for (int i = 0; i < 2; ++i) {
+        if (p.side.copy_dst[i]) *p.side.copy_dst[i] = *p.side.copy_src[i];
+        if (p.side.zero_dst[i]) *p.side.zero_dst[i] = 0.0f;
+      }
+    }
+    if (blockIdx.x == 0 && ew == 1)  // warp 3 of CTA 0; the mainloop runs meanwhile
+      for (int i = 0; i < p.nfin; ++i) ring_finalize_warp(p.fin[i], lane);
     const float inv0 = 1.0f / (*p.pr[0].scale_a * *p.pr[0].scale_b);
     const float binv0 = (p.pr[0].bias_kind >= 2) ? 1.0f / *p.pr[0].bias_scale : 1.0f;
     float inv1 = 1.0f, binv1 = 1.0f;
@@ -291,24 +350,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
       int tm, tn;
       const int pi = tile_coords(p, t, tm, tn);
-      const GemmProblem& q = p.pr[pi];
+      // The tile's constants go to registers and its bias values are fetched
+      // BEFORE the wait for the accumulator, so that no parameter read and no
+      // global-memory latency sits between the TMEM read and the store.
+      const int qm = FP8_PR(m), qn = FP8_PR(n), bias_kind = FP8_PR(bias_kind);
+      const bool tma_store = FP8_PR(tma_store) != 0;
+      const bool have_k = FP8_PR(k_blocks) > 0;
+      void* const qd_ptr = FP8_PR(d);
+      const int64_t ldd = FP8_PR(ldd);
+      const void* const bias = FP8_PR(bias);
       const CUtensorMap* tma_d = pi ? &td1 : &td0;
       const float tinv = pi ? inv1 : inv0;
-      const float tbinv = pi ? binv1 : binv0;
-      const bool have_k = q.k_blocks > 0;
+      const int col_half = tn * BN + half * (BN / 2);
+      const int live_steps = min(kSteps, max(0, (qn - col_half + kEpiCols - 1) / kEpiCols));
+      float bl[kSteps];
+      #pragma unroll
+      for (int st = 0; st < kSteps; ++st) {
+        const int j = col_half + st * kEpiCols + lane;
+        bl[st] = (bias_kind && j < qn) ? bias_value(bias, bias_kind, j, pi ? binv1 : binv0) : 0.0f;
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag)) break;
       tc_fence_after();
       const int row = tm * C::kTileM + row_in_tile;
-      const int col_half = tn * BN + half * (BN / 2);
-      const int live_steps = min(kSteps, max(0, (q.n - col_half + kEpiCols - 1) / kEpiCols));
       #pragma unroll 1
       for (int st = 0; st < kSteps; ++st) {
         const int col0 = col_half + st * kEpiCols;
         uint32_t r[32];
         if (st < live_steps) {
-          __syncwarp();  // tcgen05.ld is .sync.aligned
-          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + half * (BN / 2) + st * kEpiCols), r);
-          tmem_ld_wait();
+          if (have_k) {
+            __syncwarp();  // tcgen05.ld is .sync.aligned
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + half * (BN / 2) + st * kEpiCols), r);
+            tmem_ld_wait();
+          } else {  // K = 0: the MMA never wrote this accumulator
+            #pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = 0u;
+          }
         }
         if (st == kSteps - 1) {  // last TMEM read of this accumulator: hand it back
           tc_fence_before();
@@ -319,15 +395,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (st >= live_steps) continue;
-        float bl = 0.0f;
-        if (q.bias_kind && col0 + lane < q.n) bl = bias_value(q, col0 + lane, tbinv);
+        // One uniform branch per step, none per element: a shuffle under a
+        // per-element condition costs a reconvergence point each.
         float v[32];
-        #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v[j] = (have_k ? __uint_as_float(r[j]) : 0.0f) * tinv;
-          if (q.bias_kind) v[j] += __shfl_sync(0xFFFFFFFFu, bl, j);
+        if (bias_kind) {
+          const float bst = pick(bl, st);
+          #pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * tinv + __shfl_sync(0xFFFFFFFFu, bst, j);
+        } else {
+          #pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * tinv;
         }
-        if (q.tma_store) {
+        if (tma_store) {
           uint8_t* buf = slabs + slab * kEpiSlab;
           if (lane == 0) bulk_wait_read<1>();  // the store that last read this slab is done
           __syncwarp();
@@ -346,11 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit();
           }
           slab ^= 1;
-        } else if (row < q.m) {
-          __nv_bfloat16* drow = static_cast<__nv_bfloat16*>(q.d) + static_cast<int64_t>(row) * q.ldd;
+        } else if (row < qm) {
+          __nv_bfloat16* drow = static_cast<__nv_bfloat16*>(qd_ptr) + static_cast<int64_t>(row) * ldd;
           #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (col0 + j < q.n) drow[col0 + j] = __float2bfloat16_rn(v[j]);
+            if (col0 + j < qn) drow[col0 + j] = __float2bfloat16_rn(v[j]);
         }
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }

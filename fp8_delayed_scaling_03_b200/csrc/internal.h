@@ -31,6 +31,8 @@ struct QuantizeParams {
   float* amax_out;
   float* scale_out;
   int vec_ok;                 // 16-byte vector loads are legal for full chunks
+  int defer_finalize;         // 1: only fold block maxima into the ring's scratch
+                              // word; the GEMM that consumes the output finalizes
 };
 
 // One or two tensors quantized by one launch: blocks [0, blocks0) work on
@@ -60,6 +62,16 @@ struct SideWrites {
   float* zero_dst[2];
 };
 
+// A scale ring whose quantize ran with defer_finalize: the GEMM launch that
+// reads the quantized output completes the ring step (fold the scratch max
+// into the history, publish the next scale, advance step, clear scratch).
+struct RingFinalize {
+  float* ring;
+  int H;
+  float fp8_max;
+  float* amax_out;
+};
+
 // One GEMM problem of a launch (a launch runs one or two of them over one
 // persistent tile schedule: the backward's dX and dW share a launch).
 struct GemmProblem {
@@ -86,6 +98,8 @@ struct GemmParams {
   int any_tma_store;
   int* status;
   SideWrites side;
+  RingFinalize fin[2];
+  int nfin;
 };
 
 struct DbiasParams {

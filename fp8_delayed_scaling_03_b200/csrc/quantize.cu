@@ -20,6 +20,12 @@
 //      quotient overflows), then rezeroes ticket and scratch.  History and
 //      step are prefetched into shared memory at kernel start, so this tail is
 //      two dependent global round trips.
+//   4'. with defer_finalize (the fused linear entry points, where a GEMM that
+//      reads the output always follows) step 4 is skipped: each block's max
+//      goes to the scratch word and the GEMM -- which starts reading only after
+//      this grid has completed -- does the finalize in one warp while its
+//      mainloop runs.  That takes the release fence, the ticket round trip and
+//      the last block's round trips (about 1.5 us) off every quantize launch.
 // The column-sum variant (quantize of g with the bias gradient) walks 2-D
 // tiles of 256 columns instead, so each thread also accumulates the column
 // sums of its 16 columns; per-tile partials meet in a workspace and the last
@@ -164,16 +170,25 @@ __device__ __forceinline__ void ring_finalize(const QuantizeParams& p, uint32_t 
     for (int i = 0; i < p.H; ++i)
       if (static_cast<uint32_t>(i) != slot) m = fmaxf(m, p.ring[i]);
   }
-  float snew = s;
-  if (m > 0.0f && !isinf(m)) {
-    const float qv = __fdiv_rn(p.fp8_max, m);
-    if (!isinf(qv)) snew = qv;
-  }
+  const float snew = next_scale(s, m, p.fp8_max);
   p.ring[slot] = a;
   p.ring[p.H] = snew;
   words[p.H + 2] = step + 1;
   atomicExch(ticket, 0u);
   if (p.amax_out) *p.amax_out = a;
+}
+
+// Thread 0's end of a block: with a deferred finalize only the block's max
+// goes to the ring's scratch word (the consuming GEMM, which starts reading
+// only after this grid completed, finishes the step); else the last-block
+// finalize above.
+__device__ __forceinline__ void ring_tail(const QuantizeParams& p, uint32_t bits, uint32_t nblocks, float s,
+                                          uint32_t step, const float* hist_s) {
+  if (p.defer_finalize) {
+    if (bits) red_max_u32(reinterpret_cast<uint32_t*>(p.ring) + p.H + 3, bits);
+    return;
+  }
+  ring_finalize(p, bits, nblocks, s, step, hist_s);
 }
 
 __device__ __forceinline__ uint32_t block_max_bits(float amax, uint32_t* warp_max) {
@@ -205,11 +220,11 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_cons
   const float s = p.ring[p.H];
   uint32_t step = 0;
   if (threadIdx.x == 0) {
-    step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
+    if (!p.defer_finalize) step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
     if (bid == 0 && p.scale_out) *p.scale_out = s;
   }
   // Only the tensor's last block writes its ring, after every block read it.
-  if (p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
+  if (!p.defer_finalize && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
 
   float amax = 0.0f;
   const int64_t stride = static_cast<int64_t>(nblocks) * kThreads;
@@ -254,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_cons
   }
 
   const uint32_t bits = block_max_bits(amax, warp_max);
-  if (threadIdx.x == 0) ring_finalize(p, bits, nblocks, s, step, hist_s);
+  if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
 }
 
 // ---------------------------------------------------------------- column-sum kernel
@@ -279,10 +294,10 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   const float s = p.ring[p.H];
   uint32_t step = 0;
   if (threadIdx.x == 0) {
-    step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
+    if (!p.defer_finalize) step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
     if (bid == 0 && p.scale_out) *p.scale_out = s;
   }
-  if (p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
+  if (!p.defer_finalize && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
 
   const int cl = threadIdx.x % kChunkLanes;
   const int rl = threadIdx.x / kChunkLanes;
@@ -325,7 +340,7 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   __syncthreads();
   // Two independent tails run side by side: thread 0 the ring's, thread 32
   // the column tile's ticket.
-  if (threadIdx.x == 0) ring_finalize(p, bits, nblocks, s, step, hist_s);
+  if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
   if (threadIdx.x == 32) {
     // the barrier above ordered every thread's partial before this fence
     __threadfence();

@@ -304,6 +304,91 @@ def time_kernels(F, lins, stream, reps=5):
     return res_ms, work, count, shapes
 
 
+# --------------------------------------------------------------------------- target shapes, per operation
+
+def _graph_us(stream, fns, reps=3):
+    """Mean device time of one call of `fns` (cycled) inside a CUDA graph of
+    len(fns) * 4 calls, replayed `reps` times between CUDA events."""
+    g = torch.cuda.CUDAGraph()
+    n = len(fns) * 4
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fns[i % len(fns)]()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * n)
+
+
+def _sets_for(bytes_per_set, floor=320 << 20, cap=12):
+    """Operand sets to cycle through so that one pass touches more than L2."""
+    return max(2, min(cap, -(-floor // max(1, bytes_per_set))))
+
+
+def time_target_shapes(F, device, stream):
+    """fwd, dX and dW as separate launches (fp8_mm, the layouts the fused
+    backward uses) at the production and large shapes, and the quantize of the
+    large activations; operand sets are cycled so each pass streams more than
+    L2.  Returns a list of per-(shape, op) records and a list of quantize
+    records."""
+    h = stream.cuda_stream
+    sc = torch.ones(2, dtype=torch.float32, device=device)
+    gemm = []
+    for s in wl.C3_SHAPES + wl.C4_SHAPES:
+        M, K, N = s.M, s.K, s.N
+        per_set = M * K + N * K + M * N + 2 * (M * N + M * K + N * K)
+        nsets = _sets_for(per_set)
+        sets = []
+        for i in range(nsets):
+            x8 = torch.randint(0x20, 0x48, (M, K), dtype=torch.uint8, device=device)
+            w8 = torch.randint(0x20, 0x48, (N, K), dtype=torch.uint8, device=device)
+            g8 = torch.randint(0x20, 0x48, (M, N), dtype=torch.uint8, device=device)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            dx = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+            dw = torch.empty((N, K), dtype=torch.bfloat16, device=device)
+            sets.append((x8, w8, g8, y, dx, dw))
+        sp = sc.data_ptr()
+        ops = {
+            "fwd": lambda t: F.MmArgs(M, N, K, t[0].data_ptr(), 0, 0, K, t[1].data_ptr(), 0, 0, K, sp, sp + 4,
+                                      None, 0, None, t[3].data_ptr(), N, 0),
+            "dX": lambda t: F.MmArgs(M, K, N, t[2].data_ptr(), 1, 0, N, t[1].data_ptr(), 0, 1, K, sp, sp + 4,
+                                     None, 0, None, t[4].data_ptr(), K, 0),
+            "dW": lambda t: F.MmArgs(N, K, M, t[2].data_ptr(), 1, 1, N, t[0].data_ptr(), 0, 1, K, sp, sp + 4,
+                                     None, 0, None, t[5].data_ptr(), K, 0),
+        }
+        for op, mk in ops.items():
+            args = [mk(t) for t in sets]
+            fns = [(lambda a=a: F._lib.fp8_mm(ctypes.byref(a), h)) for a in args]
+            us = _graph_us(stream, fns)
+            tf = 2.0 * M * N * K / us / 1e6
+            gemm.append({"shape": f"M={M} K={K} N={N}", "op": op, "us": round(us, 2), "tflops": round(tf, 1),
+                         "frac_nominal_4.5PF": round(tf / NOMINAL_FP8_TFLOPS, 3)})
+        del sets
+    quant = []
+    ring = torch.empty(F.fp8_ring_bytes(wl.HIST_LEN) // 4, dtype=torch.float32, device=device)
+    F.fp8_ring_init(ring, wl.HIST_LEN)
+    for rows, cols in ((4096, 4096), (4096, 11008), (2048, 6912)):
+        per_set = rows * cols * 3
+        nsets = _sets_for(per_set)
+        sets = [(torch.randn(rows, cols, device=device).to(torch.bfloat16),
+                 torch.empty(rows, cols, dtype=torch.uint8, device=device)) for _ in range(nsets)]
+        fns = [(lambda x=x, o=o: F._lib.fp8_quantize(x.data_ptr(), 0, rows, cols, cols, 0, ring.data_ptr(),
+                                                     wl.HIST_LEN, o.data_ptr(), cols, None, None, h))
+               for x, o in sets]
+        us = _graph_us(stream, fns)
+        gbs = per_set / us / 1e3
+        quant.append({"shape": f"{rows}x{cols} bf16->e4m3", "us": round(us, 2), "gbs": round(gbs, 1)})
+        del sets
+    return gemm, quant
+
+
 # --------------------------------------------------------------------------- GEMM traffic (ncu summary)
 
 def gemm_source_sha():
@@ -496,6 +581,14 @@ def main(argv=None):
                          "note": "bf16 in + fp8 out; x+w in one launch, g with its bias gradient in one launch; "
                                  "class graph replay"},
             "gemm_by_shape": shapes}
+        tg, tq = time_target_shapes(F, device, stream)
+        for r in tq:
+            r["frac_hbm"] = round(r["gbs"] / pk["hbm_gbs"], 3)
+        line["targets"] = {
+            "gemm": tg, "quantize": tq,
+            "note": "separate fp8_mm launches per operation (dX, dW in the fused backward's in-place "
+                    "transposed layouts), operand sets cycled so each pass streams more than L2; quantize "
+                    "standalone (in-kernel ring finalize)"}
 
         # ---- end to end through the C ABI with host buffers
         host_in = [[t.cpu().pin_memory() for t in L.inputs()] for L in lins]

@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "libfp8lin.so")
 FP8_E4M3, FP8_E5M2 = 0, 1
 FP8_DT_BF16, FP8_DT_FP16, FP8_DT_FP32, FP8_DT_E4M3, FP8_DT_E5M2 = 0, 1, 2, 3, 4
 FP8_K_MAJOR, FP8_MN_MAJOR = 0, 1
-FP8_TILE_AUTO, FP8_TILE_128x128, FP8_TILE_128x256, FP8_TILE_PAIR_256x256 = 0, 1, 2, 3
+FP8_TILE_AUTO, FP8_TILE_128x128, FP8_TILE_128x256, FP8_TILE_PAIR_256x256, FP8_TILE_SPLITK_128x128 = 0, 1, 2, 3, 4
 FP8_OK = 0
 FP8_ERR_INVALID_ARG, FP8_ERR_UNSUPPORTED, FP8_ERR_MISALIGNED = -1, -2, -3
 FP8_ERR_CUDA, FP8_ERR_DEVICE_TIMEOUT, FP8_ERR_WORKSPACE = -4, -5, -6

@@ -127,7 +127,7 @@ int validate_mm(const MmCall& c) {
   s = check_fp8_matrix(c.b, c.ldb, c.b_major == FP8_K_MAJOR ? c.k : c.n);
   if (s) return s;
   if (c.ldd < c.n || !aligned(c.d, 2)) return FP8_ERR_INVALID_ARG;
-  if (c.tile_cfg < FP8_TILE_AUTO || c.tile_cfg > FP8_TILE_PAIR_256x256) return FP8_ERR_INVALID_ARG;
+  if (c.tile_cfg < FP8_TILE_AUTO || c.tile_cfg > FP8_TILE_SPLITK_128x128) return FP8_ERR_INVALID_ARG;
   if (c.bias) {
     if (c.bias_dtype != FP8_DT_BF16 && !is_fp8(c.bias_dtype)) return FP8_ERR_INVALID_ARG;
     if (is_fp8(c.bias_dtype) && !c.bias_scale) return FP8_ERR_INVALID_ARG;
@@ -142,7 +142,7 @@ int validate_mm(const MmCall& c) {
 // tile shape, plus a fixed fill/drain cost.  Measured: 0.34 us per 128x128x128
 // k-block on one SM, 0.45 us per 128x256x128 on one SM and per 256x256x128 on
 // an SM pair; ~4-5 us fill + epilogue + launch.
-int pick_tile(const MmCall* calls, int n, int sms) {
+int pick_tile(const MmCall* calls, int n, int sms, double* est_us = nullptr) {
   struct Opt { int cfg; int64_t tm, tn, units; double t_kb, fixed; };
   const Opt opts[3] = {{kGemm128, 128, 128, sms, 0.34, 4.0}, {kGemm256, 128, 256, sms, 0.45, 4.0},
                        {kGemmPair256, 256, 256, sms / 2, 0.45, 5.0}};
@@ -161,12 +161,13 @@ int pick_tile(const MmCall* calls, int n, int sms) {
     const double t = static_cast<double>(waves) * avg_kb * o.t_kb + o.fixed;
     if (best_t < 0 || t < best_t) { best = o.cfg; best_t = t; }
   }
+  if (est_us) *est_us = best_t;
   return best;
 }
 
 // Problem description and tensor maps of one GEMM for tile configuration cfg.
 int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) {
-  const int bn = cfg == kGemm128 ? 128 : 256;
+  const int bn = (cfg == kGemm128 || cfg == kGemmSplit128) ? 128 : 256;
   const int tile_m = cfg == kGemmPair256 ? 256 : 128;
   const int b_box_rows = cfg == kGemm256 ? 256 : 128;   // rows of B one CTA loads
   std::memset(maps, 0, 3 * sizeof(CUtensorMap));
@@ -215,13 +216,33 @@ int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) 
 // tile schedule.  side: writes folded into the launch; fin: rings whose
 // quantize deferred its finalize to this launch.
 int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_t st,
-                 const RingFinalize* fin = nullptr, int nfin = 0) {
+                 const RingFinalize* fin = nullptr, int nfin = 0, const DbiasFinish* dbf = nullptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   const int sms = num_sms(dev);
   if (sms <= 0) return cuda_fail(cudaGetLastError());
-  const int cfg = calls[0].tile_cfg != FP8_TILE_AUTO ? calls[0].tile_cfg : pick_tile(calls, n, sms);
+  double est = 0.0;
+  int cfg = calls[0].tile_cfg != FP8_TILE_AUTO ? calls[0].tile_cfg : pick_tile(calls, n, sms, &est);
+  // Split-K (single-problem launches): few 128 x 128 tiles and a long K leave
+  // most SMs idle, so a cluster of S CTAs shares each tile's k-blocks.
+  int split = 1;
+  if (cfg == kGemmSplit128 && n != 1) cfg = kGemm128;
+  if (n == 1 && (calls[0].tile_cfg == FP8_TILE_AUTO || cfg == kGemmSplit128)) {
+    const bool forced = cfg == kGemmSplit128;
+    const int64_t tiles = ((calls[0].m + 127) / 128) * ((calls[0].n + 127) / 128);
+    const int64_t kb = (calls[0].k + 127) / 128;
+    if (tiles <= sms && kb >= 2) split = gemm_split_factor(static_cast<int>(tiles), static_cast<int>(kb), sms, forced);
+    if (split >= 2) {
+      // measured on a B200: moving a 128 x 128 fp32 partial between the SMs of
+      // a cluster costs ~1.6 us, parking it ~0.9 us, the cluster launch ~0.5 us
+      const double t_split = static_cast<double>(kb / split) * 0.34 + 4.0 + 3.0;
+      if (forced || t_split < est) cfg = kGemmSplit128;
+      else split = 1;
+    } else if (forced) {
+      cfg = kGemm128;
+    }
+  }
   CUtensorMap maps[6];
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -232,20 +253,22 @@ int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_
     p.any_tma_store |= p.pr[i].tma_store;
   }
   p.nprob = n;
+  p.split = cfg == kGemmSplit128 ? split : 1;
   p.tiles0 = p.pr[0].num_tiles;
   p.total_tiles = p.pr[0].num_tiles + (n > 1 ? p.pr[1].num_tiles : 0);
   p.status = status_ptr(dev);
   if (side) p.side = *side;
   for (int i = 0; i < nfin; ++i) p.fin[i] = fin[i];
   p.nfin = nfin;
+  if (dbf) p.dbias = *dbf;
   e = launch_gemm(maps, p, cfg, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return FP8_OK;
 }
 
 int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st, const RingFinalize* fin = nullptr,
-           int nfin = 0) {
-  return run_mm_group(&c, 1, side, st, fin, nfin);
+           int nfin = 0, const DbiasFinish* dbf = nullptr) {
+  return run_mm_group(&c, 1, side, st, fin, nfin, dbf);
 }
 
 RingFinalize ring_fin(void* ring, int H, int fmt, float* amax_out) {
@@ -294,8 +317,10 @@ int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
 
+// defer: leave both the ring finalize and the column sums to the GEMM
+// launch that follows; *dbf then describes the sums it must do.
 int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace, cudaStream_t st,
-                       bool defer = false) {
+                       bool defer = false, DbiasFinish* dbf = nullptr) {
   ColsumParams cp;
   std::memset(&cp, 0, sizeof(cp));
   cp.q = make_qparams(g.in, g.in_dtype, g.rows, g.cols, g.ld_in, g.fmt, g.ring, g.hist_len, g.out, g.ld_out,
@@ -306,6 +331,8 @@ int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace,
   const size_t part = (static_cast<size_t>(cp.R) * static_cast<size_t>(g.cols) * 4u + 15u) & ~size_t(15);
   cp.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + part);
   cp.dbias = dbias;
+  cp.defer_sum = defer ? 1 : 0;
+  if (defer && dbf) *dbf = DbiasFinish{cp.partial, dbias, g.cols, cp.R};
   cudaError_t e = launch_quantize_colsum(g.in_dtype, g.fmt, cp, st);
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
@@ -587,6 +614,7 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   const bool gemm_follows = a->need_dx || a->need_dw;
   RingFinalize fin[1];
   int nfin = 0;
+  DbiasFinish dbf{};
   if (!gq && gemm_follows) fin[nfin++] = ring_fin(a->ring_g, a->hist_len, a->fmt_g, a->amax_g_out);
   if (gq) {
     side.copy_src[0] = a->g_scale_in; side.copy_dst[0] = a->sg_out; side.zero_dst[0] = a->amax_g_out;
@@ -595,7 +623,7 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
     // quantize g and sum its columns in the same pass over g
     const fp8_quantize_args qg = {a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len,
                                   a->g8, a->ldg8, a->amax_g_out, a->sg_out};
-    if ((s = run_quantize_dbias(qg, a->dbias, a->workspace, st, gemm_follows))) return s;
+    if ((s = run_quantize_dbias(qg, a->dbias, a->workspace, st, gemm_follows, &dbf))) return s;
     dbias_done = true;
   } else if ((s = run_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
                                a->amax_g_out, a->sg_out, st, gemm_follows))) {
@@ -603,10 +631,13 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   }
   if (a->need_dx && a->need_dw) {  // one launch for both (they share the G8 operand)
     const MmCall both[2] = {cdx, cdw};
-    if ((s = run_mm_group(both, 2, side_pending ? &side : nullptr, st, fin, nfin))) return s;
+    if ((s = run_mm_group(both, 2, side_pending ? &side : nullptr, st, fin, nfin, dbf.partial ? &dbf : nullptr)))
+      return s;
     side_pending = false;
   } else if (a->need_dx || a->need_dw) {
-    if ((s = run_mm(a->need_dx ? cdx : cdw, side_pending ? &side : nullptr, st, fin, nfin))) return s;
+    if ((s = run_mm(a->need_dx ? cdx : cdw, side_pending ? &side : nullptr, st, fin, nfin,
+                    dbf.partial ? &dbf : nullptr)))
+      return s;
     side_pending = false;
   }
   if (side_pending) {

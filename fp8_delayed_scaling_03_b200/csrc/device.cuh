@@ -56,6 +56,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// try_wait with acquire at cluster scope: for barriers that other CTAs of the
+// cluster arrive on (release.cluster) after writing shared memory this CTA
+// then reads through distributed shared memory.
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -71,19 +86,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed.  Bounded: returns
 // false (and records a timeout in *status) after FP8LIN_WAIT_LIMIT_NS, or as
 // soon as *abort becomes nonzero (another role of the CTA gave up).  status and
-// abort may be NULL.
+// abort may be NULL.  kCluster: acquire at cluster scope (see above).
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
                                           volatile int* abort) {
   const uint32_t a = smem_u32(bar);
+  auto probe = [&]() { return kCluster ? mbar_try_wait_acq_cluster(a, parity) : mbar_try_wait(a, parity); };
   #pragma unroll 1
   for (int i = 0; i < 64; ++i)
-    if (mbar_try_wait(a, parity)) return true;
+    if (probe()) return true;
   const uint64_t t0 = globaltimer_ns();
   #pragma unroll 1
   while (true) {
     #pragma unroll 1
     for (int i = 0; i < 256; ++i)
-      if (mbar_try_wait(a, parity)) return true;
+      if (probe()) return true;
     if (abort && *abort) return false;
     if (globaltimer_ns() - t0 > FP8LIN_WAIT_LIMIT_NS) {
       if (status) atomicExch(status, kDevTimeout);
@@ -118,6 +135,16 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* s
                "r"(smem_u32(src)), "r"(x), "r"(y)
                : "memory");
 }
+// Bulk copy from this CTA's shared memory into another CTA's of the cluster
+// (dst and bar from mapa_shared), completion counted in bytes on bar.  Both
+// addresses 16-byte aligned, bytes a multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N committed bulk groups still read their shared source.
 template <int N>
@@ -239,6 +266,34 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// 16-byte store into the shared memory of a CTA of the cluster (an address
+// from mapa_shared).
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
+// The two halves of cluster_sync, for work that can run between them (not
+// .aligned: a warp may reach them diverged).
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
+// 16-byte load from the shared memory of a CTA of the cluster (an address
+// from mapa_shared).
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
 // Arrive on an mbarrier of any CTA of the cluster (release at cluster scope).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");

@@ -40,6 +40,7 @@
 #include "device.cuh"
 #include "internal.h"
 #include "launch.h"
+#include "partials.cuh"
 
 namespace fp8lin {
 namespace {
@@ -52,6 +53,16 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiCols = 32;          // columns per epilogue step
 constexpr int kEpiSlab = 32 * kEpiCols * 2;  // one 32x32 bf16 staging slab
 constexpr int kRingBytes = 192 * 1024;       // operand stages
+// A split-K partial: 128 x 128 fp32 as [column / 4][row][4] (a warp's 16-byte
+// accesses for one column quad are 512 contiguous bytes, conflict-free).  The
+// split kernel gives the top (S - 1) partials' worth of the operand ring to a
+// partial region: rank r > 0 parks its partial in slot 0 of its own region
+// and one bulk copy moves it to slot r - 1 of rank 0's, completing on rank 0's
+// barrier; the ring keeps (192 KB - (S - 1) 64 KB) / 32 KB stages (4 for S = 2,
+// 2 for S = 3).
+constexpr int kPartBytes = kBM * 128 * 4;
+constexpr int kMaxSplit = 3;
+static_assert((kMaxSplit - 1) * kPartBytes < kRingBytes, "partials leave room for operand stages");
 
 template <int BN, bool kPair>
 struct Cfg {
@@ -141,38 +152,57 @@ __device__ __forceinline__ void ring_finalize_warp(const RingFinalize& f, int la
   }
 }
 
-template <int BN, bool kPair>
+// dbias[c] = bf16(fixed-order sum of the R partials of column c) for the
+// columns c = 32 * (blockIdx.x + k * gridDim.x) + lane: one warp per CTA,
+// 32 consecutive columns (coalesced rows of partials) at a time.
+__device__ __forceinline__ void dbias_finish_warp(const DbiasFinish& f, int lane) {
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * 32 + lane; c < f.cols;
+       c += static_cast<int64_t>(gridDim.x) * 32)
+    static_cast<__nv_bfloat16*>(f.dbias)[c] = __float2bfloat16_rn(sum_partials(f.partial + c, f.cols, f.R));
+}
+
+template <int BN, bool kPair, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
                     const __grid_constant__ CUtensorMap td0, const __grid_constant__ CUtensorMap ta1,
                     const __grid_constant__ CUtensorMap tb1, const __grid_constant__ CUtensorMap td1,
                     const __grid_constant__ GemmParams p) {
+  static_assert(!kSplit || (BN == 128 && !kPair), "split-K runs 128 x 128 single-CTA tiles");
   using C = Cfg<BN, kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nsplit = kSplit ? p.split : 1;
+  const int nstages = kSplit ? (kRingBytes - (nsplit - 1) * kPartBytes) / C::kStageBytes : C::kStages;
   uint8_t* sA = smem;
-  uint8_t* sB = smem + C::kStages * C::kABytes;
-  uint8_t* sEpi = sB + C::kStages * C::kBBytes;
+  uint8_t* sB = smem + nstages * C::kABytes;
+  uint8_t* sPart = smem + nstages * C::kStageBytes;   // split-K partial region
+  uint8_t* sEpi = smem + C::kStages * C::kStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::kEpiBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* pbar = drain + 1;  // split-K rank 0: partials landed (bytes); rank r > 0: partial parked (warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = kPair ? cluster_rank() : 0u;   // 0 = the pair's MMA issuer
-  const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int units = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // Pair: rank 0 issues the 2-SM MMAs, rank 1 holds the tile's lower half.
+  // Split-K: the cluster's S CTAs share one tile, rank r taking k-blocks
+  // [r kb / S, (r + 1) kb / S); rank 0 sums the partials and stores.
+  const uint32_t rank = (kPair || kSplit) ? cluster_rank() : 0u;
+  const uint32_t prank = kPair ? rank : 0u;            // rank in the tile's row geometry
+  const int per_unit = kPair ? 2 : nsplit;            // CTAs per unit of work
+  const int unit = static_cast<int>(blockIdx.x) / per_unit;
+  const int units = static_cast<int>(gridDim.x) / per_unit;
 
   // Barrier set-up (warp 2), TMEM allocation (warp 1) and the producer's
   // first tile coordinates (warp 0) proceed side by side.
   int first_tm = 0, first_tn = 0, first_pi = 0;
   if (threadIdx.x == 0 && unit < p.total_tiles) first_pi = tile_coords(p, unit, first_tm, first_tn);
   if (threadIdx.x == 64) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < nstages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -181,8 +211,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[a], C::kTempty);
     }
     mbar_init(drain, 1);
+    if constexpr (kSplit) mbar_init(pbar, rank == 0 ? 1u : static_cast<uint32_t>(kEpiWarps));
     *abort_flag = 0;
     fence_mbar_init();
+    // split-K rank 0: its partial region fills with (S - 1) bulk copies
+    if (kSplit && rank == 0) mbar_arrive_expect_tx(pbar, static_cast<uint32_t>((nsplit - 1) * kPartBytes));
     for (int i = 0; i < p.nprob; ++i) {
       if (p.pr[i].k_blocks > 0) {
         prefetch_tmap(i ? &ta1 : &ta0);
@@ -201,8 +234,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   tc_fence_before();
-  if constexpr (kPair) cluster_sync();  // both CTAs' barriers exist before either signals the other
-  else __syncthreads();
+  if constexpr (kPair) {
+    cluster_sync();  // both CTAs' barriers exist before either signals the other
+  } else {
+    __syncthreads();
+    // Split-K: the first remote access comes at the end of the mainloop, so
+    // the cluster barrier's wait (every CTA's barriers initialized) is taken
+    // there (epilogue) or at teardown (the other warps), not here.
+    if constexpr (kSplit) cluster_arrive();
+  }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // The next kernel on the stream may start its own set-up now; it reads what
@@ -218,8 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const int a_row0 = static_cast<int>(rank) * kBM;      // this CTA's rows within the tile
-      const int b_row0 = static_cast<int>(rank) * C::kBRows;
+      const int a_row0 = static_cast<int>(prank) * kBM;      // this CTA's rows within the tile
+      const int b_row0 = static_cast<int>(prank) * C::kBRows;
       bool dep_done = false;
       int issued = 0;  // k-blocks loaded so far; the first kStages find their stage free
       for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
@@ -231,8 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bn0 = tn * BN + b_row0;
         const int k_blocks = FP8_PR(k_blocks);
         const bool a_mn = FP8_PR(a_major) != 0, b_mn = FP8_PR(b_major) != 0;
-        for (int kb = 0; kb < k_blocks; ++kb, ++issued) {
-          if (issued >= C::kStages && !mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) break;
+        const int kb_lo = kSplit ? static_cast<int>(rank) * k_blocks / nsplit : 0;
+        const int kb_hi = kSplit ? (static_cast<int>(rank) + 1) * k_blocks / nsplit : k_blocks;
+        for (int kb = kb_lo; kb < kb_hi; ++kb, ++issued) {
+          if (issued >= nstages && !mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) break;
           if (!dep_done) {  // operands are the previous kernel's output
             pdl_wait();
             dep_done = true;
@@ -259,13 +301,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_2d(b_dst + h * 128 * kBK, tma_b, &full[stage], bn0 + h * 128, kb * kBK);
             }
           }
-          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == nstages) { stage = 0; phase ^= 1u; }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && rank == 0) {
+    if (lane == 0 && (!kPair || rank == 0)) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -275,10 +317,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int k_blocks = FP8_PR(k_blocks);
         const bool a_mn = FP8_PR(a_major) != 0, b_mn = FP8_PR(b_major) != 0;
         const uint32_t idesc = FP8_PR(idesc);
+        const int kb_lo = kSplit ? static_cast<int>(rank) * k_blocks / nsplit : 0;
+        const int kb_hi = kSplit ? (static_cast<int>(rank) + 1) * k_blocks / nsplit : k_blocks;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) break;
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + stage * C::kABytes);
@@ -292,8 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       : smem_desc_sw128(a_base + kk * kUmmaK * 128, 128 * kBK, 1024);
             const uint64_t bd = !b_mn ? smem_desc_sw128(b_base + kk * kUmmaK, 16, 1024)
                                       : smem_desc_sw128(b_base + kk * kUmmaK * 128, 128 * kBK, 1024);
-            if constexpr (kPair) umma_f8f6f4_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-            else                 umma_f8f6f4(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            const uint32_t accum = (kb != kb_lo || kk != 0) ? 1u : 0u;
+            if constexpr (kPair) umma_f8f6f4_pair(d_tmem, ad, bd, idesc, accum);
+            else                 umma_f8f6f4(d_tmem, ad, bd, idesc, accum);
           }
           if constexpr (kPair) {
             const uint32_t e = smem_u32(&empty[stage]);
@@ -302,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             umma_commit(&empty[stage]);
           }
-          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == nstages) { stage = 0; phase ^= 1u; }
         }
         if constexpr (kPair) {
           const uint32_t f = smem_u32(&tfull[acc]);
@@ -324,7 +369,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - 2;                 // 0..7
     const int qd = warp & 3;                 // TMEM lane quadrant this warp may access
     const int half = ew >> 2;                // which half of the tile's columns
-    const int row_in_tile = static_cast<int>(rank) * kBM + qd * 32 + lane;
+    const int row_in_tile = static_cast<int>(prank) * kBM + qd * 32 + lane;
+    // split-K: this thread's row in slot 0 of the partial region; column quad
+    // c4 of row i is float4 c4 * 128 + i of a slot
+    float4* const part_row = reinterpret_cast<float4*>(sPart) + (qd * 32 + lane);
+    bool cluster_ready = !kSplit;  // split-K: the start-up cluster barrier's wait is taken
     pdl_wait();
     if (blockIdx.x == 0 && threadIdx.x == 64) {
       for (int i = 0; i < 2; ++i) {
@@ -334,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (blockIdx.x == 0 && ew == 1)  // warp 3 of CTA 0; the mainloop runs meanwhile
       for (int i = 0; i < p.nfin; ++i) ring_finalize_warp(p.fin[i], lane);
+    if (p.dbias.partial && ew == 2) dbias_finish_warp(p.dbias, lane);  // warp 4 of every CTA
     const float inv0 = 1.0f / (*p.pr[0].scale_a * *p.pr[0].scale_b);
     const float binv0 = (p.pr[0].bias_kind >= 2) ? 1.0f / *p.pr[0].bias_scale : 1.0f;
     float inv1 = 1.0f, binv1 = 1.0f;
@@ -355,7 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // global-memory latency sits between the TMEM read and the store.
       const int qm = FP8_PR(m), qn = FP8_PR(n), bias_kind = FP8_PR(bias_kind);
       const bool tma_store = FP8_PR(tma_store) != 0;
-      const bool have_k = FP8_PR(k_blocks) > 0;
+      const bool have_k = kSplit ? (static_cast<int>(rank) + 1) * FP8_PR(k_blocks) / nsplit >
+                                       static_cast<int>(rank) * FP8_PR(k_blocks) / nsplit
+                                 : FP8_PR(k_blocks) > 0;
       void* const qd_ptr = FP8_PR(d);
       const int64_t ldd = FP8_PR(ldd);
       const void* const bias = FP8_PR(bias);
@@ -371,6 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag)) break;
       tc_fence_after();
+      if constexpr (kSplit) {
+        if (!cluster_ready) { cluster_wait(); cluster_ready = true; }
+        // rank 0: the other ranks' partials have landed in its partial region
+        if (rank == 0 && !mbar_wait(pbar, 0, p.status, abort_flag)) break;
+      }
       const int row = tm * C::kTileM + row_in_tile;
       #pragma unroll 1
       for (int st = 0; st < kSteps; ++st) {
@@ -395,6 +452,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (st >= live_steps) continue;
+        if constexpr (kSplit) {
+          const int pq = (half * (BN / 2) + st * kEpiCols) / 4;  // column quad of r[0..3]
+          if (rank != 0) {  // park the partial; rank 0 finishes the tile
+            #pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              part_row[(pq + j / 4) * kBM] = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                                         __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+            continue;
+          }
+          // rank order: ((p0 + p1) + p2) + ..., the same for every launch
+          for (int q = 1; q < nsplit; ++q) {
+            const float4* src = part_row + (q - 1) * (kPartBytes / 16) + pq * kBM;
+            #pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 o = src[(j / 4) * kBM];
+              r[j] = __float_as_uint(__uint_as_float(r[j]) + o.x);
+              r[j + 1] = __float_as_uint(__uint_as_float(r[j + 1]) + o.y);
+              r[j + 2] = __float_as_uint(__uint_as_float(r[j + 2]) + o.z);
+              r[j + 3] = __float_as_uint(__uint_as_float(r[j + 3]) + o.w);
+            }
+          }
+        }
         // One uniform branch per step, none per element: a shuffle under a
         // per-element condition costs a reconvergence point each.
         float v[32];
@@ -421,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(tma_d, buf, col0, tm * C::kTileM + static_cast<int>(rank) * kBM + qd * 32);
+            tma_store_2d(tma_d, buf, col0, tm * C::kTileM + static_cast<int>(prank) * kBM + qd * 32);
             bulk_commit();
           }
           slab ^= 1;
@@ -432,15 +511,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (col0 + j < qn) drow[col0 + j] = __float2bfloat16_rn(v[j]);
         }
       }
+      if (kSplit && rank != 0) {  // partial parked: one bulk copy into rank 0's region
+        fence_proxy_async_smem();  // this thread's parked bytes, visible to the copy engine
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pbar);
+        if (ew == 0 && lane == 0 && mbar_wait(pbar, 0, p.status, abort_flag))  // all eight warps parked
+          bulk_copy_to_cluster(mapa_shared(smem_u32(sPart + (rank - 1) * kPartBytes), 0), sPart, kPartBytes,
+                               mapa_shared(smem_u32(pbar), 0));
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
     // The stores' global writes complete on their own; the CTA only has to
     // outlive their reads of its shared memory.
     if (p.any_tma_store && lane == 0) bulk_wait_read<0>();
+    if (!cluster_ready) cluster_wait();
+  }
+  if constexpr (kSplit) {
+    if (warp < 2) cluster_wait();  // producer and MMA warps close the start-up cluster barrier
   }
 
   tc_fence_before();
-  if constexpr (kPair) cluster_sync();  // no CTA leaves while its pair still signals or reads it
+  if constexpr (kPair || kSplit) cluster_sync();  // no CTA leaves while another still signals or reads it
   else __syncthreads();
   if (warp == 1) {
     __syncwarp();
@@ -458,14 +549,14 @@ cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t 
   static bool configured[64] = {};
   if (dev < 64 && !configured[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int sms = num_sms(dev);
   if (!kPair) {
     const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-    return launch_pdl(fp8_gemm_kernel<BN, kPair>, dim3(grid), dim3(kThreads), C::kSmem, s, mp[0], mp[1], mp[2], mp[3],
+    return launch_pdl(fp8_gemm_kernel<BN, kPair, false>, dim3(grid), dim3(kThreads), C::kSmem, s, mp[0], mp[1], mp[2], mp[3],
                       mp[4], mp[5], p);
   }
   cudaLaunchConfig_t cfg = {};
@@ -486,19 +577,88 @@ cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t 
   if (dev < 64 && max_pairs[dev] == 0) {
     cfg.gridDim = dim3(2 * (sms / 2));
     int clusters = 0;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<BN, kPair>, &cfg);
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<BN, kPair, false>, &cfg);
     if (e != cudaSuccess) return e;
     max_pairs[dev] = clusters > 0 ? clusters : 1;
   }
   const int cap = dev < 64 ? max_pairs[dev] : 1;
   const int pairs = p.total_tiles < cap ? p.total_tiles : cap;
   cfg.gridDim = dim3(2 * pairs);
-  return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BN, kPair>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
+  return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BN, kPair, false>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
+}
+
+// Largest number of clusters of `split` CTAs of the split-K kernel that can be
+// resident at once (cached per device and split factor).
+int split_clusters(int dev, int split) {
+  static int cache[64][kMaxSplit + 1] = {};
+  if (split < 2 || split > kMaxSplit) return 0;
+  if (dev < 64 && cache[dev][split]) return cache[dev][split];
+  using C = Cfg<128, false>;
+  cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<128, false, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.gridDim = dim3(split * (num_sms(dev) / split));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(split);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<128, false, true>, &cfg) != cudaSuccess) return 0;
+  if (dev < 64) cache[dev][split] = clusters;
+  return clusters;
+}
+
+// Split-K launch: one cluster of p.split CTAs per 128 x 128 tile.
+cudaError_t launch_split(const CUtensorMap* mp, const GemmParams& p, cudaStream_t s) {
+  using C = Cfg<128, false>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (split_clusters(dev, p.split) <= 0) return cudaErrorInvalidConfiguration;  // also sets the smem limit
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cfg.gridDim = dim3(static_cast<unsigned>(p.total_tiles * p.split));
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.split);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<128, false, true>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
 }
 
 }  // namespace
 
+int gemm_split_factor(int tiles, int k_blocks, int sms, bool forced) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || tiles <= 0 || k_blocks < 2) return 1;
+  int best = 1;
+  for (int s = 2; s <= kMaxSplit; ++s) {
+    if (s > k_blocks) break;
+    if (!forced && k_blocks / s < 4) break;  // at least 4 k-blocks a rank
+    const int clusters = split_clusters(dev, s);
+    if (clusters <= 0) break;
+    if (tiles > clusters) {  // a second wave of clusters: never worth it
+      if (forced && best == 1) best = s;
+      break;
+    }
+    best = s;
+  }
+  return best;
+}
+
 cudaError_t launch_gemm(const CUtensorMap* maps, const GemmParams& p, int cfg, cudaStream_t s) {
+  if (cfg == kGemmSplit128) return launch_split(maps, p, s);
   if (cfg == kGemmPair256) return launch_cfg<256, true>(maps, p, s);
   if (cfg == kGemm256) return launch_cfg<256, false>(maps, p, s);
   return launch_cfg<128, false>(maps, p, s);

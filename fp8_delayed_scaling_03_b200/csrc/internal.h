@@ -52,6 +52,8 @@ struct ColsumParams {
   void* dbias;                // bf16 [cols]
   int64_t rows_per_split;
   int R;
+  int defer_sum;              // 1: only write the partials; the GEMM that
+                              // follows sums them (DbiasFinish)
 };
 
 // Side writes a GEMM launch performs once (block 0), for operands that arrive
@@ -70,6 +72,17 @@ struct RingFinalize {
   int H;
   float fp8_max;
   float* amax_out;
+};
+
+// The bias gradient of a quantize whose column sums ran with defer_sum: the
+// GEMM launch that follows turns the R x cols partials into dbias (bf16),
+// each column summed in the same fixed order as the quantize's own last
+// block would have.
+struct DbiasFinish {
+  const float* partial;
+  void* dbias;
+  int64_t cols;
+  int R;
 };
 
 // One GEMM problem of a launch (a launch runs one or two of them over one
@@ -100,6 +113,8 @@ struct GemmParams {
   SideWrites side;
   RingFinalize fin[2];
   int nfin;
+  DbiasFinish dbias;          // partial == nullptr: none
+  int split;                  // split-K launches: CTAs per tile (cluster size)
 };
 
 struct DbiasParams {
@@ -124,7 +139,11 @@ cudaError_t launch_ring_set(float* ring, int H, float scale, cudaStream_t s);
 cudaError_t launch_side_writes(const SideWrites& w, cudaStream_t s);
 // GEMM tile configurations: 128x128 and 128x256 on one CTA, 256x256 on a pair
 // of CTAs (2-SM MMA).
-enum : int { kGemm128 = 1, kGemm256 = 2, kGemmPair256 = 3 };
+enum : int { kGemm128 = 1, kGemm256 = 2, kGemmPair256 = 3, kGemmSplit128 = 4 };
+// Split factor (2..3, or 1 for none) for a 128 x 128-tile problem: the largest
+// S with every rank given >= 4 k-blocks and all tiles' clusters resident in
+// one wave; forced: the largest S <= min(3, k_blocks) fitting one wave, else 2.
+int gemm_split_factor(int tiles, int k_blocks, int sms, bool forced);
 // maps[0..2]: A, B, D of pr[0]; maps[3..5]: those of pr[1] (zeroed if unused).
 cudaError_t launch_gemm(const CUtensorMap* maps, const GemmParams& p, int cfg, cudaStream_t s);
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s);

@@ -31,6 +31,9 @@
 // sums of its 16 columns; per-tile partials meet in a workspace and the last
 // block of each column tile (its own ticket) sums them in a fixed order
 // (astrai @4019dda: the column sum runs only when the bias needs a gradient).
+// With defer_sum (a GEMM follows in the fused backward) the blocks stop after
+// writing their partials and the GEMM's idle epilogue warps do the fixed-order
+// sums, as they do the deferred ring finalize.
 // No block ever waits on another, so nothing here can hang.
 #include <type_traits>
 
@@ -337,6 +340,10 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   #pragma unroll
   for (int y = 0; y < kRowLanes; ++y) part += red[y][threadIdx.x];
   if (ccol < p.cols) cp.partial[static_cast<int64_t>(blockIdx.y) * p.cols + ccol] = part;
+  if (cp.defer_sum) {  // the GEMM that follows sums the partials
+    if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
+    return;
+  }
   __syncthreads();
   // Two independent tails run side by side: thread 0 the ring's, thread 32
   // the column tile's ticket.

@@ -56,9 +56,17 @@ typedef enum {
 typedef enum { FP8_K_MAJOR = 0, FP8_MN_MAJOR = 1 } fp8_major;
 
 /* GEMM output tiles: 128x128 or 128x256 per CTA, or 256x256 per pair of CTAs
- * (2-SM MMA, cluster of 2).  Results do not depend on the choice beyond the
- * fp32 summation order inside the tensor cores. */
-typedef enum { FP8_TILE_AUTO = 0, FP8_TILE_128x128 = 1, FP8_TILE_128x256 = 2, FP8_TILE_PAIR_256x256 = 3 } fp8_tile_cfg;
+ * (2-SM MMA, cluster of 2), or 128x128 tiles each shared by a cluster of S = 2..3
+ * CTAs that split K (FP8_TILE_SPLITK_128x128: rank r takes k-blocks
+ * [r kb/S, (r+1) kb/S) and rank 0 adds the partial fp32 accumulators in rank
+ * order before the epilogue; fp8_mm only -- a two-GEMM launch falls back to
+ * 128x128).  FP8_TILE_AUTO chooses per shape, split-K included when the output
+ * has few tiles and K is long.  Results do not depend on the choice beyond the
+ * fp32 summation order. */
+typedef enum {
+  FP8_TILE_AUTO = 0, FP8_TILE_128x128 = 1, FP8_TILE_128x256 = 2, FP8_TILE_PAIR_256x256 = 3,
+  FP8_TILE_SPLITK_128x128 = 4
+} fp8_tile_cfg;
 
 typedef enum {
   FP8_OK = 0,

@@ -100,7 +100,7 @@ def test_mm_validation(fp8):
     assert mm(fp8, ldd=100) == E.FP8_ERR_INVALID_ARG
     assert mm(fp8, bias=A, bias_dtype=E.FP8_DT_E4M3) == E.FP8_ERR_INVALID_ARG  # fp8 bias needs a scale
     assert mm(fp8, bias=A, bias_dtype=E.FP8_DT_FP32) == E.FP8_ERR_INVALID_ARG
-    assert mm(fp8, tile_cfg=4) == E.FP8_ERR_INVALID_ARG
+    assert mm(fp8, tile_cfg=5) == E.FP8_ERR_INVALID_ARG
     assert mm(fp8, tile_cfg=-1) == E.FP8_ERR_INVALID_ARG
     assert mm(fp8, m=0) == E.FP8_OK
     assert mm(fp8, k=0) == E.FP8_OK

@@ -92,7 +92,9 @@ def run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=0, fmt_b=0, sa=1.0, sb=1
 
 
 LAYOUTS = [(0, 0), (0, 1), (1, 1), (1, 0)]
-TILES = [1, 2, 3]   # 128x128, 128x256 (one CTA), 256x256 (CTA pair, 2-SM MMA)
+# 128x128, 128x256 (one CTA), 256x256 (CTA pair, 2-SM MMA), 128x128 split-K
+# over a cluster (forced: S = 2..3 by k-blocks and residency; one k-block runs unsplit)
+TILES = [1, 2, 3, 4]
 
 
 @pytest.mark.parametrize("tile", TILES)
@@ -173,7 +175,8 @@ def test_mm_long_k_accumulation(fp8, a_major, b_major, tile):
 @pytest.mark.parametrize("tile", [0] + TILES)
 @pytest.mark.parametrize("m,n,k,a_major,b_major", [
     (2048, 1024, 1024, 0, 0), (2048, 1024, 4096, 0, 1), (4096, 1024, 2048, 1, 1), (512, 6912, 1536, 0, 0),
-    (1536, 1536, 512, 1, 1), (640, 2304, 4096, 0, 0), (4096, 11008, 512, 0, 0)])
+    (1536, 1536, 512, 1, 1), (640, 2304, 4096, 0, 0), (4096, 11008, 512, 0, 0),
+    (512, 1536, 6912, 0, 0), (512, 1536, 6912, 0, 1), (512, 1536, 1536, 1, 1)])
 def test_mm_large_sampled(fp8, m, n, k, a_major, b_major, tile):
     rng = np.random.default_rng(m + n + k)
     run_case(fp8, rng, m, n, k, a_major, b_major, sa=3.0, sb=0.25, full=False, tile=tile)
@@ -188,7 +191,8 @@ def test_mm_no_device_timeouts(fp8):
 def test_mm_pair_matches_two_calls(fp8, tile):
     """fp8_mm_pair runs dX-like (K x MN-major) and dW-like (MN x MN-major) GEMMs
     of different shapes in one launch; each output equals its own fp8_mm call
-    with the same tile configuration bit for bit."""
+    with the same tile configuration bit for bit (split-K, which two-GEMM
+    launches do not use, against the 128x128 fallback)."""
     rng = np.random.default_rng(31)
     M, N, K = 700, 520, 300
     g8 = codes_like_tensor(rng, 1, (M, N), 3000.0)
@@ -221,10 +225,23 @@ def test_mm_pair_matches_two_calls(fp8, tile):
         want, _ = oracle.epilogue(gemm_dw, 3.0, 0.25)
         assert_gemm_close(dw1.cpu().view(torch.int16).numpy().view(np.uint16), want, sab, 3.0, 0.25, "pair dw")
     else:
-        a2, b2 = args(dx2, dw2, tile)
+        # a two-GEMM launch does not split K: forced split-K falls back to 128x128
+        a2, b2 = args(dx2, dw2, 1 if tile == 4 else tile)
         fp8._lib.fp8_mm(ctypes.byref(a2), torch.cuda.current_stream().cuda_stream)
         fp8._lib.fp8_mm(ctypes.byref(b2), torch.cuda.current_stream().cuda_stream)
         torch.cuda.synchronize()
         assert torch.equal(dx1.view(torch.int16), dx2.view(torch.int16))
         assert torch.equal(dw1.view(torch.int16), dw2.view(torch.int16))
     assert fp8.fp8_get_device_status() == 0
+
+
+@pytest.mark.parametrize("m,n,k,a_major,b_major", [(300, 260, 1000, 0, 0), (512, 1536, 6912, 0, 1)])
+def test_mm_split_k_deterministic(fp8, m, n, k, a_major, b_major):
+    """Split-K sums the ranks' partials in rank order, so two launches give the
+    same bits; and AUTO on a few-tile, long-K shape agrees with forced split-K
+    within the GEMM tolerance (AUTO may or may not split)."""
+    rng = np.random.default_rng(77)
+    _, y1, _ = run_case(fp8, rng, m, n, k, a_major, b_major, full=False, tile=4)
+    rng = np.random.default_rng(77)
+    _, y2, _ = run_case(fp8, rng, m, n, k, a_major, b_major, full=False, tile=4)
+    assert np.array_equal(y1, y2)

@@ -121,21 +121,21 @@ __global__ void __launch_bounds__(kRowLanes * 32) dbias_kernel(const DbiasParams
   }
   #pragma unroll
   for (int j = 0; j < 8; ++j) red[ty][tx * 8 + j] = acc[j];
-  __syncthreads();
+  cta_sync();
 
   const int64_t col = c_base + threadIdx.x;
   float s = 0.0f;
   #pragma unroll
   for (int y = 0; y < kRowLanes; ++y) s += red[y][threadIdx.x];
   if (col < p.N) p.partial[static_cast<int64_t>(blockIdx.y) * p.N + col] = s;
-  __syncthreads();
+  cta_sync();
   if (threadIdx.x == 0) {
     // the barrier above ordered every thread's partial before this fence
     __threadfence();
     last = atomicAdd(&p.counters[blockIdx.x], 1u) == static_cast<unsigned>(p.R - 1);
     if (last) __threadfence();
   }
-  __syncthreads();
+  cta_sync();
   if (!last) return;
   if (col < p.N)
     static_cast<__nv_bfloat16*>(p.dbias)[col] = __float2bfloat16_rn(sum_partials(p.partial + col, p.N, p.R));

@@ -263,9 +263,17 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
+// CTA and cluster barriers in their non-.aligned forms, which count threads
+// one by one.  In the warp-specialized GEMM one lane of a warp runs the
+// producer or MMA loop while its other lanes go ahead (timestamps on a B200
+// show them reaching the teardown barrier ~0.7 us apart); the .aligned forms
+// (what __syncthreads() emits) require the whole warp at the instruction
+// together and leave that to the compiler's reconvergence, the non-.aligned
+// forms are correct whatever the arrival order.
 __device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
+__device__ __forceinline__ void cta_sync() { asm volatile("barrier.sync 0;" ::: "memory"); }
 // 16-byte store into the shared memory of a CTA of the cluster (an address
 // from mapa_shared).
 __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float4 v) {

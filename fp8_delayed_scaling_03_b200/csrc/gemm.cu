@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (kPair) {
     cluster_sync();  // both CTAs' barriers exist before either signals the other
   } else {
-    __syncthreads();
+    cta_sync();
     // Split-K: the first remote access comes at the end of the mainloop, so
     // the cluster barrier's wait (every CTA's barriers initialized) is taken
     // there (epilogue) or at teardown (the other warps), not here.
@@ -532,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   if constexpr (kPair || kSplit) cluster_sync();  // no CTA leaves while another still signals or reads it
-  else __syncthreads();
+  else cta_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

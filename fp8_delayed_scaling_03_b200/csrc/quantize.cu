@@ -197,7 +197,7 @@ __device__ __forceinline__ void ring_tail(const QuantizeParams& p, uint32_t bits
 __device__ __forceinline__ uint32_t block_max_bits(float amax, uint32_t* warp_max) {
   uint32_t bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
   if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = bits;
-  __syncthreads();
+  cta_sync();
   #pragma unroll
   for (int w = 0; w < kThreads / 32; ++w) bits = max(bits, warp_max[w]);
   return bits;
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   #pragma unroll
   for (int j = 0; j < 16; j += 4)
     *reinterpret_cast<float4*>(&red[rl][cl * kChunk + j]) = make_float4(csum[j], csum[j + 1], csum[j + 2], csum[j + 3]);
-  const uint32_t bits = block_max_bits(amax, warp_max);  // includes __syncthreads
+  const uint32_t bits = block_max_bits(amax, warp_max);  // includes a CTA barrier
   const int64_t ccol = static_cast<int64_t>(blockIdx.x) * kColTile + threadIdx.x;
   float part = 0.0f;
   #pragma unroll
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
     if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
     return;
   }
-  __syncthreads();
+  cta_sync();
   // Two independent tails run side by side: thread 0 the ring's, thread 32
   // the column tile's ticket.
   if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
     last_tile = atomicAdd(&cp.counters[blockIdx.x], 1u) == gridDim.y - 1;
     if (last_tile) __threadfence();
   }
-  __syncthreads();
+  cta_sync();
   if (!last_tile) return;
   if (ccol < p.cols)
     static_cast<__nv_bfloat16*>(cp.dbias)[ccol] =

@@ -199,6 +199,31 @@ class Ring:
         return self.scale
 
 
+def dynamic_scale(amax_value: float, fmt: int) -> np.float32:
+    """Current (dynamic) scaling, the pages' alternative to the ring (AstrAI
+    commits: astrai @4019dda, recipe bullet -- one recipe with a dynamic flag;
+    astrai/extension/fp8.py @3e57cc8, DynamicScaling bullet -- no rings, the
+    scale measured inline): the scale of a tensor is fp8_max / its own amax,
+    one fp32 IEEE division, and 1.0 when amax is 0, not finite, or the
+    quotient overflows (the ring's keep rule with 1.0 as the kept scale)."""
+    a = np.float32(amax_value)
+    if not (np.isfinite(a) and a > 0):
+        return np.float32(1.0)
+    with np.errstate(over="ignore"):
+        q = np.float32(np.float32(FP8_MAX[fmt]) / a)
+    return q if np.isfinite(q) else np.float32(1.0)
+
+
+def quantize_dynamic(x: np.ndarray, dtype: int, fmt: int, cols: int | None = None,
+                     ld_out: int | None = None):
+    """Quantize with the tensor's own scale: amax over the raw input first, then
+    s = dynamic_scale(amax), then the same cast.  Returns (codes, amax, s)."""
+    a = amax(x, dtype, cols)
+    s = dynamic_scale(a, fmt)
+    q = quantize_codes(x, dtype, fmt, s, cols, ld_out)
+    return q, a, s
+
+
 def quantize(x: np.ndarray, dtype: int, fmt: int, ring: Ring, cols: int | None = None,
              ld_out: int | None = None):
     """One quantize launch as the pages define it: read the ring's current scale
@@ -296,15 +321,18 @@ def _operand(t, dtype, fmt, ring, scale_in, cols, ld8):
     if dtype in (DT_E4M3, DT_E5M2):
         assert (dtype - DT_E4M3) == fmt, "pre-quantized operand must match fmt"
         return np.ascontiguousarray(t), np.float32(0.0), np.float32(scale_in)
+    if ring is None:  # current (dynamic) scaling
+        return quantize_dynamic(t, dtype, fmt, cols=cols, ld_out=ld8)
     q, a, s = quantize(t, dtype, fmt, ring, cols=cols, ld_out=ld8)
     return q, a, s
 
 
-def linear_forward(M, N, K, x, x_dtype, w, w_dtype, ring_x: Ring, ring_w: Ring,
+def linear_forward(M, N, K, x, x_dtype, w, w_dtype, ring_x: Ring | None, ring_w: Ring | None,
                    fmt_x=E4M3, fmt_w=E4M3, bias=None, bias_dtype=DT_BF16, bias_scale=1.0,
                    x_scale_in=1.0, w_scale_in=1.0, ldx8=None, ldw8=None, sumabs=True):
-    """Forward of the FP8 linear: quantize x and w (each with its own ring, or
-    skipped when pre-quantized), then Y = bf16(X8 W8^T / (sx sw) + bias).
+    """Forward of the FP8 linear: quantize x and w (each with its own ring,
+    with its own amax when the ring is None, or skipped when pre-quantized),
+    then Y = bf16(X8 W8^T / (sx sw) + bias).
     Returns a dict with y (bf16 bits), x8, w8, the scale snapshots sx, sw, the
     amaxes, the fp32 accumulator and sum|ab|."""
     x8, ax, sx = _operand(x, x_dtype, fmt_x, ring_x, x_scale_in, K, ldx8)
@@ -314,7 +342,7 @@ def linear_forward(M, N, K, x, x_dtype, w, w_dtype, ring_x: Ring, ring_w: Ring,
     return dict(y=y, y_f32=yf, x8=x8, w8=w8, sx=sx, sw=sw, amax_x=ax, amax_w=aw, acc=acc, sumabs=sab)
 
 
-def linear_backward(M, N, K, g, g_dtype, ring_g: Ring, x8, fmt_x, sx, w8, fmt_w, sw,
+def linear_backward(M, N, K, g, g_dtype, ring_g: Ring | None, x8, fmt_x, sx, w8, fmt_w, sw,
                     fmt_g=E5M2, g_scale_in=1.0, ldg8=None, need_dx=True, need_dw=True,
                     need_dbias=False, sumabs=True):
     """Backward: quantize g with its ring (E5M2; skipped when pre-quantized),

@@ -534,6 +534,82 @@ def test_no_scale_ratio_leak():
         assert 0.8 < ratio < 1.2, (step, ratio)
 
 
+# ---------------------------------------------------------------- dynamic (current) scaling
+
+def test_dynamic_scale_worked_values():
+    """amax 3.5 -> s = 448 / 3.5 = 128 exactly; codes of +-3.5, 1.75, 0.5
+    are the grid points 448, 224, 64 (all exact powers-of-two multiples)."""
+    x = torch.tensor([[3.5, -3.5, 1.75, 0.5, 0.0, -0.0]], dtype=torch.bfloat16)
+    q, a, s = oracle.quantize_dynamic(_bits(x), DT_BF16, E4M3)
+    assert a == np.float32(3.5) and s == np.float32(128.0)
+    v = oracle.decode(E4M3, q[0])
+    assert list(v[:5]) == [448.0, -448.0, 224.0, 64.0, 0.0] and np.signbit(v[5])
+    q5, a5, s5 = oracle.quantize_dynamic(_bits(x), DT_BF16, E5M2)
+    assert s5 == np.float32(57344.0 / 3.5)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_dynamic_scale_maps_amax_to_fp8_max(fmt):
+    """The element of largest magnitude lands on the format's largest finite
+    code (fp32 rounding of x*s can only nudge it to the saturated maximum)."""
+    rng = np.random.default_rng(40 + fmt)
+    for std in (1e-3, 1.0, 300.0):
+        x = _bf16(rng.standard_normal((37, 51)) * std)
+        q, a, s = oracle.quantize_dynamic(_bits(x), DT_BF16, fmt)
+        xf = x.float().numpy()
+        i = np.unravel_index(np.argmax(np.abs(xf)), xf.shape)
+        assert abs(oracle.decode(fmt, q[i[0], i[1]:i[1] + 1])[0]) == FP8_MAX[fmt]
+        assert a == np.float32(np.abs(xf).max())
+        # every other code stays inside the grid (no saturation beyond amax)
+        assert np.all(np.abs(oracle.decode(fmt, q)) <= FP8_MAX[fmt])
+
+
+def test_dynamic_scale_keep_rules():
+    """amax 0 (all zeros / all NaN), inf, or an overflowing quotient -> 1.0."""
+    z = np.zeros((2, 8), np.float32)
+    assert oracle.quantize_dynamic(z, DT_FP32, E4M3)[2] == 1.0
+    n = np.full((2, 8), np.nan, np.float32)
+    qn, an, sn = oracle.quantize_dynamic(n, DT_FP32, E4M3)
+    assert an == 0.0 and sn == 1.0 and np.all((qn & 0x7F) == 0x7F)
+    inf = np.array([[1.0, np.inf]], np.float32)
+    assert oracle.quantize_dynamic(inf, DT_FP32, E5M2)[2] == 1.0
+    tiny = np.array([[1e-40, 0.0]], np.float32)  # 57344 / 1e-40 overflows fp32
+    assert oracle.quantize_dynamic(tiny, DT_FP32, E5M2)[2] == 1.0
+
+
+def test_dynamic_linear_has_no_saturation_and_no_ring():
+    """With ring None the forward uses each operand's own amax: unlike the
+    delayed path's first step (scale 1, x ~ 2^step saturating), no element
+    saturates except at the amax, and Y tracks the float64 GEMM."""
+    rng = np.random.default_rng(41)
+    M, N, K = 64, 192, 128
+    x = _bf16(rng.standard_normal((M, K)) * 1e3)
+    w = _bf16(rng.standard_normal((N, K)) * 0.02)
+    f = oracle.linear_forward(M, N, K, _bits(x), DT_BF16, _bits(w), DT_BF16, None, None)
+    assert f["sx"] == oracle.dynamic_scale(f["amax_x"], E4M3)
+    assert f["sw"] == oracle.dynamic_scale(f["amax_w"], E4M3)
+    # codes at the maximum come only from |x| s at or above 432, the midpoint
+    # to the next grid value 416 (RNE), never from saturation of larger values
+    sat = np.abs(oracle.decode(E4M3, f["x8"])) == 448.0
+    prod = (np.abs(x.float().numpy()) * f["sx"]).astype(np.float32)
+    assert sat.any() and np.all(prod[sat] >= 432.0) and np.all(prod <= np.float32(448.0) * (1 + 2.0 ** -23))
+    y = oracle.bf16_to_f32(f["y"]).astype(np.float64)
+    ref = x.double().numpy() @ w.double().numpy().T
+    assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.1
+
+
+def test_mutant_dynamic_scale_from_quantized_max_is_caught():
+    """A dynamic path that measured amax after a scale-1 cast (saturating at
+    448) would give s = 1 for |x| >> 448: the worked-value pin above rejects
+    any s other than fp8_max / raw amax."""
+    x = torch.tensor([[5000.0, 1.0]], dtype=torch.bfloat16)
+    raw = oracle.amax(_bits(x), DT_BF16)
+    q1 = oracle.quantize_codes(_bits(x), DT_BF16, E4M3, np.float32(1.0))
+    wrong = oracle.dynamic_scale(np.abs(oracle.decode(E4M3, q1)).max(), E4M3)
+    assert wrong != oracle.quantize_dynamic(_bits(x), DT_BF16, E4M3)[2]
+    assert oracle.quantize_dynamic(_bits(x), DT_BF16, E4M3)[2] == np.float32(448.0) / raw
+
+
 # ---------------------------------------------------------------- mutants
 
 def test_mutant_window_without_current_amax_is_caught():

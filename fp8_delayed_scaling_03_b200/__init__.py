@@ -303,15 +303,16 @@ class ScaleRing:
         return self.buf.view(torch.int32)
 
 
-def quantize(x: torch.Tensor, fmt: int, ring: ScaleRing, out: torch.Tensor | None = None):
-    """Quantize x with its ring; returns (codes [rows, cols] uint8 view with a
-    16-aligned row stride, amax (1-elem fp32), scale used (1-elem fp32))."""
+def quantize(x: torch.Tensor, fmt: int, ring: ScaleRing | None, out: torch.Tensor | None = None):
+    """Quantize x with its ring (ring None: current scaling from x's own amax);
+    returns (codes [rows, cols] uint8 view with a 16-aligned row stride, amax
+    (1-elem fp32), scale used (1-elem fp32))."""
     rows, cols = x.shape
     if out is None:
         out = fp8_alloc(rows, cols, x.device)
     amax = torch.empty(1, dtype=torch.float32, device=x.device)
     scale = torch.empty(1, dtype=torch.float32, device=x.device)
-    fp8_quantize(x, fmt, ring.buf, ring.H, out, amax, scale)
+    fp8_quantize(x, fmt, ring.buf if ring is not None else None, ring.H if ring is not None else 0, out, amax, scale)
     return out, amax, scale
 
 

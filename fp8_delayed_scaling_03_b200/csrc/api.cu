@@ -305,6 +305,24 @@ QuantizeParams make_qparams(const void* in, int in_dtype, int64_t rows, int64_t 
   return p;
 }
 
+// Current scaling's first pass for the ring-less ones of a and b (either may
+// be NULL): zero each one's amax_out, point its dyn_amax there, and reduce
+// max |x| into it in one launch.
+int amax_pass(int in_dtype, QuantizeParams* a, QuantizeParams* b, cudaStream_t st) {
+  const QuantizeParams* d[2] = {nullptr, nullptr};
+  int n = 0;
+  for (QuantizeParams* q : {a, b}) {
+    if (!q || q->ring) continue;
+    q->dyn_amax = q->amax_out;
+    cudaError_t e = cudaMemsetAsync(q->amax_out, 0, sizeof(float), st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    d[n++] = q;
+  }
+  if (n == 0) return FP8_OK;
+  cudaError_t e = launch_amax(in_dtype, d[0], d[1], st);
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
 // defer: leave the ring's finalize to the GEMM launch that follows (which
 // must then list the ring in its RingFinalize set).
 int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt, void* ring,
@@ -312,7 +330,9 @@ int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
                  bool defer = false) {
   QuantizeParams p =
       make_qparams(in, in_dtype, rows, cols, ld_in, fmt, ring, H, out, ld_out, amax_out, scale_out, true);
-  p.defer_finalize = defer ? 1 : 0;
+  p.defer_finalize = defer && ring ? 1 : 0;
+  int s = amax_pass(in_dtype, &p, nullptr, st);
+  if (s) return s;
   cudaError_t e = launch_quantize(in_dtype, fmt, &p, nullptr, st);
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
@@ -325,7 +345,9 @@ int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace,
   std::memset(&cp, 0, sizeof(cp));
   cp.q = make_qparams(g.in, g.in_dtype, g.rows, g.cols, g.ld_in, g.fmt, g.ring, g.hist_len, g.out, g.ld_out,
                       g.amax_out, g.scale_out, false);
-  cp.q.defer_finalize = defer ? 1 : 0;
+  cp.q.defer_finalize = defer && g.ring ? 1 : 0;
+  int s = amax_pass(g.in_dtype, &cp.q, nullptr, st);
+  if (s) return s;
   dbias_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
   cp.partial = static_cast<float*>(workspace);
   const size_t part = (static_cast<size_t>(cp.R) * static_cast<size_t>(g.cols) * 4u + 15u) & ~size_t(15);
@@ -337,13 +359,19 @@ int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace,
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
 
+// ring NULL selects current scaling, which reduces the amax into *amax_out
+// (required then).
 int validate_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt,
-                      void* ring, int H, uint8_t* out, int64_t ld_out) {
+                      void* ring, int H, uint8_t* out, int64_t ld_out, const float* amax_out) {
   if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
   if (!is_wide(in_dtype) || !is_fmt(fmt)) return FP8_ERR_INVALID_ARG;
-  if (!ring_len_ok(H)) return FP8_ERR_INVALID_ARG;
-  if (!in || !ring || !out) return FP8_ERR_INVALID_ARG;
-  if (!aligned(ring, 4) || !aligned(in, esize(in_dtype))) return FP8_ERR_INVALID_ARG;
+  if (!in || !out) return FP8_ERR_INVALID_ARG;
+  if (ring) {
+    if (!ring_len_ok(H) || !aligned(ring, 4)) return FP8_ERR_INVALID_ARG;
+  } else if (!amax_out || !aligned(amax_out, 4)) {
+    return FP8_ERR_INVALID_ARG;
+  }
+  if (!aligned(in, esize(in_dtype))) return FP8_ERR_INVALID_ARG;
   if (ld_in < cols) return FP8_ERR_INVALID_ARG;
   return check_fp8_matrix(out, ld_out, cols);
 }
@@ -390,7 +418,7 @@ int fp8_ring_seed(void* ring, int hist_len, int fmt, float amax, fp8_stream_t st
 int fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt, void* ring,
                  int hist_len, uint8_t* out, int64_t ld_out, float* amax_out, float* scale_out,
                  fp8_stream_t stream) {
-  int s = validate_quantize(in, in_dtype, rows, cols, ld_in, fmt, ring, hist_len, out, ld_out);
+  int s = validate_quantize(in, in_dtype, rows, cols, ld_in, fmt, ring, hist_len, out, ld_out, amax_out);
   if (s) return s;
   if (rows == 0 || cols == 0) return FP8_OK;
   return run_quantize(in, in_dtype, rows, cols, ld_in, fmt, ring, hist_len, out, ld_out, amax_out, scale_out,
@@ -400,12 +428,13 @@ int fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
 int fp8_quantize_dual(const fp8_quantize_args* a, const fp8_quantize_args* b, fp8_stream_t stream) {
   if (!a || !b) return FP8_ERR_INVALID_ARG;
   int s = validate_quantize(a->in, a->in_dtype, a->rows, a->cols, a->ld_in, a->fmt, a->ring, a->hist_len, a->out,
-                            a->ld_out);
+                            a->ld_out, a->amax_out);
   if (s) return s;
   s = validate_quantize(b->in, b->in_dtype, b->rows, b->cols, b->ld_in, b->fmt, b->ring, b->hist_len, b->out,
-                        b->ld_out);
+                        b->ld_out, b->amax_out);
   if (s) return s;
-  if (a->in_dtype != b->in_dtype || a->fmt != b->fmt || a->ring == b->ring) return FP8_ERR_INVALID_ARG;
+  if (a->in_dtype != b->in_dtype || a->fmt != b->fmt || (a->ring && a->ring == b->ring)) return FP8_ERR_INVALID_ARG;
+  if (!a->ring && !b->ring && a->amax_out == b->amax_out) return FP8_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool ea = a->rows == 0 || a->cols == 0, eb = b->rows == 0 || b->cols == 0;
   if (ea && eb) return FP8_OK;
@@ -414,10 +443,11 @@ int fp8_quantize_dual(const fp8_quantize_args* a, const fp8_quantize_args* b, fp
     return run_quantize(o->in, o->in_dtype, o->rows, o->cols, o->ld_in, o->fmt, o->ring, o->hist_len, o->out,
                         o->ld_out, o->amax_out, o->scale_out, st);
   }
-  const QuantizeParams qa = make_qparams(a->in, a->in_dtype, a->rows, a->cols, a->ld_in, a->fmt, a->ring, a->hist_len,
-                                         a->out, a->ld_out, a->amax_out, a->scale_out, true);
-  const QuantizeParams qb = make_qparams(b->in, b->in_dtype, b->rows, b->cols, b->ld_in, b->fmt, b->ring, b->hist_len,
-                                         b->out, b->ld_out, b->amax_out, b->scale_out, true);
+  QuantizeParams qa = make_qparams(a->in, a->in_dtype, a->rows, a->cols, a->ld_in, a->fmt, a->ring, a->hist_len,
+                                   a->out, a->ld_out, a->amax_out, a->scale_out, true);
+  QuantizeParams qb = make_qparams(b->in, b->in_dtype, b->rows, b->cols, b->ld_in, b->fmt, b->ring, b->hist_len,
+                                   b->out, b->ld_out, b->amax_out, b->scale_out, true);
+  if ((s = amax_pass(a->in_dtype, &qa, &qb, st))) return s;
   cudaError_t e = launch_quantize(a->in_dtype, a->fmt, &qa, &qb, st);
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
@@ -426,7 +456,7 @@ int fp8_quantize_dbias(const fp8_quantize_args* g, void* dbias, void* workspace,
                        fp8_stream_t stream) {
   if (!g) return FP8_ERR_INVALID_ARG;
   int s = validate_quantize(g->in, g->in_dtype, g->rows, g->cols, g->ld_in, g->fmt, g->ring, g->hist_len, g->out,
-                            g->ld_out);
+                            g->ld_out, g->amax_out);
   if (s) return s;
   if (g->rows > kMaxDim || g->cols > kMaxDim) return FP8_ERR_INVALID_ARG;
   if (!dbias || !aligned(dbias, 2)) return FP8_ERR_INVALID_ARG;
@@ -520,17 +550,18 @@ int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
     if (a->x_dtype - FP8_DT_E4M3 != a->fmt_x || !a->x_scale_in) return FP8_ERR_INVALID_ARG;
     if ((s = check_fp8_matrix(a->x, a->ldx, K))) return s;
   } else if ((s = validate_quantize(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8,
-                                    a->ldx8))) {
+                                    a->ldx8, a->amax_x_out))) {
     return s;
   }
   if (wq) {
     if (a->w_dtype - FP8_DT_E4M3 != a->fmt_w || !a->w_scale_in) return FP8_ERR_INVALID_ARG;
     if ((s = check_fp8_matrix(a->w, a->ldw, K))) return s;
   } else if ((s = validate_quantize(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8,
-                                    a->ldw8))) {
+                                    a->ldw8, a->amax_w_out))) {
     return s;
   }
-  if (!xq && !wq && a->ring_x == a->ring_w) return FP8_ERR_INVALID_ARG;
+  if (!xq && !wq && a->ring_x && a->ring_x == a->ring_w) return FP8_ERR_INVALID_ARG;
+  if (!xq && !wq && !a->ring_x && !a->ring_w && a->amax_x_out == a->amax_w_out) return FP8_ERR_INVALID_ARG;
   const uint8_t* x8 = xq ? static_cast<const uint8_t*>(a->x) : a->x8;
   const uint8_t* w8 = wq ? static_cast<const uint8_t*>(a->w) : a->w8;
   MmCall c{M, N, K, x8, a->fmt_x, FP8_K_MAJOR, xq ? a->ldx : a->ldx8, w8, a->fmt_w, FP8_K_MAJOR,
@@ -548,15 +579,17 @@ int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
   // waits for them to complete anyway, finishes both ring steps.
   RingFinalize fin[2];
   int nfin = 0;
-  if (!xq) fin[nfin++] = ring_fin(a->ring_x, a->hist_len, a->fmt_x, a->amax_x_out);
-  if (!wq) fin[nfin++] = ring_fin(a->ring_w, a->hist_len, a->fmt_w, a->amax_w_out);
+  if (!xq && a->ring_x) fin[nfin++] = ring_fin(a->ring_x, a->hist_len, a->fmt_x, a->amax_x_out);
+  if (!wq && a->ring_w) fin[nfin++] = ring_fin(a->ring_w, a->hist_len, a->fmt_w, a->amax_w_out);
   if (!xq && !wq && a->x_dtype == a->w_dtype && a->fmt_x == a->fmt_w) {
     // x and w in one launch
     QuantizeParams qx = make_qparams(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8,
                                      a->ldx8, a->amax_x_out, a->sx_out, true);
     QuantizeParams qw = make_qparams(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8,
                                      a->ldw8, a->amax_w_out, a->sw_out, true);
-    qx.defer_finalize = qw.defer_finalize = 1;
+    qx.defer_finalize = a->ring_x ? 1 : 0;
+    qw.defer_finalize = a->ring_w ? 1 : 0;
+    if ((s = amax_pass(a->x_dtype, &qx, &qw, st))) return s;
     cudaError_t e = launch_quantize(a->x_dtype, a->fmt_x, &qx, &qw, st);
     if (e != cudaSuccess) return cuda_fail(e);
   } else {
@@ -583,7 +616,7 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
     if (a->g_dtype - FP8_DT_E4M3 != a->fmt_g || !a->g_scale_in) return FP8_ERR_INVALID_ARG;
     if ((s = check_fp8_matrix(a->g, a->ldg, N))) return s;
   } else if ((s = validate_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8,
-                                    a->ldg8))) {
+                                    a->ldg8, a->amax_g_out))) {
     return s;
   }
   const uint8_t* g8 = gq ? static_cast<const uint8_t*>(a->g) : a->g8;
@@ -615,7 +648,7 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   RingFinalize fin[1];
   int nfin = 0;
   DbiasFinish dbf{};
-  if (!gq && gemm_follows) fin[nfin++] = ring_fin(a->ring_g, a->hist_len, a->fmt_g, a->amax_g_out);
+  if (!gq && gemm_follows && a->ring_g) fin[nfin++] = ring_fin(a->ring_g, a->hist_len, a->fmt_g, a->amax_g_out);
   if (gq) {
     side.copy_src[0] = a->g_scale_in; side.copy_dst[0] = a->sg_out; side.zero_dst[0] = a->amax_g_out;
     side_pending = true;

@@ -33,6 +33,8 @@ struct QuantizeParams {
   int vec_ok;                 // 16-byte vector loads are legal for full chunks
   int defer_finalize;         // 1: only fold block maxima into the ring's scratch
                               // word; the GEMM that consumes the output finalizes
+  const float* dyn_amax;      // current scaling: ring unused, s = fp8_max / *dyn_amax
+                              // (the amax pass reduced it there before this launch)
 };
 
 // One or two tensors quantized by one launch: blocks [0, blocks0) work on
@@ -135,6 +137,9 @@ int num_sms(int device);
 // b may be NULL (one tensor); both tensors share in_dtype and fmt.
 cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, const QuantizeParams* b, cudaStream_t s);
 cudaError_t launch_quantize_colsum(int in_dtype, int fmt, const ColsumParams& cp, cudaStream_t s);
+// Current scaling's first pass: max |x| of one or two tensors (b may be NULL)
+// reduced into each one's dyn_amax word, which must be zero beforehand.
+cudaError_t launch_amax(int in_dtype, const QuantizeParams* a, const QuantizeParams* b, cudaStream_t s);
 cudaError_t launch_ring_set(float* ring, int H, float scale, cudaStream_t s);
 cudaError_t launch_side_writes(const SideWrites& w, cudaStream_t s);
 // GEMM tile configurations: 128x128 and 128x256 on one CTA, 256x256 on a pair

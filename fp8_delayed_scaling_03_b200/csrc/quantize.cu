@@ -181,6 +181,13 @@ __device__ __forceinline__ void ring_finalize(const QuantizeParams& p, uint32_t 
   if (p.amax_out) *p.amax_out = a;
 }
 
+// The scale a launch multiplies by: the ring's current scale (delayed), or
+// fp8_max / this tensor's amax (current scaling; 1.0 when amax is 0 or not
+// finite or the quotient overflows -- the ring's keep rule with 1.0 kept).
+__device__ __forceinline__ float scale_of(const QuantizeParams& p) {
+  return p.dyn_amax ? next_scale(1.0f, *p.dyn_amax, p.fp8_max) : p.ring[p.H];
+}
+
 // Thread 0's end of a block: with a deferred finalize only the block's max
 // goes to the ring's scratch word (the consuming GEMM, which starts reading
 // only after this grid completed, finishes the step); else the last-block
@@ -220,14 +227,15 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_cons
   const uint32_t bid = second ? blockIdx.x - pair.blocks0 : blockIdx.x;
   const uint32_t nblocks = second ? gridDim.x - pair.blocks0 : pair.blocks0;
 
-  const float s = p.ring[p.H];
+  const float s = scale_of(p);
+  const bool ring_step = p.ring && !p.defer_finalize;  // this launch finalizes the ring
   uint32_t step = 0;
   if (threadIdx.x == 0) {
-    if (!p.defer_finalize) step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
+    if (ring_step) step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
     if (bid == 0 && p.scale_out) *p.scale_out = s;
   }
   // Only the tensor's last block writes its ring, after every block read it.
-  if (!p.defer_finalize && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
+  if (ring_step && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
 
   float amax = 0.0f;
   const int64_t stride = static_cast<int64_t>(nblocks) * kThreads;
@@ -271,8 +279,51 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_cons
     c = cn;
   }
 
+  if (!p.ring) return;  // current scaling: amax was reduced by the amax pass
   const uint32_t bits = block_max_bits(amax, warp_max);
   if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
+}
+
+// ---------------------------------------------------------------- amax pass
+
+// Current scaling's first pass: the same chunk walk as the quantize, max |x|
+// only (NaN ignored), one red.max per block into the tensor's dyn_amax word.
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 4) amax_kernel(const __grid_constant__ QuantizePair pair) {
+  __shared__ uint32_t warp_max[kThreads / 32];
+  constexpr int U = unroll_for(sizeof(T));
+  pdl_wait();
+  pdl_trigger();
+  const bool second = blockIdx.x >= pair.blocks0;
+  const QuantizeParams& p = second ? pair.t[1] : pair.t[0];
+  const uint32_t bid = second ? blockIdx.x - pair.blocks0 : blockIdx.x;
+  const uint32_t nblocks = second ? gridDim.x - pair.blocks0 : pair.blocks0;
+  float amax = 0.0f;
+  const int64_t stride = static_cast<int64_t>(nblocks) * kThreads;
+  #pragma unroll 1
+  for (int64_t c = static_cast<int64_t>(bid) * kThreads + threadIdx.x; c < p.total_chunks; c += U * stride) {
+    Raw<T> raw[U];
+    #pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t cu = c + u * stride;
+      if (cu < p.total_chunks) {
+        int64_t r, col;
+        chunk_pos(p, cu, r, col);
+        load_raw<T>(p, r, col, raw[u]);
+      }
+    }
+    #pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (c + u * stride < p.total_chunks) {
+        float v[16];
+        to_floats<T>(raw[u], v);
+        #pragma unroll
+        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+      }
+    }
+  }
+  const uint32_t bits = block_max_bits(amax, warp_max);
+  if (threadIdx.x == 0 && bits) red_max_u32(reinterpret_cast<uint32_t*>(const_cast<float*>(p.dyn_amax)), bits);
 }
 
 // ---------------------------------------------------------------- column-sum kernel
@@ -294,13 +345,14 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   const QuantizeParams& p = cp.q;
   const uint32_t nblocks = gridDim.x * gridDim.y;
   const uint32_t bid = blockIdx.y * gridDim.x + blockIdx.x;
-  const float s = p.ring[p.H];
+  const float s = scale_of(p);
+  const bool ring_step = p.ring && !p.defer_finalize;
   uint32_t step = 0;
   if (threadIdx.x == 0) {
-    if (!p.defer_finalize) step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
+    if (ring_step) step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
     if (bid == 0 && p.scale_out) *p.scale_out = s;
   }
-  if (!p.defer_finalize && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
+  if (ring_step && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
 
   const int cl = threadIdx.x % kChunkLanes;
   const int rl = threadIdx.x / kChunkLanes;
@@ -341,13 +393,13 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   for (int y = 0; y < kRowLanes; ++y) part += red[y][threadIdx.x];
   if (ccol < p.cols) cp.partial[static_cast<int64_t>(blockIdx.y) * p.cols + ccol] = part;
   if (cp.defer_sum) {  // the GEMM that follows sums the partials
-    if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
+    if (threadIdx.x == 0 && p.ring) ring_tail(p, bits, nblocks, s, step, hist_s);
     return;
   }
   cta_sync();
   // Two independent tails run side by side: thread 0 the ring's, thread 32
   // the column tile's ticket.
-  if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
+  if (threadIdx.x == 0 && p.ring) ring_tail(p, bits, nblocks, s, step, hist_s);
   if (threadIdx.x == 32) {
     // the barrier above ordered every thread's partial before this fence
     __threadfence();
@@ -413,14 +465,14 @@ cudaError_t launch_cs(const ColsumParams& cp, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, const QuantizeParams* b,
-                            cudaStream_t s) {
+// One or two tensors over one resident wave of blocks, shared in proportion to
+// their chunks; returns the grid size.
+static int make_pair(const QuantizeParams* a, const QuantizeParams* b, QuantizePair* pair) {
   int dev = 0;
   cudaGetDevice(&dev);
   const int sms = num_sms(dev);
-  QuantizePair pair;
-  pair.t[0] = *a;
-  pair.t[1] = b ? *b : *a;
+  pair->t[0] = *a;
+  pair->t[1] = b ? *b : *a;
   int64_t g0 = blocks_for(*a, sms);
   int64_t g1 = b ? blocks_for(*b, sms) : 0;
   const int64_t cap = static_cast<int64_t>(sms) * kBlocksPerSm;  // one resident wave
@@ -430,8 +482,14 @@ cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, cons
     g0 = g0 < 1 ? 1 : (g0 > cap - 1 ? cap - 1 : g0);
     g1 = cap - g0;
   }
-  pair.blocks0 = static_cast<int>(g0);
-  const int grid = static_cast<int>(g0 + g1);
+  pair->blocks0 = static_cast<int>(g0);
+  return static_cast<int>(g0 + g1);
+}
+
+cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, const QuantizeParams* b,
+                            cudaStream_t s) {
+  QuantizePair pair;
+  const int grid = make_pair(a, b, &pair);
   if (fmt == kE4M3) {
     if (in_dtype == kBF16) return launch_q<__nv_bfloat16, kE4M3>(pair, grid, s);
     if (in_dtype == kFP16) return launch_q<__half, kE4M3>(pair, grid, s);
@@ -440,6 +498,14 @@ cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, cons
   if (in_dtype == kBF16) return launch_q<__nv_bfloat16, kE5M2>(pair, grid, s);
   if (in_dtype == kFP16) return launch_q<__half, kE5M2>(pair, grid, s);
   return launch_q<float, kE5M2>(pair, grid, s);
+}
+
+cudaError_t launch_amax(int in_dtype, const QuantizeParams* a, const QuantizeParams* b, cudaStream_t s) {
+  QuantizePair pair;
+  const int grid = make_pair(a, b, &pair);
+  if (in_dtype == kBF16) return launch_pdl(amax_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, s, pair);
+  if (in_dtype == kFP16) return launch_pdl(amax_kernel<__half>, dim3(grid), dim3(kThreads), 0, s, pair);
+  return launch_pdl(amax_kernel<float>, dim3(grid), dim3(kThreads), 0, s, pair);
 }
 
 cudaError_t launch_quantize_colsum(int in_dtype, int fmt, const ColsumParams& cp, cudaStream_t s) {

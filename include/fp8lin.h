@@ -111,9 +111,16 @@ FP8LIN_API int fp8_ring_seed(void* ring, int hist_len, int fmt, float amax, fp8_
  * quotient overflows), advances step, and rezeroes ticket and scratch.
  *   in        bf16/fp16/fp32 [rows, ld_in]            (in_dtype FP8_DT_BF16/FP16/FP32)
  *   fmt       FP8_E4M3 (max 448) or FP8_E5M2 (max 57344)
- *   ring      required; fp8_ring_bytes(hist_len) bytes, initialized
+ *   ring      fp8_ring_bytes(hist_len) bytes, initialized (delayed scaling); or
+ *             NULL for current (dynamic) scaling ([astrai@4019dda] recipe with
+ *             a dynamic flag; [astrai/extension/fp8.py@3e57cc8] DynamicScaling:
+ *             no rings, scales measured inline): a first launch reduces this
+ *             tensor's amax into *amax_out (required then; zeroed first), and
+ *             s = fp8_max / amax (1.0 when amax is 0 or not finite or the
+ *             quotient overflows); hist_len is ignored.  Reads the input twice
+ *             (the second read mostly from L2 for tensors up to ~100 MB).
  *   out       fp8 codes [rows, ld_out], ld_out % 16 == 0, 16-byte aligned
- *   amax_out  optional fp32: the amax of this launch
+ *   amax_out  optional fp32 (required when ring is NULL): the amax of this launch
  *   scale_out optional fp32: the scale this launch multiplied by (the snapshot
  *             taken before the ring overwrites it, [astrai/extension/ops@057c0d3])
  * NaN inputs give the NaN code and do not enter amax; +-inf saturate to +-max. */
@@ -133,13 +140,15 @@ typedef struct fp8_quantize_args {
 /* Two quantizes in ONE launch ([astrai@4019dda] quantize_dual: x and w of a
  * forward).  Each tensor keeps its own ring and last-block finalize, exactly
  * as two fp8_quantize calls would.  Both must share in_dtype and fmt, and use
- * different rings. */
+ * different rings.  Either ring may be NULL (current scaling, amax_out
+ * required and distinct); the amax passes of such tensors share one launch. */
 FP8LIN_API int fp8_quantize_dual(const fp8_quantize_args* a, const fp8_quantize_args* b, fp8_stream_t stream);
 
 /* fp8_quantize of g [rows, cols] plus, in the same pass over g, its column
  * sums: dbias[c] = bf16( sum_r g[r, c] ) as fp8_dbias computes them (fp32
  * sums in a fixed order).  workspace as fp8_dbias (size from
- * fp8_dbias_workspace_bytes(rows, cols), zero-filled before first use). */
+ * fp8_dbias_workspace_bytes(rows, cols), zero-filled before first use).
+ * g->ring NULL: current scaling as in fp8_quantize. */
 FP8LIN_API int fp8_quantize_dbias(const fp8_quantize_args* g, void* dbias, void* workspace, size_t workspace_bytes,
                                   fp8_stream_t stream);
 
@@ -224,7 +233,12 @@ FP8LIN_API int fp8_dbias_noalloc(const void* g, int g_dtype, int64_t M, int64_t 
  * Outputs: y (bf16 [M, ldy]); x8/w8 (fp8, kept by the caller for the
  * backward; unused when that operand arrives fp8); sx_out/sw_out (required:
  * the scales the GEMM dequantized with); amax_x_out/amax_w_out (optional).
- * 2 to 3 launches.  hist_len is the H of both rings. */
+ * A NULL ring_x / ring_w selects current scaling for that operand, as in
+ * fp8_quantize (its amax output is then required; one extra amax launch for
+ * one or both).  Inside this call a ring's step is completed by the GEMM
+ * launch, not by the quantize's last block (same ring words; one launch
+ * fewer on the critical path).  2 to 4 launches.  hist_len is the H of both
+ * rings. */
 typedef struct fp8_linear_fwd_args {
   int64_t M, N, K;
   const void* x; int x_dtype; int64_t ldx; const float* x_scale_in;
@@ -241,7 +255,8 @@ FP8LIN_API int fp8_linear_forward(const fp8_linear_fwd_args* args, fp8_stream_t 
 
 /* Backward of the FP8 linear ([astrai/extension/ops@057c0d3]):
  *   g [M, N] is bf16/fp16/fp32, quantized with ring_g (fmt_g, normally E5M2)
- *   into g8, or already fp8 (then *g_scale_in is its scale, amax_g_out = 0).
+ *   into g8 (ring_g NULL: current scaling, amax_g_out required), or already
+ *   fp8 (then *g_scale_in is its scale, amax_g_out = 0).
  *   dx = bf16( G8 W8 / (sg sw) )    [M, K]  when need_dx
  *   dw = bf16( G8^T X8 / (sg sx) )  [N, K]  when need_dw
  *   dbias = bf16( sum_m g )         [N]     when need_dbias ([astrai@4019dda]:

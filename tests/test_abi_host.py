@@ -61,7 +61,7 @@ def q(fp8, **kw):
 def test_quantize_validation(fp8):
     E = fp8
     assert q(fp8, inp=None) == E.FP8_ERR_INVALID_ARG
-    assert q(fp8, ring=None) == E.FP8_ERR_INVALID_ARG
+    assert q(fp8, ring=None) == E.FP8_ERR_INVALID_ARG                # current scaling needs amax_out
     assert q(fp8, out=None) == E.FP8_ERR_INVALID_ARG
     assert q(fp8, dt=E.FP8_DT_E4M3) == E.FP8_ERR_INVALID_ARG       # fp8 input is not quantized again
     assert q(fp8, dt=9) == E.FP8_ERR_INVALID_ARG

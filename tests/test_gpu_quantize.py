@@ -177,7 +177,8 @@ def test_quantize_dbias_entry(fp8, rows, cols):
         g = wl.normal((rows, cols), 1e-3 * (1 + 3 * step), 970 + step)
         out = fp8_buffer(rows, cols)
         db = torch.empty(cols, dtype=torch.bfloat16, device="cuda")
-        fp8.fp8_quantize_dbias(fp8.quantize_args(g.cuda(), 1, ring.buf, H, out), db, ws)
+        gd = g.cuda()  # the args hold a raw pointer: keep the tensor alive
+        fp8.fp8_quantize_dbias(fp8.quantize_args(gd, 1, ring.buf, H, out), db, ws)
         torch.cuda.synchronize()
         q, a, s = oracle.quantize(bits(g), oracle.DT_BF16, 1, orr)
         assert_codes_equal(host_rows(out), q, 1)

@@ -100,6 +100,7 @@ _SIGS = {
     "fp8_quantize_dbias": (_I, [ctypes.POINTER(QuantizeArgs), _P, _P, _SZ, _P]),
     "fp8_mm": (_I, [ctypes.POINTER(MmArgs), _P]),
     "fp8_mm_pair": (_I, [ctypes.POINTER(MmArgs), ctypes.POINTER(MmArgs), _P]),
+    "fp8_mm_batched": (_I, [ctypes.POINTER(MmArgs), _I64, _I64, _I64, _I64, _P]),
     "fp8_dbias_workspace_bytes": (_SZ, [_I64, _I64]),
     "fp8_dbias": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "fp8_dbias_noalloc": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P]),
@@ -209,6 +210,12 @@ def fp8_quantize_dbias(g: QuantizeArgs, dbias: torch.Tensor, workspace: torch.Te
 
 def fp8_mm_pair(a: MmArgs, b: MmArgs, device=None) -> None:
     _check(_lib.fp8_mm_pair(ctypes.byref(a), ctypes.byref(b), _stream(device)), "fp8_mm_pair")
+
+
+def fp8_mm_batched(a: MmArgs, batch: int, stride_a: int, stride_b: int, stride_d: int, device=None) -> None:
+    """batch GEMMs of a's shape; element strides between batches (0 shares an operand)."""
+    _check(_lib.fp8_mm_batched(ctypes.byref(a), batch, stride_a, stride_b, stride_d, _stream(device)),
+           "fp8_mm_batched")
 
 
 def fp8_mm(m, n, k, a, fmt_a, a_major, lda, b, fmt_b, b_major, ldb, scale_a, scale_b, d, ldd,

@@ -80,18 +80,23 @@ int check_fp8_matrix(const void* p, int64_t ld, int64_t cols) {
 }
 
 // 2-D tensor map with zero fill out of bounds (loads) / clipping (stores).
+// Every GEMM tensor map is 3-D: (inner, outer, batch) with a box one batch
+// deep.  An unbatched or broadcast operand has batch extent 1 (its batch
+// stride is then only formal: one matrix, rounded up to 16 bytes).
 int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-             uint64_t ld_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+             uint64_t ld_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz,
+             uint64_t batch = 1, uint64_t batch_bytes = 0) {
   EncodeTiledFn enc = encoder();
   if (!enc) {
     snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled unavailable");
     return FP8_ERR_CUDA;
   }
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+  if (batch <= 1) batch_bytes = (ld_bytes * outer + 15) / 16 * 16;
+  cuuint64_t dims[3] = {inner, outer, batch};
+  cuuint64_t strides[2] = {ld_bytes, batch_bytes};
+  cuuint32_t box[3] = {box_inner, box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -101,8 +106,10 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t 
 }
 
 // fp8 operand map: 128-byte rows of a 128 x `rows` box, 128-byte swizzle.
-int make_fp8_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_rows) {
-  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, inner, outer, ld, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+int make_fp8_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_rows,
+                 uint64_t batch = 1, uint64_t batch_stride = 0) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, inner, outer, ld, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B,
+                  batch, batch_stride);
 }
 
 struct MmCall {
@@ -113,6 +120,9 @@ struct MmCall {
   const void* bias; int bias_dtype; const float* bias_scale;
   void* d; int64_t ldd;
   int tile_cfg;
+  // batched GEMMs (fp8_mm_batched): element strides between batches; a zero
+  // operand stride shares that operand across the batch
+  int64_t batch = 1, stride_a = 0, stride_b = 0, stride_d = 0;
 };
 
 int validate_mm(const MmCall& c) {
@@ -152,7 +162,7 @@ int pick_tile(const MmCall* calls, int n, int sms, double* est_us = nullptr) {
     int64_t tiles = 0;
     double work = 0.0;
     for (int i = 0; i < n; ++i) {
-      const int64_t ti = ((calls[i].m + o.tm - 1) / o.tm) * ((calls[i].n + o.tn - 1) / o.tn);
+      const int64_t ti = ((calls[i].m + o.tm - 1) / o.tm) * ((calls[i].n + o.tn - 1) / o.tn) * calls[i].batch;
       tiles += ti;
       work += static_cast<double>(ti) * static_cast<double>((calls[i].k + 127) / 128);
     }
@@ -171,22 +181,25 @@ int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) 
   const int tile_m = cfg == kGemmPair256 ? 256 : 128;
   const int b_box_rows = cfg == kGemm256 ? 256 : 128;   // rows of B one CTA loads
   std::memset(maps, 0, 3 * sizeof(CUtensorMap));
+  const bool bcast_a = c.batch > 1 && c.stride_a == 0, bcast_b = c.batch > 1 && c.stride_b == 0;
+  const uint64_t ba = bcast_a ? 1 : static_cast<uint64_t>(c.batch), bb = bcast_b ? 1 : static_cast<uint64_t>(c.batch);
   if (c.k > 0) {
-    int s = c.a_major == FP8_K_MAJOR ? make_fp8_map(&maps[0], c.a, c.k, c.m, c.lda, 128)
-                                     : make_fp8_map(&maps[0], c.a, c.m, c.k, c.lda, 128);
+    int s = c.a_major == FP8_K_MAJOR ? make_fp8_map(&maps[0], c.a, c.k, c.m, c.lda, 128, ba, c.stride_a)
+                                     : make_fp8_map(&maps[0], c.a, c.m, c.k, c.lda, 128, ba, c.stride_a);
     if (s) return s;
-    s = c.b_major == FP8_K_MAJOR ? make_fp8_map(&maps[1], c.b, c.k, c.n, c.ldb, b_box_rows)
-                                 : make_fp8_map(&maps[1], c.b, c.n, c.k, c.ldb, 128);
+    s = c.b_major == FP8_K_MAJOR ? make_fp8_map(&maps[1], c.b, c.k, c.n, c.ldb, b_box_rows, bb, c.stride_b)
+                                 : make_fp8_map(&maps[1], c.b, c.n, c.k, c.ldb, 128, bb, c.stride_b);
     if (s) return s;
   }
   // bf16 output through TMA stores when the rows are 16-byte addressable and
   // end on a 16-byte boundary (a B200 run showed the store clipping the row
   // end at 16-byte granularity, writing up to 7 columns past n otherwise):
   // 32 x 32 boxes, 64-byte swizzle (matches the epilogue's staging layout).
-  const bool tma_store = aligned(c.d, 16) && ((c.ldd * 2) % 16 == 0) && (c.n % 8 == 0);
+  const bool tma_store = aligned(c.d, 16) && ((c.ldd * 2) % 16 == 0) && (c.n % 8 == 0) &&
+                         (c.batch <= 1 || (c.stride_d * 2) % 16 == 0);
   if (tma_store) {
     int s = make_map(&maps[2], c.d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.n, c.m, c.ldd * 2, 32, 32,
-                     CU_TENSOR_MAP_SWIZZLE_64B);
+                     CU_TENSOR_MAP_SWIZZLE_64B, static_cast<uint64_t>(c.batch), static_cast<uint64_t>(c.stride_d) * 2);
     if (s) return s;
   }
   std::memset(pr, 0, sizeof(*pr));
@@ -195,7 +208,11 @@ int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) 
   pr->k = static_cast<int>(c.k);
   pr->tiles_m = static_cast<int>((c.m + tile_m - 1) / tile_m);
   pr->tiles_n = static_cast<int>((c.n + bn - 1) / bn);
-  pr->num_tiles = pr->tiles_m * pr->tiles_n;
+  pr->num_tiles = pr->tiles_m * pr->tiles_n * static_cast<int>(c.batch);
+  pr->batch = static_cast<int>(c.batch);
+  pr->bcast_a = bcast_a ? 1 : 0;
+  pr->bcast_b = bcast_b ? 1 : 0;
+  pr->stride_d = c.stride_d;
   pr->k_blocks = static_cast<int>((c.k + 127) / 128);
   pr->raster_group = 8;
   pr->idesc = idesc_f8(c.fmt_a, c.fmt_b, c.a_major, c.b_major, tile_m, bn);
@@ -228,7 +245,8 @@ int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_
   // most SMs idle, so a cluster of S CTAs shares each tile's k-blocks.
   int split = 1;
   if (cfg == kGemmSplit128 && n != 1) cfg = kGemm128;
-  if (n == 1 && (calls[0].tile_cfg == FP8_TILE_AUTO || cfg == kGemmSplit128)) {
+  if (cfg == kGemmSplit128 && calls[0].batch > 1) cfg = kGemm128;  // batches already give the tiles
+  if (n == 1 && calls[0].batch == 1 && (calls[0].tile_cfg == FP8_TILE_AUTO || cfg == kGemmSplit128)) {
     const bool forced = cfg == kGemmSplit128;
     const int64_t tiles = ((calls[0].m + 127) / 128) * ((calls[0].n + 127) / 128);
     const int64_t kb = (calls[0].k + 127) / 128;
@@ -490,6 +508,26 @@ int fp8_mm(const fp8_mm_args* a, fp8_stream_t stream) {
   int s = validate_mm(c);
   if (s) return s;
   if (c.m == 0 || c.n == 0 || c.k == 0) return FP8_OK;
+  return run_mm(c, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fp8_mm_batched(const fp8_mm_args* a, int64_t batch, int64_t stride_a, int64_t stride_b, int64_t stride_d,
+                   fp8_stream_t stream) {
+  if (!a || batch < 0 || stride_a < 0 || stride_b < 0 || stride_d < 0) return FP8_ERR_INVALID_ARG;
+  MmCall c{a->m, a->n, a->k, a->a, a->fmt_a, a->a_major, a->lda, a->b, a->fmt_b, a->b_major, a->ldb,
+           a->scale_a, a->scale_b, a->bias, a->bias_dtype, a->bias_scale, a->d, a->ldd, a->tile_cfg,
+           batch, stride_a, stride_b, stride_d};
+  int s = validate_mm(c);
+  if (s) return s;
+  if (batch == 0 || c.m == 0 || c.n == 0 || c.k == 0) return FP8_OK;
+  if (batch > 1) {
+    // batch strides of the fp8 operands are TMA strides: multiples of 16 bytes
+    if (stride_a % 16 || stride_b % 16) return FP8_ERR_MISALIGNED;
+    // the batches' outputs must not overlap
+    if (stride_d < (c.m - 1) * c.ldd + c.n) return FP8_ERR_INVALID_ARG;
+    const int64_t tiles = ((c.m + 127) / 128) * ((c.n + 127) / 128) * batch;
+    if (tiles > (int64_t(1) << 30)) return FP8_ERR_INVALID_ARG;
+  }
   return run_mm(c, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 

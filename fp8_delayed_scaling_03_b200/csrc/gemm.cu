@@ -88,9 +88,13 @@ struct Cfg {
 // two fixed-offset parameter reads instead of one at a run-time offset.
 #define FP8_PR(f) (pi ? p.pr[1].f : p.pr[0].f)
 
-__device__ __forceinline__ int tile_coords(const GemmParams& p, int t, int& tm, int& tn) {
+__device__ __forceinline__ int tile_coords(const GemmParams& p, int t, int& tb, int& tm, int& tn) {
   const int pi = t >= p.tiles0 ? 1 : 0;
   if (pi) t -= p.tiles0;
+  // batches one after another, each with its own raster
+  const int per_batch = FP8_PR(tiles_m) * FP8_PR(tiles_n);
+  tb = t / per_batch;
+  t -= tb * per_batch;
   const int raster_group = FP8_PR(raster_group);
   const int per_group = raster_group * FP8_PR(tiles_n);
   const int g = t / per_group;
@@ -199,8 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Barrier set-up (warp 2), TMEM allocation (warp 1) and the producer's
   // first tile coordinates (warp 0) proceed side by side.
-  int first_tm = 0, first_tn = 0, first_pi = 0;
-  if (threadIdx.x == 0 && unit < p.total_tiles) first_pi = tile_coords(p, unit, first_tm, first_tn);
+  int first_tb = 0, first_tm = 0, first_tn = 0, first_pi = 0;
+  if (threadIdx.x == 0 && unit < p.total_tiles) first_pi = tile_coords(p, unit, first_tb, first_tm, first_tn);
   if (threadIdx.x == 64) {
     for (int s = 0; s < nstages; ++s) {
       mbar_init(&full[s], 1);
@@ -263,8 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool dep_done = false;
       int issued = 0;  // k-blocks loaded so far; the first kStages find their stage free
       for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
-        int tm = first_tm, tn = first_tn;
-        const int pi = t == unit ? first_pi : tile_coords(p, t, tm, tn);
+        int tb = first_tb, tm = first_tm, tn = first_tn;
+        const int pi = t == unit ? first_pi : tile_coords(p, t, tb, tm, tn);
+        const int za = FP8_PR(bcast_a) ? 0 : tb, zb = FP8_PR(bcast_b) ? 0 : tb;  // batch coordinates
         const CUtensorMap* tma_a = pi ? &ta1 : &ta0;
         const CUtensorMap* tma_b = pi ? &tb1 : &tb0;
         const int am = tm * C::kTileM + a_row0;
@@ -285,20 +290,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             // both CTAs' bytes are counted on the even CTA's full barrier
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
-            if (!a_mn) tma_load_2d_pair(a_dst, tma_a, bar, kb * kBK, am);
-            else       tma_load_2d_pair(a_dst, tma_a, bar, am, kb * kBK);
-            if (!b_mn) tma_load_2d_pair(b_dst, tma_b, bar, kb * kBK, bn0);
-            else       tma_load_2d_pair(b_dst, tma_b, bar, bn0, kb * kBK);
+            if (!a_mn) tma_load_3d_pair(a_dst, tma_a, bar, kb * kBK, am, za);
+            else       tma_load_3d_pair(a_dst, tma_a, bar, am, kb * kBK, za);
+            if (!b_mn) tma_load_3d_pair(b_dst, tma_b, bar, kb * kBK, bn0, zb);
+            else       tma_load_3d_pair(b_dst, tma_b, bar, bn0, kb * kBK, zb);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-            if (!a_mn) tma_load_2d(a_dst, tma_a, &full[stage], kb * kBK, am);
-            else       tma_load_2d(a_dst, tma_a, &full[stage], am, kb * kBK);
+            if (!a_mn) tma_load_3d(a_dst, tma_a, &full[stage], kb * kBK, am, za);
+            else       tma_load_3d(a_dst, tma_a, &full[stage], am, kb * kBK, za);
             if (!b_mn) {
-              tma_load_2d(b_dst, tma_b, &full[stage], kb * kBK, bn0);
+              tma_load_3d(b_dst, tma_b, &full[stage], kb * kBK, bn0, zb);
             } else {
               #pragma unroll
               for (int h = 0; h < C::kBRows / 128; ++h)
-                tma_load_2d(b_dst + h * 128 * kBK, tma_b, &full[stage], bn0 + h * 128, kb * kBK);
+                tma_load_3d(b_dst + h * 128 * kBK, tma_b, &full[stage], bn0 + h * 128, kb * kBK, zb);
             }
           }
           if (++stage == nstages) { stage = 0; phase ^= 1u; }
@@ -398,8 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     constexpr int kSteps = BN / 2 / kEpiCols;
     for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
-      int tm, tn;
-      const int pi = tile_coords(p, t, tm, tn);
+      int tb, tm, tn;
+      const int pi = tile_coords(p, t, tb, tm, tn);
       // The tile's constants go to registers and its bias values are fetched
       // BEFORE the wait for the accumulator, so that no parameter read and no
       // global-memory latency sits between the TMEM read and the store.
@@ -408,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool have_k = kSplit ? (static_cast<int>(rank) + 1) * FP8_PR(k_blocks) / nsplit >
                                        static_cast<int>(rank) * FP8_PR(k_blocks) / nsplit
                                  : FP8_PR(k_blocks) > 0;
-      void* const qd_ptr = FP8_PR(d);
+      void* const qd_ptr = static_cast<__nv_bfloat16*>(FP8_PR(d)) + static_cast<int64_t>(tb) * FP8_PR(stride_d);
       const int64_t ldd = FP8_PR(ldd);
       const void* const bias = FP8_PR(bias);
       const CUtensorMap* tma_d = pi ? &td1 : &td0;
@@ -500,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(tma_d, buf, col0, tm * C::kTileM + static_cast<int>(prank) * kBM + qd * 32);
+            tma_store_3d(tma_d, buf, col0, tm * C::kTileM + static_cast<int>(prank) * kBM + qd * 32, tb);
             bulk_commit();
           }
           slab ^= 1;

@@ -103,6 +103,9 @@ struct GemmProblem {
   void* d;
   int64_t ldd;
   int tma_store;              // D is addressable by TMA (16-byte aligned base, pitch and row end)
+  int batch;                  // independent GEMMs of this shape; tiles enumerate batch x tiles_m x tiles_n
+  int bcast_a, bcast_b;       // operand shared by every batch (batch stride 0): batch coordinate 0
+  int64_t stride_d;           // elements between consecutive batches of D
 };
 
 struct GemmParams {

@@ -182,6 +182,21 @@ typedef struct fp8_mm_args {
 } fp8_mm_args;
 FP8LIN_API int fp8_mm(const fp8_mm_args* args, fp8_stream_t stream);
 
+/* A batch of GEMMs of one shape in one launch ([astrai@4019dda] mm_fp8 bullet:
+ * 3-D operands through the same signature, batches sliced by strides, a
+ * size-1 batch broadcast with stride 0, transposed views folded into the
+ * layout tag at zero copy):
+ *   D_b = args applied to A_b = a + b*stride_a, B_b = b + b*stride_b,
+ *         D_b = d + b*stride_d, for b < batch (strides in ELEMENTS)
+ * stride_a / stride_b 0 shares that operand across the batch; other operand
+ * strides must be multiples of 16 bytes (FP8_ERR_MISALIGNED); stride_d >=
+ * (m - 1) * ldd + n so that outputs do not overlap (FP8_ERR_INVALID_ARG).
+ * Scales and bias are shared by the batch.  The tile configuration counts
+ * batch x per-matrix tiles; split-K is not used for batch > 1 (the batch
+ * already fills the SMs).  batch == 0 is a no-op; batch == 1 equals fp8_mm. */
+FP8LIN_API int fp8_mm_batched(const fp8_mm_args* args, int64_t batch, int64_t stride_a, int64_t stride_b,
+                              int64_t stride_d, fp8_stream_t stream);
+
 /* Two independent GEMMs in ONE launch over one persistent tile schedule (the
  * backward's dX and dW).  Same results as two fp8_mm calls; the tile
  * configuration (a->tile_cfg, or chosen for the pair when AUTO) is shared. */

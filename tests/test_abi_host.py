@@ -26,7 +26,7 @@ def header_functions():
 
 def test_exports_every_header_symbol(fp8):
     names = header_functions()
-    assert len(names) >= 17
+    assert len(names) >= 18
     for n in names:
         assert hasattr(fp8._lib, n), n
         assert n in fp8.EXPORTED, n
@@ -85,6 +85,30 @@ def mm(fp8, **kw):
     a.update(kw)
     args = fp8.MmArgs(**a)
     return fp8._lib.fp8_mm(ctypes.byref(args), None)
+
+
+def mmb(fp8, batch, sa, sb, sd, **kw):
+    a = dict(m=128, n=128, k=128, a=A, fmt_a=0, a_major=0, lda=128, b=A + 0x10000, fmt_b=0, b_major=0, ldb=128,
+             scale_a=A + 0x20000, scale_b=A + 0x20010, bias=None, bias_dtype=0, bias_scale=None, d=A + 0x30000,
+             ldd=128)
+    a.update(kw)
+    args = fp8.MmArgs(**a)
+    return fp8._lib.fp8_mm_batched(ctypes.byref(args), batch, sa, sb, sd, None)
+
+
+def test_mm_batched_validation(fp8):
+    """Checked before anything is enqueued (no GPU needed)."""
+    E = fp8
+    big = 128 * 128
+    assert mmb(fp8, -1, big, big, big) == E.FP8_ERR_INVALID_ARG
+    assert mmb(fp8, 2, -16, big, big) == E.FP8_ERR_INVALID_ARG
+    assert mmb(fp8, 2, big + 8, big, big) == E.FP8_ERR_MISALIGNED         # fp8 batch stride: 16-byte multiple
+    assert mmb(fp8, 2, big, 24, big) == E.FP8_ERR_MISALIGNED
+    assert mmb(fp8, 2, big, big, big - 1) == E.FP8_ERR_INVALID_ARG        # outputs of two batches overlap
+    assert mmb(fp8, 2, big, big, 0) == E.FP8_ERR_INVALID_ARG
+    assert mmb(fp8, 0, big, big, big) == E.FP8_OK                         # empty batch: nothing enqueued
+    assert mmb(fp8, 3, 0, 0, big, m=0) == E.FP8_OK
+    assert mmb(fp8, 2, big, big, big, scale_a=None) == E.FP8_ERR_INVALID_ARG
 
 
 def test_mm_validation(fp8):

@@ -245,3 +245,114 @@ def test_mm_split_k_deterministic(fp8, m, n, k, a_major, b_major):
     rng = np.random.default_rng(77)
     _, y2, _ = run_case(fp8, rng, m, n, k, a_major, b_major, full=False, tile=4)
     assert np.array_equal(y1, y2)
+
+
+# ---------------------------------------------------------------- batched (3-D) GEMMs
+
+def stack_operand(mats, major):
+    """Per-batch logical operands -> one storage array of the batches one after
+    another, its row stride and its batch stride (elements)."""
+    sts = [store(x, major, 0) for x in mats]
+    rows, ld = sts[0][0].shape
+    return np.concatenate([s_ for s_, _ in sts], axis=0), ld, rows * ld, [s_ for s_, _ in sts]
+
+
+def run_batched(fp8, rng, batch, m, n, k, a_major, b_major, bcast_a=False, bcast_b=False, tile=0, bias=False,
+                d_gap=0, full=True):
+    As = [codes_like_tensor(rng, 0, (m, k), 60.0) for _ in range(1 if bcast_a else batch)]
+    Bs = [codes_like_tensor(rng, 1, (n, k), 3000.0) for _ in range(1 if bcast_b else batch)]
+    a_buf, lda, sa, a_sts = stack_operand(As, a_major)
+    b_buf, ldb, sb, b_sts = stack_operand(Bs, b_major)
+    ldd = n + (8 if d_gap else 0)
+    sd = m * ldd + d_gap
+    dflat = torch.full((batch * sd,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    A, B = torch.from_numpy(a_buf).cuda(), torch.from_numpy(b_buf).cuda()
+    sc = torch.tensor([2.5, 0.125], dtype=torch.float32, device="cuda")
+    bias_np = bias_dev = None
+    if bias:
+        bt = torch.from_numpy((rng.standard_normal(n) * 3).astype(np.float32)).to(torch.bfloat16)
+        bias_dev, bias_np = bt.cuda(), bt.view(torch.int16).numpy().view(np.uint16)
+    args = fp8.MmArgs(m, n, k, A.data_ptr(), 0, a_major, lda, B.data_ptr(), 1, b_major, ldb, sc.data_ptr(),
+                      sc.data_ptr() + 4, bias_dev.data_ptr() if bias else None, 0, None, dflat.data_ptr(), ldd, tile)
+    fp8.fp8_mm_batched(args, batch, 0 if bcast_a else sa, 0 if bcast_b else sb, sd)
+    torch.cuda.synchronize()
+    assert fp8.fp8_get_device_status() == 0
+    allbits = dflat.cpu().view(torch.int16).numpy().view(np.uint16)
+    a_si, a_sk = strides(a_major, lda)
+    b_sj, b_sk = strides(b_major, ldb)
+    outs = []
+    for bi in range(batch):
+        blk = allbits[bi * sd: bi * sd + m * ldd].reshape(m, ldd)
+        y = blk[:, :n]
+        if ldd > n:
+            assert np.all(blk[:, n:] == 0x7FC0), "columns past n must stay untouched"
+        if d_gap:
+            assert np.all(allbits[bi * sd + m * ldd: (bi + 1) * sd] == 0x7FC0), "gap between batches untouched"
+        a_st = a_sts[0 if bcast_a else bi]
+        b_st = b_sts[0 if bcast_b else bi]
+        if full:
+            acc, _, sab = oracle.gemm_acc(a_st, 0, a_si, a_sk, b_st, 1, b_sj, b_sk, m, n, k)
+            want, _ = oracle.epilogue(acc, 2.5, 0.125, bias_np, oracle.DT_BF16 if bias else 0)
+            assert_gemm_close(y, want, sab, 2.5, 0.125, f"batched b={bi}")
+        else:
+            pi, pj = sample_points(rng, m, n)
+            acc, sab = oracle.gemm_acc_points(pi, pj, a_st, 0, a_si, a_sk, b_st, 1, b_sj, b_sk, k)
+            want, _ = oracle.epilogue(acc, 2.5, 0.125, bias_np, oracle.DT_BF16 if bias else 0, col_idx=pj)
+            assert_gemm_close(y[pi, pj], want, sab, 2.5, 0.125, f"batched b={bi} sampled")
+        outs.append(y.copy())
+    return outs
+
+
+@pytest.mark.parametrize("tile", [0, 1, 2, 3])
+@pytest.mark.parametrize("a_major,b_major", LAYOUTS)
+def test_mm_batched_layouts(fp8, a_major, b_major, tile):
+    """Three batches of a ragged shape, every layout and tile configuration,
+    a padded output row stride and a gap between the batches' outputs."""
+    rng = np.random.default_rng(50 + 4 * a_major + b_major + 10 * tile)
+    run_batched(fp8, rng, 3, 200, 300, 333, a_major, b_major, tile=tile, bias=True, d_gap=24)
+
+
+@pytest.mark.parametrize("bcast_a,bcast_b", [(False, True), (True, False)])
+@pytest.mark.parametrize("a_major,b_major", [(0, 0), (0, 1), (1, 1)])
+def test_mm_batched_broadcast(fp8, a_major, b_major, bcast_a, bcast_b):
+    """A zero batch stride shares that operand across the batch (the pages'
+    size-1 batch broadcast): a shared weight, or a shared activation."""
+    rng = np.random.default_rng(60 + a_major + 2 * b_major + 4 * bcast_a)
+    run_batched(fp8, rng, 4, 130, 257, 200, a_major, b_major, bcast_a=bcast_a, bcast_b=bcast_b)
+
+
+def test_mm_batched_single_equals_mm(fp8):
+    """batch = 1 is fp8_mm bit for bit; a batch whose matrices are copies of one
+    operand pair gives identical outputs."""
+    rng = np.random.default_rng(70)
+    m, n, k = 300, 260, 1000
+    A8 = codes_like_tensor(rng, 0, (m, k), 60.0)
+    B8 = codes_like_tensor(rng, 1, (n, k), 3000.0)
+    a_st, lda = store(A8, 0, 0)
+    b_st, ldb = store(B8, 0, 0)
+    A, B = torch.from_numpy(a_st).cuda(), torch.from_numpy(b_st).cuda()
+    A3 = torch.from_numpy(np.concatenate([a_st] * 3)).cuda()
+    sc = torch.tensor([1.5, 0.5], dtype=torch.float32, device="cuda")
+    d1 = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    d2 = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    d3 = torch.empty((3, m, n), dtype=torch.bfloat16, device="cuda")
+    mk = lambda a_, d_: fp8.MmArgs(m, n, k, a_.data_ptr(), 0, 0, lda, B.data_ptr(), 1, 0, ldb,  # noqa: E731
+                                   sc.data_ptr(), sc.data_ptr() + 4, None, 0, None, d_.data_ptr(), n, 0)
+    a1, a2, a3 = mk(A, d1), mk(A, d2), mk(A3, d3)
+    fp8._lib.fp8_mm(ctypes.byref(a1), torch.cuda.current_stream().cuda_stream)
+    fp8.fp8_mm_batched(a2, 1, 0, 0, 0)
+    fp8.fp8_mm_batched(a3, 3, m * lda, 0, m * n)
+    torch.cuda.synchronize()
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+    for bi in range(3):
+        # batched launches pick their tile configuration on batch x tiles, so
+        # compare within the GEMM tolerance rather than bit for bit
+        assert torch.equal(d3[bi].view(torch.int16), d3[0].view(torch.int16))
+
+
+@pytest.mark.parametrize("batch,m,n,k,a_major,b_major", [(64, 512, 512, 512, 0, 0), (8, 1024, 2048, 1024, 0, 1),
+                                                         (4, 2048, 1024, 4096, 1, 1)])
+def test_mm_batched_large_sampled(fp8, batch, m, n, k, a_major, b_major):
+    """The pages' bmm shapes (64 x 512^3, 8 x 1024 x 2048) and a dW-like batch."""
+    rng = np.random.default_rng(batch + m + k)
+    run_batched(fp8, rng, batch, m, n, k, a_major, b_major, full=False)

@@ -101,6 +101,8 @@ _SIGS = {
     "fp8_mm": (_I, [ctypes.POINTER(MmArgs), _P]),
     "fp8_mm_pair": (_I, [ctypes.POINTER(MmArgs), ctypes.POINTER(MmArgs), _P]),
     "fp8_mm_batched": (_I, [ctypes.POINTER(MmArgs), _I64, _I64, _I64, _I64, _P]),
+    "fp8_quantize_ex": (_I, [ctypes.POINTER(QuantizeArgs), _I, _P]),
+    "fp8_ring_finalize": (_I, [_P, _I, _I, _P, _P]),
     "fp8_dbias_workspace_bytes": (_SZ, [_I64, _I64]),
     "fp8_dbias": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "fp8_dbias_noalloc": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P]),
@@ -196,6 +198,18 @@ def quantize_args(x: torch.Tensor, fmt: int, ring: torch.Tensor, hist_len: int, 
     rows, cols = x.shape
     return QuantizeArgs(_ptr(x), _dtype_code(x), rows, cols, _ld(x), fmt, _ptr(ring), hist_len, _ptr(out), _ld(out),
                         _ptr(amax_out), _ptr(scale_out))
+
+
+FP8_QUANTIZE_DEFER_RING_STEP = 1
+
+
+def fp8_quantize_ex(a: QuantizeArgs, flags: int, device=None) -> None:
+    _check(_lib.fp8_quantize_ex(ctypes.byref(a), flags, _stream(device)), "fp8_quantize_ex")
+
+
+def fp8_ring_finalize(ring: torch.Tensor, hist_len: int, fmt: int, amax_out: torch.Tensor | None = None) -> None:
+    _check(_lib.fp8_ring_finalize(_ptr(ring), hist_len, fmt, _ptr(amax_out), _stream(ring.device)),
+           "fp8_ring_finalize")
 
 
 def fp8_quantize_dual(a: QuantizeArgs, b: QuantizeArgs, device=None) -> None:

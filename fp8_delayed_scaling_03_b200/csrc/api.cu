@@ -443,6 +443,25 @@ int fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
+int fp8_quantize_ex(const fp8_quantize_args* q, int flags, fp8_stream_t stream) {
+  if (!q || (flags & ~FP8_QUANTIZE_DEFER_RING_STEP)) return FP8_ERR_INVALID_ARG;
+  const bool defer = (flags & FP8_QUANTIZE_DEFER_RING_STEP) != 0;
+  if (defer && !q->ring) return FP8_ERR_INVALID_ARG;  // a pending step needs a ring
+  int s = validate_quantize(q->in, q->in_dtype, q->rows, q->cols, q->ld_in, q->fmt, q->ring, q->hist_len, q->out,
+                            q->ld_out, q->amax_out);
+  if (s) return s;
+  if (q->rows == 0 || q->cols == 0) return FP8_OK;
+  return run_quantize(q->in, q->in_dtype, q->rows, q->cols, q->ld_in, q->fmt, q->ring, q->hist_len, q->out,
+                      q->ld_out, q->amax_out, q->scale_out, reinterpret_cast<cudaStream_t>(stream), defer);
+}
+
+int fp8_ring_finalize(void* ring, int hist_len, int fmt, float* amax_out, fp8_stream_t stream) {
+  if (!ring || !aligned(ring, 4) || !ring_len_ok(hist_len) || !is_fmt(fmt)) return FP8_ERR_INVALID_ARG;
+  if (amax_out && !aligned(amax_out, 4)) return FP8_ERR_INVALID_ARG;
+  cudaError_t e = launch_ring_finalize(ring_fin(ring, hist_len, fmt, amax_out), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
 int fp8_quantize_dual(const fp8_quantize_args* a, const fp8_quantize_args* b, fp8_stream_t stream) {
   if (!a || !b) return FP8_ERR_INVALID_ARG;
   int s = validate_quantize(a->in, a->in_dtype, a->rows, a->cols, a->ld_in, a->fmt, a->ring, a->hist_len, a->out,

@@ -41,6 +41,7 @@
 #include "internal.h"
 #include "launch.h"
 #include "partials.cuh"
+#include "ring.cuh"
 
 namespace fp8lin {
 namespace {
@@ -127,33 +128,6 @@ __device__ __forceinline__ float bias_value(const void* bias, int bias_kind, int
   const uint16_t b = __ldg(static_cast<const uint8_t*>(bias) + j);
   const float2 f = bias_kind == 2 ? dec_e4m3x2(b) : dec_e5m2x2(b);
   return f.x * binv;
-}
-
-// Completes a delayed-scaling step for a ring whose quantize deferred it (its
-// blocks only max-reduced into the scratch word).  Runs after
-// griddepcontrol.wait, so every block's reduction is visible and nothing else
-// touches the ring until this grid completes.  Same rule as the quantize's
-// own last-block finalize: hist[step % H] = amax, window max over the history
-// with the new amax in place of the overwritten slot, next scale, step + 1.
-__device__ __forceinline__ void ring_finalize_warp(const RingFinalize& f, int lane) {
-  uint32_t* words = reinterpret_cast<uint32_t*>(f.ring);
-  const int H = f.H;
-  const uint32_t step = words[H + 2];
-  const float a = __uint_as_float(words[H + 3]);
-  const float s = f.ring[H];
-  const uint32_t slot = step % static_cast<uint32_t>(H);
-  float m = a;
-  for (int i = lane; i < H; i += 32)
-    if (static_cast<uint32_t>(i) != slot) m = fmaxf(m, f.ring[i]);
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  if (lane == 0) {
-    f.ring[slot] = a;
-    f.ring[H] = next_scale(s, m, f.fp8_max);
-    words[H + 2] = step + 1;
-    words[H + 3] = 0u;
-    if (f.amax_out) *f.amax_out = a;
-  }
 }
 
 // dbias[c] = bf16(fixed-order sum of the R partials of column c) for the

@@ -145,6 +145,7 @@ cudaError_t launch_quantize_colsum(int in_dtype, int fmt, const ColsumParams& cp
 cudaError_t launch_amax(int in_dtype, const QuantizeParams* a, const QuantizeParams* b, cudaStream_t s);
 cudaError_t launch_ring_set(float* ring, int H, float scale, cudaStream_t s);
 cudaError_t launch_side_writes(const SideWrites& w, cudaStream_t s);
+cudaError_t launch_ring_finalize(const RingFinalize& f, cudaStream_t s);
 // GEMM tile configurations: 128x128 and 128x256 on one CTA, 256x256 on a pair
 // of CTAs (2-SM MMA).
 enum : int { kGemm128 = 1, kGemm256 = 2, kGemmPair256 = 3, kGemmSplit128 = 4 };

@@ -41,6 +41,7 @@
 #include "internal.h"
 #include "launch.h"
 #include "partials.cuh"
+#include "ring.cuh"
 
 namespace fp8lin {
 namespace {
@@ -429,6 +430,13 @@ __global__ void ring_set_kernel(float* ring, int H, float scale) {
   }
 }
 
+// The pending ring step of one ring (fp8_ring_finalize): one warp.
+__global__ void ring_finalize_kernel(const RingFinalize f) {
+  pdl_wait();
+  pdl_trigger();
+  ring_finalize_warp(f, static_cast<int>(threadIdx.x));
+}
+
 __global__ void side_writes_kernel(const SideWrites w) {
   pdl_wait();
   pdl_trigger();
@@ -521,6 +529,10 @@ cudaError_t launch_quantize_colsum(int in_dtype, int fmt, const ColsumParams& cp
 
 cudaError_t launch_ring_set(float* ring, int H, float scale, cudaStream_t s) {
   return launch_pdl(ring_set_kernel, dim3(1), dim3(128), 0, s, ring, H, scale);
+}
+
+cudaError_t launch_ring_finalize(const RingFinalize& f, cudaStream_t s) {
+  return launch_pdl(ring_finalize_kernel, dim3(1), dim3(32), 0, s, f);
 }
 
 cudaError_t launch_side_writes(const SideWrites& w, cudaStream_t s) {

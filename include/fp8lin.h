@@ -144,6 +144,26 @@ typedef struct fp8_quantize_args {
  * required and distinct); the amax passes of such tensors share one launch. */
 FP8LIN_API int fp8_quantize_dual(const fp8_quantize_args* a, const fp8_quantize_args* b, fp8_stream_t stream);
 
+/* fp8_quantize with flags.  FP8_QUANTIZE_DEFER_RING_STEP (ring required):
+ * the launch quantizes with the ring's scale and writes scale_out as usual,
+ * but only max-reduces this launch's amax into the ring's scratch word
+ * (32-bit word hist_len + 3, i.e. byte offset (hist_len + 3) * 4); the
+ * history, scale, step and amax_out wait for fp8_ring_finalize.  Between the
+ * two, data-parallel ranks all-reduce that word with MAX (non-negative floats
+ * order like their bit patterns, so an unsigned or signed 32-bit integer MAX
+ * is exact), so every rank's ring takes the same step -- the one exchange the
+ * method needs across data-parallel replicas.  Since delayed scaling casts
+ * with the previous scale, the all-reduce can overlap the GEMM. */
+enum { FP8_QUANTIZE_DEFER_RING_STEP = 1 };
+FP8LIN_API int fp8_quantize_ex(const fp8_quantize_args* q, int flags, fp8_stream_t stream);
+
+/* The pending step of a ring left by FP8_QUANTIZE_DEFER_RING_STEP: a = the
+ * scratch word (as float), hist[step % H] = a, window max, scale = fp8_max(fmt)
+ * / max with the keep-old rule, step + 1, scratch = 0, *amax_out = a (if
+ * given) -- exactly the step the quantize's last block would have taken.  One
+ * 32-thread launch.  Calling it with no pending step folds an amax of 0. */
+FP8LIN_API int fp8_ring_finalize(void* ring, int hist_len, int fmt, float* amax_out, fp8_stream_t stream);
+
 /* fp8_quantize of g [rows, cols] plus, in the same pass over g, its column
  * sums: dbias[c] = bf16( sum_r g[r, c] ) as fp8_dbias computes them (fp32
  * sums in a fixed order).  workspace as fp8_dbias (size from

@@ -26,7 +26,7 @@ def header_functions():
 
 def test_exports_every_header_symbol(fp8):
     names = header_functions()
-    assert len(names) >= 18
+    assert len(names) >= 20
     for n in names:
         assert hasattr(fp8._lib, n), n
         assert n in fp8.EXPORTED, n
@@ -109,6 +109,22 @@ def test_mm_batched_validation(fp8):
     assert mmb(fp8, 0, big, big, big) == E.FP8_OK                         # empty batch: nothing enqueued
     assert mmb(fp8, 3, 0, 0, big, m=0) == E.FP8_OK
     assert mmb(fp8, 2, big, big, big, scale_a=None) == E.FP8_ERR_INVALID_ARG
+
+
+def test_quantize_ex_and_ring_finalize_validation(fp8):
+    E = fp8
+    f = fp8._lib
+    qa = fp8.QuantizeArgs(A, 0, 4, 32, 32, 0, A + 0x1000, 16, A + 0x2000, 32, None, None)
+    qn = fp8.QuantizeArgs(A, 0, 4, 32, 32, 0, None, 16, A + 0x2000, 32, A + 0x3000, None)
+    assert f.fp8_quantize_ex(ctypes.byref(qa), 2, None) == E.FP8_ERR_INVALID_ARG          # unknown flag
+    assert f.fp8_quantize_ex(ctypes.byref(qn), E.FP8_QUANTIZE_DEFER_RING_STEP, None) == E.FP8_ERR_INVALID_ARG
+    assert f.fp8_quantize_ex(None, 0, None) == E.FP8_ERR_INVALID_ARG
+    empty = fp8.QuantizeArgs(A, 0, 0, 32, 32, 0, A + 0x1000, 16, A + 0x2000, 32, None, None)
+    assert f.fp8_quantize_ex(ctypes.byref(empty), E.FP8_QUANTIZE_DEFER_RING_STEP, None) == E.FP8_OK
+    assert f.fp8_ring_finalize(None, 16, 0, None, None) == E.FP8_ERR_INVALID_ARG
+    assert f.fp8_ring_finalize(A + 2, 16, 0, None, None) == E.FP8_ERR_INVALID_ARG
+    assert f.fp8_ring_finalize(A, 0, 0, None, None) == E.FP8_ERR_INVALID_ARG
+    assert f.fp8_ring_finalize(A, 16, 3, None, None) == E.FP8_ERR_INVALID_ARG
 
 
 def test_mm_validation(fp8):

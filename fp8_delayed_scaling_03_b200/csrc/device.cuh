@@ -136,6 +136,14 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
                "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
+// Asynchronous L2 prefetch of a global byte range (16-byte aligned address,
+// size a multiple of 16).  Only a hint; L2 is the point of coherence, so a
+// line fetched early is updated by any later write to it.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
+
 // Bulk copy from this CTA's shared memory into another CTA's of the cluster
 // (dst and bar from mapa_shared), completion counted in bytes on bar.  Both
 // addresses 16-byte aligned, bytes a multiple of 16.  No multicast.

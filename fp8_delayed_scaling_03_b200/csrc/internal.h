@@ -42,6 +42,7 @@ struct QuantizeParams {
 struct QuantizePair {
   QuantizeParams t[2];
   int blocks0;
+  int pf_blocks;              // the first pf_blocks blocks prefetch the inputs into L2
 };
 
 // Quantize of a [rows, cols] tensor (not flattened) that also produces its

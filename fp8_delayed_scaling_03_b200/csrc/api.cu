@@ -9,7 +9,11 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
+#include <functional>
+#include <queue>
+#include <vector>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -146,12 +150,60 @@ int validate_mm(const MmCall& c) {
   return FP8_OK;
 }
 
+// Per-tile cost, in k-blocks, of the schedule models: the mainloop plus the
+// part of the epilogue a following tile does not hide.
+constexpr int kTileFixedKb = 2;
+
+// Longest-processing-time list schedule of a launch's tiles (problem 0's
+// count0 tiles of cost0 k-blocks, then count1 of cost1) over `units` CTAs:
+// tiles in decreasing cost, each to the least loaded unit (ties: lowest unit,
+// so equal-cost tiles keep their raster order).  Returns the makespan in
+// k-blocks; with `order`, writes slot round * units + unit (kNoTile: none) and
+// *nslots, or returns -1 when the slots would exceed kMaxOrder.
+int64_t lpt_schedule(int64_t count0, int64_t cost0, int64_t count1, int64_t cost1, int64_t units, uint16_t* order,
+                     int* nslots) {
+  const int64_t total = count0 + count1;
+  if (total <= 0 || units <= 0) return 0;
+  units = std::min(units, total);
+  std::vector<int64_t> tiles(static_cast<size_t>(total));
+  for (int64_t t = 0; t < total; ++t) tiles[static_cast<size_t>(t)] = t;
+  auto cost = [&](int64_t t) { return (t < count0 ? cost0 : cost1) + kTileFixedKb; };
+  std::stable_sort(tiles.begin(), tiles.end(), [&](int64_t a, int64_t b) { return cost(a) > cost(b); });
+  using Load = std::pair<int64_t, int64_t>;  // (load, unit)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int64_t u = 0; u < units; ++u) heap.push({0, u});
+  std::vector<std::vector<int64_t>> lists(order ? static_cast<size_t>(units) : 0);
+  int64_t makespan = 0;
+  for (int64_t t : tiles) {
+    Load l = heap.top();
+    heap.pop();
+    l.first += cost(t);
+    makespan = std::max(makespan, l.first);
+    if (order) lists[static_cast<size_t>(l.second)].push_back(t);
+    heap.push(l);
+  }
+  if (order) {
+    size_t rounds = 0;
+    for (const auto& v : lists) rounds = std::max(rounds, v.size());
+    if (static_cast<int64_t>(rounds) * units > kMaxOrder) return -1;
+    for (size_t r = 0; r < rounds; ++r)
+      for (int64_t u = 0; u < units; ++u) {
+        const auto& v = lists[static_cast<size_t>(u)];
+        order[r * static_cast<size_t>(units) + static_cast<size_t>(u)] =
+            r < v.size() ? static_cast<uint16_t>(v[r]) : kNoTile;
+      }
+    *nslots = static_cast<int>(rounds * static_cast<size_t>(units));
+  }
+  return makespan;
+}
+
 // Tile configuration with the smallest modelled time for a launch of one or
-// two problems: waves of tiles over the SMs (pairs of SMs for 2-SM tiles)
-// times the tile's mainloop at the k-block time measured on a B200 for that
-// tile shape, plus a fixed fill/drain cost.  Measured: 0.34 us per 128x128x128
-// k-block on one SM, 0.45 us per 128x256x128 on one SM and per 256x256x128 on
-// an SM pair; ~4-5 us fill + epilogue + launch.
+// two problems: the makespan (k-blocks) of the launch's tile schedule -- the
+// LPT schedule the single-CTA configurations run for two problems of unequal
+// k, round robin otherwise -- times the k-block time measured on a B200 for
+// that tile shape, plus a fixed fill/drain cost.  Measured: 0.34 us per
+// 128x128x128 k-block on one SM, 0.45 us per 128x256x128 on one SM and per
+// 256x256x128 on an SM pair; ~4-5 us fill + epilogue + launch.
 int pick_tile(const MmCall* calls, int n, int sms, double* est_us = nullptr) {
   struct Opt { int cfg; int64_t tm, tn, units; double t_kb, fixed; };
   const Opt opts[3] = {{kGemm128, 128, 128, sms, 0.34, 4.0}, {kGemm256, 128, 256, sms, 0.45, 4.0},
@@ -159,16 +211,26 @@ int pick_tile(const MmCall* calls, int n, int sms, double* est_us = nullptr) {
   int best = kGemm128;
   double best_t = -1.0;
   for (const Opt& o : opts) {
-    int64_t tiles = 0;
-    double work = 0.0;
+    int64_t cnt[2] = {0, 0}, kb[2] = {0, 0};
     for (int i = 0; i < n; ++i) {
-      const int64_t ti = ((calls[i].m + o.tm - 1) / o.tm) * ((calls[i].n + o.tn - 1) / o.tn) * calls[i].batch;
-      tiles += ti;
-      work += static_cast<double>(ti) * static_cast<double>((calls[i].k + 127) / 128);
+      cnt[i] = ((calls[i].m + o.tm - 1) / o.tm) * ((calls[i].n + o.tn - 1) / o.tn) * calls[i].batch;
+      kb[i] = (calls[i].k + 127) / 128;
     }
-    const double avg_kb = tiles ? work / static_cast<double>(tiles) : 0.0;
-    const int64_t waves = (tiles + o.units - 1) / o.units;
-    const double t = static_cast<double>(waves) * avg_kb * o.t_kb + o.fixed;
+    int64_t span;
+    if (o.cfg != kGemmPair256 && n == 2 && kb[0] != kb[1]) {
+      span = lpt_schedule(cnt[0], kb[0], cnt[1], kb[1], o.units, nullptr, nullptr);
+    } else {  // round robin: unit u runs tiles u, u + units, ...
+      span = 0;
+      const int64_t total = cnt[0] + cnt[1];
+      const int64_t units = std::max<int64_t>(1, std::min(o.units, total));
+      for (int64_t u = 0; u < std::min(units, total); ++u) {
+        int64_t load = 0;
+        // tiles of problem 0 at u, u + units, ... then problem 1
+        for (int64_t t = u; t < total; t += units) load += (t < cnt[0] ? kb[0] : kb[1]) + kTileFixedKb;
+        span = std::max(span, load);
+      }
+    }
+    const double t = static_cast<double>(span - kTileFixedKb) * o.t_kb + o.fixed;
     if (best_t < 0 || t < best_t) { best = o.cfg; best_t = t; }
   }
   if (est_us) *est_us = best_t;
@@ -274,6 +336,18 @@ int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_
   p.split = cfg == kGemmSplit128 ? split : 1;
   p.tiles0 = p.pr[0].num_tiles;
   p.total_tiles = p.pr[0].num_tiles + (n > 1 ? p.pr[1].num_tiles : 0);
+  p.nslots = p.total_tiles;
+  p.use_order = 0;
+  // Two problems of unequal k on single-CTA tiles: LPT schedule instead of
+  // round robin (the launch's grid is min(tiles, SMs), the schedule's units).
+  if (n == 2 && (cfg == kGemm128 || cfg == kGemm256) && p.pr[0].k_blocks != p.pr[1].k_blocks) {
+    int nslots = 0;
+    if (lpt_schedule(p.pr[0].num_tiles, p.pr[0].k_blocks, p.pr[1].num_tiles, p.pr[1].k_blocks, sms, p.order,
+                     &nslots) >= 0) {
+      p.nslots = nslots;
+      p.use_order = 1;
+    }
+  }
   p.status = status_ptr(dev);
   if (side) p.side = *side;
   for (int i = 0; i < nfin; ++i) p.fin[i] = fin[i];

@@ -107,6 +107,13 @@ __device__ __forceinline__ int tile_coords(const GemmParams& p, int t, int& tb, 
   return pi;
 }
 
+// The tile a schedule slot holds (-1: none).
+__device__ __forceinline__ int slot_tile(const GemmParams& p, int slot) {
+  if (!p.use_order) return slot;
+  const uint16_t t = p.order[slot];
+  return t == kNoTile ? -1 : static_cast<int>(t);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -178,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Barrier set-up (warp 2), TMEM allocation (warp 1) and the producer's
   // first tile coordinates (warp 0) proceed side by side.
   int first_tb = 0, first_tm = 0, first_tn = 0, first_pi = 0;
-  if (threadIdx.x == 0 && unit < p.total_tiles) first_pi = tile_coords(p, unit, first_tb, first_tm, first_tn);
+  const int first_t = unit < p.nslots ? slot_tile(p, unit) : -1;
+  if (threadIdx.x == 0 && first_t >= 0) first_pi = tile_coords(p, first_t, first_tb, first_tm, first_tn);
   if (threadIdx.x == 64) {
     for (int s = 0; s < nstages; ++s) {
       mbar_init(&full[s], 1);
@@ -240,9 +248,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b_row0 = static_cast<int>(prank) * C::kBRows;
       bool dep_done = false;
       int issued = 0;  // k-blocks loaded so far; the first kStages find their stage free
-      for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
+      for (int slot = unit; slot < p.nslots && !*abort_flag; slot += units) {
+        const int t = slot_tile(p, slot);
+        if (t < 0) continue;
         int tb = first_tb, tm = first_tm, tn = first_tn;
-        const int pi = t == unit ? first_pi : tile_coords(p, t, tb, tm, tn);
+        const int pi = t == first_t ? first_pi : tile_coords(p, t, tb, tm, tn);
         const int za = FP8_PR(bcast_a) ? 0 : tb, zb = FP8_PR(bcast_b) ? 0 : tb;  // batch coordinates
         const CUtensorMap* tma_a = pi ? &ta1 : &ta0;
         const CUtensorMap* tma_b = pi ? &tb1 : &tb0;
@@ -291,7 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
+      for (int slot = unit; slot < p.nslots && !*abort_flag; slot += units) {
+        const int t = slot_tile(p, slot);
+        if (t < 0) continue;
         const int pi = t >= p.tiles0 ? 1 : 0;
         const int k_blocks = FP8_PR(k_blocks);
         const bool a_mn = FP8_PR(a_major) != 0, b_mn = FP8_PR(b_major) != 0;
@@ -376,7 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     constexpr int kSteps = BN / 2 / kEpiCols;
-    for (int t = unit; t < p.total_tiles && !*abort_flag; t += units) {
+    for (int slot = unit; slot < p.nslots && !*abort_flag; slot += units) {
+      const int t = slot_tile(p, slot);
+      if (t < 0) continue;
       int tb, tm, tn;
       const int pi = tile_coords(p, t, tb, tm, tn);
       // The tile's constants go to registers and its bias values are fetched

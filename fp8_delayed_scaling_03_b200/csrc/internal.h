@@ -121,7 +121,15 @@ struct GemmParams {
   int nfin;
   DbiasFinish dbias;          // partial == nullptr: none
   int split;                  // split-K launches: CTAs per tile (cluster size)
+  // Tile schedule.  CTA (or pair) u runs slots u, u + units, u + 2 units, ...
+  // below nslots; with use_order, slot s holds tile order[s] (kNoTile: none),
+  // else tile s.
+  int nslots;
+  int use_order;
+  uint16_t order[1024];
 };
+constexpr int kMaxOrder = 1024;
+constexpr uint16_t kNoTile = 0xFFFF;
 
 struct DbiasParams {
   const void* g;

@@ -39,7 +39,7 @@ class Fp8Error(RuntimeError):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m fp8_delayed_scaling_03_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python fp8_delayed_scaling_03_b200/build.py` "
                       "(there is no CPU fallback)")
 
 _lib = ctypes.CDLL(LIB_PATH)

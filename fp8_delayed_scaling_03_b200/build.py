@@ -1,6 +1,6 @@
 """Build libfp8lin.so (sm_100a) in-tree with nvcc.
 
-    python -m fp8_delayed_scaling_03_b200.build [--force] [-v]
+    python fp8_delayed_scaling_03_b200/build.py [--force] [-v] [--ptxas-v]
 
 Each .cu under csrc/ is compiled in parallel to an object under _build/, then
 linked with the static CUDA runtime into fp8_delayed_scaling_03_b200/lib/.

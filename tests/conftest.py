@@ -8,8 +8,20 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def build_library():
+    """Compile libfp8lin.so in-tree if it is missing or stale.  The build script
+    is loaded by path: the package's __init__ refuses to import without it."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "fp8lin_build", os.path.join(ROOT, "fp8_delayed_scaling_03_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs an sm_100 GPU and the built CUDA library")
+    build_library()
 
 
 def _have_sm100():

@@ -13,8 +13,6 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def fp8():
-    from fp8_delayed_scaling_03_b200 import build as b
-    b.build()
     import fp8_delayed_scaling_03_b200 as m
     return m
 

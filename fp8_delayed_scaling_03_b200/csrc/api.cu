@@ -201,13 +201,17 @@ int64_t lpt_schedule(int64_t count0, int64_t cost0, int64_t count1, int64_t cost
 // two problems: the makespan (k-blocks) of the launch's tile schedule -- the
 // LPT schedule the single-CTA configurations run for two problems of unequal
 // k, round robin otherwise -- times the k-block time measured on a B200 for
-// that tile shape, plus a fixed fill/drain cost.  Measured: 0.34 us per
-// 128x128x128 k-block on one SM, 0.45 us per 128x256x128 on one SM and per
-// 256x256x128 on an SM pair; ~4-5 us fill + epilogue + launch.
+// that tile shape, plus a fixed fill/drain cost.  Measured on a B200 (1965
+// MHz): 0.31 us per 128x128x128 k-block on one SM; per 128x256x128 of work
+// on one SM, 0.35 us for a single-CTA 128x256 tile and 0.37 us for a 256x256
+// pair tile while each CTA runs at most 3 tiles, 0.40 and 0.365 us in longer
+// launches (the single-CTA tile moves 1.5x the operand bytes per SM through
+// L2, which tells once the whole chip streams for long); ~4-5 us fill +
+// epilogue + launch.
 int pick_tile(const MmCall* calls, int n, int sms, double* est_us = nullptr) {
-  struct Opt { int cfg; int64_t tm, tn, units; double t_kb, fixed; };
-  const Opt opts[3] = {{kGemm128, 128, 128, sms, 0.34, 4.0}, {kGemm256, 128, 256, sms, 0.45, 4.0},
-                       {kGemmPair256, 256, 256, sms / 2, 0.45, 5.0}};
+  struct Opt { int cfg; int64_t tm, tn, units; double t_kb, t_kb_long, fixed; };
+  const Opt opts[3] = {{kGemm128, 128, 128, sms, 0.31, 0.31, 4.0}, {kGemm256, 128, 256, sms, 0.35, 0.40, 4.0},
+                       {kGemmPair256, 256, 256, sms / 2, 0.37, 0.365, 5.0}};
   int best = kGemm128;
   double best_t = -1.0;
   for (const Opt& o : opts) {
@@ -230,7 +234,9 @@ int pick_tile(const MmCall* calls, int n, int sms, double* est_us = nullptr) {
         span = std::max(span, load);
       }
     }
-    const double t = static_cast<double>(span - kTileFixedKb) * o.t_kb + o.fixed;
+    const int64_t tiles = cnt[0] + cnt[1];
+    const int64_t rounds = (tiles + o.units - 1) / std::max<int64_t>(1, o.units);
+    const double t = static_cast<double>(span - kTileFixedKb) * (rounds > 3 ? o.t_kb_long : o.t_kb) + o.fixed;
     if (best_t < 0 || t < best_t) { best = o.cfg; best_t = t; }
   }
   if (est_us) *est_us = best_t;

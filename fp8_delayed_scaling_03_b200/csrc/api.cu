@@ -435,6 +435,17 @@ int run_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
 
+// Bytes of a dbias workspace's per-tile counters (16-byte rounded); the
+// R x N fp32 partials follow them.
+size_t dbias_counter_bytes(int64_t N) {
+  const size_t tiles = static_cast<size_t>((N + kDbiasColsPerTile - 1) / kDbiasColsPerTile);
+  return (tiles * 4u + 15u) & ~size_t(15);
+}
+
+size_t dbias_partial_bytes(int R, int64_t N) {
+  return (static_cast<size_t>(R) * static_cast<size_t>(N) * 4u + 15u) & ~size_t(15);
+}
+
 // defer: leave both the ring finalize and the column sums to the GEMM
 // launch that follows; *dbf then describes the sums it must do.
 int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace, cudaStream_t st,
@@ -446,10 +457,10 @@ int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace,
   cp.q.defer_finalize = defer && g.ring ? 1 : 0;
   int s = amax_pass(g.in_dtype, &cp.q, nullptr, st);
   if (s) return s;
-  dbias_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
-  cp.partial = static_cast<float*>(workspace);
-  const size_t part = (static_cast<size_t>(cp.R) * static_cast<size_t>(g.cols) * 4u + 15u) & ~size_t(15);
-  cp.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + part);
+  if (defer) colsum_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
+  else dbias_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
+  cp.counters = static_cast<unsigned*>(workspace);
+  cp.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dbias_counter_bytes(g.cols));
   cp.dbias = dbias;
   cp.defer_sum = defer ? 1 : 0;
   if (defer && dbf) *dbf = DbiasFinish{cp.partial, dbias, g.cols, cp.R};
@@ -635,9 +646,7 @@ size_t fp8_dbias_workspace_bytes(int64_t M, int64_t N) {
   int R;
   int64_t rps;
   dbias_geometry(M, N, &R, &rps);
-  const int64_t tiles = (N + kDbiasColsPerTile - 1) / kDbiasColsPerTile;
-  const size_t part = (static_cast<size_t>(R) * static_cast<size_t>(N) * 4u + 15u) & ~size_t(15);
-  return part + ((static_cast<size_t>(tiles) * 4u + 15u) & ~size_t(15));
+  return dbias_counter_bytes(N) + dbias_partial_bytes(R, N);
 }
 
 int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg, const float* g_scale, void* dbias,
@@ -659,9 +668,8 @@ int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg, con
   p.g_scale = g_scale;
   p.dbias = dbias;
   dbias_geometry(M, N, &p.R, &p.rows_per_split);
-  p.partial = static_cast<float*>(workspace);
-  const size_t part = (static_cast<size_t>(p.R) * static_cast<size_t>(N) * 4u + 15u) & ~size_t(15);
-  p.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + part);
+  p.counters = static_cast<unsigned*>(workspace);
+  p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dbias_counter_bytes(N));
   const int es = esize(g_dtype);
   p.vec_ok = is_fp8(g_dtype) ? (aligned(g, 8) && (ldg % 8 == 0)) : (aligned(g, 16) && ((ldg * es) % 16 == 0));
   cudaError_t e = launch_dbias(p, reinterpret_cast<cudaStream_t>(stream));
@@ -670,7 +678,12 @@ int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg, con
 
 size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   (void)K;
-  return fp8_dbias_workspace_bytes(M, N);
+  if (M <= 0 || N <= 0) return 0;
+  int Rd, Rc;
+  int64_t rps;
+  dbias_geometry(M, N, &Rd, &rps);
+  colsum_geometry(M, N, &Rc, &rps);
+  return dbias_counter_bytes(N) + dbias_partial_bytes(std::max(Rd, Rc), N);
 }
 
 int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
@@ -767,7 +780,7 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
              sg, a->sx, nullptr, 0, nullptr, a->dw, a->lddw, FP8_TILE_AUTO};
   if (a->need_dx && (s = validate_mm(cdx))) return s;
   if (a->need_dw && (s = validate_mm(cdw))) return s;
-  const size_t ws_need = a->need_dbias ? fp8_dbias_workspace_bytes(M, N) : 0;
+  const size_t ws_need = a->need_dbias ? fp8_linear_workspace_bytes(M, N, K) : 0;
   if (a->need_dbias) {
     if (!a->dbias || !aligned(a->dbias, 2)) return FP8_ERR_INVALID_ARG;
     if (ws_need && (!a->workspace || a->workspace_bytes < ws_need || !aligned(a->workspace, 16)))

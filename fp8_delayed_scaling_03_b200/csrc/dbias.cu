@@ -144,11 +144,14 @@ __global__ void __launch_bounds__(kRowLanes * 32) dbias_kernel(const DbiasParams
 
 }  // namespace
 
-void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
-  // About 296 blocks (two per SM of a B200) in total, at least 64 rows each.
+namespace {
+
+// Row splits of an [M, N] column sum over 256-column tiles: about `blocks`
+// (col tile, row split) blocks in total, each split at least min_rows rows.
+void split_geometry(int64_t M, int64_t N, int64_t blocks, int64_t min_rows, int* R, int64_t* rows_per_split) {
   const int64_t col_tiles = (N + kCols - 1) / kCols;
-  int64_t r = (296 + col_tiles - 1) / (col_tiles > 0 ? col_tiles : 1);
-  const int64_t rmax = (M + 63) / 64;
+  int64_t r = (blocks + col_tiles - 1) / (col_tiles > 0 ? col_tiles : 1);
+  const int64_t rmax = (M + min_rows - 1) / min_rows;
   if (r > rmax) r = rmax;
   if (r < 1) r = 1;
   int64_t rps = (M + r - 1) / r;
@@ -157,6 +160,21 @@ void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
   if (r < 1) r = 1;
   *R = static_cast<int>(r);
   *rows_per_split = rps;
+}
+
+}  // namespace
+
+// The dbias kernel: about 296 blocks (two per SM of a B200), at least 64 rows each.
+void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
+  split_geometry(M, N, 296, 64, R, rows_per_split);
+}
+
+// The column-sum quantize whose sums a GEMM launch finishes (the linear
+// backward): about 592 blocks, at least 32 rows each.  Measured on a B200 in
+// the dim1024 training step (g of 2048 x 1024 and 2048 x 4096): 2% faster
+// than the dbias kernel's geometry; 16-row or 1184-block splits were slower.
+void colsum_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
+  split_geometry(M, N, 592, 32, R, rows_per_split);
 }
 
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s) {

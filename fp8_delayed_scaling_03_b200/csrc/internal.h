@@ -166,8 +166,14 @@ int gemm_split_factor(int tiles, int k_blocks, int sms, bool forced);
 cudaError_t launch_gemm(const CUtensorMap* maps, const GemmParams& p, int cfg, cudaStream_t s);
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s);
 
-// dbias geometry shared by the size query and the launcher.
+// Column-sum geometry (R row splits of rows_per_split rows over 256-column
+// tiles) shared by the size queries and the launchers: dbias_geometry for the
+// dbias kernel and the standalone column-sum quantize, colsum_geometry for
+// the column-sum quantize of the linear backward (its sums finished by the
+// GEMM launch).  Workspaces hold the per-tile counters first (16-byte
+// rounded), then the R x N fp32 partials.
 constexpr int kDbiasColsPerTile = 256;
 void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split);
+void colsum_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split);
 
 }  // namespace fp8lin

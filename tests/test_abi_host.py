@@ -150,7 +150,10 @@ def test_dbias_workspace_rules(fp8):
     assert fp8.fp8_dbias_workspace_bytes(0, 10) == 0
     need = fp8.fp8_dbias_workspace_bytes(2048, 1024)
     assert need > 0 and need % 16 == 0
-    assert fp8.fp8_linear_workspace_bytes(2048, 1024, 4096) == need
+    # the linear backward's column sums may split rows more finely than fp8_dbias
+    lin = fp8.fp8_linear_workspace_bytes(2048, 1024, 4096)
+    assert lin >= need and lin % 16 == 0
+    assert fp8.fp8_linear_workspace_bytes(0, 1024, 4096) == 0
     f = fp8._lib.fp8_dbias
     assert f(A, E.FP8_DT_BF16, 2048, 1024, 1024, None, A + 0x100, None, 0, None) == E.FP8_ERR_WORKSPACE
     assert f(A, E.FP8_DT_BF16, 2048, 1024, 1024, None, A + 0x100, A, need - 16, None) == E.FP8_ERR_WORKSPACE

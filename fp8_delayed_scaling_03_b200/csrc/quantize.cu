@@ -363,6 +363,22 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   __shared__ float hist_s[kHistCache];
   __shared__ __align__(16) float red[kRowLanes][kColTile];
   __shared__ int last_tile;
+  // Before the dependency wait: the first block of each row split prefetches
+  // its band of rows into L2 (one contiguous range when the rows are 16-byte
+  // aligned), so the DRAM latency overlaps the previous kernel's tail; as in
+  // the flat kernel, only inputs up to kPrefetchMaxBytes.
+  if (threadIdx.x == 0 && blockIdx.x == 0 && cp.q.vec_ok) {
+    const QuantizeParams& q = cp.q;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * cp.rows_per_split;
+    const int64_t r1 = min(q.rows, r0 + cp.rows_per_split);
+    const uint64_t total = static_cast<uint64_t>(q.rows) * static_cast<uint64_t>(q.ld_in) * sizeof(T);
+    if (r1 > r0 && total <= kPrefetchMaxBytes) {
+      const uint64_t bytes =
+          (static_cast<uint64_t>((r1 - r0 - 1) * q.ld_in + q.cols) * sizeof(T)) & ~uint64_t(15);
+      if (bytes > 0)
+        prefetch_l2_bulk(static_cast<const T*>(q.in) + r0 * q.ld_in, static_cast<uint32_t>(bytes));
+    }
+  }
   pdl_wait();
   pdl_trigger();
   const QuantizeParams& p = cp.q;

@@ -273,8 +273,10 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_cons
       load_raw<T>(p, r, col, cur[u]);
     }
   }
+  // Every round but the last: the next round's loads are issued before the
+  // current chunks are converted and stored.
   #pragma unroll 1
-  while (c < p.total_chunks) {
+  while (c + U * stride < p.total_chunks) {
     const int64_t cn = c + U * stride;
     Raw<T> nxt[U];
     #pragma unroll
@@ -301,10 +303,35 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_cons
     for (int u = 0; u < U; ++u) cur[u] = nxt[u];
     c = cn;
   }
-
-  if (!p.ring) return;  // current scaling: amax was reduced by the amax pass
-  const uint32_t bits = block_max_bits(amax, warp_max);
-  if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
+  // Last round: its amax first, then the block's ring tail, then its stores.
+  // The tail's release (the last-block ticket) then waits only for the
+  // stores of earlier rounds, which drain while these loads are in flight,
+  // and the finalize runs beside the other blocks' last stores.
+  #pragma unroll
+  for (int u = 0; u < U; ++u) {
+    if (c + u * stride < p.total_chunks) {
+      float v[16];
+      to_floats<T>(cur[u], v);
+      #pragma unroll
+      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    }
+  }
+  if (p.ring) {  // current scaling: amax was reduced by the amax pass
+    const uint32_t bits = block_max_bits(amax, warp_max);
+    if (threadIdx.x == 0) ring_tail(p, bits, nblocks, s, step, hist_s);
+  }
+  float unused = 0.0f;
+  #pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t cu = c + u * stride;
+    if (cu < p.total_chunks) {
+      int64_t r, col;
+      chunk_pos(p, cu, r, col);
+      float v[16];
+      to_floats<T>(cur[u], v);
+      cast_store<FMT>(p, r, col, v, s, unused);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- amax pass

@@ -5,7 +5,8 @@ One step = forward + backward of every linear of the 12L/dim1024/B4xT512 model
 (12 layers x {q, k, v, o: 1024x1024; up: 1024x4096; down: 4096x1024}, M = 2048
 tokens): per linear, quantize x and w (E4M3, delayed scaling rings), the
 forward GEMM with fused dequant + bf16 bias, quantize g (E5M2), dX, dW and
-dbias -- 504 kernel launches, replayed as one CUDA graph of C-ABI calls.
+dbias -- 288 kernel launches (4 per linear), replayed as one CUDA graph of
+C-ABI calls.
 The value is TFLOP/s of the three GEMMs (6 M N K per linear) over the whole
 step.  Inputs are synthetic, seeded and resident in HBM; the step's working
 set (about 3 GB) is far larger than L2.

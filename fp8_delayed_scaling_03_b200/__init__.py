@@ -56,6 +56,10 @@ class MmArgs(ctypes.Structure):
                 ("tile_cfg", _I)]
 
 
+class MmPlanInfo(ctypes.Structure):
+    _fields_ = [("tile_cfg", _I), ("tiles", _I64), ("units", _I), ("est_us", ctypes.c_double)]
+
+
 class QuantizeArgs(ctypes.Structure):
     _fields_ = [("in_", _P), ("in_dtype", _I), ("rows", _I64), ("cols", _I64), ("ld_in", _I64),
                 ("fmt", _I), ("ring", _P), ("hist_len", _I),
@@ -99,6 +103,7 @@ _SIGS = {
     "fp8_quantize_dual": (_I, [ctypes.POINTER(QuantizeArgs), ctypes.POINTER(QuantizeArgs), _P]),
     "fp8_quantize_dbias": (_I, [ctypes.POINTER(QuantizeArgs), _P, _P, _SZ, _P]),
     "fp8_mm": (_I, [ctypes.POINTER(MmArgs), _P]),
+    "fp8_mm_plan": (_I, [ctypes.POINTER(MmArgs), ctypes.POINTER(MmArgs), _I, ctypes.POINTER(MmPlanInfo)]),
     "fp8_mm_pair": (_I, [ctypes.POINTER(MmArgs), ctypes.POINTER(MmArgs), _P]),
     "fp8_mm_batched": (_I, [ctypes.POINTER(MmArgs), _I64, _I64, _I64, _I64, _P]),
     "fp8_quantize_ex": (_I, [ctypes.POINTER(QuantizeArgs), _I, _P]),
@@ -238,6 +243,15 @@ def fp8_mm(m, n, k, a, fmt_a, a_major, lda, b, fmt_b, b_major, ldb, scale_a, sca
                   _ptr(scale_a), _ptr(scale_b), _ptr(bias), bias_dtype, _ptr(bias_scale), _ptr(d), ldd, tile_cfg)
     s = stream if stream is not None else _stream(d.device if isinstance(d, torch.Tensor) else None)
     _check(_lib.fp8_mm(ctypes.byref(args), s), "fp8_mm")
+
+
+def fp8_mm_plan(a: MmArgs, b: MmArgs | None = None, num_sms: int = 148) -> MmPlanInfo:
+    """The tile configuration fp8_mm (or fp8_mm_pair with b) would choose on a
+    GPU with num_sms SMs; host arithmetic only (no device needed)."""
+    info = MmPlanInfo()
+    _check(_lib.fp8_mm_plan(ctypes.byref(a), ctypes.byref(b) if b is not None else None, num_sms,
+                            ctypes.byref(info)), "fp8_mm_plan")
+    return info
 
 
 def fp8_dbias_workspace_bytes(M: int, N: int) -> int:

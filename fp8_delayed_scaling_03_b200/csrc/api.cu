@@ -641,6 +641,35 @@ int fp8_mm_batched(const fp8_mm_args* a, int64_t batch, int64_t stride_a, int64_
   return run_mm(c, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int fp8_mm_plan(const fp8_mm_args* a, const fp8_mm_args* b, int num_sms, fp8_mm_plan_info* out) {
+  if (!a || !out || num_sms <= 0) return FP8_ERR_INVALID_ARG;
+  MmCall c[2];
+  int n = 0;
+  for (const fp8_mm_args* x : {a, b}) {
+    if (!x) continue;
+    MmCall m{x->m, x->n, x->k, x->a, x->fmt_a, x->a_major, x->lda, x->b, x->fmt_b, x->b_major, x->ldb,
+             x->scale_a, x->scale_b, x->bias, x->bias_dtype, x->bias_scale, x->d, x->ldd, a->tile_cfg};
+    int s = validate_mm(m);
+    if (s) return s;
+    if (m.m == 0 || m.n == 0 || m.k == 0) continue;  // an empty problem launches nothing
+    c[n++] = m;
+  }
+  std::memset(out, 0, sizeof(*out));
+  if (n == 0) return FP8_OK;
+  double est = 0.0;
+  const int cfg = c[0].tile_cfg != FP8_TILE_AUTO ? c[0].tile_cfg : pick_tile(c, n, num_sms, &est);
+  const int64_t tm = cfg == kGemmPair256 ? 256 : 128;
+  const int64_t tn = (cfg == kGemm256 || cfg == kGemmPair256) ? 256 : 128;
+  int64_t tiles = 0;
+  for (int i = 0; i < n; ++i) tiles += ((c[i].m + tm - 1) / tm) * ((c[i].n + tn - 1) / tn);
+  const int64_t cap = cfg == kGemmPair256 ? num_sms / 2 : num_sms;
+  out->tile_cfg = cfg;
+  out->tiles = tiles;
+  out->units = static_cast<int>(std::max<int64_t>(1, std::min(tiles, cap)));
+  out->est_us = c[0].tile_cfg != FP8_TILE_AUTO ? 0.0 : est;
+  return FP8_OK;
+}
+
 size_t fp8_dbias_workspace_bytes(int64_t M, int64_t N) {
   if (M <= 0 || N <= 0) return 0;
   int R;

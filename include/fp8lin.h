@@ -222,6 +222,29 @@ FP8LIN_API int fp8_mm_batched(const fp8_mm_args* args, int64_t batch, int64_t st
  * configuration (a->tile_cfg, or chosen for the pair when AUTO) is shared. */
 FP8LIN_API int fp8_mm_pair(const fp8_mm_args* a, const fp8_mm_args* b, fp8_stream_t stream);
 
+/* The tile configuration fp8_mm (b == NULL) or fp8_mm_pair (b != NULL) would
+ * choose for these arguments on a GPU with num_sms SMs -- host arithmetic
+ * only: nothing is launched, the GPU is not touched and the operands are not
+ * read, so it works without a device.  The arguments are validated as
+ * fp8_mm validates them (same status codes).  Split-K, which FP8_TILE_AUTO
+ * may also pick for a single few-tile, long-K problem, depends on the
+ * device's cluster occupancy and is not considered here.  Output (host
+ * pointer):
+ *   tile_cfg  the fp8_tile_cfg value (a forced a->tile_cfg comes back as given;
+ *             FP8_TILE_AUTO when every problem is empty);
+ *   tiles     output tiles of that configuration over the problem(s);
+ *   units     CTAs (CTA pairs for FP8_TILE_PAIR_256x256) the launch keeps
+ *             busy: min(tiles, num_sms) (pairs: num_sms / 2);
+ *   est_us    the cost model's estimate of the launch in microseconds (fitted
+ *             to B200 timings; 0 for a forced configuration). */
+typedef struct {
+  int tile_cfg;
+  int64_t tiles;
+  int units;
+  double est_us;
+} fp8_mm_plan_info;
+FP8LIN_API int fp8_mm_plan(const fp8_mm_args* a, const fp8_mm_args* b, int num_sms, fp8_mm_plan_info* out);
+
 /* ------------------------------------------------------------------ dbias
  * dbias[n] = bf16_rne( sum_m g(m, n) ), fp32 sums, for n < N.  g is bf16,
  * fp16 or fp32 [M, ldg], or fp8 (E4M3/E5M2) [M, ldg] with g_scale required:

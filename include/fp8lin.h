@@ -339,6 +339,11 @@ typedef struct fp8_linear_bwd_args {
 } fp8_linear_bwd_args;
 FP8LIN_API int fp8_linear_backward(const fp8_linear_bwd_args* args, fp8_stream_t stream);
 
+/* Workspace bytes fp8_linear_backward needs for need_dbias (0 when M or N is
+ * 0).  At least fp8_dbias_workspace_bytes(M, N): the column-sum quantize of
+ * the backward may split g's rows more finely than fp8_dbias does.  Zero-fill
+ * it once before first use, like fp8_dbias's workspace; every call leaves it
+ * ready for the next.  K does not enter. */
 FP8LIN_API size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------ status

@@ -206,6 +206,23 @@ def test_linear_backward_validation(fp8):
     assert bwd(fp8, g_dtype=E.FP8_DT_E5M2) == E.FP8_ERR_INVALID_ARG         # pre-quantized g needs its scale
     assert bwd(fp8, sg_out=None) == E.FP8_ERR_INVALID_ARG
     assert bwd(fp8, N=0) == E.FP8_OK
+    # the backward's column sums need fp8_linear_workspace_bytes, which can
+    # exceed what fp8_dbias needs; a workspace sized for fp8_dbias is refused
+    M, N, K = 2048, 1024, 1024
+    lin, dbw = fp8.fp8_linear_workspace_bytes(M, N, K), fp8.fp8_dbias_workspace_bytes(M, N)
+    assert lin > dbw
+    big = dict(M=M, N=N, K=K, ldg=N, ldg8=N, ldx8=K, ldw8=K, lddx=K, lddw=K, need_dbias=1, dbias=A + 0xA0000,
+               workspace=A + 0x100000)
+    assert bwd(fp8, workspace_bytes=dbw, **big) == E.FP8_ERR_WORKSPACE
+    assert bwd(fp8, workspace_bytes=lin, workspace=A + 0x100008, **{k: v for k, v in big.items()
+                                                                   if k != "workspace"}) == E.FP8_ERR_WORKSPACE
+
+
+def test_linear_workspace_covers_dbias(fp8):
+    for M in (1, 3, 64, 100, 512, 2048, 4096, 65536):
+        for N in (1, 100, 192, 1024, 1536, 4096, 6912, 11008):
+            lin, dbw = fp8.fp8_linear_workspace_bytes(M, N, 64), fp8.fp8_dbias_workspace_bytes(M, N)
+            assert lin >= dbw > 0 and lin % 16 == 0
 
 
 def test_fused_entry_points_validation(fp8):

@@ -245,7 +245,10 @@ void orc_gemm(int64_t I, int64_t J, int64_t Kc,
 }
 
 /* The same dot products for a list of n (i, j) output coordinates only, for
- * sampled checks of shapes whose full product is too slow on the CPU. */
+ * sampled checks of shapes whose full product is too slow on the CPU.  Each
+ * point is the loop of orc_gemm for that (i, j): fp32 accumulation with k
+ * ascending, sum |a_k b_k| in double, and a NaN or infinite operand makes
+ * both results NaN. */
 void orc_gemm_points(int64_t n, const int64_t* ii, const int64_t* jj, int64_t Kc,
                      const uint8_t* a, int fmt_a, int64_t a_si, int64_t a_sk,
                      const uint8_t* b, int fmt_b, int64_t b_sj, int64_t b_sk,
@@ -258,15 +261,17 @@ void orc_gemm_points(int64_t n, const int64_t* ii, const int64_t* jj, int64_t Kc
     int64_t i = ii[t], j = jj[t];
     float acc = 0.0f;
     double sa = 0.0;
+    int nan = 0;
     for (int64_t k = 0; k < Kc; ++k) {
       double va = ta[a[i * a_si + k * a_sk]];
       double vb = tb[b[j * b_sj + k * b_sk]];
+      if (isnan(va) || isnan(vb) || isinf(va) || isinf(vb)) { nan = 1; break; }
       float p = (float)(va * vb);
       acc = acc + p;
       sa += fabs(va * vb);
     }
-    acc_f32[t] = acc;
-    sumabs[t] = sa;
+    acc_f32[t] = nan ? NAN : acc;
+    sumabs[t] = nan ? NAN : sa;
   }
 }
 

@@ -1,15 +1,25 @@
 #!/usr/bin/env python
 """Throughput of the FP8 linear layer with delayed scaling on B200.
 
-One step = forward + backward of every linear of the 12L/dim1024/B4xT512 model
-(12 layers x {q, k, v, o: 1024x1024; up: 1024x4096; down: 4096x1024}, M = 2048
-tokens): per linear, quantize x and w (E4M3, delayed scaling rings), the
-forward GEMM with fused dequant + bf16 bias, quantize g (E5M2), dX, dW and
-dbias -- 288 kernel launches (4 per linear), replayed as one CUDA graph of
-C-ABI calls.
-The value is TFLOP/s of the three GEMMs (6 M N K per linear) over the whole
-step.  Inputs are synthetic, seeded and resident in HBM; the step's working
-set (about 3 GB) is far larger than L2.
+One step = forward + backward of every linear of a workload through the C ABI
+(fp8_linear_forward, then fp8_linear_backward in reverse order), replayed as
+one CUDA graph: per linear, quantize x and w (E4M3, delayed-scaling rings),
+the forward GEMM with fused dequant (+ bias), quantize g (E5M2, + bias
+gradient), dX and dW.  The headline workload is the generic large shapes at
+M = 4096 tokens: three linears {4096x11008, 11008x4096, 4096x4096} (K x N),
+x ~ N(0,1) with 0.1% outliers x50, w ~ N(0, 1/sqrt(K)), g ~ N(0, 1e-3), no
+bias.  The value is TFLOP/s of the three GEMMs (6 M N K per linear) over the
+whole step.  Inputs are synthetic, seeded and resident in HBM; the step's
+working set (about 1.6 GB) is far larger than L2.
+
+Extra keys of the same JSON line: `roofline` (the GEMM class of the headline
+step), `kernels` (per-class times), `steps` (the dim1024 training step of the
+pages' 12L/dim1024/B4xT512 model with bf16 bias + dbias, and the production
+24L/dim1536/ffn6912 linears at M in {512, 2048} with an E4M3 bias and dbias),
+`targets` (fwd, dX and dW as single launches at the production and large
+shapes, warm and cold L2, against the measured peak, the nominal peak and
+each shape's own roofline; standalone quantize GB/s), `e2e` (the headline
+step with host buffers), `cpu_baseline` (the oracle on a sample).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -43,8 +53,8 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_PER_BF16 = 2.0          # nominal dense fp8 : bf16 tensor-core ratio (4.5 : 2.25 PFLOP/s)
 NOMINAL_FP8_TFLOPS = 4500.0
-REF_TOKENS = 128            # tokens of one layer per reference-arm step
-CPU_SAMPLE_TOKENS = 1024      # tokens of one layer for the cpu_baseline sample
+REF_TOKENS = 16             # tokens of the headline linears per reference-arm step
+CPU_SAMPLE_TOKENS = 128     # tokens of the headline linears for the cpu_baseline sample
 
 
 # --------------------------------------------------------------------------- helpers
@@ -137,16 +147,27 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- workload
 
-class Linear:
-    """Device buffers and prebuilt C-ABI argument structs of one FP8 linear."""
+BIAS_NONE, BIAS_BF16, BIAS_E4M3 = "none", "bf16", "e4m3"
 
-    def __init__(self, F, shape, seed_base, device, H=wl.HIST_LEN):
+
+class Linear:
+    """Device buffers and prebuilt C-ABI argument structs of one FP8 linear.
+    bias: BIAS_NONE, BIAS_BF16 (bf16 bias, bf16 dbias) or BIAS_E4M3 (the bias
+    stored as E4M3 codes with its own scale, quantized once here by the
+    library's current-scaling quantize; bf16 dbias)."""
+
+    def __init__(self, F, shape, seed_base, device, H=wl.HIST_LEN, bias=BIAS_BF16, outliers=False):
         M, K, N = shape.M, shape.K, shape.N
         self.shape = shape
+        self.bias = bias
         ldk, ldn = (K + 15) // 16 * 16, (N + 15) // 16 * 16
-        self.x = wl.normal_device((M, K), 1.0, seed_base + wl.OP_X, device)
+        if outliers:
+            self.x = wl.normal_with_outliers_device((M, K), 1.0, seed_base + wl.OP_X, seed_base + wl.OP_MASK, device)
+        else:
+            self.x = wl.normal_device((M, K), 1.0, seed_base + wl.OP_X, device)
         self.w = wl.normal_device((N, K), wl.weight_std(K), seed_base + wl.OP_W, device)
-        self.b = wl.normal_device((N,), wl.BENCH_BIAS_STD, seed_base + wl.OP_BIAS, device)
+        self.b = wl.normal_device((N,), wl.BENCH_BIAS_STD, seed_base + wl.OP_BIAS, device) if bias != BIAS_NONE \
+            else None
         self.g = wl.normal_device((M, N), 1e-3, seed_base + wl.OP_G, device)
         self.x8 = torch.zeros((M, ldk), dtype=torch.uint8, device=device)
         self.w8 = torch.zeros((N, ldk), dtype=torch.uint8, device=device)
@@ -154,32 +175,52 @@ class Linear:
         self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
         self.dx = torch.empty((M, K), dtype=torch.bfloat16, device=device)
         self.dw = torch.empty((N, K), dtype=torch.bfloat16, device=device)
-        self.db = torch.empty((N,), dtype=torch.bfloat16, device=device)
+        self.db = torch.empty((N,), dtype=torch.bfloat16, device=device) if bias != BIAS_NONE else None
         words = F.fp8_ring_bytes(H) // 4
         self.rings = torch.empty((3, words), dtype=torch.float32, device=device)
         for i in range(3):
             F.fp8_ring_init(self.rings[i], H)
-        self.sc = torch.zeros(6, dtype=torch.float32, device=device)
-        self.ws = torch.zeros(max(16, F.fp8_linear_workspace_bytes(M, N, K)), dtype=torch.uint8, device=device)
-        p = lambda t: t.data_ptr()  # noqa: E731
+        # sx, sw, sg, amax_x, amax_w, amax_g, bias_scale, bias amax
+        self.sc = torch.zeros(8, dtype=torch.float32, device=device)
         sc = self.sc.data_ptr()
+        self.bias_ptr, self.bias_dtype, self.bias_scale_ptr = None, F.FP8_DT_BF16, None
+        if bias == BIAS_BF16:
+            self.bias_ptr = self.b.data_ptr()
+        elif bias == BIAS_E4M3:
+            self.b8 = torch.zeros((1, ldn), dtype=torch.uint8, device=device)
+            F.fp8_quantize(self.b.view(1, N), F.FP8_E4M3, None, 0, self.b8[:, :N], self.sc[7:8], self.sc[6:7])
+            self.bias_ptr, self.bias_dtype, self.bias_scale_ptr = self.b8.data_ptr(), F.FP8_DT_E4M3, sc + 24
+        need_dbias = bias != BIAS_NONE
+        # backward: bias-gradient + stream-K scratch; forward: stream-K scratch
+        self.ws = torch.zeros(max(16, F.fp8_linear_workspace_bytes(M, N, K)), dtype=torch.uint8, device=device)
+        self.wsf = torch.zeros(max(16, F.fp8_mm_workspace_bytes(M, N, K)), dtype=torch.uint8, device=device)
+        # where the stream-K part starts in the backward workspace
+        sk_need = max(F.fp8_mm_workspace_bytes(M, K, N), F.fp8_mm_workspace_bytes(N, K, M))
+        self.sk_offset = self.ws.numel() - sk_need
+        p = lambda t: t.data_ptr() if t is not None else None  # noqa: E731
         self.fwd = F.LinearFwdArgs(M, N, K, p(self.x), F.FP8_DT_BF16, K, None, p(self.w), F.FP8_DT_BF16, K, None,
-                                   p(self.b), F.FP8_DT_BF16, None, F.FP8_E4M3, F.FP8_E4M3, H,
+                                   self.bias_ptr, self.bias_dtype, self.bias_scale_ptr, F.FP8_E4M3, F.FP8_E4M3, H,
                                    p(self.rings[0]), p(self.rings[1]), p(self.x8), ldk, p(self.w8), ldk,
-                                   sc, sc + 4, sc + 12, sc + 16, p(self.y), N)
+                                   sc, sc + 4, sc + 12, sc + 16, p(self.y), N, p(self.wsf), self.wsf.numel())
         self.bwd = F.LinearBwdArgs(M, N, K, p(self.g), F.FP8_DT_BF16, N, None, F.FP8_E5M2, H, p(self.rings[2]),
                                    p(self.g8), ldn, sc + 8, sc + 20, p(self.x8), ldk, sc, F.FP8_E4M3,
-                                   p(self.w8), ldk, sc + 4, F.FP8_E4M3, 1, 1, 1, p(self.dx), K, p(self.dw), K,
-                                   p(self.db), p(self.ws), self.ws.numel())
+                                   p(self.w8), ldk, sc + 4, F.FP8_E4M3, 1, 1, int(need_dbias), p(self.dx), K,
+                                   p(self.dw), K, p(self.db), p(self.ws), self.ws.numel())
 
     def inputs(self):
-        return [self.x, self.w, self.b, self.g]
+        return [t for t in (self.x, self.w, self.b, self.g) if t is not None]
 
     def outputs(self):
-        return [self.y, self.dx, self.dw, self.db]
+        return [t for t in (self.y, self.dx, self.dw, self.db) if t is not None]
 
 
-def build_model(F, device, rank):
+# Workloads: (description, builder).  Each builder returns the step's linears.
+def _c4_linears(F, device, rank):
+    return [Linear(F, s, wl.seed_for(4, 0, 0, extra=1 + rank * 1000 + j) * 10, device, bias=BIAS_NONE,
+                   outliers=True) for j, s in enumerate(wl.C4_SHAPES)]
+
+
+def _dim1024_linears(F, device, rank):
     lins = []
     for layer in range(wl.BENCH_LAYERS):
         for j, s in enumerate(wl.BENCH_LAYER):
@@ -187,8 +228,36 @@ def build_model(F, device, rank):
     return lins
 
 
+def _c3_linears(F, device, rank):
+    return [Linear(F, s, wl.seed_for(3, 0, 0, extra=1 + rank * 1000 + j) * 10, device, bias=BIAS_E4M3)
+            for j, s in enumerate(wl.C3_SHAPES)]
+
+
+WORKLOADS = {
+    "c4": ("generic large linears at M=4096 tokens: {4096x11008, 11008x4096, 4096x4096} (K x N), fwd+dX+dW, "
+           "x ~ N(0,1) with 0.1% outliers x50, E4M3 x/w, E5M2 g, delayed scaling H=16, no bias",
+           _c4_linears),
+    "dim1024": ("12L/dim1024/B4xT512 linears: 12 layers x {q,k,v,o 1024x1024, up 1024x4096, down 4096x1024}, "
+                "M=2048 tokens, fwd+dX+dW, E4M3 x/w, E5M2 g, delayed scaling H=16, bf16 bias + dbias",
+                _dim1024_linears),
+    "c3": ("production 24L/dim1536/ffn6912 linears: M in {512, 2048} x {1536x1536, 1536x6912, 6912x1536}, "
+           "fwd+dX+dW, E4M3 x/w, E5M2 g, delayed scaling H=16, E4M3 bias with its own scale + dbias",
+           _c3_linears),
+}
+HEADLINE = "c4"
+
+
+def build_model(F, device, rank, workload=HEADLINE):
+    return WORKLOADS[workload][1](F, device, rank)
+
+
+def step_flops(lins) -> int:
+    """fwd + dX + dW: 3 GEMMs of 2 M N K flops per linear."""
+    return sum(6 * L.shape.M * L.shape.N * L.shape.K for L in lins)
+
+
 def run_step(F, lins, stream_handle):
-    """Forward over the layers in order, then backward in reverse, through the C ABI."""
+    """Forward over the linears in order, then backward in reverse, through the C ABI."""
     fwd, bwd = F._lib.fp8_linear_forward, F._lib.fp8_linear_backward
     for L in lins:
         s = fwd(ctypes.byref(L.fwd), stream_handle)
@@ -200,16 +269,18 @@ def run_step(F, lins, stream_handle):
             raise F.Fp8Error(s, "fp8_linear_backward")
 
 
-LAUNCHES_PER_LINEAR = 4  # quantize x+w, fwd GEMM, quantize g + dbias, dX+dW GEMMs
+# quantize x+w, fwd GEMM, quantize g (+ dbias partials), dX+dW GEMMs (dX and
+# dW as two launches when both are long: the count comes from the graph)
+LAUNCHES_PER_LINEAR = 4
 
 
 # --------------------------------------------------------------------------- kernel-level timing
 
 def step_primitives(F, lins, h):
     """The step's kernel launches as (class, algorithmic work, label, call) in
-    launch order, through the same fused entry points fp8_linear_forward /
-    fp8_linear_backward use: quantize x+w, forward GEMM (+bias); then in
-    reverse, quantize g (+dbias), dX+dW GEMMs."""
+    launch order, through the standalone entry points that do the same work as
+    the fused fp8_linear_forward / fp8_linear_backward: quantize x+w, forward
+    GEMM (+bias); then in reverse, quantize g (+ dbias), dX+dW GEMMs."""
     lib = F._lib
     out = []
     keep = []  # ctypes argument structs must outlive the calls and the graphs
@@ -226,7 +297,8 @@ def step_primitives(F, lins, h):
         qw = F.QuantizeArgs(L.w.data_ptr(), 0, N, K, K, 0, L.rings[1].data_ptr(), wl.HIST_LEN, L.w8.data_ptr(), ldk,
                             sc + 16, sc + 4)
         fwd = F.MmArgs(M, N, K, L.x8.data_ptr(), 0, 0, ldk, L.w8.data_ptr(), 0, 0, ldk, sc, sc + 4,
-                       L.b.data_ptr(), 0, None, L.y.data_ptr(), N, 0)
+                       L.bias_ptr, L.bias_dtype, L.bias_scale_ptr, L.y.data_ptr(), N, 0,
+                       L.wsf.data_ptr(), L.wsf.numel())
         out.append(("quantize", (M * K + N * K) * 3, None, call(lib.fp8_quantize_dual, qx, qw)))
         out.append(("gemm", 2 * M * N * K, f"fwd {M}x{N}x{K}", call(lib.fp8_mm, fwd)))
     for L in reversed(lins):
@@ -235,15 +307,22 @@ def step_primitives(F, lins, h):
         sc = L.sc.data_ptr()
         qg = F.QuantizeArgs(L.g.data_ptr(), 0, M, N, N, 1, L.rings[2].data_ptr(), wl.HIST_LEN, L.g8.data_ptr(), ldn,
                             sc + 20, sc + 8)
+        # the same stream-K scratch the fused backward uses (after its bias-gradient part)
+        sk = L.ws.data_ptr() + L.sk_offset
+        sk_bytes = L.ws.numel() - L.sk_offset
         dx = F.MmArgs(M, K, N, L.g8.data_ptr(), 1, 0, ldn, L.w8.data_ptr(), 0, 1, ldk, sc + 8, sc + 4,
-                      None, 0, None, L.dx.data_ptr(), K, 0)
+                      None, 0, None, L.dx.data_ptr(), K, 0, sk, sk_bytes)
         dw = F.MmArgs(N, K, M, L.g8.data_ptr(), 1, 1, ldn, L.x8.data_ptr(), 0, 1, ldk, sc + 8, sc,
-                      None, 0, None, L.dw.data_ptr(), K, 0)
-        ws = L.ws
-        out.append(("quantize", M * N * 3, None,
-                    (lambda qg=qg, L=L, ws=ws: lib.fp8_quantize_dbias(ctypes.byref(qg), L.db.data_ptr(), ws.data_ptr(),
-                                                                      ws.numel(), h))))
-        keep.append((qg,))
+                      None, 0, None, L.dw.data_ptr(), K, 0, sk, sk_bytes)
+        if L.db is not None:
+            ws = L.ws
+            out.append(("quantize", M * N * 3, None,
+                        (lambda qg=qg, L=L, ws=ws: lib.fp8_quantize_dbias(ctypes.byref(qg), L.db.data_ptr(),
+                                                                          ws.data_ptr(), ws.numel(), h))))
+            keep.append((qg,))
+        else:
+            out.append(("quantize", M * N * 3, None, (lambda qg=qg: lib.fp8_quantize_ex(ctypes.byref(qg), 0, h))))
+            keep.append((qg,))
         out.append(("gemm", 4 * M * N * K, f"dX+dW {M}x{N}x{K}", call(lib.fp8_mm_pair, dx, dw)))
     return out, keep
 
@@ -278,13 +357,12 @@ def time_kernels(F, lins, stream, reps=5):
         torch.cuda.synchronize()
         res_ms[cls] = e0.elapsed_time(e1) / reps
         del g
-    # per-shape GEMM times: one graph per distinct GEMM of a layer, 12 launches each
+    # per-shape GEMM times: one graph per distinct GEMM launch of the step, 12 launches each
     shapes = {}
-    layer = len(wl.BENCH_LAYER)
-    first_layer = [c for c in prims if c[0] == "gemm"]
     seen = {}
-    for c in first_layer:
-        seen.setdefault(c[2], c)
+    for c in prims:
+        if c[0] == "gemm":
+            seen.setdefault(c[2], c)
     for name, c in seen.items():
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
@@ -301,7 +379,7 @@ def time_kernels(F, lins, stream, reps=5):
         us = e0.elapsed_time(e1) * 1e3 / 12
         shapes[name] = {"us": us, "tflops": c[1] / us / 1e6, "note": "same operands back to back (warm L2)"}
         del g
-    del layer, keep
+    del keep
     return res_ms, work, count, shapes
 
 
@@ -333,45 +411,88 @@ def _sets_for(bytes_per_set, floor=320 << 20, cap=12):
     return max(2, min(cap, -(-floor // max(1, bytes_per_set))))
 
 
-def time_target_shapes(F, device, stream):
+def gemm_min_bytes(op: str, M: int, N: int, K: int, bias_bytes: int = 0) -> int:
+    """Compulsory DRAM bytes of one GEMM: fp8 operands read once, bf16 output
+    written once (fwd MK + NK + 2MN, dX MN + NK + 2MK, dW MN + MK + 2NK)."""
+    if op == "fwd":
+        return M * K + N * K + 2 * M * N + bias_bytes
+    if op == "dX":
+        return M * N + N * K + 2 * M * K
+    return M * N + M * K + 2 * N * K
+
+
+def roofline_tflops(flops: float, nbytes: float, peak_tflops: float, hbm_gbs: float) -> float:
+    """min(peak, AI x BW) in TFLOP/s for arithmetic intensity AI = flops / bytes."""
+    return min(peak_tflops, flops / nbytes * hbm_gbs * 1e9 / 1e12)
+
+
+def time_target_shapes(F, device, stream, fp8_peak, hbm_gbs):
     """fwd, dX and dW as separate launches (fp8_mm, the layouts the fused
-    backward uses) at the production and large shapes, and the quantize of the
-    large activations; operand sets are cycled so each pass streams more than
-    L2.  Returns a list of per-(shape, op) records and a list of quantize
-    records."""
+    backward uses) at the production (config 3, the forward with its E4M3
+    bias and bias scale) and large (config 4) shapes, each timed warm (the
+    same operands back to back: L2 holds what fits) and cold (operand sets
+    cycled so that each pass streams more than L2); and the standalone
+    quantize of the large activations (cold).  Each GEMM record carries its
+    fraction of the measured fp8 peak, of the 4.5 PFLOP/s nominal peak and of
+    its own roofline min(peak, AI x HBM bandwidth) -- the HBM term binds only
+    the cold case; warm operands come from L2."""
     h = stream.cuda_stream
-    sc = torch.ones(2, dtype=torch.float32, device=device)
+    sc = torch.ones(3, dtype=torch.float32, device=device)
+    sc[2] = 448.0 / 0.04
     gemm = []
-    for s in wl.C3_SHAPES + wl.C4_SHAPES:
-        M, K, N = s.M, s.K, s.N
-        per_set = M * K + N * K + M * N + 2 * (M * N + M * K + N * K)
-        nsets = _sets_for(per_set)
-        sets = []
-        for i in range(nsets):
-            x8 = torch.randint(0x20, 0x48, (M, K), dtype=torch.uint8, device=device)
-            w8 = torch.randint(0x20, 0x48, (N, K), dtype=torch.uint8, device=device)
-            g8 = torch.randint(0x20, 0x48, (M, N), dtype=torch.uint8, device=device)
-            y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-            dx = torch.empty((M, K), dtype=torch.bfloat16, device=device)
-            dw = torch.empty((N, K), dtype=torch.bfloat16, device=device)
-            sets.append((x8, w8, g8, y, dx, dw))
-        sp = sc.data_ptr()
-        ops = {
-            "fwd": lambda t: F.MmArgs(M, N, K, t[0].data_ptr(), 0, 0, K, t[1].data_ptr(), 0, 0, K, sp, sp + 4,
-                                      None, 0, None, t[3].data_ptr(), N, 0),
-            "dX": lambda t: F.MmArgs(M, K, N, t[2].data_ptr(), 1, 0, N, t[1].data_ptr(), 0, 1, K, sp, sp + 4,
-                                     None, 0, None, t[4].data_ptr(), K, 0),
-            "dW": lambda t: F.MmArgs(N, K, M, t[2].data_ptr(), 1, 1, N, t[0].data_ptr(), 0, 1, K, sp, sp + 4,
-                                     None, 0, None, t[5].data_ptr(), K, 0),
-        }
-        for op, mk in ops.items():
-            args = [mk(t) for t in sets]
-            fns = [(lambda a=a: F._lib.fp8_mm(ctypes.byref(a), h)) for a in args]
-            us = _graph_us(stream, fns)
-            tf = 2.0 * M * N * K / us / 1e6
-            gemm.append({"shape": f"M={M} K={K} N={N}", "op": op, "us": round(us, 2), "tflops": round(tf, 1),
-                         "frac_nominal_4.5PF": round(tf / NOMINAL_FP8_TFLOPS, 3)})
-        del sets
+    for cfg_id, shapes in ((3, wl.C3_SHAPES), (4, wl.C4_SHAPES)):
+        for s in shapes:
+            M, K, N = s.M, s.K, s.N
+            per_set = M * K + N * K + M * N + 2 * (M * N + M * K + N * K)
+            nsets = _sets_for(per_set)
+            sets = []
+            for i in range(nsets):
+                x8 = torch.randint(0x20, 0x48, (M, K), dtype=torch.uint8, device=device)
+                w8 = torch.randint(0x20, 0x48, (N, K), dtype=torch.uint8, device=device)
+                g8 = torch.randint(0x20, 0x48, (M, N), dtype=torch.uint8, device=device)
+                b8 = torch.randint(0, 0xFF, (N,), dtype=torch.uint8, device=device) & 0xF7   # no NaN code
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+                dx = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+                dw = torch.empty((N, K), dtype=torch.bfloat16, device=device)
+                sets.append((x8, w8, g8, y, dx, dw, b8))
+            sp = sc.data_ptr()
+            with_bias = cfg_id == 3
+            # one stream-K workspace for the shape's three GEMMs (calls are stream-ordered)
+            ws = torch.zeros(max(16, F.fp8_mm_workspace_bytes(M, N, K), F.fp8_mm_workspace_bytes(M, K, N),
+                                 F.fp8_mm_workspace_bytes(N, K, M)), dtype=torch.uint8, device=device)
+            wp, wn = ws.data_ptr(), ws.numel()
+            ops = {
+                "fwd": lambda t: F.MmArgs(M, N, K, t[0].data_ptr(), 0, 0, K, t[1].data_ptr(), 0, 0, K, sp, sp + 4,
+                                          t[6].data_ptr() if with_bias else None, F.FP8_DT_E4M3,
+                                          sp + 8 if with_bias else None, t[3].data_ptr(), N, 0, wp, wn),
+                "dX": lambda t: F.MmArgs(M, K, N, t[2].data_ptr(), 1, 0, N, t[1].data_ptr(), 0, 1, K, sp, sp + 4,
+                                         None, 0, None, t[4].data_ptr(), K, 0, wp, wn),
+                "dW": lambda t: F.MmArgs(N, K, M, t[2].data_ptr(), 1, 1, N, t[0].data_ptr(), 0, 1, K, sp, sp + 4,
+                                         None, 0, None, t[5].data_ptr(), K, 0, wp, wn),
+            }
+            flops = 2.0 * M * N * K
+            for op, mk in ops.items():
+                nbytes = gemm_min_bytes(op, M, N, K, N if (op == "fwd" and with_bias) else 0)
+                roof = roofline_tflops(flops, nbytes, fp8_peak, hbm_gbs)
+                rec = {"config": cfg_id, "shape": f"M={M} K={K} N={N}", "op": op,
+                       "bias": "e4m3 + bias_scale" if (op == "fwd" and with_bias) else None,
+                       "gflop": round(flops / 1e9, 2), "min_bytes": nbytes,
+                       "ai_flop_per_byte": round(flops / nbytes, 1),
+                       "roofline_cold_tflops": round(roof, 1)}
+                for mode, ss in (("warm", sets[:1]), ("cold", sets)):
+                    args = [mk(t) for t in ss]
+                    fns = [(lambda a=a: F._lib.fp8_mm(ctypes.byref(a), h)) for a in args]
+                    us = _graph_us(stream, fns)
+                    tf = flops / us / 1e6
+                    plan = F.fp8_mm_plan(args[0], None, torch.cuda.get_device_properties(device).multi_processor_count)
+                    rec["plan"] = {"tile_cfg": plan.tile_cfg, "stream_k_ctas": plan.stream_k_ctas,
+                                   "dp_tiles": plan.dp_tiles}
+                    rec[mode] = {"us": round(us, 2), "tflops": round(tf, 1),
+                                 "frac_measured_peak": round(tf / fp8_peak, 3),
+                                 "frac_nominal_4.5PF": round(tf / NOMINAL_FP8_TFLOPS, 3),
+                                 "frac_roofline": round(tf / (fp8_peak if mode == "warm" else roof), 3)}
+                gemm.append(rec)
+            del sets, ws
     quant = []
     ring = torch.empty(F.fp8_ring_bytes(wl.HIST_LEN) // 4, dtype=torch.float32, device=device)
     F.fp8_ring_init(ring, wl.HIST_LEN)
@@ -385,7 +506,8 @@ def time_target_shapes(F, device, stream):
                for x, o in sets]
         us = _graph_us(stream, fns)
         gbs = per_set / us / 1e3
-        quant.append({"shape": f"{rows}x{cols} bf16->e4m3", "us": round(us, 2), "gbs": round(gbs, 1)})
+        quant.append({"shape": f"{rows}x{cols} bf16->e4m3", "us": round(us, 2), "gbs": round(gbs, 1),
+                      "frac_hbm": round(gbs / hbm_gbs, 3)})
         del sets
     return gemm, quant
 
@@ -398,10 +520,17 @@ def gemm_source_sha():
         return hashlib.sha256(fh.read()).hexdigest()[:16]
 
 
-def gemm_traffic_per_launch():
-    """DRAM bytes per GEMM launch from the committed ncu summary, or None when
-    the summary is missing or was taken on a different gemm.cu."""
-    p = os.path.join(ROOT, "profiles", "gemm_dram_traffic_dim1024_layer.txt")
+TRAFFIC_SUMMARY = {"c4": "gemm_dram_traffic_c4_step.txt", "dim1024": "gemm_dram_traffic_dim1024_layer.txt"}
+
+
+def gemm_traffic_per_launch(workload=HEADLINE):
+    """DRAM bytes per GEMM launch of the workload's step from the committed ncu
+    summary, or None when the summary is missing or was taken on a different
+    gemm.cu."""
+    name = TRAFFIC_SUMMARY.get(workload)
+    if name is None:
+        return None
+    p = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(p):
         return None
     kv = {}
@@ -420,32 +549,35 @@ def gemm_traffic_per_launch():
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def oracle_layer_sample(tokens: int, seed: int = 1234):
-    """The oracle's forward + backward of one dim1024 layer's six linears on
-    `tokens` tokens (quantize x/w/g with rings, fwd/dX/dW GEMMs, bias, dbias).
-    Returns (seconds, flops)."""
+def oracle_sample(tokens: int, seed: int = 1234):
+    """The oracle's forward + backward of the headline linears (the three
+    M=4096 shapes) on `tokens` tokens: quantize x (with outliers), w and g
+    with rings, fwd/dX/dW GEMMs with fp32 accumulation.  The weights are
+    quantized whole, as in a training step.  Returns (seconds, flops)."""
     import numpy as np
 
     import oracle
-    rng_seed = seed
     flops = 0
     prepared = []
-    for j, s in enumerate(wl.BENCH_LAYER):
-        x = wl.normal((tokens, s.K), 1.0, rng_seed + 10 * j)
-        w = wl.normal((s.N, s.K), wl.weight_std(s.K), rng_seed + 10 * j + 1)
-        b = wl.normal((s.N,), wl.BENCH_BIAS_STD, rng_seed + 10 * j + 2)
-        g = wl.normal((tokens, s.N), 1e-3, rng_seed + 10 * j + 3)
-        bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
-        prepared.append((s, bits(x), bits(w), bits(b), bits(g)))
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    for j, s in enumerate(wl.C4_SHAPES):
+        x = wl.normal_with_outliers((tokens, s.K), 1.0, seed + 10 * j, seed + 10 * j + 4)
+        w = wl.normal((s.N, s.K), wl.weight_std(s.K), seed + 10 * j + 1)
+        g = wl.normal((tokens, s.N), 1e-3, seed + 10 * j + 3)
+        prepared.append((s, bits(x), bits(w), bits(g)))
         flops += 6 * tokens * s.N * s.K
     t0 = time.perf_counter()
-    for s, x, w, b, g in prepared:
+    for s, x, w, g in prepared:
         rx, rw, rg = oracle.Ring(wl.HIST_LEN), oracle.Ring(wl.HIST_LEN), oracle.Ring(wl.HIST_LEN)
-        f = oracle.linear_forward(tokens, s.N, s.K, x, oracle.DT_BF16, w, oracle.DT_BF16, rx, rw, bias=b,
-                                  sumabs=False)
+        f = oracle.linear_forward(tokens, s.N, s.K, x, oracle.DT_BF16, w, oracle.DT_BF16, rx, rw, sumabs=False)
         oracle.linear_backward(tokens, s.N, s.K, g, oracle.DT_BF16, rg, f["x8"], oracle.E4M3, f["sx"], f["w8"],
-                               oracle.E4M3, f["sw"], need_dbias=True, sumabs=False)
+                               oracle.E4M3, f["sw"], sumabs=False)
     return time.perf_counter() - t0, flops
+
+
+def sample_text(tokens: int) -> str:
+    return (f"{tokens} of 4096 tokens of the three M=4096 linears (quantize x/w/g with rings -- the weights "
+            f"whole --, fwd+dX+dW GEMMs with fp32 accumulation)")
 
 
 def oracle_threads():
@@ -458,33 +590,37 @@ def run_reference(args):
     if rank != 0:
         return 0
     for _ in range(args.warmup):
-        oracle_layer_sample(REF_TOKENS)
+        oracle_sample(REF_TOKENS)
     secs, flops = [], 0
     for i in range(args.steps):
-        s, flops = oracle_layer_sample(REF_TOKENS, seed=4321 + i)
+        s, flops = oracle_sample(REF_TOKENS, seed=4321 + i)
         secs.append(s)
     total = sum(secs)
     value = flops * len(secs) / total / 1e12
-    sample = (f"{REF_TOKENS} of 2048 tokens of one of the 12 dim1024 layers per step (6 linears: quantize x/w/g "
-              f"with rings, fwd+dX+dW GEMMs, bf16 bias, dbias)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(secs),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8 e4m3/e5m2 (fp32 accumulate)",
-            "data": "synthetic", "config": config_dict(),
+            "data": "synthetic", "config": config_dict(HEADLINE),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample_text(REF_TOKENS) + " per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-def config_dict():
-    return {"workload": "12L/dim1024/B4xT512 linears: 12 layers x {q,k,v,o 1024x1024, up 1024x4096, "
-                        "down 4096x1024}, M=2048 tokens, fwd+dX+dW, E4M3 x/w, E5M2 g, delayed scaling H=16, "
-                        "bf16 bias + dbias",
-            "M": 2048, "layers": wl.BENCH_LAYERS, "linears_per_step": wl.BENCH_LAYERS * len(wl.BENCH_LAYER),
-            "hist_len": wl.HIST_LEN, "l2": "inputs larger than L2 (step working set ~3 GB, 126 MB L2)",
-            "timing": "CUDA graph of the step's C-ABI calls, CUDA events, max over ranks"}
+def config_dict(workload=HEADLINE, lins=None):
+    d = {"workload": WORKLOADS[workload][0], "hist_len": wl.HIST_LEN,
+         "timing": "CUDA graph of the step's C-ABI calls, CUDA events, max over ranks"}
+    if workload == "c4":
+        d.update(M=4096, linears_per_step=3,
+                 l2="inputs larger than L2 (step working set ~1.6 GB, 126 MB L2)")
+    elif workload == "dim1024":
+        d.update(M=2048, layers=wl.BENCH_LAYERS, linears_per_step=wl.BENCH_LAYERS * len(wl.BENCH_LAYER),
+                 l2="inputs larger than L2 (step working set ~3 GB, 126 MB L2)")
+    else:
+        d.update(M=[512, 2048], linears_per_step=len(wl.C3_SHAPES),
+                 l2="inputs larger than L2 (step working set ~0.5 GB, 126 MB L2)")
+    return d
 
 
 # --------------------------------------------------------------------------- end to end
@@ -563,16 +699,87 @@ def time_e2e(F, lins, host_in, host_out, comp, device, steps):
 
 # --------------------------------------------------------------------------- main
 
+def working_set_bytes(lins) -> int:
+    ts = []
+    for L in lins:
+        ts += L.inputs() + L.outputs() + [L.x8, L.w8, L.g8]
+    return sum(t.numel() * t.element_size() for t in ts)
+
+
+def graph_kernel_nodes(graph):
+    """Kernel nodes of a captured CUDA graph -- the kernel launches one replay
+    runs (None when the graph cannot be inspected)."""
+    try:
+        from cuda.bindings import runtime as rt
+        g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(g, numNodes=0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(g, numNodes=n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        count = 0
+        for nd in nodes[:n]:
+            err, t = rt.cudaGraphNodeGetType(nd)
+            if err == rt.cudaError_t.cudaSuccess and t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                count += 1
+        return count
+    except Exception:
+        return None
+
+
+def capture_step(F, lins, stream, warmup):
+    """Eager step (first-launch set-up outside the capture), then the step
+    captured as one CUDA graph (kept, so its kernel nodes can be counted) and
+    replayed `warmup` times."""
+    with torch.cuda.stream(stream):
+        run_step(F, lins, stream.cuda_stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(graph, stream=stream):
+        run_step(F, lins, stream.cuda_stream)
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    return graph
+
+
+def time_graph_ms(graph, stream, reps):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def fp8_peak_for(pk, clocks):
+    """The measured fp8 denominator: measured bf16 GEMM x the nominal fp8:bf16
+    ratio -- the burst figure while the timed region held the maximum SM
+    clock with no power-cap reason, the sustained figure (seconds-long loop
+    under the power cap) otherwise."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    capped = "sw_power_cap" in clocks.get("reasons", []) or (mhz is not None and mx and mhz < 0.97 * mx)
+    key = "bf16_tflops_sustained" if capped and "bf16_tflops_sustained" in pk else "bf16_tflops"
+    return pk[key] * FP8_PER_BF16, key
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--layers", type=int, default=wl.BENCH_LAYERS, help="layers per step (profiling runs only)")
-    ap.add_argument("--no-extras", action="store_true", help="skip e2e, kernel timing and cpu baseline")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS),
+                    help="workload of the timed step (the headline by default)")
+    ap.add_argument("--layers", type=int, default=wl.BENCH_LAYERS, help="layers of the dim1024 workload "
+                    "(profiling runs only)")
+    ap.add_argument("--no-extras", action="store_true", help="skip e2e, kernel timing, targets and cpu baseline")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    wl.BENCH_LAYERS = args.layers
     if args.impl == "reference":
         return run_reference(args)
 
@@ -587,66 +794,53 @@ def main(argv=None):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
 
-    wl.BENCH_LAYERS = args.layers
-    lins = build_model(F, device, rank)
+    lins = build_model(F, device, rank, args.workload)
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize()
-    flops_step = wl.bench_flops_per_step(args.layers)
-
-    # eager warm-up (first-launch set-up happens outside the capture), then capture
-    with torch.cuda.stream(stream):
-        run_step(F, lins, stream.cuda_stream)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        run_step(F, lins, stream.cuda_stream)
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
+    flops_step = step_flops(lins)
+    graph = capture_step(F, lins, stream, args.warmup)
 
     # ---- timed region
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
-        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(args.steps):
-                graph.replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
+        ms = time_graph_ms(graph, stream, args.steps)
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
     max_ms = reduce_max(ms, world, device)
     value = aggregate_throughput(flops_step * args.steps, world, max_ms / 1e3) / 1e12
     status = F.fp8_get_device_status()
     if status:
         raise F.Fp8Error(status, "device status after timed region")
+    clocks = clk.report()
+    cfg = config_dict(args.workload)
+    cfg["working_set_bytes"] = working_set_bytes(lins)
 
+    kernels_per_step = graph_kernel_nodes(graph)
+    cfg["kernels_per_step"] = kernels_per_step if kernels_per_step is not None else \
+        f"not inspectable; at least {LAUNCHES_PER_LINEAR * len(lins)}"
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8 e4m3/e5m2 (fp32 accumulate, bf16 out)", "data": "synthetic",
-            "config": config_dict(), "clocks": clk.report(),
-            "gpu_launches": LAUNCHES_PER_LINEAR * len(lins) * args.steps}
+            "config": cfg, "clocks": clocks,
+            "gpu_launches": (kernels_per_step or LAUNCHES_PER_LINEAR * len(lins)) * args.steps}
 
     if not args.no_extras:
         pk, pk_kind = peaks()
-        # ---- kernel-level timing and roofline of the dominant kernel
+        fp8_peak, peak_key = fp8_peak_for(pk, clocks)
+        # ---- kernel-level timing and roofline of the dominant kernel (the GEMM class)
         tot, work, count, shapes = time_kernels(F, lins, stream)
         gemm_tflops = work["gemm"] / (tot["gemm"] / 1e3) / 1e12
-        fp8_peak = pk["bf16_tflops"] * FP8_PER_BF16
-        traffic = gemm_traffic_per_launch()
+        traffic = gemm_traffic_per_launch(args.workload)
         line["roofline"] = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                             "frac": gemm_tflops / fp8_peak, "traffic": traffic,
-                            "kernel": "fp8_gemm_kernel (the step's 144 launches: 72 forward, 72 dX+dW pairs, "
-                                      "replayed as one graph)",
-                            "peak_source": f"{pk_kind} bf16 burst x {FP8_PER_BF16} (nominal fp8:bf16)",
+                            "kernel": f"fp8_gemm_kernel (the step's {count['gemm']} GEMM launches: forward and "
+                                      f"dX+dW pairs, replayed as one graph)",
+                            "peak_source": f"{pk_kind} {peak_key} x {FP8_PER_BF16} (nominal fp8:bf16)",
                             "frac_of_nominal_4.5PF": gemm_tflops / NOMINAL_FP8_TFLOPS}
         # Inside fp8_linear_forward/backward the quantize launches leave the
-        # ring finalize and the bias-gradient sums to the GEMM that follows;
+        # ring finalize (and any bias-gradient sums) to the GEMM that follows;
         # the standalone quantize calls the class graph replays finalize in
         # their last block.  The step's quantize time is therefore taken as
         # the step minus the GEMM class.
@@ -660,17 +854,43 @@ def main(argv=None):
             "quantize_standalone_class_ms": tot["quantize"],
             "quantize": {"achieved_gbs": q_gbs, "peak_gbs": pk["hbm_gbs"], "frac": q_gbs / pk["hbm_gbs"],
                          "bytes_per_elem": 3,
-                         "note": "bf16 in + fp8 out; x+w in one launch, g with its bias-gradient partials in one "
-                                 "launch; time = step minus the GEMM class graph"},
+                         "note": "bf16 in + fp8 out; x+w in one launch, g (with its bias-gradient partials when "
+                                 "the bias needs a gradient) in one launch; time = step minus the GEMM class graph"},
             "gemm_by_shape": shapes}
-        tg, tq = time_target_shapes(F, device, stream)
-        for r in tq:
-            r["frac_hbm"] = round(r["gbs"] / pk["hbm_gbs"], 3)
+
+        # ---- the other workloads' steps, timed the same way
+        others = {}
+        for wname in WORKLOADS:
+            if wname == args.workload:
+                continue
+            olins = build_model(F, device, rank, wname)
+            og = capture_step(F, olins, stream, args.warmup)
+            oreps = max(5, args.steps // 2)
+            if world > 1:
+                dist.barrier()
+            oms = reduce_max(time_graph_ms(og, stream, oreps), world, device)
+            ofl = step_flops(olins)
+            ot, owork, ocount, _ = time_kernels(F, olins, stream)
+            otf = owork["gemm"] / (ot["gemm"] / 1e3) / 1e12
+            others[wname] = {"workload": WORKLOADS[wname][0],
+                             "value": aggregate_throughput(ofl * oreps, world, oms / 1e3) / 1e12, "unit": UNIT,
+                             "ms_per_step": oms / oreps,
+                             "gpu_launches_per_step": graph_kernel_nodes(og) or LAUNCHES_PER_LINEAR * len(olins),
+                             "gemm_class": {"tflops": otf, "frac_measured_peak": otf / fp8_peak,
+                                            "ms_per_step": ot["gemm"]}}
+            del og, olins
+            torch.cuda.synchronize()
+        if F.fp8_get_device_status():
+            raise F.Fp8Error(F.fp8_get_device_status(), "device status after the other workloads")
+        line["steps_other_workloads"] = others
+
+        tg, tq = time_target_shapes(F, device, stream, fp8_peak, pk["hbm_gbs"])
         line["targets"] = {
-            "gemm": tg, "quantize": tq,
+            "gemm": tg, "quantize": tq, "fp8_peak_tflops": fp8_peak, "hbm_gbs": pk["hbm_gbs"],
             "note": "separate fp8_mm launches per operation (dX, dW in the fused backward's in-place "
-                    "transposed layouts), operand sets cycled so each pass streams more than L2; quantize "
-                    "standalone (in-kernel ring finalize)"}
+                    "transposed layouts); warm = the same operands back to back, cold = operand sets cycled so "
+                    "each pass streams more than L2; frac_roofline = achieved / min(peak, AI x HBM BW) cold, "
+                    "achieved / peak warm; quantize standalone (in-kernel ring finalize), cold"}
 
         # ---- end to end through the C ABI with host buffers
         host_in = [[t.cpu().pin_memory() for t in L.inputs()] for L in lins]
@@ -685,19 +905,16 @@ def main(argv=None):
         line["e2e"] = {"value": aggregate_throughput(flops_step * e2e_steps, world, e2e_ms / 1e3) / 1e12,
                        "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps,
-                       "path": "pinned host -> device copies of x, w, b, g (copy stream), fp8_linear_forward/"
-                               "backward per linear (compute stream), device -> pinned host copies of y, dX, dW, "
-                               "dbias (second copy stream); per-linear events, so the two copy directions and the "
-                               "kernels overlap"}
+                       "path": "pinned host -> device copies of each linear's inputs (copy stream), "
+                               "fp8_linear_forward/backward per linear (compute stream), device -> pinned host copies "
+                               "of its outputs (second copy stream); per-linear events, so the two copy directions "
+                               "and the kernels overlap"}
 
         # ---- CPU oracle baseline (rank 0, one GPU only)
         if rank == 0 and world == 1:
-            secs, flops = oracle_layer_sample(CPU_SAMPLE_TOKENS)
-            line["cpu_baseline"] = {
-                "value": flops / secs / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                "sample": f"{CPU_SAMPLE_TOKENS} of 2048 tokens of one of the 12 dim1024 layers (6 linears: quantize "
-                          f"x/w/g with rings, fwd+dX+dW GEMMs with fp32 accumulation, bf16 bias, dbias), "
-                          f"{secs:.1f} s"}
+            secs, flops = oracle_sample(CPU_SAMPLE_TOKENS)
+            line["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": UNIT, "cores": oracle_threads(),
+                                    "kind": "oracle", "sample": sample_text(CPU_SAMPLE_TOKENS) + f", {secs:.1f} s"}
 
     if world > 1:
         del graph

@@ -25,6 +25,7 @@ FP8_E4M3, FP8_E5M2 = 0, 1
 FP8_DT_BF16, FP8_DT_FP16, FP8_DT_FP32, FP8_DT_E4M3, FP8_DT_E5M2 = 0, 1, 2, 3, 4
 FP8_K_MAJOR, FP8_MN_MAJOR = 0, 1
 FP8_TILE_AUTO, FP8_TILE_128x128, FP8_TILE_128x256, FP8_TILE_PAIR_256x256, FP8_TILE_SPLITK_128x128 = 0, 1, 2, 3, 4
+FP8_TILE_STREAMK = 8
 FP8_OK = 0
 FP8_ERR_INVALID_ARG, FP8_ERR_UNSUPPORTED, FP8_ERR_MISALIGNED = -1, -2, -3
 FP8_ERR_CUDA, FP8_ERR_DEVICE_TIMEOUT, FP8_ERR_WORKSPACE = -4, -5, -6
@@ -53,11 +54,13 @@ class MmArgs(ctypes.Structure):
                 ("scale_a", _P), ("scale_b", _P),
                 ("bias", _P), ("bias_dtype", _I), ("bias_scale", _P),
                 ("d", _P), ("ldd", _I64),
-                ("tile_cfg", _I)]
+                ("tile_cfg", _I),
+                ("workspace", _P), ("workspace_bytes", _SZ)]
 
 
 class MmPlanInfo(ctypes.Structure):
-    _fields_ = [("tile_cfg", _I), ("tiles", _I64), ("units", _I), ("est_us", ctypes.c_double)]
+    _fields_ = [("tile_cfg", _I), ("tiles", _I64), ("units", _I), ("est_us", ctypes.c_double),
+                ("stream_k_ctas", _I), ("dp_tiles", _I64)]
 
 
 class QuantizeArgs(ctypes.Structure):
@@ -77,7 +80,8 @@ class LinearFwdArgs(ctypes.Structure):
                 ("x8", _P), ("ldx8", _I64),
                 ("w8", _P), ("ldw8", _I64),
                 ("sx_out", _P), ("sw_out", _P), ("amax_x_out", _P), ("amax_w_out", _P),
-                ("y", _P), ("ldy", _I64)]
+                ("y", _P), ("ldy", _I64),
+                ("workspace", _P), ("workspace_bytes", _SZ)]
 
 
 class LinearBwdArgs(ctypes.Structure):
@@ -106,6 +110,7 @@ _SIGS = {
     "fp8_mm_plan": (_I, [ctypes.POINTER(MmArgs), ctypes.POINTER(MmArgs), _I, ctypes.POINTER(MmPlanInfo)]),
     "fp8_mm_pair": (_I, [ctypes.POINTER(MmArgs), ctypes.POINTER(MmArgs), _P]),
     "fp8_mm_batched": (_I, [ctypes.POINTER(MmArgs), _I64, _I64, _I64, _I64, _P]),
+    "fp8_mm_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "fp8_quantize_ex": (_I, [ctypes.POINTER(QuantizeArgs), _I, _P]),
     "fp8_ring_finalize": (_I, [_P, _I, _I, _P, _P]),
     "fp8_dbias_workspace_bytes": (_SZ, [_I64, _I64]),
@@ -160,6 +165,10 @@ def _dtype_code(t: torch.Tensor, fp8_fmt: int | None = None) -> int:
     if t.dtype == torch.uint8 and fp8_fmt is not None:
         return FP8_DT_E4M3 + fp8_fmt
     raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 def _ld(t: torch.Tensor) -> int:
@@ -238,11 +247,23 @@ def fp8_mm_batched(a: MmArgs, batch: int, stride_a: int, stride_b: int, stride_d
 
 
 def fp8_mm(m, n, k, a, fmt_a, a_major, lda, b, fmt_b, b_major, ldb, scale_a, scale_b, d, ldd,
-           bias=None, bias_dtype=FP8_DT_BF16, bias_scale=None, stream=None, tile_cfg=FP8_TILE_AUTO) -> None:
+           bias=None, bias_dtype=FP8_DT_BF16, bias_scale=None, stream=None, tile_cfg=FP8_TILE_AUTO,
+           workspace=None) -> None:
     args = MmArgs(m, n, k, _ptr(a), fmt_a, a_major, lda, _ptr(b), fmt_b, b_major, ldb,
-                  _ptr(scale_a), _ptr(scale_b), _ptr(bias), bias_dtype, _ptr(bias_scale), _ptr(d), ldd, tile_cfg)
+                  _ptr(scale_a), _ptr(scale_b), _ptr(bias), bias_dtype, _ptr(bias_scale), _ptr(d), ldd, tile_cfg,
+                  _ptr(workspace), _nbytes(workspace))
     s = stream if stream is not None else _stream(d.device if isinstance(d, torch.Tensor) else None)
     _check(_lib.fp8_mm(ctypes.byref(args), s), "fp8_mm")
+
+
+def fp8_mm_workspace_bytes(m: int, n: int, k: int) -> int:
+    return _lib.fp8_mm_workspace_bytes(m, n, k)
+
+
+def mm_workspace(m: int, n: int, k: int, device) -> torch.Tensor | None:
+    """A zero-filled stream-K workspace for GEMMs of this size (None when empty)."""
+    nb = fp8_mm_workspace_bytes(m, n, k)
+    return torch.zeros(nb, dtype=torch.uint8, device=device) if nb else None
 
 
 def fp8_mm_plan(a: MmArgs, b: MmArgs | None = None, num_sms: int = 148) -> MmPlanInfo:
@@ -364,9 +385,12 @@ class ForwardResult:
 
 def linear_forward(x, w, ring_x: ScaleRing | None, ring_w: ScaleRing | None, bias=None, bias_scale=None,
                    fmt_x=FP8_E4M3, fmt_w=FP8_E4M3, x_scale_in=None, w_scale_in=None, hist_len=16,
-                   y=None, x8=None, w8=None) -> ForwardResult:
+                   y=None, x8=None, w8=None, scales=None, workspace=None) -> ForwardResult:
     """y = x w^T + bias through fp8_linear_forward.  x/w may be bf16/fp16/fp32
-    or fp8 codes (torch.float8_* or uint8 with their fmt, plus *_scale_in)."""
+    or fp8 codes (torch.float8_* or uint8 with their fmt, plus *_scale_in).
+    scales: optional 4-element fp32 device buffer receiving sx, sw, amax_x,
+    amax_w (allocated here when None).  workspace: optional zero-filled
+    stream-K workspace of the GEMM (mm_workspace(M, N, K))."""
     M, K = x.shape
     N = w.shape[0]
     dev = x.device
@@ -377,7 +401,7 @@ def linear_forward(x, w, ring_x: ScaleRing | None, ring_w: ScaleRing | None, bia
         x8 = x.view(torch.uint8) if xq else fp8_alloc(M, K, dev)
     if w8 is None:
         w8 = w.view(torch.uint8) if wq else fp8_alloc(N, K, dev)
-    sc = torch.empty(4, dtype=torch.float32, device=dev)
+    sc = torch.empty(4, dtype=torch.float32, device=dev) if scales is None else scales
     H = ring_x.H if ring_x is not None else (ring_w.H if ring_w is not None else hist_len)
     bias_dtype = FP8_DT_BF16
     if bias is not None and bias.dtype != torch.bfloat16:
@@ -391,7 +415,7 @@ def linear_forward(x, w, ring_x: ScaleRing | None, ring_w: ScaleRing | None, bia
         _ptr(ring_x.buf) if ring_x is not None else None, _ptr(ring_w.buf) if ring_w is not None else None,
         _ptr(x8), _ld(x8), _ptr(w8), _ld(w8),
         _ptr(sc[0:1]), _ptr(sc[1:2]), _ptr(sc[2:3]), _ptr(sc[3:4]),
-        _ptr(y), _ld(y))
+        _ptr(y), _ld(y), _ptr(workspace), _nbytes(workspace))
     fp8_linear_forward(args, dev)
     return ForwardResult(y, x8, w8, sc[0:1], sc[1:2], sc[2:3], sc[3:4])
 
@@ -421,6 +445,7 @@ def linear_backward(g, fwd: ForwardResult, ring_g: ScaleRing | None, fmt_g=FP8_E
     dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if (need_dw and dw is None) else dw
     dbias = torch.empty(N, dtype=torch.bfloat16, device=dev) if (need_dbias and dbias is None) else dbias
     if need_dbias and workspace is None:
+        # the bias-gradient scratch and the dX + dW launch's stream-K scratch
         workspace = torch.zeros(max(16, fp8_linear_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
     sc = torch.empty(2, dtype=torch.float32, device=dev)
     H = ring_g.H if ring_g is not None else 16

@@ -76,7 +76,11 @@ float fp8_max(int fmt) { return fmt == FP8_E4M3 ? 448.0f : 57344.0f; }
 bool ring_len_ok(int H) { return H >= 1 && H <= 4096; }
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
-int check_fp8_matrix(const void* p, int64_t ld, int64_t cols) {
+// An fp8 matrix [rows, ld] the kernels read or write with TMA or 16-byte
+// accesses.  An empty one (no rows or no columns) is never touched, so its
+// pointer and stride are not checked.
+int check_fp8_matrix(const void* p, int64_t ld, int64_t rows, int64_t cols) {
+  if (rows == 0 || cols == 0) return FP8_OK;
   if (!p) return FP8_ERR_INVALID_ARG;
   if (ld < cols) return FP8_ERR_INVALID_ARG;
   if (ld % 16 != 0 || !aligned(p, 16)) return FP8_ERR_MISALIGNED;
@@ -127,7 +131,32 @@ struct MmCall {
   // batched GEMMs (fp8_mm_batched): element strides between batches; a zero
   // operand stride shares that operand across the batch
   int64_t batch = 1, stride_a = 0, stride_b = 0, stride_d = 0;
+  // stream-K workspace (optional): zero-at-rest flags, then partial slots
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
 };
+
+// Stream-K scratch: a fixed block of flags (one per epilogue warp of up to
+// kSkMaxCtas CTAs, zero at rest), then one partial accumulator slot per CTA.
+constexpr int kSkMaxCtas = 160;
+constexpr int kSkWarps = 8;
+constexpr size_t kSkFlagBytes = static_cast<size_t>(kSkMaxCtas) * kSkWarps * 4;
+constexpr size_t kSkSlotBytes = 128 * 256 * 4;   // the largest tile's fp32 accumulator
+constexpr int64_t kSkMinUnits = 4;               // k-blocks per CTA below which stream-K is not used
+constexpr int64_t kSkMaxParts = 6;               // partials a finishing CTA stages (24 KB per epilogue warp)
+
+// Slots a stream-K launch of this size can use: at most one per CTA and per
+// 128 x 128 x 128 block of work.
+int64_t sk_slots_for(int64_t m, int64_t n, int64_t k) {
+  if (m <= 0 || n <= 0 || k <= 0) return 0;
+  const int64_t blocks = ((m + 127) / 128) * ((n + 127) / 128) * ((k + 127) / 128);
+  return std::min<int64_t>(kSkMaxCtas, blocks);
+}
+
+size_t sk_bytes_for(int64_t m, int64_t n, int64_t k) {
+  const int64_t slots = sk_slots_for(m, n, k);
+  return slots ? kSkFlagBytes + static_cast<size_t>(slots) * kSkSlotBytes : 0;
+}
 
 int validate_mm(const MmCall& c) {
   if (c.m < 0 || c.n < 0 || c.k < 0 || c.m > kMaxDim || c.n > kMaxDim || c.k > kMaxDim) return FP8_ERR_INVALID_ARG;
@@ -135,19 +164,33 @@ int validate_mm(const MmCall& c) {
   if ((c.a_major != FP8_K_MAJOR && c.a_major != FP8_MN_MAJOR) ||
       (c.b_major != FP8_K_MAJOR && c.b_major != FP8_MN_MAJOR))
     return FP8_ERR_INVALID_ARG;
-  if (!c.scale_a || !c.scale_b || !c.d) return FP8_ERR_INVALID_ARG;
-  int s = check_fp8_matrix(c.a, c.lda, c.a_major == FP8_K_MAJOR ? c.k : c.m);
+  if (!c.scale_a || !c.scale_b) return FP8_ERR_INVALID_ARG;
+  int s = c.a_major == FP8_K_MAJOR ? check_fp8_matrix(c.a, c.lda, c.m, c.k) : check_fp8_matrix(c.a, c.lda, c.k, c.m);
   if (s) return s;
-  s = check_fp8_matrix(c.b, c.ldb, c.b_major == FP8_K_MAJOR ? c.k : c.n);
+  s = c.b_major == FP8_K_MAJOR ? check_fp8_matrix(c.b, c.ldb, c.n, c.k) : check_fp8_matrix(c.b, c.ldb, c.k, c.n);
   if (s) return s;
-  if (c.ldd < c.n || !aligned(c.d, 2)) return FP8_ERR_INVALID_ARG;
-  if (c.tile_cfg < FP8_TILE_AUTO || c.tile_cfg > FP8_TILE_SPLITK_128x128) return FP8_ERR_INVALID_ARG;
+  if (c.m > 0 && c.n > 0 && (!c.d || c.ldd < c.n || !aligned(c.d, 2))) return FP8_ERR_INVALID_ARG;
+  const int base_cfg = c.tile_cfg & ~FP8_TILE_STREAMK;
+  if (base_cfg < FP8_TILE_AUTO || base_cfg > FP8_TILE_SPLITK_128x128) return FP8_ERR_INVALID_ARG;
+  if ((c.tile_cfg & FP8_TILE_STREAMK) && base_cfg != FP8_TILE_128x128 && base_cfg != FP8_TILE_128x256)
+    return FP8_ERR_INVALID_ARG;
+  if (c.ws_bytes && (!c.ws || !aligned(c.ws, 16))) return FP8_ERR_WORKSPACE;
   if (c.bias) {
     if (c.bias_dtype != FP8_DT_BF16 && !is_fp8(c.bias_dtype)) return FP8_ERR_INVALID_ARG;
     if (is_fp8(c.bias_dtype) && !c.bias_scale) return FP8_ERR_INVALID_ARG;
     if (c.bias_dtype == FP8_DT_BF16 && !aligned(c.bias, 2)) return FP8_ERR_INVALID_ARG;
   }
   return FP8_OK;
+}
+
+// The call an fp8_mm_args describes (tile configuration and workspace from
+// `lead`, the first GEMM of a launch).
+MmCall mm_call(const fp8_mm_args* x, const fp8_mm_args* lead) {
+  MmCall c{x->m, x->n, x->k, x->a, x->fmt_a, x->a_major, x->lda, x->b, x->fmt_b, x->b_major, x->ldb,
+           x->scale_a, x->scale_b, x->bias, x->bias_dtype, x->bias_scale, x->d, x->ldd, lead->tile_cfg};
+  c.ws = lead->workspace;
+  c.ws_bytes = lead->workspace_bytes;
+  return c;
 }
 
 // Per-tile cost, in k-blocks, of the schedule models: the mainloop plus the
@@ -197,6 +240,15 @@ int64_t lpt_schedule(int64_t count0, int64_t cost0, int64_t count1, int64_t cost
   return makespan;
 }
 
+// A launch's tile configuration and schedule.
+struct TilePlan {
+  int cfg = kGemm128;
+  int sk_ctas = 0;         // stream-K: CTAs sharing the cut tiles' k-blocks (0: none)
+  int dp_tiles = 0;        // stream-K: tiles run whole first
+  int64_t sk_total = 0, sk_u0 = 0;
+  double est_us = 0.0;
+};
+
 // Tile configuration with the smallest modelled time for a launch of one or
 // two problems: the makespan (k-blocks) of the launch's tile schedule -- the
 // LPT schedule the single-CTA configurations run for two problems of unequal
@@ -208,38 +260,98 @@ int64_t lpt_schedule(int64_t count0, int64_t cost0, int64_t count1, int64_t cost
 // launches (the single-CTA tile moves 1.5x the operand bytes per SM through
 // L2, which tells once the whole chip streams for long); ~4-5 us fill +
 // epilogue + launch.
-int pick_tile(const MmCall* calls, int n, int sms, double* est_us = nullptr) {
-  struct Opt { int cfg; int64_t tm, tn, units; double t_kb, t_kb_long, fixed; };
-  const Opt opts[3] = {{kGemm128, 128, 128, sms, 0.31, 0.31, 4.0}, {kGemm256, 128, 256, sms, 0.35, 0.40, 4.0},
-                       {kGemmPair256, 256, 256, sms / 2, 0.37, 0.365, 5.0}};
-  int best = kGemm128;
-  double best_t = -1.0;
+// With sk_slots > 0 (a stream-K workspace of that many partial slots), the
+// single-CTA configurations are also costed with stream-K: whole waves but
+// the last one or two run data-parallel, the remaining tiles' k-blocks are
+// split evenly over min(SMs, slots) CTAs (at least kSkMinUnits each, and few
+// enough that a tile has at most kSkMaxParts partials), plus a fixup for the
+// cut tiles: the partials' release and acquire, then the finishing CTA's bulk
+// copies of the partials into its idle operand ring (one round per six 4 KB
+// (step, partial) blocks of each epilogue warp).  force_sk: only stream-K
+// plans of the given configuration.
+TilePlan pick_tile(const MmCall* calls, int n, int sms, int64_t sk_slots = 0, int force_cfg = 0,
+                   bool force_sk = false) {
+  struct Opt { int cfg; int64_t tm, tn, units; double t_kb, t_kb_long, fixed, fixup; };
+  const Opt opts[3] = {{kGemm128, 128, 128, sms, 0.31, 0.31, 4.0, 1.5},
+                       {kGemm256, 128, 256, sms, 0.35, 0.40, 4.0, 1.5},
+                       {kGemmPair256, 256, 256, sms / 2, 0.37, 0.365, 5.0, 0.0}};
+  TilePlan best;
+  bool have = false;
+  bool batched = false;
+  for (int i = 0; i < n; ++i) batched = batched || calls[i].batch > 1;
   for (const Opt& o : opts) {
+    if (force_cfg && o.cfg != force_cfg) continue;
     int64_t cnt[2] = {0, 0}, kb[2] = {0, 0};
     for (int i = 0; i < n; ++i) {
       cnt[i] = ((calls[i].m + o.tm - 1) / o.tm) * ((calls[i].n + o.tn - 1) / o.tn) * calls[i].batch;
       kb[i] = (calls[i].k + 127) / 128;
     }
-    int64_t span;
-    if (o.cfg != kGemmPair256 && n == 2 && kb[0] != kb[1]) {
-      span = lpt_schedule(cnt[0], kb[0], cnt[1], kb[1], o.units, nullptr, nullptr);
-    } else {  // round robin: unit u runs tiles u, u + units, ...
-      span = 0;
-      const int64_t total = cnt[0] + cnt[1];
-      const int64_t units = std::max<int64_t>(1, std::min(o.units, total));
-      for (int64_t u = 0; u < std::min(units, total); ++u) {
-        int64_t load = 0;
-        // tiles of problem 0 at u, u + units, ... then problem 1
-        for (int64_t t = u; t < total; t += units) load += (t < cnt[0] ? kb[0] : kb[1]) + kTileFixedKb;
-        span = std::max(span, load);
+    const int64_t tiles = cnt[0] + cnt[1];
+    if (!force_sk) {
+      int64_t span;
+      if (o.cfg != kGemmPair256 && n == 2 && kb[0] != kb[1]) {
+        span = lpt_schedule(cnt[0], kb[0], cnt[1], kb[1], o.units, nullptr, nullptr);
+      } else {  // round robin: unit u runs tiles u, u + units, ...
+        span = 0;
+        const int64_t units = std::max<int64_t>(1, std::min(o.units, tiles));
+        for (int64_t u = 0; u < std::min(units, tiles); ++u) {
+          int64_t load = 0;
+          // tiles of problem 0 at u, u + units, ... then problem 1
+          for (int64_t t = u; t < tiles; t += units) load += (t < cnt[0] ? kb[0] : kb[1]) + kTileFixedKb;
+          span = std::max(span, load);
+        }
+      }
+      const int64_t rounds = (tiles + o.units - 1) / std::max<int64_t>(1, o.units);
+      const double t = static_cast<double>(span - kTileFixedKb) * (rounds > 3 ? o.t_kb_long : o.t_kb) + o.fixed;
+      if (!have || t < best.est_us) {
+        best = TilePlan{};
+        best.cfg = o.cfg;
+        best.est_us = t;
+        have = true;
       }
     }
-    const int64_t tiles = cnt[0] + cnt[1];
-    const int64_t rounds = (tiles + o.units - 1) / std::max<int64_t>(1, o.units);
-    const double t = static_cast<double>(span - kTileFixedKb) * (rounds > 3 ? o.t_kb_long : o.t_kb) + o.fixed;
-    if (best_t < 0 || t < best_t) { best = o.cfg; best_t = t; }
+    // stream-K (single-CTA tiles, unbatched)
+    if (o.cfg == kGemmPair256 || batched || sk_slots <= 0) continue;
+    const int64_t P = std::min<int64_t>(sms, kSkMaxCtas);
+    const int64_t D = tiles >= 2 * P ? (tiles / P - 1) * P : 0;
+    const int64_t u0 = D < cnt[0] ? (cnt[0] - D) * kb[0] : 0;
+    const int64_t u1 = (tiles - std::max(D, cnt[0])) * kb[1];
+    const int64_t U = u0 + u1;
+    // at least kSkMinUnits k-blocks per CTA, and ranges long enough that a
+    // tile is cut into at most kSkMaxParts + 1 parts (the finishing CTA stages
+    // at most kSkMaxParts partials): ceil((kb - 1) / floor(U / ctas)) <= 6
+    const int64_t kbmax = std::max(kb[0], kb[1]);
+    const int64_t min_units = std::max<int64_t>(kSkMinUnits, (kbmax - 1 + kSkMaxParts - 1) / kSkMaxParts);
+    int64_t ctas = std::min({P, sk_slots, std::max<int64_t>(force_sk ? 1 : 0, U / min_units)});
+    while (ctas > 1 && (kbmax - 1 + U / ctas - 1) / (U / ctas) > kSkMaxParts) --ctas;
+    if (ctas < (force_sk ? 1 : 2)) continue;
+    const int64_t nparts = U / ctas > 0 ? (kbmax - 1 + U / ctas - 1) / (U / ctas) : 0;
+    int64_t dp_span = 0;
+    for (int64_t u = 0; u < std::min(P, D); ++u) {
+      int64_t load = 0;
+      for (int64_t t = u; t < D; t += P) load += (t < cnt[0] ? kb[0] : kb[1]) + kTileFixedKb;
+      dp_span = std::max(dp_span, load);
+    }
+    const int64_t sk_span = (U + ctas - 1) / ctas + kTileFixedKb;
+    // fixup: flags, then the staged partials in rounds of 6 (step, part) blocks
+    const int64_t steps = o.tn / 64;
+    const int64_t rounds = nparts > 0 ? (steps + std::max<int64_t>(1, kSkMaxParts / nparts) - 1) /
+                                            std::max<int64_t>(1, kSkMaxParts / nparts)
+                                      : 0;
+    const double fixup = nparts > 0 ? o.fixup + 0.6 * static_cast<double>(rounds) : 0.0;
+    const double t = static_cast<double>(dp_span + sk_span - kTileFixedKb) * o.t_kb_long + o.fixed + fixup;
+    // stream-K only for a clear gain (5 %) over the data-parallel plans
+    if (!have || (force_sk ? t < best.est_us : t < 0.95 * best.est_us)) {
+      best = TilePlan{};
+      best.cfg = o.cfg;
+      best.sk_ctas = static_cast<int>(ctas);
+      best.dp_tiles = static_cast<int>(D);
+      best.sk_total = U;
+      best.sk_u0 = u0;
+      best.est_us = t;
+      have = true;
+    }
   }
-  if (est_us) *est_us = best_t;
   return best;
 }
 
@@ -300,6 +412,88 @@ int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) 
 // Enqueue one launch running n (1 or 2) validated GEMMs over one persistent
 // tile schedule.  side: writes folded into the launch; fin: rings whose
 // quantize deferred its finalize to this launch.
+// Stream-K slots the calls' workspace holds (0: no usable workspace).  A
+// two-GEMM launch shares calls[0]'s workspace.
+int64_t sk_slots_available(const MmCall* calls, int n) {
+  if (!calls[0].ws || calls[0].ws_bytes < kSkFlagBytes + kSkSlotBytes) return 0;
+  int64_t need = 0;
+  for (int i = 0; i < n; ++i) need = std::max(need, sk_slots_for(calls[i].m, calls[i].n, calls[i].k));
+  const int64_t have = static_cast<int64_t>((calls[0].ws_bytes - kSkFlagBytes) / kSkSlotBytes);
+  return std::min(need, have);
+}
+
+// The plan of a launch: the forced configuration (stream-K when flagged), or
+// the cost model's choice over data-parallel, stream-K and split-K schedules.
+int plan_launch(const MmCall* calls, int n, int sms, TilePlan* plan, int* split) {
+  const int req = calls[0].tile_cfg;
+  const bool force_sk = (req & FP8_TILE_STREAMK) != 0;
+  const int req_cfg = req & ~FP8_TILE_STREAMK;
+  bool batched = false;
+  for (int i = 0; i < n; ++i) batched = batched || calls[i].batch > 1;
+  const int64_t slots = batched ? 0 : sk_slots_available(calls, n);
+  *split = 1;
+  if (force_sk) {
+    if (batched) return FP8_ERR_INVALID_ARG;
+    if (slots < 1) return FP8_ERR_WORKSPACE;
+    *plan = pick_tile(calls, n, sms, slots, req_cfg, true);
+    return plan->sk_ctas > 0 ? FP8_OK : FP8_ERR_WORKSPACE;
+  }
+  if (req_cfg != FP8_TILE_AUTO) {
+    *plan = TilePlan{};
+    plan->cfg = req_cfg;
+  } else {
+    *plan = pick_tile(calls, n, sms, slots);
+  }
+  int& cfg = plan->cfg;
+  // Split-K (single-problem launches): few 128 x 128 tiles and a long K leave
+  // most SMs idle, so a cluster of S CTAs shares each tile's k-blocks.
+  if (cfg == kGemmSplit128 && n != 1) cfg = kGemm128;
+  if (cfg == kGemmSplit128 && calls[0].batch > 1) cfg = kGemm128;  // batches already give the tiles
+  if (n == 1 && calls[0].batch == 1 && plan->sk_ctas == 0 && (req_cfg == FP8_TILE_AUTO || cfg == kGemmSplit128)) {
+    const bool forced = cfg == kGemmSplit128;
+    const int64_t tiles = ((calls[0].m + 127) / 128) * ((calls[0].n + 127) / 128);
+    const int64_t kb = (calls[0].k + 127) / 128;
+    int s = 1;
+    if (tiles <= sms && kb >= 2) s = gemm_split_factor(static_cast<int>(tiles), static_cast<int>(kb), sms, forced);
+    if (s >= 2) {
+      // measured on a B200: moving a 128 x 128 fp32 partial between the SMs of
+      // a cluster costs ~1.6 us, parking it ~0.9 us, the cluster launch ~0.5 us
+      const double t_split = static_cast<double>(kb / s) * 0.34 + 4.0 + 3.0;
+      if (forced || t_split < plan->est_us) {
+        cfg = kGemmSplit128;
+        *split = s;
+      }
+    } else if (forced) {
+      cfg = kGemm128;
+    }
+  }
+  return FP8_OK;
+}
+
+// Two GEMMs (the backward's dX and dW) in one launch save a launch's fixed
+// cost (a few us), which matters for short launches; long ones run as two
+// launches, each with its own tile choice and an operand set that stays in L2
+// (measured on a B200 at M = 4096 with a 4096 x 11008 weight: one launch
+// 283 us, two 255 us).
+constexpr double kFuseMaxUs = 50.0;
+
+bool fuse_pair(const MmCall& dx, const MmCall& dw) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return true;
+  const int sms = num_sms(dev);
+  if (sms <= 0) return true;
+  const MmCall both[2] = {dx, dw};
+  TilePlan pb, px, pw;
+  int split = 1;
+  if (plan_launch(both, 2, sms, &pb, &split) || plan_launch(&dx, 1, sms, &px, &split) ||
+      plan_launch(&dw, 1, sms, &pw, &split))
+    return true;
+  return pb.est_us < kFuseMaxUs && pb.est_us <= px.est_us + pw.est_us;
+}
+
+// Enqueue one launch running n (1 or 2) validated GEMMs over one persistent
+// tile schedule.  side: writes folded into the launch; fin: rings whose
+// quantize deferred its finalize to this launch.
 int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_t st,
                  const RingFinalize* fin = nullptr, int nfin = 0, const DbiasFinish* dbf = nullptr) {
   int dev = 0;
@@ -307,35 +501,17 @@ int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_
   if (e != cudaSuccess) return cuda_fail(e);
   const int sms = num_sms(dev);
   if (sms <= 0) return cuda_fail(cudaGetLastError());
-  double est = 0.0;
-  int cfg = calls[0].tile_cfg != FP8_TILE_AUTO ? calls[0].tile_cfg : pick_tile(calls, n, sms, &est);
-  // Split-K (single-problem launches): few 128 x 128 tiles and a long K leave
-  // most SMs idle, so a cluster of S CTAs shares each tile's k-blocks.
+  TilePlan plan;
   int split = 1;
-  if (cfg == kGemmSplit128 && n != 1) cfg = kGemm128;
-  if (cfg == kGemmSplit128 && calls[0].batch > 1) cfg = kGemm128;  // batches already give the tiles
-  if (n == 1 && calls[0].batch == 1 && (calls[0].tile_cfg == FP8_TILE_AUTO || cfg == kGemmSplit128)) {
-    const bool forced = cfg == kGemmSplit128;
-    const int64_t tiles = ((calls[0].m + 127) / 128) * ((calls[0].n + 127) / 128);
-    const int64_t kb = (calls[0].k + 127) / 128;
-    if (tiles <= sms && kb >= 2) split = gemm_split_factor(static_cast<int>(tiles), static_cast<int>(kb), sms, forced);
-    if (split >= 2) {
-      // measured on a B200: moving a 128 x 128 fp32 partial between the SMs of
-      // a cluster costs ~1.6 us, parking it ~0.9 us, the cluster launch ~0.5 us
-      const double t_split = static_cast<double>(kb / split) * 0.34 + 4.0 + 3.0;
-      if (forced || t_split < est) cfg = kGemmSplit128;
-      else split = 1;
-    } else if (forced) {
-      cfg = kGemm128;
-    }
-  }
+  int s = plan_launch(calls, n, sms, &plan, &split);
+  if (s) return s;
+  const int cfg = plan.cfg;
   CUtensorMap maps[6];
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   std::memset(maps, 0, sizeof(maps));
   for (int i = 0; i < n; ++i) {
-    int s = build_problem(calls[i], cfg, &p.pr[i], &maps[3 * i]);
-    if (s) return s;
+    if ((s = build_problem(calls[i], cfg, &p.pr[i], &maps[3 * i]))) return s;
     p.any_tma_store |= p.pr[i].tma_store;
   }
   p.nprob = n;
@@ -344,9 +520,18 @@ int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_
   p.total_tiles = p.pr[0].num_tiles + (n > 1 ? p.pr[1].num_tiles : 0);
   p.nslots = p.total_tiles;
   p.use_order = 0;
-  // Two problems of unequal k on single-CTA tiles: LPT schedule instead of
-  // round robin (the launch's grid is min(tiles, SMs), the schedule's units).
-  if (n == 2 && (cfg == kGemm128 || cfg == kGemm256) && p.pr[0].k_blocks != p.pr[1].k_blocks) {
+  if (plan.sk_ctas > 0) {
+    // stream-K: whole tiles [0, dp_tiles) round robin, the rest by k-block ranges
+    p.nslots = plan.dp_tiles;
+    p.sk_ctas = plan.sk_ctas;
+    p.dp_tiles = plan.dp_tiles;
+    p.sk_total = plan.sk_total;
+    p.sk_u0 = plan.sk_u0;
+    p.sk_flag = static_cast<unsigned*>(calls[0].ws);
+    p.sk_part = reinterpret_cast<float*>(static_cast<uint8_t*>(calls[0].ws) + kSkFlagBytes);
+  } else if (n == 2 && (cfg == kGemm128 || cfg == kGemm256) && p.pr[0].k_blocks != p.pr[1].k_blocks) {
+    // Two problems of unequal k on single-CTA tiles: LPT schedule instead of
+    // round robin (the launch's grid is min(tiles, SMs), the schedule's units).
     int nslots = 0;
     if (lpt_schedule(p.pr[0].num_tiles, p.pr[0].k_blocks, p.pr[1].num_tiles, p.pr[1].k_blocks, sms, p.order,
                      &nslots) >= 0) {
@@ -367,6 +552,45 @@ int run_mm_group(const MmCall* calls, int n, const SideWrites* side, cudaStream_
 int run_mm(const MmCall& c, const SideWrites* side, cudaStream_t st, const RingFinalize* fin = nullptr,
            int nfin = 0, const DbiasFinish* dbf = nullptr) {
   return run_mm_group(&c, 1, side, st, fin, nfin, dbf);
+}
+
+// D of a GEMM whose contraction is empty (K = 0): every accumulator is 0, so
+// D = bias broadcast over the rows (or zero).  Also used for gradients of a
+// linear whose contraction dimension is empty.
+int run_fill(const MmCall& c, cudaStream_t st) {
+  FillParams f;
+  std::memset(&f, 0, sizeof(f));
+  f.d = c.d;
+  f.ldd = c.ldd;
+  f.stride_d = c.batch > 1 ? c.stride_d : 0;
+  f.m = c.m;
+  f.n = c.n;
+  f.batch = c.batch;
+  f.bias = c.bias;
+  f.bias_kind = !c.bias ? 0 : (c.bias_dtype == FP8_DT_BF16 ? 1 : (c.bias_dtype == FP8_DT_E4M3 ? 2 : 3));
+  f.bias_scale = c.bias_scale;
+  cudaError_t e = launch_fill(f, st);
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
+// A bf16 [rows, cols] output (row stride ld) set to zero: the gradient of an
+// empty contraction.
+int run_zero(void* d, int64_t rows, int64_t cols, int64_t ld, cudaStream_t st) {
+  MmCall c{};
+  c.m = rows;
+  c.n = cols;
+  c.d = d;
+  c.ldd = ld;
+  c.batch = 1;
+  return run_fill(c, st);
+}
+
+// One validated GEMM call: nothing for an empty output, the fill for an empty
+// contraction, else the GEMM kernel.
+int run_mm_any(const MmCall& c, cudaStream_t st) {
+  if (c.m == 0 || c.n == 0 || c.batch == 0) return FP8_OK;
+  if (c.k == 0) return run_fill(c, st);
+  return run_mm(c, nullptr, st);
 }
 
 RingFinalize ring_fin(void* ring, int H, int fmt, float* amax_out) {
@@ -468,24 +692,41 @@ int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace,
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
 
+// The backward workspace's bias-gradient part: the tile counters, then the
+// partials of the larger of the two column-sum geometries (0 when M or N is 0).
+size_t linear_dbias_bytes(int64_t M, int64_t N) {
+  if (M <= 0 || N <= 0) return 0;
+  int Rd, Rc;
+  int64_t rps;
+  dbias_geometry(M, N, &Rd, &rps);
+  colsum_geometry(M, N, &Rc, &rps);
+  return dbias_counter_bytes(N) + dbias_partial_bytes(std::max(Rd, Rc), N);
+}
+
+// Offset of the stream-K part in the backward workspace.
+size_t linear_sk_offset(int64_t M, int64_t N) { return (linear_dbias_bytes(M, N) + 255) & ~size_t(255); }
+
 // ring NULL selects current scaling, which reduces the amax into *amax_out
 // (required then).
 int validate_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt,
                       void* ring, int H, uint8_t* out, int64_t ld_out, const float* amax_out) {
   if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
   if (!is_wide(in_dtype) || !is_fmt(fmt)) return FP8_ERR_INVALID_ARG;
-  if (!in || !out) return FP8_ERR_INVALID_ARG;
   if (ring) {
     if (!ring_len_ok(H) || !aligned(ring, 4)) return FP8_ERR_INVALID_ARG;
   } else if (!amax_out || !aligned(amax_out, 4)) {
     return FP8_ERR_INVALID_ARG;
   }
+  if (rows == 0 || cols == 0) return FP8_OK;  // empty: nothing is read or written
+  if (!in || !out) return FP8_ERR_INVALID_ARG;
   if (!aligned(in, esize(in_dtype))) return FP8_ERR_INVALID_ARG;
   if (ld_in < cols) return FP8_ERR_INVALID_ARG;
-  return check_fp8_matrix(out, ld_out, cols);
+  return check_fp8_matrix(out, ld_out, rows, cols);
 }
 
 }  // namespace
+
+int record_cuda_error(cudaError_t e) { return cuda_fail(e); }
 
 int num_sms(int dev) {
   if (dev < 0 || dev >= 64) return 0;
@@ -596,40 +837,38 @@ int fp8_quantize_dbias(const fp8_quantize_args* g, void* dbias, void* workspace,
 
 int fp8_mm_pair(const fp8_mm_args* a, const fp8_mm_args* b, fp8_stream_t stream) {
   if (!a || !b) return FP8_ERR_INVALID_ARG;
-  const MmCall c[2] = {
-      {a->m, a->n, a->k, a->a, a->fmt_a, a->a_major, a->lda, a->b, a->fmt_b, a->b_major, a->ldb, a->scale_a,
-       a->scale_b, a->bias, a->bias_dtype, a->bias_scale, a->d, a->ldd, a->tile_cfg},
-      {b->m, b->n, b->k, b->a, b->fmt_a, b->a_major, b->lda, b->b, b->fmt_b, b->b_major, b->ldb, b->scale_a,
-       b->scale_b, b->bias, b->bias_dtype, b->bias_scale, b->d, b->ldd, a->tile_cfg}};
+  const MmCall c[2] = {mm_call(a, a), mm_call(b, a)};
   int s = validate_mm(c[0]);
   if (s) return s;
   if ((s = validate_mm(c[1]))) return s;
-  const bool ea = c[0].m == 0 || c[0].n == 0 || c[0].k == 0, eb = c[1].m == 0 || c[1].n == 0 || c[1].k == 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (ea && eb) return FP8_OK;
-  if (ea || eb) return run_mm(ea ? c[1] : c[0], nullptr, st);
-  return run_mm_group(c, 2, nullptr, st);
+  const bool ga = c[0].m > 0 && c[0].n > 0 && c[0].k > 0, gb = c[1].m > 0 && c[1].n > 0 && c[1].k > 0;
+  // one launch, unless both are long enough that two launches run faster
+  // (forced tile configurations always share one launch)
+  if (ga && gb && (c[0].tile_cfg != FP8_TILE_AUTO || fuse_pair(c[0], c[1]))) return run_mm_group(c, 2, nullptr, st);
+  if ((s = run_mm_any(c[0], st))) return s;
+  return run_mm_any(c[1], st);
 }
 
 int fp8_mm(const fp8_mm_args* a, fp8_stream_t stream) {
   if (!a) return FP8_ERR_INVALID_ARG;
-  MmCall c{a->m, a->n, a->k, a->a, a->fmt_a, a->a_major, a->lda, a->b, a->fmt_b, a->b_major, a->ldb,
-           a->scale_a, a->scale_b, a->bias, a->bias_dtype, a->bias_scale, a->d, a->ldd, a->tile_cfg};
+  const MmCall c = mm_call(a, a);
   int s = validate_mm(c);
   if (s) return s;
-  if (c.m == 0 || c.n == 0 || c.k == 0) return FP8_OK;
-  return run_mm(c, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return run_mm_any(c, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fp8_mm_batched(const fp8_mm_args* a, int64_t batch, int64_t stride_a, int64_t stride_b, int64_t stride_d,
                    fp8_stream_t stream) {
   if (!a || batch < 0 || stride_a < 0 || stride_b < 0 || stride_d < 0) return FP8_ERR_INVALID_ARG;
-  MmCall c{a->m, a->n, a->k, a->a, a->fmt_a, a->a_major, a->lda, a->b, a->fmt_b, a->b_major, a->ldb,
-           a->scale_a, a->scale_b, a->bias, a->bias_dtype, a->bias_scale, a->d, a->ldd, a->tile_cfg,
-           batch, stride_a, stride_b, stride_d};
+  MmCall c = mm_call(a, a);
+  c.batch = batch;
+  c.stride_a = stride_a;
+  c.stride_b = stride_b;
+  c.stride_d = stride_d;
   int s = validate_mm(c);
   if (s) return s;
-  if (batch == 0 || c.m == 0 || c.n == 0 || c.k == 0) return FP8_OK;
+  if (batch == 0 || c.m == 0 || c.n == 0) return FP8_OK;
   if (batch > 1) {
     // batch strides of the fp8 operands are TMA strides: multiples of 16 bytes
     if (stride_a % 16 || stride_b % 16) return FP8_ERR_MISALIGNED;
@@ -638,7 +877,7 @@ int fp8_mm_batched(const fp8_mm_args* a, int64_t batch, int64_t stride_a, int64_
     const int64_t tiles = ((c.m + 127) / 128) * ((c.n + 127) / 128) * batch;
     if (tiles > (int64_t(1) << 30)) return FP8_ERR_INVALID_ARG;
   }
-  return run_mm(c, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return run_mm_any(c, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fp8_mm_plan(const fp8_mm_args* a, const fp8_mm_args* b, int num_sms, fp8_mm_plan_info* out) {
@@ -647,28 +886,43 @@ int fp8_mm_plan(const fp8_mm_args* a, const fp8_mm_args* b, int num_sms, fp8_mm_
   int n = 0;
   for (const fp8_mm_args* x : {a, b}) {
     if (!x) continue;
-    MmCall m{x->m, x->n, x->k, x->a, x->fmt_a, x->a_major, x->lda, x->b, x->fmt_b, x->b_major, x->ldb,
-             x->scale_a, x->scale_b, x->bias, x->bias_dtype, x->bias_scale, x->d, x->ldd, a->tile_cfg};
+    const MmCall m = mm_call(x, a);
     int s = validate_mm(m);
     if (s) return s;
-    if (m.m == 0 || m.n == 0 || m.k == 0) continue;  // an empty problem launches nothing
+    if (m.m == 0 || m.n == 0 || m.k == 0) continue;  // no GEMM tiles (an empty contraction is a fill)
     c[n++] = m;
   }
   std::memset(out, 0, sizeof(*out));
   if (n == 0) return FP8_OK;
-  double est = 0.0;
-  const int cfg = c[0].tile_cfg != FP8_TILE_AUTO ? c[0].tile_cfg : pick_tile(c, n, num_sms, &est);
+  const int req_cfg = a->tile_cfg & ~FP8_TILE_STREAMK;
+  const bool force_sk = (a->tile_cfg & FP8_TILE_STREAMK) != 0;
+  const int64_t slots = sk_slots_available(c, n);
+  TilePlan plan;
+  if (force_sk) {
+    if (slots < 1) return FP8_ERR_WORKSPACE;
+    plan = pick_tile(c, n, num_sms, slots, req_cfg, true);
+  } else if (req_cfg != FP8_TILE_AUTO) {
+    plan.cfg = req_cfg;
+  } else {
+    plan = pick_tile(c, n, num_sms, slots);
+  }
+  const int cfg = plan.cfg;
   const int64_t tm = cfg == kGemmPair256 ? 256 : 128;
   const int64_t tn = (cfg == kGemm256 || cfg == kGemmPair256) ? 256 : 128;
   int64_t tiles = 0;
   for (int i = 0; i < n; ++i) tiles += ((c[i].m + tm - 1) / tm) * ((c[i].n + tn - 1) / tn);
   const int64_t cap = cfg == kGemmPair256 ? num_sms / 2 : num_sms;
-  out->tile_cfg = cfg;
+  out->tile_cfg = plan.sk_ctas ? (cfg | FP8_TILE_STREAMK) : cfg;
   out->tiles = tiles;
-  out->units = static_cast<int>(std::max<int64_t>(1, std::min(tiles, cap)));
-  out->est_us = c[0].tile_cfg != FP8_TILE_AUTO ? 0.0 : est;
+  out->units = plan.sk_ctas ? static_cast<int>(std::max<int64_t>(plan.sk_ctas, std::min<int64_t>(plan.dp_tiles, std::min(num_sms, kSkMaxCtas))))
+                            : static_cast<int>(std::max<int64_t>(1, std::min(tiles, cap)));
+  out->est_us = req_cfg != FP8_TILE_AUTO && !force_sk ? 0.0 : plan.est_us;
+  out->stream_k_ctas = plan.sk_ctas;
+  out->dp_tiles = plan.dp_tiles;
   return FP8_OK;
 }
+
+size_t fp8_mm_workspace_bytes(int64_t m, int64_t n, int64_t k) { return sk_bytes_for(m, n, k); }
 
 size_t fp8_dbias_workspace_bytes(int64_t M, int64_t N) {
   if (M <= 0 || N <= 0) return 0;
@@ -706,13 +960,9 @@ int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg, con
 }
 
 size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  (void)K;
   if (M <= 0 || N <= 0) return 0;
-  int Rd, Rc;
-  int64_t rps;
-  dbias_geometry(M, N, &Rd, &rps);
-  colsum_geometry(M, N, &Rc, &rps);
-  return dbias_counter_bytes(N) + dbias_partial_bytes(std::max(Rd, Rc), N);
+  // the bias-gradient part, then the stream-K part of the dX + dW launch
+  return linear_sk_offset(M, N) + std::max(sk_bytes_for(M, K, N), sk_bytes_for(N, K, M));
 }
 
 int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
@@ -720,21 +970,23 @@ int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
   const int64_t M = a->M, N = a->N, K = a->K;
   if (M < 0 || N < 0 || K < 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8_ERR_INVALID_ARG;
   if (!is_fmt(a->fmt_x) || !is_fmt(a->fmt_w)) return FP8_ERR_INVALID_ARG;
-  if (!a->x || !a->w || !a->y || !a->sx_out || !a->sw_out) return FP8_ERR_INVALID_ARG;
+  if (!a->sx_out || !a->sw_out) return FP8_ERR_INVALID_ARG;
+  // operands and output with elements need their buffers (validated below)
+  if ((M > 0 && K > 0 && !a->x) || (N > 0 && K > 0 && !a->w)) return FP8_ERR_INVALID_ARG;
   const bool xq = is_fp8(a->x_dtype), wq = is_fp8(a->w_dtype);
   if (!xq && !is_wide(a->x_dtype)) return FP8_ERR_INVALID_ARG;
   if (!wq && !is_wide(a->w_dtype)) return FP8_ERR_INVALID_ARG;
   int s;
   if (xq) {
     if (a->x_dtype - FP8_DT_E4M3 != a->fmt_x || !a->x_scale_in) return FP8_ERR_INVALID_ARG;
-    if ((s = check_fp8_matrix(a->x, a->ldx, K))) return s;
+    if ((s = check_fp8_matrix(a->x, a->ldx, M, K))) return s;
   } else if ((s = validate_quantize(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8,
                                     a->ldx8, a->amax_x_out))) {
     return s;
   }
   if (wq) {
     if (a->w_dtype - FP8_DT_E4M3 != a->fmt_w || !a->w_scale_in) return FP8_ERR_INVALID_ARG;
-    if ((s = check_fp8_matrix(a->w, a->ldw, K))) return s;
+    if ((s = check_fp8_matrix(a->w, a->ldw, N, K))) return s;
   } else if ((s = validate_quantize(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8,
                                     a->ldw8, a->amax_w_out))) {
     return s;
@@ -746,14 +998,35 @@ int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
   MmCall c{M, N, K, x8, a->fmt_x, FP8_K_MAJOR, xq ? a->ldx : a->ldx8, w8, a->fmt_w, FP8_K_MAJOR,
            wq ? a->ldw : a->ldw8, xq ? a->x_scale_in : a->sx_out, wq ? a->w_scale_in : a->sw_out,
            a->bias, a->bias_dtype, a->bias_scale, a->y, a->ldy, FP8_TILE_AUTO};
+  c.ws = a->workspace;
+  c.ws_bytes = a->workspace_bytes;
   if ((s = validate_mm(c))) return s;
-  if (M == 0 || N == 0 || K == 0) return FP8_OK;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Empty sizes: an operand with no elements is neither quantized nor
+  // side-written (its ring does not step); a non-empty one is, whatever the
+  // other sizes.  y is written when it has elements: the GEMM, or the bias
+  // alone (zero without one) when the contraction K is empty.
+  const bool x_live = M > 0 && K > 0, w_live = N > 0 && K > 0;
+  const bool gemm = M > 0 && N > 0 && K > 0;
   SideWrites side;
   std::memset(&side, 0, sizeof(side));
-  if (xq) { side.copy_src[0] = a->x_scale_in; side.copy_dst[0] = a->sx_out; side.zero_dst[0] = a->amax_x_out; }
-  if (wq) { side.copy_src[1] = a->w_scale_in; side.copy_dst[1] = a->sw_out; side.zero_dst[1] = a->amax_w_out; }
+  if (xq && x_live) { side.copy_src[0] = a->x_scale_in; side.copy_dst[0] = a->sx_out; side.zero_dst[0] = a->amax_x_out; }
+  if (wq && w_live) { side.copy_src[1] = a->w_scale_in; side.copy_dst[1] = a->sw_out; side.zero_dst[1] = a->amax_w_out; }
+  if (!gemm) {
+    // No GEMM follows: a quantize finishes its ring step in its own last block.
+    if (!xq && x_live && (s = run_quantize(a->x, a->x_dtype, M, K, a->ldx, a->fmt_x, a->ring_x, a->hist_len, a->x8,
+                                           a->ldx8, a->amax_x_out, a->sx_out, st)))
+      return s;
+    if (!wq && w_live && (s = run_quantize(a->w, a->w_dtype, N, K, a->ldw, a->fmt_w, a->ring_w, a->hist_len, a->w8,
+                                           a->ldw8, a->amax_w_out, a->sw_out, st)))
+      return s;
+    if (side.copy_dst[0] || side.copy_dst[1]) {
+      cudaError_t e = launch_side_writes(side, st);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return run_mm_any(c, st);  // M, N > 0 here means K == 0: y = bias
+  }
   // The quantize launches only max-reduce into their rings; the GEMM, which
   // waits for them to complete anyway, finishes both ring steps.
   RingFinalize fin[2];
@@ -787,13 +1060,13 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   const int64_t M = a->M, N = a->N, K = a->K;
   if (M < 0 || N < 0 || K < 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8_ERR_INVALID_ARG;
   if (!is_fmt(a->fmt_g) || !is_fmt(a->fmt_x) || !is_fmt(a->fmt_w)) return FP8_ERR_INVALID_ARG;
-  if (!a->g || !a->sg_out) return FP8_ERR_INVALID_ARG;
+  if (!a->sg_out || (M > 0 && N > 0 && !a->g)) return FP8_ERR_INVALID_ARG;
   const bool gq = is_fp8(a->g_dtype);
   if (!gq && !is_wide(a->g_dtype)) return FP8_ERR_INVALID_ARG;
   int s;
   if (gq) {
     if (a->g_dtype - FP8_DT_E4M3 != a->fmt_g || !a->g_scale_in) return FP8_ERR_INVALID_ARG;
-    if ((s = check_fp8_matrix(a->g, a->ldg, N))) return s;
+    if ((s = check_fp8_matrix(a->g, a->ldg, M, N))) return s;
   } else if ((s = validate_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8,
                                     a->ldg8, a->amax_g_out))) {
     return s;
@@ -807,47 +1080,64 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   // dW[N,K] = G8^T . X8: A(i=n, m) = G8[m, n] MN-major, B(j=k, m) = X8[m, k] MN-major.
   MmCall cdw{N, K, M, g8, a->fmt_g, FP8_MN_MAJOR, ldg8, a->x8, a->fmt_x, FP8_MN_MAJOR, a->ldx8,
              sg, a->sx, nullptr, 0, nullptr, a->dw, a->lddw, FP8_TILE_AUTO};
+  // the stream-K part of the workspace, when the caller gave the whole size
+  const size_t sk_off = linear_sk_offset(M, N);
+  if (a->workspace && aligned(a->workspace, 16) && a->workspace_bytes > sk_off) {
+    cdx.ws = cdw.ws = static_cast<uint8_t*>(a->workspace) + sk_off;
+    cdx.ws_bytes = cdw.ws_bytes = a->workspace_bytes - sk_off;
+  }
   if (a->need_dx && (s = validate_mm(cdx))) return s;
   if (a->need_dw && (s = validate_mm(cdw))) return s;
-  const size_t ws_need = a->need_dbias ? fp8_linear_workspace_bytes(M, N, K) : 0;
-  if (a->need_dbias) {
+  const size_t ws_need = a->need_dbias ? linear_dbias_bytes(M, N) : 0;
+  if (a->need_dbias && N > 0) {
     if (!a->dbias || !aligned(a->dbias, 2)) return FP8_ERR_INVALID_ARG;
     if (ws_need && (!a->workspace || a->workspace_bytes < ws_need || !aligned(a->workspace, 16)))
       return FP8_ERR_WORKSPACE;
   }
-  if (M == 0 || N == 0 || K == 0) return FP8_OK;
-
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Empty sizes: g is quantized (or side-written) only when it has elements;
+  // each requested gradient with elements is written -- by its GEMM, or as
+  // zero when its contraction is empty (dX: N = 0; dW: M = 0; dbias: M = 0).
+  const bool g_live = M > 0 && N > 0;
+  const bool dx_live = a->need_dx && M > 0 && K > 0, dw_live = a->need_dw && N > 0 && K > 0;
+  const bool db_live = a->need_dbias && N > 0;
+  const bool dx_gemm = dx_live && N > 0, dw_gemm = dw_live && M > 0;
   SideWrites side;
   std::memset(&side, 0, sizeof(side));
   bool side_pending = false;
   bool dbias_done = false;
   // With a GEMM to follow, the quantize of g leaves its ring step to it.
-  const bool gemm_follows = a->need_dx || a->need_dw;
+  const bool gemm_follows = dx_gemm || dw_gemm;
   RingFinalize fin[1];
   int nfin = 0;
   DbiasFinish dbf{};
-  if (!gq && gemm_follows && a->ring_g) fin[nfin++] = ring_fin(a->ring_g, a->hist_len, a->fmt_g, a->amax_g_out);
-  if (gq) {
-    side.copy_src[0] = a->g_scale_in; side.copy_dst[0] = a->sg_out; side.zero_dst[0] = a->amax_g_out;
-    side_pending = true;
-  } else if (a->need_dbias) {
-    // quantize g and sum its columns in the same pass over g
-    const fp8_quantize_args qg = {a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len,
-                                  a->g8, a->ldg8, a->amax_g_out, a->sg_out};
-    if ((s = run_quantize_dbias(qg, a->dbias, a->workspace, st, gemm_follows, &dbf))) return s;
-    dbias_done = true;
-  } else if ((s = run_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
-                               a->amax_g_out, a->sg_out, st, gemm_follows))) {
-    return s;
+  if (g_live) {
+    if (!gq && gemm_follows && a->ring_g) fin[nfin++] = ring_fin(a->ring_g, a->hist_len, a->fmt_g, a->amax_g_out);
+    if (gq) {
+      side.copy_src[0] = a->g_scale_in; side.copy_dst[0] = a->sg_out; side.zero_dst[0] = a->amax_g_out;
+      side_pending = true;
+    } else if (db_live) {
+      // quantize g and sum its columns in the same pass over g
+      const fp8_quantize_args qg = {a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len,
+                                    a->g8, a->ldg8, a->amax_g_out, a->sg_out};
+      if ((s = run_quantize_dbias(qg, a->dbias, a->workspace, st, gemm_follows, &dbf))) return s;
+      dbias_done = true;
+    } else if ((s = run_quantize(a->g, a->g_dtype, M, N, a->ldg, a->fmt_g, a->ring_g, a->hist_len, a->g8, a->ldg8,
+                                 a->amax_g_out, a->sg_out, st, gemm_follows))) {
+      return s;
+    }
   }
-  if (a->need_dx && a->need_dw) {  // one launch for both (they share the G8 operand)
+  if (dx_gemm && dw_gemm && fuse_pair(cdx, cdw)) {  // one launch for both (they share the G8 operand)
     const MmCall both[2] = {cdx, cdw};
     if ((s = run_mm_group(both, 2, side_pending ? &side : nullptr, st, fin, nfin, dbf.partial ? &dbf : nullptr)))
       return s;
     side_pending = false;
-  } else if (a->need_dx || a->need_dw) {
-    if ((s = run_mm(a->need_dx ? cdx : cdw, side_pending ? &side : nullptr, st, fin, nfin,
+  } else if (dx_gemm && dw_gemm) {  // two launches; the first completes the deferred steps
+    if ((s = run_mm(cdx, side_pending ? &side : nullptr, st, fin, nfin, dbf.partial ? &dbf : nullptr))) return s;
+    if ((s = run_mm(cdw, nullptr, st))) return s;
+    side_pending = false;
+  } else if (dx_gemm || dw_gemm) {
+    if ((s = run_mm(dx_gemm ? cdx : cdw, side_pending ? &side : nullptr, st, fin, nfin,
                     dbf.partial ? &dbf : nullptr)))
       return s;
     side_pending = false;
@@ -856,10 +1146,15 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
     cudaError_t e = launch_side_writes(side, st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
-  if (a->need_dbias && !dbias_done) {
-    if ((s = fp8_dbias(a->g, a->g_dtype, M, N, a->ldg, a->g_scale_in, a->dbias, a->workspace, a->workspace_bytes,
-                       stream)))
+  if (dx_live && !dx_gemm && (s = run_zero(a->dx, M, K, a->lddx, st))) return s;
+  if (dw_live && !dw_gemm && (s = run_zero(a->dw, N, K, a->lddw, st))) return s;
+  if (db_live && !dbias_done) {
+    if (M == 0) {
+      if ((s = run_zero(a->dbias, 1, N, N, st))) return s;
+    } else if ((s = fp8_dbias(a->g, a->g_dtype, M, N, a->ldg, a->g_scale_in, a->dbias, a->workspace,
+                              a->workspace_bytes, stream))) {
       return s;
+    }
   }
   return FP8_OK;
 }

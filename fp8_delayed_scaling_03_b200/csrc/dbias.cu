@@ -250,9 +250,10 @@ extern "C" int fp8_dbias_noalloc(const void* g, int g_dtype, int64_t M, int64_t 
   const size_t need = fp8_dbias_workspace_bytes(M, N);
   if (need > kNoAllocScratchBytes) return FP8_ERR_TOO_LARGE;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FP8_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_error(e);
   unsigned char* scratch = nullptr;
-  if (noalloc_scratch(dev, &scratch) != cudaSuccess) return FP8_ERR_CUDA;
+  if ((e = noalloc_scratch(dev, &scratch)) != cudaSuccess) return record_cuda_error(e);
   DbiasParams p;
   std::memset(&p, 0, sizeof(p));
   p.g = g;
@@ -272,7 +273,7 @@ extern "C" int fp8_dbias_noalloc(const void* g, int g_dtype, int64_t M, int64_t 
   // The array keeps the previous call's contents: the tile counters must start
   // at zero (the kernel also leaves them at zero when it completes).
   const size_t tiles = static_cast<size_t>((N + kDbiasColsPerTile - 1) / kDbiasColsPerTile);
-  if (cudaMemsetAsync(p.counters, 0, tiles * sizeof(unsigned), st) != cudaSuccess) return FP8_ERR_CUDA;
-  if (launch_dbias(p, st) != cudaSuccess) return FP8_ERR_CUDA;
+  if ((e = cudaMemsetAsync(p.counters, 0, tiles * sizeof(unsigned), st)) != cudaSuccess) return record_cuda_error(e);
+  if ((e = launch_dbias(p, st)) != cudaSuccess) return record_cuda_error(e);
   return FP8_OK;
 }

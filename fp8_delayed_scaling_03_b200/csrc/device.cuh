@@ -355,6 +355,74 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// ---------------------------------------------------------------- gpu-scope flags
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait, with the whole warp, until the global flag *f is nonzero (another CTA
+// raised it with a release store after writing the data it guards).  Lane 0
+// polls; once it sees the flag every lane reads it again with acquire
+// semantics, so each lane's later loads see the guarded data.  Bounded like
+// mbar_wait: after FP8LIN_WAIT_LIMIT_NS a timeout is recorded in *status and
+// false returned (also as soon as *abort is set).
+__device__ __forceinline__ bool flag_wait_warp(const uint32_t* f, int* status, volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0 && !ld_acquire_u32(f)) {
+    ok = 0;
+    const uint64_t t0 = globaltimer_ns();
+    #pragma unroll 1
+    while (true) {
+      #pragma unroll 1
+      for (int i = 0; i < 64 && !ok; ++i) ok = ld_acquire_u32(f) != 0;
+      if (ok) break;
+      if (abort && *abort) break;
+      if (globaltimer_ns() - t0 > FP8LIN_WAIT_LIMIT_NS) {
+        if (status) atomicExch(status, kDevTimeout);
+        if (abort) *abort = 1;
+        break;
+      }
+    }
+  }
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  if (ok) (void)ld_acquire_u32(f);
+  return ok != 0;
+}
+
+// Release a flag for the CTAs of another SM after every lane of the warp has
+// written the data it guards: the warp barrier orders the lanes' stores
+// before lane 0's fence (cumulative), the fence before the flag store.
+__device__ __forceinline__ void warp_release_flag(uint32_t* f, uint32_t v) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+  }
+}
+
+// Order this thread's generic-proxy accesses of global memory (e.g. the
+// acquire of a flag) before its later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bulk copy global -> this CTA's shared memory (no tensor map), completion
+// counted in bytes on `bar`.  Both addresses 16-byte aligned, bytes a
+// multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- gpu-scope atomics
 
 // Relaxed max on a global word, no return value.

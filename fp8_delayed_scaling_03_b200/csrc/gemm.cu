@@ -37,6 +37,8 @@
 //     per-element stores instead.
 // Every mbarrier wait is bounded (see device.cuh); a timeout records
 // FP8_ERR_DEVICE_TIMEOUT and the CTA winds down instead of hanging.
+#include <algorithm>
+
 #include "device.cuh"
 #include "internal.h"
 #include "launch.h"
@@ -63,6 +65,14 @@ constexpr int kRingBytes = 192 * 1024;       // operand stages
 // 2 for S = 3).
 constexpr int kPartBytes = kBM * 128 * 4;
 constexpr int kMaxSplit = 3;
+// Stream-K fixup: the finishing CTA's epilogue warps stage the partials of a
+// cut tile in the operand ring (free by then: the owner part is the CTA's
+// last work item), kSkStageBytes per warp, one 4 KB block per 32-column step
+// and partial; at most kSkMaxParts partials per tile (the planner's bound).
+constexpr int kSkBlock = 32 * kEpiCols * 4;
+constexpr int kSkStageBytes = kRingBytes / kEpiWarps;
+constexpr int kSkMaxParts = kSkStageBytes / kSkBlock;
+static_assert(kSkMaxParts == 6, "stream-K stage: 24 KB per epilogue warp");
 static_assert((kMaxSplit - 1) * kPartBytes < kRingBytes, "partials leave room for operand stages");
 
 template <int BN, bool kPair>
@@ -112,6 +122,92 @@ __device__ __forceinline__ int slot_tile(const GemmParams& p, int slot) {
   if (!p.use_order) return slot;
   const uint16_t t = p.order[slot];
   return t == kNoTile ? -1 : static_cast<int>(t);
+}
+
+// ---------------------------------------------------------------- work items
+// One work item of a CTA (or pair): k-blocks [kb_lo, kb_hi) of tile t.
+//   kFull    the whole tile: its own epilogue;
+//   kPartial a later part of a stream-K tile: the fp32 accumulator goes to
+//            this CTA's partial slot, then its epilogue warps raise their flags;
+//   kOwner   the part holding a stream-K tile's first k-block: the partials of
+//            CTAs part0 .. part0 + nparts - 1 (the ranges right after this
+//            CTA's, which start with them) are added, in CTA order, before the
+//            epilogue.
+// A CTA's stream-K range runs [tail of one tile][whole tiles][head of another]:
+// its one partial (the tail) is stored first and its owner part (the head)
+// comes last, so an owner only waits for partials written at the start of
+// later CTAs' ranges, and no CTA waits while holding a partial -- no cycle.
+enum : int { kFull = 0, kOwner = 1, kPartial = 2 };
+struct Work {
+  int t, kb_lo, kb_hi, kind, part0, nparts;
+};
+struct Sched {
+  int slot;        // next data-parallel slot
+  int64_t u, ue;   // next stream-K k-block unit, end of this CTA's range
+};
+
+__device__ __forceinline__ int64_t sk_begin(const GemmParams& p, int c) {
+  return static_cast<int64_t>(c) * p.sk_total / p.sk_ctas;
+}
+// The CTA whose stream-K range holds unit u: the largest c with
+// floor(c total / ctas) <= u, i.e. c = ceil((u + 1) ctas / total) - 1.
+__device__ __forceinline__ int sk_cta_of(const GemmParams& p, int64_t u) {
+  return static_cast<int>(((u + 1) * p.sk_ctas + p.sk_total - 1) / p.sk_total) - 1;
+}
+
+__device__ __forceinline__ void sched_init(const GemmParams& p, int unit, Sched& s) {
+  s.slot = unit;
+  s.u = s.ue = 0;
+  if (unit < p.sk_ctas) {
+    s.u = sk_begin(p, unit);
+    s.ue = sk_begin(p, unit + 1);
+  }
+}
+
+__device__ __forceinline__ bool sched_next(const GemmParams& p, int unit, int units, Sched& s, Work& w) {
+  while (s.slot < p.nslots) {
+    const int t = slot_tile(p, s.slot);
+    s.slot += units;
+    if (t < 0) continue;
+    w.t = t;
+    w.kb_lo = 0;
+    w.kb_hi = t >= p.tiles0 ? p.pr[1].k_blocks : p.pr[0].k_blocks;
+    w.kind = kFull;
+    w.part0 = 0;
+    w.nparts = 0;
+    return true;
+  }
+  if (s.u >= s.ue) return false;
+  // stream-K unit -> (tile, k-block); problem 0's stream-K tiles come first
+  int t, kbt;
+  int64_t ut;  // the tile's first unit
+  if (s.u < p.sk_u0) {
+    kbt = p.pr[0].k_blocks;
+    t = p.dp_tiles + static_cast<int>(s.u / kbt);
+    ut = static_cast<int64_t>(t - p.dp_tiles) * kbt;
+  } else {
+    kbt = p.pr[1].k_blocks;
+    const int t1 = max(p.dp_tiles, p.tiles0);
+    t = t1 + static_cast<int>((s.u - p.sk_u0) / kbt);
+    ut = p.sk_u0 + static_cast<int64_t>(t - t1) * kbt;
+  }
+  const int kb = static_cast<int>(s.u - ut);
+  const int take = static_cast<int>(min(static_cast<int64_t>(kbt - kb), s.ue - s.u));
+  s.u += take;
+  w.t = t;
+  w.kb_lo = kb;
+  w.kb_hi = kb + take;
+  w.part0 = unit + 1;
+  w.nparts = 0;
+  if (kb > 0) {
+    w.kind = kPartial;
+  } else if (take == kbt) {
+    w.kind = kFull;
+  } else {
+    w.kind = kOwner;
+    w.nparts = sk_cta_of(p, ut + kbt - 1) - unit;
+  }
+  return true;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -168,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* pbar = drain + 1;  // split-K rank 0: partials landed (bytes); rank r > 0: partial parked (warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
+  uint64_t* skbar = pbar + 1;  // stream-K: one per epilogue warp, its staged partials landed (bytes)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(skbar + kEpiWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -198,6 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain, 1);
     if constexpr (kSplit) mbar_init(pbar, rank == 0 ? 1u : static_cast<uint32_t>(kEpiWarps));
+    if constexpr (!kPair && !kSplit)
+      for (int i = 0; i < kEpiWarps; ++i) mbar_init(&skbar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
     // split-K rank 0: its partial region fills with (S - 1) bulk copies
@@ -248,9 +347,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b_row0 = static_cast<int>(prank) * C::kBRows;
       bool dep_done = false;
       int issued = 0;  // k-blocks loaded so far; the first kStages find their stage free
-      for (int slot = unit; slot < p.nslots && !*abort_flag; slot += units) {
-        const int t = slot_tile(p, slot);
-        if (t < 0) continue;
+      Sched sc;
+      sched_init(p, unit, sc);
+      Work w;
+      while (!*abort_flag && sched_next(p, unit, units, sc, w)) {
+        const int t = w.t;
         int tb = first_tb, tm = first_tm, tn = first_tn;
         const int pi = t == first_t ? first_pi : tile_coords(p, t, tb, tm, tn);
         const int za = FP8_PR(bcast_a) ? 0 : tb, zb = FP8_PR(bcast_b) ? 0 : tb;  // batch coordinates
@@ -260,8 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bn0 = tn * BN + b_row0;
         const int k_blocks = FP8_PR(k_blocks);
         const bool a_mn = FP8_PR(a_major) != 0, b_mn = FP8_PR(b_major) != 0;
-        const int kb_lo = kSplit ? static_cast<int>(rank) * k_blocks / nsplit : 0;
-        const int kb_hi = kSplit ? (static_cast<int>(rank) + 1) * k_blocks / nsplit : k_blocks;
+        const int kb_lo = kSplit ? static_cast<int>(rank) * k_blocks / nsplit : w.kb_lo;
+        const int kb_hi = kSplit ? (static_cast<int>(rank) + 1) * k_blocks / nsplit : w.kb_hi;
         for (int kb = kb_lo; kb < kb_hi; ++kb, ++issued) {
           if (issued >= nstages && !mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) break;
           if (!dep_done) {  // operands are the previous kernel's output
@@ -301,15 +402,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int slot = unit; slot < p.nslots && !*abort_flag; slot += units) {
-        const int t = slot_tile(p, slot);
-        if (t < 0) continue;
+      Sched sc;
+      sched_init(p, unit, sc);
+      Work w;
+      while (!*abort_flag && sched_next(p, unit, units, sc, w)) {
+        const int t = w.t;
         const int pi = t >= p.tiles0 ? 1 : 0;
         const int k_blocks = FP8_PR(k_blocks);
         const bool a_mn = FP8_PR(a_major) != 0, b_mn = FP8_PR(b_major) != 0;
         const uint32_t idesc = FP8_PR(idesc);
-        const int kb_lo = kSplit ? static_cast<int>(rank) * k_blocks / nsplit : 0;
-        const int kb_hi = kSplit ? (static_cast<int>(rank) + 1) * k_blocks / nsplit : k_blocks;
+        const int kb_lo = kSplit ? static_cast<int>(rank) * k_blocks / nsplit : w.kb_lo;
+        const int kb_hi = kSplit ? (static_cast<int>(rank) + 1) * k_blocks / nsplit : w.kb_hi;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -388,9 +491,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     constexpr int kSteps = BN / 2 / kEpiCols;
-    for (int slot = unit; slot < p.nslots && !*abort_flag; slot += units) {
-      const int t = slot_tile(p, slot);
-      if (t < 0) continue;
+    // stream-K partial slots, one per CTA: [epilogue warp][32-column step]
+    // [column quad][lane] float4s, so each (warp, step) block is 4 KB of
+    // contiguous fp32 (one bulk copy) and a warp's stores of one column quad
+    // are 512 contiguous bytes
+    float4* const sk_part = reinterpret_cast<float4*>(p.sk_part);
+    uint8_t* const sk_stage = sA + ew * kSkStageBytes;
+    uint32_t sk_phase = 0;
+    auto sk_block = [&](int slot, int st) {
+      return sk_part + ((static_cast<int64_t>(slot) * kEpiWarps + ew) * kSteps + st) * (kSkBlock / 16);
+    };
+    Sched sc;
+    sched_init(p, unit, sc);
+    Work w;
+    while (!*abort_flag && sched_next(p, unit, units, sc, w)) {
+      const int t = w.t;
       int tb, tm, tn;
       const int pi = tile_coords(p, t, tb, tm, tn);
       // The tile's constants go to registers and its bias values are fetched
@@ -400,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool tma_store = FP8_PR(tma_store) != 0;
       const bool have_k = kSplit ? (static_cast<int>(rank) + 1) * FP8_PR(k_blocks) / nsplit >
                                        static_cast<int>(rank) * FP8_PR(k_blocks) / nsplit
-                                 : FP8_PR(k_blocks) > 0;
+                                 : w.kb_hi > w.kb_lo;
       void* const qd_ptr = static_cast<__nv_bfloat16*>(FP8_PR(d)) + static_cast<int64_t>(tb) * FP8_PR(stride_d);
       const int64_t ldd = FP8_PR(ldd);
       const void* const bias = FP8_PR(bias);
@@ -421,10 +536,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         // rank 0: the other ranks' partials have landed in its partial region
         if (rank == 0 && !mbar_wait(pbar, 0, p.status, abort_flag)) break;
       }
+      // owner: the later parts' partials are in their slots; they are staged
+      // `spr` steps at a time in this warp's share of the (now idle) operand ring
+      int spr = kSteps;
+      if (w.kind == kOwner) {
+        bool ok = w.nparts >= 1 && w.nparts <= kSkMaxParts;
+        if (!ok && lane == 0 && p.status) atomicExch(p.status, kDevTimeout);  // outside the planner's bound: give up
+        for (int q = 0; q < w.nparts && ok; ++q)
+          ok = flag_wait_warp(p.sk_flag + static_cast<int64_t>(w.part0 + q) * kEpiWarps + ew, p.status, abort_flag);
+        if (!ok) {
+          *abort_flag = 1;
+          break;
+        }
+        spr = min(kSteps, kSkMaxParts / w.nparts);
+        fence_proxy_async_global();  // the acquires above come before the bulk copies' reads
+      }
       const int row = tm * C::kTileM + row_in_tile;
       #pragma unroll 1
       for (int st = 0; st < kSteps; ++st) {
         const int col0 = col_half + st * kEpiCols;
+        if (w.kind == kOwner && st % spr == 0) {  // stage the partials of steps [st, st + spr)
+          const int nst = min(spr, kSteps - st);
+          fence_proxy_async_smem();  // this warp's reads of the previous round come first
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&skbar[ew], static_cast<uint32_t>(w.nparts * nst * kSkBlock));
+            for (int q = 0; q < w.nparts; ++q)
+              bulk_copy_g2s(sk_stage + q * nst * kSkBlock, sk_block(w.part0 + q, st),
+                            static_cast<uint32_t>(nst * kSkBlock), &skbar[ew]);
+          }
+          if (!mbar_wait(&skbar[ew], sk_phase, p.status, abort_flag)) break;
+          sk_phase ^= 1u;
+        }
         uint32_t r[32];
         if (st < live_steps) {
           if (have_k) {
@@ -460,6 +603,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             #pragma unroll
             for (int j = 0; j < 32; j += 4) {
               const float4 o = src[(j / 4) * kBM];
+              r[j] = __float_as_uint(__uint_as_float(r[j]) + o.x);
+              r[j + 1] = __float_as_uint(__uint_as_float(r[j + 1]) + o.y);
+              r[j + 2] = __float_as_uint(__uint_as_float(r[j + 2]) + o.z);
+              r[j + 3] = __float_as_uint(__uint_as_float(r[j + 3]) + o.w);
+            }
+          }
+        }
+        if (w.kind != kFull) {
+          if (w.kind == kPartial) {  // this part's accumulator goes to the CTA's slot
+            float4* dst = sk_block(unit, st) + lane;
+            #pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              __stcg(dst + (j / 4) * 32, make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                                     __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])));
+            continue;
+          }
+          // owner: ((acc + p[part0]) + p[part0 + 1]) + ..., the same for every launch
+          const int nst = min(spr, kSteps - (st - st % spr));
+          for (int q = 0; q < w.nparts; ++q) {
+            const float4* src =
+                reinterpret_cast<const float4*>(sk_stage + (q * nst + st % spr) * kSkBlock) + lane;
+            #pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 o = src[(j / 4) * 32];
               r[j] = __float_as_uint(__uint_as_float(r[j]) + o.x);
               r[j + 1] = __float_as_uint(__uint_as_float(r[j + 1]) + o.y);
               r[j + 2] = __float_as_uint(__uint_as_float(r[j + 2]) + o.z);
@@ -503,6 +670,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j)
             if (col0 + j < qn) drow[col0 + j] = __float2bfloat16_rn(v[j]);
         }
+      }
+      if (w.kind == kPartial) {  // this warp's share of the partial is written: raise its flag
+        warp_release_flag(p.sk_flag + static_cast<int64_t>(unit) * kEpiWarps + ew, 1u);
+      } else if (w.kind == kOwner) {  // every lane has read the partials: clear their flags
+        __syncwarp();
+        if (lane == 0)
+          for (int q = 0; q < w.nparts; ++q) p.sk_flag[static_cast<int64_t>(w.part0 + q) * kEpiWarps + ew] = 0u;
       }
       if (kSplit && rank != 0) {  // partial parked: one bulk copy into rank 0's region
         fence_proxy_async_smem();  // this thread's parked bytes, visible to the copy engine
@@ -548,7 +722,10 @@ cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t 
   }
   const int sms = num_sms(dev);
   if (!kPair) {
-    const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+    // stream-K: the whole-tile waves use one CTA per SM (at most 160, the
+    // planner's CTA count), the k-block ranges the first sk_ctas of them
+    int grid = p.total_tiles < sms ? p.total_tiles : sms;
+    if (p.sk_ctas > 0) grid = p.dp_tiles > 0 ? (sms < 160 ? sms : 160) : p.sk_ctas;
     return launch_pdl(fp8_gemm_kernel<BN, kPair, false>, dim3(grid), dim3(kThreads), C::kSmem, s, mp[0], mp[1], mp[2], mp[3],
                       mp[4], mp[5], p);
   }
@@ -630,7 +807,33 @@ cudaError_t launch_split(const CUtensorMap* mp, const GemmParams& p, cudaStream_
   return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<128, false, true>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
 }
 
+// The output of an empty contraction: every accumulator is zero, so each
+// element is 0 + bias[j] rounded once to bf16 (the epilogue's arithmetic with
+// acc = 0), or zero without a bias.  Grid-stride over batch x m x n.
+__global__ void __launch_bounds__(256) fill_kernel(const FillParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const float binv = p.bias_kind >= 2 ? 1.0f / *p.bias_scale : 1.0f;
+  const int64_t per = p.m * p.n;
+  const int64_t total = per * p.batch;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = i / per, r = (i - b * per) / p.n, c = i - b * per - r * p.n;
+    const float v = 0.0f + (p.bias_kind ? bias_value(p.bias, p.bias_kind, static_cast<int>(c), binv) : 0.0f);
+    static_cast<__nv_bfloat16*>(p.d)[b * p.stride_d + r * p.ldd + c] = __float2bfloat16_rn(v);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_fill(const FillParams& p, cudaStream_t s) {
+  const int64_t total = p.m * p.n * p.batch;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int64_t cap = static_cast<int64_t>(num_sms(dev) > 0 ? num_sms(dev) : 1) * 8;
+  const int64_t blocks = std::min<int64_t>(cap, std::max<int64_t>(1, (total + 255) / 256));
+  return launch_pdl(fill_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
+}
 
 int gemm_split_factor(int tiles, int k_blocks, int sms, bool forced) {
   int dev = 0;

@@ -126,10 +126,36 @@ struct GemmParams {
   // else tile s.
   int nslots;
   int use_order;
+  // Stream-K (single-CTA tiles; sk_ctas = 0: off).  The slots above cover the
+  // whole tiles [0, dp_tiles); the k-blocks of tiles [dp_tiles, total_tiles),
+  // sk_total of them in tile order (sk_u0 belong to problem 0), are split
+  // into sk_ctas contiguous ranges, range c = [c sk_total / sk_ctas,
+  // (c + 1) sk_total / sk_ctas) for CTA c.  A tile cut by range boundaries
+  // is finished by the CTA whose range holds its first k-block: the CTAs
+  // holding its later k-blocks store their fp32 partial accumulators in
+  // sk_part (one slot per CTA) and raise one flag per epilogue warp in
+  // sk_flag; the finishing CTA adds them in CTA order and clears the flags.
+  int sk_ctas;
+  int dp_tiles;
+  int64_t sk_total;
+  int64_t sk_u0;
+  float* sk_part;             // [sk_ctas][BN / 4][128][4]
+  unsigned* sk_flag;          // [sk_ctas][8]
   uint16_t order[1024];
 };
 constexpr int kMaxOrder = 1024;
 constexpr uint16_t kNoTile = 0xFFFF;
+
+// D = bias broadcast over the rows (bf16, or fp8 / bias_scale), or zero: the
+// GEMM of an empty contraction (K = 0), where every accumulator is 0.
+struct FillParams {
+  void* d;
+  int64_t ldd, stride_d;      // elements
+  int64_t m, n, batch;
+  const void* bias;
+  int bias_kind;              // 0 none, 1 bf16, 2 e4m3, 3 e5m2
+  const float* bias_scale;
+};
 
 struct DbiasParams {
   const void* g;
@@ -145,6 +171,9 @@ struct DbiasParams {
 };
 
 int num_sms(int device);
+// Keeps e's name for fp8_status_string(FP8_ERR_CUDA) on this host thread and
+// returns FP8_ERR_CUDA.
+int record_cuda_error(cudaError_t e);
 
 // b may be NULL (one tensor); both tensors share in_dtype and fmt.
 cudaError_t launch_quantize(int in_dtype, int fmt, const QuantizeParams* a, const QuantizeParams* b, cudaStream_t s);
@@ -165,6 +194,7 @@ int gemm_split_factor(int tiles, int k_blocks, int sms, bool forced);
 // maps[0..2]: A, B, D of pr[0]; maps[3..5]: those of pr[1] (zeroed if unused).
 cudaError_t launch_gemm(const CUtensorMap* maps, const GemmParams& p, int cfg, cudaStream_t s);
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s);
+cudaError_t launch_fill(const FillParams& p, cudaStream_t s);
 
 // Column-sum geometry (R row splits of rows_per_split rows over 256-column
 // tiles) shared by the size queries and the launchers: dbias_geometry for the

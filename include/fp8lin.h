@@ -19,10 +19,20 @@
  *   - Work is enqueued on `stream` in stream order; no call synchronizes the
  *     host.  A ring (and a workspace) must not be used by two launches that can
  *     run concurrently.
+ *   - The library caches a few per-device facts on first use (SM count, the
+ *     device address of its status word and of fp8_dbias_noalloc's scratch);
+ *     keep one CUDA context per device while it is in use (no
+ *     cudaDeviceReset in between).
  *   - Arguments are validated before anything is enqueued.  A failed check
  *     returns a negative fp8_status and enqueues nothing.  A launch failure
  *     returns FP8_ERR_CUDA; fp8_status_string(FP8_ERR_CUDA) then names the CUDA
- *     error.  Sizes of zero are accepted and do nothing (rings untouched).
+ *     error.
+ *   - Sizes of zero are accepted.  A matrix with no elements is neither read
+ *     nor written and its pointer and stride are not checked (NULL is fine):
+ *     an empty operand is not quantized and its ring does not step.  An
+ *     output that has elements is always written: a GEMM whose contraction
+ *     is empty (K = 0 in fp8_mm, N = 0 for dX, M = 0 for dW) writes the bias
+ *     alone (zero without one), and dbias over M = 0 rows is zero.
  *   - Matrices are row-major with an explicit row stride `ld` in ELEMENTS.
  *     fp8 matrices (read or written) need ld % 16 == 0 and a 16-byte aligned
  *     base (the GEMMs read them with TMA); bf16/fp16/fp32 inputs may have any
@@ -60,12 +70,21 @@ typedef enum { FP8_K_MAJOR = 0, FP8_MN_MAJOR = 1 } fp8_major;
  * CTAs that split K (FP8_TILE_SPLITK_128x128: rank r takes k-blocks
  * [r kb/S, (r+1) kb/S) and rank 0 adds the partial fp32 accumulators in rank
  * order before the epilogue; fp8_mm only -- a two-GEMM launch falls back to
- * 128x128).  FP8_TILE_AUTO chooses per shape, split-K included when the output
- * has few tiles and K is long.  Results do not depend on the choice beyond the
- * fp32 summation order. */
+ * 128x128).
+ * Stream-K (FP8_TILE_STREAMK, or'ed with FP8_TILE_128x128 or
+ * FP8_TILE_128x256; needs a workspace): one CTA per SM; whole waves of tiles
+ * run data-parallel and the k-blocks of the remaining tiles are split evenly
+ * over the CTAs, so that no SM idles while others finish a last partial wave.
+ * A tile cut between CTAs is finished by the CTA holding its first k-block,
+ * which adds the others' fp32 partial accumulators (stored in the workspace)
+ * in CTA order: the result is deterministic for a given GPU.
+ * FP8_TILE_AUTO chooses per shape with a cost model fitted to B200 timings --
+ * split-K when the output has few tiles and K is long, stream-K when a
+ * workspace is given and it pays.  Results do not depend on the choice beyond
+ * the fp32 summation order. */
 typedef enum {
   FP8_TILE_AUTO = 0, FP8_TILE_128x128 = 1, FP8_TILE_128x256 = 2, FP8_TILE_PAIR_256x256 = 3,
-  FP8_TILE_SPLITK_128x128 = 4
+  FP8_TILE_SPLITK_128x128 = 4, FP8_TILE_STREAMK = 8
 } fp8_tile_cfg;
 
 typedef enum {
@@ -190,7 +209,9 @@ FP8LIN_API int fp8_quantize_dbias(const fp8_quantize_args* g, void* dbias, void*
  *                     ([csrc@2eeac02] FP8Params bias bullet: fp8 bias
  *                     dequantized after the operand scaling)
  *   d                 bf16 [m, ldd], ldd >= n
- * Out-of-range rows/columns/k of partial tiles contribute nothing. */
+ * Out-of-range rows/columns/k of partial tiles contribute nothing.  k = 0
+ * (m, n > 0): every sum is empty, so D = bf16(0 + bias[j]), or 0 without a
+ * bias (a small fill launch; the operands and scales are not read). */
 typedef struct fp8_mm_args {
   int64_t m, n, k;
   const uint8_t* a; int fmt_a; int a_major; int64_t lda;
@@ -199,8 +220,22 @@ typedef struct fp8_mm_args {
   const void* bias; int bias_dtype; const float* bias_scale;
   void* d; int64_t ldd;
   int tile_cfg;   /* FP8_TILE_AUTO (0, chosen per shape) or one of fp8_tile_cfg */
+  /* Optional stream-K workspace (NULL / 0: none; results are the same, only
+   * the schedule differs): >= fp8_mm_workspace_bytes(m, n, k) bytes, 256-byte
+   * aligned, ZERO-FILLED before its first use; every call leaves its flags at
+   * zero again, so it may be reused by later calls of the same sizes that are
+   * ordered after this one (same stream).  A forced FP8_TILE_STREAMK without
+   * it returns FP8_ERR_WORKSPACE. */
+  void* workspace; size_t workspace_bytes;
 } fp8_mm_args;
 FP8LIN_API int fp8_mm(const fp8_mm_args* args, fp8_stream_t stream);
+
+/* Bytes of the stream-K workspace of an m x n x k GEMM (or of a two-GEMM
+ * launch: the larger of the two): a fixed block of 1280 zero-at-rest flags,
+ * then one 128 x 256 fp32 partial accumulator per CTA that can hold a cut
+ * tile (at most 160, and at most one per 128 x 128 x 128 block of work).
+ * 0 when m, n or k is 0. */
+FP8LIN_API size_t fp8_mm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /* A batch of GEMMs of one shape in one launch ([astrai@4019dda] mm_fp8 bullet:
  * 3-D operands through the same signature, batches sliced by strides, a
@@ -217,9 +252,15 @@ FP8LIN_API int fp8_mm(const fp8_mm_args* args, fp8_stream_t stream);
 FP8LIN_API int fp8_mm_batched(const fp8_mm_args* args, int64_t batch, int64_t stride_a, int64_t stride_b,
                               int64_t stride_d, fp8_stream_t stream);
 
-/* Two independent GEMMs in ONE launch over one persistent tile schedule (the
- * backward's dX and dW).  Same results as two fp8_mm calls; the tile
- * configuration (a->tile_cfg, or chosen for the pair when AUTO) is shared. */
+/* Two independent GEMMs (the backward's dX and dW) in ONE launch over one
+ * persistent tile schedule.  Same results as two fp8_mm calls; the tile
+ * configuration (a->tile_cfg, or chosen for the pair when AUTO) and the
+ * stream-K workspace (a->workspace, >= fp8_mm_workspace_bytes of either
+ * problem) are shared.  With FP8_TILE_AUTO, two GEMMs long enough that the
+ * launch's fixed cost no longer matters (the cost model's estimate of the
+ * shared launch is 50 us or more, or above the two separate launches) run
+ * as two launches instead: each gets its own tile choice and operand set in
+ * L2 (at M = 4096 with a 4096 x 11008 weight on a B200: 255 us vs 283 us). */
 FP8LIN_API int fp8_mm_pair(const fp8_mm_args* a, const fp8_mm_args* b, fp8_stream_t stream);
 
 /* The tile configuration fp8_mm (b == NULL) or fp8_mm_pair (b != NULL) would
@@ -234,7 +275,7 @@ FP8LIN_API int fp8_mm_pair(const fp8_mm_args* a, const fp8_mm_args* b, fp8_strea
  *             FP8_TILE_AUTO when every problem is empty);
  *   tiles     output tiles of that configuration over the problem(s);
  *   units     CTAs (CTA pairs for FP8_TILE_PAIR_256x256) the launch keeps
- *             busy: min(tiles, num_sms) (pairs: num_sms / 2);
+ *             busy: min(tiles, num_sms) (pairs: num_sms / 2; stream-K: all);
  *   est_us    the cost model's estimate of the launch in microseconds (fitted
  *             to B200 timings; 0 for a forced configuration). */
 typedef struct {
@@ -242,6 +283,8 @@ typedef struct {
   int64_t tiles;
   int units;
   double est_us;
+  int stream_k_ctas;   /* CTAs sharing the stream-K k-blocks (0: no stream-K) */
+  int64_t dp_tiles;    /* tiles run whole before the stream-K part */
 } fp8_mm_plan_info;
 FP8LIN_API int fp8_mm_plan(const fp8_mm_args* a, const fp8_mm_args* b, int num_sms, fp8_mm_plan_info* out);
 
@@ -273,7 +316,9 @@ FP8LIN_API int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64
  *   - It calls no cudaMalloc, cudaFree or allocating library routine.
  *   - The first call on a device looks up the array's device address (once
  *     per device, under a lock); make that first call before any stream
- *     capture.
+ *     capture.  The address is kept for the life of the process, so the
+ *     device must keep one CUDA context meanwhile: no cudaDeviceReset (or
+ *     other context teardown) while the library is in use.
  *   - All calls share the one array: calls that can overlap on the GPU (other
  *     streams, other host threads) race and must be serialized by the caller.
  *     Each call clears the tile counters it needs before its kernel. */
@@ -308,6 +353,8 @@ typedef struct fp8_linear_fwd_args {
   uint8_t* w8; int64_t ldw8;
   float* sx_out; float* sw_out; float* amax_x_out; float* amax_w_out;
   void* y; int64_t ldy;
+  void* workspace; size_t workspace_bytes;   /* optional stream-K workspace of the GEMM, as
+                                                fp8_mm_args (size fp8_mm_workspace_bytes(M, N, K)) */
 } fp8_linear_fwd_args;
 FP8LIN_API int fp8_linear_forward(const fp8_linear_fwd_args* args, fp8_stream_t stream);
 
@@ -321,8 +368,12 @@ FP8LIN_API int fp8_linear_forward(const fp8_linear_fwd_args* args, fp8_stream_t 
  *                                           only when the bias needs a grad)
  * sx, sw, x8, w8 are the FORWARD's snapshots and quantized operands: the
  * backward reuses the forward's scales.  Outputs are bf16 whatever the input
- * dtypes.  workspace: as fp8_dbias, needed only when need_dbias (size from
- * fp8_linear_workspace_bytes).  Up to 4 launches. */
+ * dtypes.  dX and dW share one launch as fp8_mm_pair decides with
+ * FP8_TILE_AUTO.  workspace: fp8_linear_workspace_bytes(M, N, K) bytes, zero-filled
+ * before first use, reusable by later calls of the same sizes on the same
+ * stream: the bias-gradient scratch (as fp8_dbias; required when need_dbias,
+ * which needs at least that part), then the stream-K scratch of the dX + dW
+ * launch (used only when the whole size is given).  Up to 4 launches. */
 typedef struct fp8_linear_bwd_args {
   int64_t M, N, K;
   const void* g; int g_dtype; int64_t ldg; const float* g_scale_in;
@@ -339,11 +390,12 @@ typedef struct fp8_linear_bwd_args {
 } fp8_linear_bwd_args;
 FP8LIN_API int fp8_linear_backward(const fp8_linear_bwd_args* args, fp8_stream_t stream);
 
-/* Workspace bytes fp8_linear_backward needs for need_dbias (0 when M or N is
- * 0).  At least fp8_dbias_workspace_bytes(M, N): the column-sum quantize of
- * the backward may split g's rows more finely than fp8_dbias does.  Zero-fill
- * it once before first use, like fp8_dbias's workspace; every call leaves it
- * ready for the next.  K does not enter. */
+/* Workspace bytes of fp8_linear_backward (0 when M or N is 0): the bias
+ * gradient's part -- at least fp8_dbias_workspace_bytes(M, N), since the
+ * column-sum quantize of the backward may split g's rows more finely than
+ * fp8_dbias does -- followed by the stream-K part of the dX + dW launch.
+ * Zero-fill it once before first use; every call leaves it ready for the next
+ * call of the same sizes. */
 FP8LIN_API size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------ status

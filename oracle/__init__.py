@@ -271,6 +271,8 @@ def epilogue(acc: np.ndarray, sa: float, sb: float, bias: np.ndarray | None = No
     (bf16 bits, fp32 pre-rounding values)."""
     acc = np.ascontiguousarray(acc, np.float32)
     shape = acc.shape
+    if acc.size == 0:  # an empty output
+        return np.zeros(shape, np.uint16), np.zeros(shape, np.float32)
     acc2 = acc.reshape(1, -1) if col_idx is not None else acc.reshape(shape[0] if acc.ndim > 1 else 1, -1)
     out = np.empty(acc2.shape, np.uint16)
     f = np.empty(acc2.shape, np.float32)
@@ -317,10 +319,19 @@ def dbias(g: np.ndarray, dtype: int, M: int, N: int, sg: float = 1.0):
 # ------------------------------------------------------------------ orchestration
 
 def _operand(t, dtype, fmt, ring, scale_in, cols, ld8):
-    """Quantize an operand with its ring, or take a pre-quantized one as is."""
+    """Quantize an operand with its ring, or take a pre-quantized one as is.
+    An operand with no elements is not quantized: it has no amax to fold, so
+    its ring does not step (the pages are silent on empty tensors; reading: a
+    quantize of nothing does nothing) and the scale returned is the one a
+    quantize would have used."""
     if dtype in (DT_E4M3, DT_E5M2):
         assert (dtype - DT_E4M3) == fmt, "pre-quantized operand must match fmt"
         return np.ascontiguousarray(t), np.float32(0.0), np.float32(scale_in)
+    if t.size == 0 or (cols is not None and cols == 0):
+        rows = t.shape[0]
+        width = cols if ld8 is None else ld8
+        s = np.float32(1.0) if ring is None else np.float32(ring.scale)
+        return np.zeros((rows, width if width is not None else t.shape[1]), np.uint8), np.float32(0.0), s
     if ring is None:  # current (dynamic) scaling
         return quantize_dynamic(t, dtype, fmt, cols=cols, ld_out=ld8)
     q, a, s = quantize(t, dtype, fmt, ring, cols=cols, ld_out=ld8)

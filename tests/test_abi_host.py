@@ -141,7 +141,8 @@ def test_mm_validation(fp8):
     assert mm(fp8, tile_cfg=5) == E.FP8_ERR_INVALID_ARG
     assert mm(fp8, tile_cfg=-1) == E.FP8_ERR_INVALID_ARG
     assert mm(fp8, m=0) == E.FP8_OK
-    assert mm(fp8, k=0) == E.FP8_OK
+    assert mm(fp8, n=0, k=0) == E.FP8_OK          # empty output: nothing enqueued (K = 0 alone writes D = bias)
+    assert mm(fp8, m=0, a=None, d=None) == E.FP8_OK   # empty operands and output are not dereferenced
     assert fp8._lib.fp8_mm(None, None) == E.FP8_ERR_INVALID_ARG
 
 
@@ -182,7 +183,8 @@ def test_linear_forward_validation(fp8):
     assert fwd(fp8, ldx8=120) == E.FP8_ERR_INVALID_ARG
     assert fwd(fp8, ldy=100) == E.FP8_ERR_INVALID_ARG
     assert fwd(fp8, hist_len=0) == E.FP8_ERR_INVALID_ARG
-    assert fwd(fp8, M=0) == E.FP8_OK
+    assert fwd(fp8, M=0, N=0) == E.FP8_OK       # x and w empty: nothing enqueued
+    assert fwd(fp8, M=0, N=0, x=None, w=None) == E.FP8_OK
     assert fp8._lib.fp8_linear_forward(None, None) == E.FP8_ERR_INVALID_ARG
 
 
@@ -205,7 +207,8 @@ def test_linear_backward_validation(fp8):
     assert bwd(fp8, ldx8=136, need_dw=1) == E.FP8_ERR_MISALIGNED
     assert bwd(fp8, g_dtype=E.FP8_DT_E5M2) == E.FP8_ERR_INVALID_ARG         # pre-quantized g needs its scale
     assert bwd(fp8, sg_out=None) == E.FP8_ERR_INVALID_ARG
-    assert bwd(fp8, N=0) == E.FP8_OK
+    assert bwd(fp8, N=0, need_dx=0) == E.FP8_OK  # g and dW empty: nothing enqueued
+    assert bwd(fp8, M=0, need_dw=0, g=None) == E.FP8_OK
     # the backward's column sums need fp8_linear_workspace_bytes, which can
     # exceed what fp8_dbias needs; a workspace sized for fp8_dbias is refused
     M, N, K = 2048, 1024, 1024

@@ -43,7 +43,7 @@ def strides(major, ld):
 
 
 def run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=0, fmt_b=0, sa=1.0, sb=1.0, bias_kind=None,
-             pad=0, ldd_extra=0, full=True, a_codes=None, b_codes=None, tile=0):
+             pad=0, ldd_extra=0, full=True, a_codes=None, b_codes=None, tile=0, workspace=None):
     A = a_codes if a_codes is not None else codes_like_tensor(rng, fmt_a, (m, k), 60.0 if fmt_a == 0 else 3000.0)
     B = b_codes if b_codes is not None else codes_like_tensor(rng, fmt_b, (n, k), 60.0 if fmt_b == 0 else 3000.0)
     a_st, lda = store(A, a_major, pad)
@@ -70,7 +70,7 @@ def run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=0, fmt_b=0, sa=1.0, sb=1
         bias_dtype = fp8.FP8_DT_E4M3 + bf
         odt = oracle.DT_E4M3 + bf
     fp8.fp8_mm(m, n, k, dev_a, fmt_a, a_major, lda, dev_b, fmt_b, b_major, ldb, scales[0:1], scales[1:2], d, ldd,
-               bias=bias_dev, bias_dtype=bias_dtype, bias_scale=bias_scale, tile_cfg=tile)
+               bias=bias_dev, bias_dtype=bias_dtype, bias_scale=bias_scale, tile_cfg=tile, workspace=workspace)
     torch.cuda.synchronize()
     assert fp8.fp8_get_device_status() == 0
     y = d.cpu().view(torch.int16).numpy().view(np.uint16)
@@ -356,3 +356,111 @@ def test_mm_batched_large_sampled(fp8, batch, m, n, k, a_major, b_major):
     """The pages' bmm shapes (64 x 512^3, 8 x 1024 x 2048) and a dW-like batch."""
     rng = np.random.default_rng(batch + m + k)
     run_batched(fp8, rng, batch, m, n, k, a_major, b_major, full=False)
+
+
+# ---------------------------------------------------------------- stream-K
+
+SK = 8                         # FP8_TILE_STREAMK
+SK_TILES = [1 | SK, 2 | SK]    # 128x128 and 128x256 tiles with stream-K forced
+SK_FLAG_BYTES = 160 * 8 * 4    # the workspace's zero-at-rest flag block
+
+
+def flags_clear(ws):
+    return int(ws[:SK_FLAG_BYTES].view(torch.int32).abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("tile", SK_TILES)
+@pytest.mark.parametrize("a_major,b_major", LAYOUTS)
+@pytest.mark.parametrize("m,n,k", [(256, 384, 2048), (300, 200, 1000), (64, 192, 640), (3, 100, 1100)])
+def test_mm_stream_k_full(fp8, a_major, b_major, m, n, k, tile):
+    """Stream-K forced on few-tile, long-K shapes (every tile cut between 2 to
+    ~6 CTAs; ragged rows, columns and k): full comparison with the oracle, and
+    every flag of the workspace back at zero after the launch."""
+    rng = np.random.default_rng(m + n + k + tile)
+    ws = fp8.mm_workspace(m, n, k, "cuda")
+    run_case(fp8, rng, m, n, k, a_major, b_major, full=True, tile=tile, workspace=ws)
+    assert flags_clear(ws)
+
+
+@pytest.mark.parametrize("tile", [0] + SK_TILES)
+@pytest.mark.parametrize("m,n,k,a_major,b_major", [
+    (2048, 1536, 6912, 0, 0), (2048, 1536, 6912, 0, 1), (1536, 1536, 2048, 1, 1),
+    (4096, 4096, 384, 0, 0), (512, 6912, 1536, 1, 1)])
+def test_mm_stream_k_large_sampled(fp8, m, n, k, a_major, b_major, tile):
+    """Production-sized shapes with a workspace: AUTO (which picks stream-K
+    where the cost model says it pays) and forced stream-K, including the
+    hybrid schedule (4096 x 4096 tiles: whole waves data-parallel, the last
+    ones stream-K), against sampled oracle outputs; the fp8 bias rides on the
+    finishing CTA's epilogue."""
+    rng = np.random.default_rng(m + k + tile)
+    ws = fp8.mm_workspace(m, n, k, "cuda")
+    run_case(fp8, rng, m, n, k, a_major, b_major, full=False, tile=tile, workspace=ws, bias_kind="e4m3")
+    assert flags_clear(ws)
+
+
+@pytest.mark.parametrize("tile", SK_TILES)
+def test_mm_stream_k_deterministic_and_reusable(fp8, tile):
+    """The finishing CTA adds the partials in CTA order: two launches reusing
+    one workspace give the same bits."""
+    m, n, k = 700, 520, 3000
+    rng = np.random.default_rng(5)
+    ws = fp8.mm_workspace(m, n, k, "cuda")
+    _, y1, _ = run_case(fp8, rng, m, n, k, 0, 1, full=False, tile=tile, workspace=ws)
+    rng = np.random.default_rng(5)
+    _, y2, _ = run_case(fp8, rng, m, n, k, 0, 1, full=False, tile=tile, workspace=ws)
+    assert np.array_equal(y1, y2) and flags_clear(ws)
+
+
+def test_mm_stream_k_needs_workspace(fp8):
+    """Forced stream-K without (or with too small) a workspace is refused
+    before anything is enqueued; AUTO without one simply runs data-parallel."""
+    m, n, k = 256, 256, 1024
+    A = torch.zeros((m, k), dtype=torch.uint8, device="cuda")
+    B = torch.zeros((n, k), dtype=torch.uint8, device="cuda")
+    sc = torch.ones(2, device="cuda")
+    d = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    small = torch.zeros(SK_FLAG_BYTES, dtype=torch.uint8, device="cuda")
+    for ws in (None, small):
+        args = fp8.MmArgs(m, n, k, A.data_ptr(), 0, 0, k, B.data_ptr(), 0, 0, k, sc.data_ptr(), sc.data_ptr() + 4,
+                          None, 0, None, d.data_ptr(), n, 1 | SK,
+                          ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0)
+        assert fp8._lib.fp8_mm(ctypes.byref(args), torch.cuda.current_stream().cuda_stream) == fp8.FP8_ERR_WORKSPACE
+    assert fp8._lib.fp8_mm(ctypes.byref(fp8.MmArgs(m, n, k, A.data_ptr(), 0, 0, k, B.data_ptr(), 0, 0, k,
+                                                   sc.data_ptr(), sc.data_ptr() + 4, None, 0, None, d.data_ptr(),
+                                                   n, 0)), torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert torch.all(d.float() == 0) and fp8.fp8_get_device_status() == 0
+
+
+@pytest.mark.parametrize("tile", [0] + SK_TILES)
+def test_mm_pair_stream_k(fp8, tile):
+    """dX and dW of one linear in one launch with stream-K over both problems'
+    k-blocks (unequal k: 520 vs 2100), against the oracle."""
+    rng = np.random.default_rng(41)
+    M, N, K = 2100, 520, 300
+    g8 = codes_like_tensor(rng, 1, (M, N), 3000.0)
+    w8 = codes_like_tensor(rng, 0, (N, K), 60.0)
+    x8 = codes_like_tensor(rng, 0, (M, K), 60.0)
+    gs, ldg = store(g8, 0, 0)
+    wst, ldw = store(w8, 0, 0)
+    xs, ldx = store(x8, 0, 0)
+    G, W, X = (torch.from_numpy(t).cuda() for t in (gs, wst, xs))
+    sc = torch.tensor([3.0, 0.5, 0.25], device="cuda")
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty(N, K, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(max(fp8.fp8_mm_workspace_bytes(M, K, N), fp8.fp8_mm_workspace_bytes(N, K, M)),
+                     dtype=torch.uint8, device="cuda")
+    p = lambda t: t.data_ptr()  # noqa: E731
+    s4 = sc.data_ptr()
+    a = fp8.MmArgs(M, K, N, p(G), 1, 0, ldg, p(W), 0, 1, ldw, s4, s4 + 4, None, 0, None, p(dx), K, tile,
+                   p(ws), ws.numel())
+    b = fp8.MmArgs(N, K, M, p(G), 1, 1, ldg, p(X), 0, 1, ldx, s4, s4 + 8, None, 0, None, p(dw), K, tile)
+    fp8.fp8_mm_pair(a, b)
+    torch.cuda.synchronize()
+    assert fp8.fp8_get_device_status() == 0 and flags_clear(ws)
+    gemm_dx, _, sab = oracle.gemm_acc(gs, 1, ldg, 1, wst, 0, 1, ldw, M, K, N)
+    want, _ = oracle.epilogue(gemm_dx, 3.0, 0.5)
+    assert_gemm_close(dx.cpu().view(torch.int16).numpy().view(np.uint16), want, sab, 3.0, 0.5, "pair sk dx")
+    gemm_dw, _, sab = oracle.gemm_acc(gs, 1, 1, ldg, xs, 0, 1, ldx, N, K, M)
+    want, _ = oracle.epilogue(gemm_dw, 3.0, 0.25)
+    assert_gemm_close(dw.cpu().view(torch.int16).numpy().view(np.uint16), want, sab, 3.0, 0.25, "pair sk dw")

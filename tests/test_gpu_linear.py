@@ -49,11 +49,21 @@ def dbias_check(got, g_bits, M, N):
     assert np.all(np.abs(g - o) <= tol), np.max(np.abs(g - o) / tol)
 
 
+def prequantized_device(codes_np, scale, rows, cols):
+    """fp8 codes (numpy [rows, >= cols]) in a 16-aligned device buffer, and the
+    scale as a 1-element device tensor."""
+    buf = torch.zeros((rows, (cols + 15) // 16 * 16), dtype=torch.uint8)
+    buf[:, :cols] = torch.from_numpy(np.ascontiguousarray(codes_np[:, :cols]))
+    return buf.cuda()[:, :cols], torch.tensor([scale], dtype=torch.float32, device="cuda")
+
+
 def linear_step(fp8, x, w, g, rings, orings, full, rng, bias=None, bias8=None, bias_scale=None,
-                need_dbias=False, w_pre=None, what=""):
+                need_dbias=False, w_pre=None, x_pre=None, what=""):
     """One forward + backward on the GPU and in the oracle; compare everything.
-    w_pre: (w8 codes [N,K] numpy, scale) for the pre-quantized weight path."""
-    M, K = x.shape
+    w_pre / x_pre: (codes [N,K] / [M,K] numpy, scale) for a pre-quantized
+    weight / activation: its quantize is skipped, its snapshot is the given
+    scale, its amax output 0 and its ring untouched."""
+    M, K = x.shape if x is not None else x_pre[0].shape
     N = w.shape[0] if w is not None else w_pre[0].shape[0]
     rx, rw, rg = rings
     orx, orw, org = orings
@@ -66,21 +76,34 @@ def linear_step(fp8, x, w, g, rings, orings, full, rng, bias=None, bias8=None, b
         dev_bsc = torch.tensor([bias_scale], dtype=torch.float32, device="cuda")
     if w_pre is not None:
         w8_np, wsc = w_pre
-        wbuf = torch.zeros((N, (K + 15) // 16 * 16), dtype=torch.uint8)
-        wbuf[:, :K] = torch.from_numpy(w8_np[:, :K])
-        w_dev = wbuf.cuda()[:, :K]
-        w_scale_in = torch.tensor([wsc], dtype=torch.float32, device="cuda")
+        w_dev, w_scale_in = prequantized_device(w8_np, wsc, N, K)
         ring_w_words = ring_words(rw)
     else:
         w_dev, w_scale_in = w.cuda(), None
-    f = fp8.linear_forward(x.cuda(), w_dev, rx, None if w_pre is not None else rw, bias=dev_bias,
-                           bias_scale=dev_bsc, w_scale_in=w_scale_in, hist_len=rx.H)
+    if x_pre is not None:
+        x8_np, xsc = x_pre
+        x_dev, x_scale_in = prequantized_device(x8_np, xsc, M, K)
+        ring_x_words = ring_words(rx)
+    else:
+        x_dev, x_scale_in = x.cuda(), None
+    # outputs start as NaN: a pre-quantized operand's snapshot and zero amax
+    # must be written by the library (the GEMM launch's side writes)
+    scales = torch.full((4,), float("nan"), dtype=torch.float32, device="cuda")
+    f = fp8.linear_forward(x_dev, w_dev, None if x_pre is not None else rx, None if w_pre is not None else rw,
+                           bias=dev_bias, bias_scale=dev_bsc, x_scale_in=x_scale_in, w_scale_in=w_scale_in,
+                           hist_len=rx.H, scales=scales)
     b = fp8.linear_backward(g.cuda(), f, rg, need_dbias=need_dbias)
     torch.cuda.synchronize()
     assert fp8.fp8_get_device_status() == 0
 
     # oracle quantize (always full) and the scale snapshots
-    x8o, ax, sx = oracle.quantize(bits(x), oracle.DT_BF16, E4, orx, ld_out=(K + 15) // 16 * 16)
+    if x_pre is not None:
+        x8o = np.zeros((M, (K + 15) // 16 * 16), np.uint8)
+        x8o[:, :K] = x8_np[:, :K]
+        ax, sx = np.float32(0.0), np.float32(x_pre[1])
+        assert np.array_equal(ring_words(rx), ring_x_words), "ring_x must stay untouched"
+    else:
+        x8o, ax, sx = oracle.quantize(bits(x), oracle.DT_BF16, E4, orx, ld_out=(K + 15) // 16 * 16)
     if w_pre is not None:
         w8o, aw, sw = np.ascontiguousarray(w8_np), np.float32(0.0), np.float32(w_pre[1])
     else:
@@ -94,7 +117,8 @@ def linear_step(fp8, x, w, g, rings, orings, full, rng, bias=None, bias8=None, b
     else:
         assert np.array_equal(ring_words(rw), ring_w_words), "ring_w must stay untouched"
     assert_codes_equal(host_rows(b.g8), g8o[:, :N], E5)
-    assert np.array_equal(ring_words(rx), oracle_ring_words(orx)), what
+    if x_pre is None:
+        assert np.array_equal(ring_words(rx), oracle_ring_words(orx)), what
     if w_pre is None:
         assert np.array_equal(ring_words(rw), oracle_ring_words(orw)), what
     assert np.array_equal(ring_words(rg), oracle_ring_words(org)), what
@@ -157,6 +181,31 @@ def test_prequantized_weight(fp8):
         linear_step(fp8, x, None, g, rings, orings, True, rng, w_pre=(w8, float(wsc)), what=f"w8 step {step}")
 
 
+@pytest.mark.parametrize("both", (False, True), ids=("x8", "x8+w8"))
+def test_prequantized_activation(fp8, both):
+    """A pre-quantized x8 skips its quantize ([ops] bullet: g/x/w may each
+    arrive fp8 in the matching format): sx = x_scale_in, amax_x = 0 and ring_x
+    untouched, written by the GEMM launch's side writes; with w8 pre-quantized
+    too no quantize runs at all and both snapshots and amaxes come from those
+    side writes.  The backward then reuses the caller's x8 and scale for dW.
+    Config 1 shapes (full comparison) and a c3-sized case (sampled)."""
+    for (M, K, N, full, cfg) in ((wl.C1.M, wl.C1.K, wl.C1.N, True, 1), (512, 1536, 1536, False, 3)):
+        rings, orings = make_rings(fp8)
+        rng = np.random.default_rng(23 + cfg)
+        w = wl.normal((N, K), wl.weight_std(K), wl.seed_for(cfg, 0, wl.OP_W))
+        w_pre = None
+        if both:
+            wsc = np.float32(448.0) / oracle.amax(bits(w), oracle.DT_BF16)
+            w_pre = (oracle.quantize_codes(bits(w), oracle.DT_BF16, E4, wsc), float(wsc))
+        for step in range(2):
+            x = wl.normal((M, K), 1.0 + step, wl.seed_for(cfg, step, wl.OP_X))
+            g = wl.normal((M, N), 1e-3, wl.seed_for(cfg, step, wl.OP_G))
+            xsc = np.float32(448.0) / oracle.amax(bits(x), oracle.DT_BF16) / np.float32(1.5)
+            x8 = oracle.quantize_codes(bits(x), oracle.DT_BF16, E4, xsc)
+            linear_step(fp8, None, None if both else w, g, rings, orings, full, rng, w_pre=w_pre,
+                        x_pre=(x8, float(xsc)), need_dbias=True, what=f"x8 M={M} step {step}")
+
+
 @pytest.mark.parametrize("shape", wl.C2_SHAPES, ids=lambda s: s.name)
 def test_config2_shapes(fp8, shape):
     rings, orings = make_rings(fp8)
@@ -217,8 +266,10 @@ def test_config5_edge_shapes(fp8, shape):
 def test_config5_twenty_step_sequence(fp8):
     """Config 5: 20 steps over 12 layers x 6 linears (216 rings), M = 2048, input
     std drifting log-uniformly in [0.5, 4] per step.  Every ring word matches
-    the oracle after every step; the backward's dX/dW use the forward's
-    snapshots (checked on sampled outputs of two linears at three steps)."""
+    the oracle after every step.  At every step one linear of each type (q,
+    up, down) in layer step % 12 is checked in depth: x8, w8 and g8 byte for
+    byte, the snapshots, and sampled y, dX and dW -- the backward dequantizing
+    with the forward's snapshots."""
     H, M = wl.HIST_LEN, 2048
     words = fp8.fp8_ring_bytes(H) // 4
     nlin = wl.C5_LAYERS * len(wl.C5_LAYER)
@@ -233,6 +284,21 @@ def test_config5_twenty_step_sequence(fp8):
     ws_dev = [w.cuda() for w in ws]
     w_bits = [bits(w) for w in ws]
     amax_w = [oracle.amax(b, oracle.DT_BF16) for b in w_bits]
+    per_layer = len(wl.C5_LAYER)
+    # one linear of each shape type within a layer: q (first), up, down
+    types = [0] + [i for i, s in enumerate(wl.C5_LAYER) if s.K != s.N]
+    assert len(types) == 3
+
+    def small_sample(I, J):
+        return sample_points(rng, I, J, nrows=4, ncols=4, nrand=2048)
+
+    def check_sampled(y_dev, a8, fmt_a, a_s, b8, fmt_b, b_s, I, J, Kc, sa, sb, what):
+        y = y_dev.cpu().view(torch.int16).numpy().view(np.uint16)
+        pi, pj = small_sample(I, J)
+        acc, sab = oracle.gemm_acc_points(pi, pj, a8, fmt_a, *a_s, b8, fmt_b, *b_s, Kc)
+        want, _ = oracle.epilogue(acc, sa, sb, col_idx=pj)
+        assert_gemm_close(y[pi, pj], want, sab, sa, sb, what)
+
     for step in range(wl.C5_STEPS):
         sigma = wl.log_uniform(0.5, 4.0, wl.seed_for(5, step, wl.OP_STD))
         xs = {K: (t.float() * sigma).to(torch.bfloat16) for K, t in base_x.items()}
@@ -241,7 +307,7 @@ def test_config5_twenty_step_sequence(fp8):
         gs_dev = {N: t.cuda() for N, t in gs.items()}
         xa = {K: oracle.amax(bits(t), oracle.DT_BF16) for K, t in xs.items()}
         ga = {N: oracle.amax(bits(t), oracle.DT_BF16) for N, t in gs.items()}
-        check_now = step in (0, 10, 19)
+        deep = {(step % wl.C5_LAYERS) * per_layer + t for t in types}
         for li, s in enumerate(wl.C5_LAYER * wl.C5_LAYERS):
             rx, rw, rg = rings[3 * li: 3 * li + 3]
             f = fp8.linear_forward(xs_dev[s.K], ws_dev[li], rx, rw)
@@ -251,14 +317,21 @@ def test_config5_twenty_step_sequence(fp8):
             orx.advance(xa[s.K], E4)
             orw.advance(amax_w[li], E4)
             org.advance(ga[s.N], E5)
-            if check_now and li in (0, nlin - 1):
+            if li in deep:
                 torch.cuda.synchronize()
-                assert (f.sx.item(), f.sw.item(), b.sg.item()) == (sx, sw, sg)
+                what = f"c5 step {step} linear {li} ({s.name})"
+                assert (f.sx.item(), f.sw.item(), b.sg.item()) == (sx, sw, sg), what
+                assert (f.amax_x.item(), f.amax_w.item(), b.amax_g.item()) == (xa[s.K], amax_w[li], ga[s.N]), what
                 x8 = oracle.quantize_codes(bits(xs[s.K]), oracle.DT_BF16, E4, sx)
                 w8 = oracle.quantize_codes(w_bits[li], oracle.DT_BF16, E4, sw)
                 g8 = oracle.quantize_codes(bits(gs[s.N]), oracle.DT_BF16, E5, sg)
-                gemm_check(b.dx, g8, 0, E5, w8, E4, M, s.K, s.N, sg, sw, "dx", False, rng, what="c5 dx")
-                gemm_check(b.dw, g8, 0, E5, x8, E4, s.N, s.K, M, sg, sx, "dw", False, rng, what="c5 dw")
+                assert_codes_equal(host_rows(f.x8), x8, E4)
+                assert_codes_equal(host_rows(f.w8), w8, E4)
+                assert_codes_equal(host_rows(b.g8), g8, E5)
+                K, N = s.K, s.N
+                check_sampled(f.y, x8, E4, (K, 1), w8, E4, (K, 1), M, N, K, sx, sw, what + " y")
+                check_sampled(b.dx, g8, E5, (N, 1), w8, E4, (1, K), M, K, N, sg, sw, what + " dx")
+                check_sampled(b.dw, g8, E5, (1, N), x8, E4, (1, K), N, K, M, sg, sx, what + " dw")
         torch.cuda.synchronize()
         got = allbuf.cpu().view(torch.int32).numpy().view(np.uint32)
         want = np.stack([oracle_ring_words(r) for r in orings])
@@ -343,3 +416,65 @@ def test_forward_mixed_input_dtypes(fp8):
         assert_codes_equal(host_rows(f.x8), x8o, E4)
         assert np.array_equal(ring_words(rx), oracle_ring_words(orx))
         gemm_check(f.y, x8o, 0, E4, w8o, E4, M, N, K, sx, sw, "fwd", True, rng, what="mixed y")
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 192, 0), (0, 192, 128), (64, 0, 128), (0, 0, 0)],
+                         ids=["K0", "M0", "N0", "all0"])
+@pytest.mark.parametrize("bias_kind", ("bf16", "e4m3"))
+def test_empty_sizes(fp8, M, N, K, bias_kind):
+    """Empty sizes: an operand with no elements is not quantized (its ring does
+    not step); a non-empty one is, with its ring step; y is the bias when the
+    contraction K is empty; a requested gradient with elements is zero when its
+    contraction is empty (dX when N = 0, dW and dbias when M = 0) and dbias is
+    the column sum of g when K = 0 -- all against the oracle's orchestration."""
+    rx, rw, rg = fp8.ScaleRing(16), fp8.ScaleRing(16), fp8.ScaleRing(16)
+    orx, orw, org = oracle.Ring(16), oracle.Ring(16), oracle.Ring(16)
+    x = wl.normal((M, K), 1.0, 61)
+    w = wl.normal((N, K), 0.05, 62)
+    g = wl.normal((M, N), 1e-3, 63)
+    b = wl.normal((N,), 0.01, 64)
+    if bias_kind == "bf16":
+        dev_bias, dev_bsc, bias_np, bias_dt, bsc = b.cuda(), None, bits(b), oracle.DT_BF16, 1.0
+    else:
+        bsc = np.float32(448.0) / max(oracle.amax(bits(b).reshape(1, -1), oracle.DT_BF16), np.float32(1e-3)) \
+            if N else np.float32(1.0)
+        b8 = oracle.quantize_codes(bits(b).reshape(1, -1), oracle.DT_BF16, E4, bsc)[0] if N else \
+            np.zeros(0, np.uint8)
+        dev_bias, dev_bsc = torch.from_numpy(np.ascontiguousarray(b8)).cuda(), \
+            torch.tensor([float(bsc)], device="cuda")
+        bias_np, bias_dt = b8, oracle.DT_E4M3
+    before = [ring_words(r).copy() for r in (rx, rw, rg)]
+    f = fp8.linear_forward(x.cuda(), w.cuda(), rx, rw, bias=dev_bias, bias_scale=dev_bsc)
+    bwd = fp8.linear_backward(g.cuda(), f, rg, need_dbias=True)
+    torch.cuda.synchronize()
+    assert fp8.fp8_get_device_status() == 0
+    of = oracle.linear_forward(M, N, K, bits(x), oracle.DT_BF16, bits(w), oracle.DT_BF16, orx, orw,
+                               bias=bias_np, bias_dtype=bias_dt, bias_scale=float(bsc),
+                               ldx8=(K + 15) // 16 * 16, ldw8=(K + 15) // 16 * 16)
+    ob = oracle.linear_backward(M, N, K, bits(g), oracle.DT_BF16, org, of["x8"], E4, of["sx"], of["w8"], E4,
+                                of["sw"], ldg8=(N + 15) // 16 * 16, need_dbias=True)
+    # rings: stepped exactly when their operand has elements
+    for ring, oring, live, b0 in ((rx, orx, M * K > 0, before[0]), (rw, orw, N * K > 0, before[1]),
+                                  (rg, org, M * N > 0, before[2])):
+        if live:
+            assert np.array_equal(ring_words(ring), oracle_ring_words(oring))
+        else:
+            assert np.array_equal(ring_words(ring), b0) and oring.step == 0
+    if M * K:
+        assert_codes_equal(host_rows(f.x8), of["x8"][:, :K], E4)
+        assert f.sx.item() == of["sx"] and f.amax_x.item() == of["amax_x"]
+    if N * K:
+        assert_codes_equal(host_rows(f.w8), of["w8"][:, :K], E4)
+        assert f.sw.item() == of["sw"] and f.amax_w.item() == of["amax_w"]
+    if M * N:
+        assert_codes_equal(host_rows(bwd.g8), ob["g8"][:, :N], E5)
+        y = f.y.cpu().view(torch.int16).numpy().view(np.uint16)
+        assert_gemm_close(y, of["y"], np.zeros(of["y"].shape), 1.0, 1.0, "y of an empty contraction")
+    if M * K:
+        assert np.array_equal(bwd.dx.cpu().view(torch.int16).numpy().view(np.uint16), ob["dx"])
+    if N * K:
+        assert np.array_equal(bwd.dw.cpu().view(torch.int16).numpy().view(np.uint16), ob["dw"])
+    if N:
+        got = bwd.dbias.cpu().view(torch.int16).numpy().view(np.uint16)
+        gv, ov = oracle.bf16_to_f32(got).astype(np.float64), oracle.bf16_to_f32(ob["dbias"]).astype(np.float64)
+        assert np.all(np.abs(gv - ov) <= np.maximum(oracle.bf16_ulp(ov), 2e-6 * ob["dbias_sumabs"]))

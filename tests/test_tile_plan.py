@@ -71,3 +71,63 @@ def test_plan_validation(fp8):
     assert (empty.tile_cfg, empty.tiles, empty.units) == (0, 0, 0)
     one = F.fp8_mm_plan(args(F, 0, 256, 256), args(F, 256, 256, 256))   # the empty problem is dropped
     assert one.tiles == 4 and one.tile_cfg == 1
+
+
+WS = 0x8000000  # fake workspace address
+
+
+def with_ws(F, a, nbytes=None):
+    a.workspace = WS
+    a.workspace_bytes = F.fp8_mm_workspace_bytes(a.m, a.n, a.k) if nbytes is None else nbytes
+    return a
+
+
+def test_workspace_bytes(fp8):
+    F = fp8
+    flags, slot = 160 * 8 * 4, 128 * 256 * 4
+    assert F.fp8_mm_workspace_bytes(0, 10, 10) == 0 and F.fp8_mm_workspace_bytes(10, 10, 0) == 0
+    assert F.fp8_mm_workspace_bytes(64, 192, 128) == flags + 2 * slot     # two 128 x 128 x 128 blocks
+    assert F.fp8_mm_workspace_bytes(2048, 1536, 6912) == flags + 160 * slot
+    lin = F.fp8_linear_workspace_bytes(2048, 1536, 6912)
+    assert lin >= F.fp8_dbias_workspace_bytes(2048, 1536) + flags + 160 * slot
+
+
+@pytest.mark.parametrize("m,n,k,a_major,b_major", [
+    (2048, 1536, 6912, 0, 1),     # dX with contraction 6912: 96 tiles of 128x256 on 148 SMs
+    (2048, 1536, 6912, 0, 0),     # forward with K = 6912
+    (512, 1536, 6912, 0, 1),
+    (2048, 6912, 1536, 0, 0),     # 432 tiles = 2.92 waves: already balanced
+])
+def test_stream_k_costed(fp8, m, n, k, a_major, b_major):
+    """With a workspace the planner also costs stream-K; AUTO takes it only
+    for a clear gain over every data-parallel plan, and never where the
+    data-parallel waves are already even (2048 x 6912 x 1536)."""
+    F = fp8
+    plain = F.fp8_mm_plan(args(F, m, n, k, a_major, b_major))
+    sk = F.fp8_mm_plan(with_ws(F, args(F, m, n, k, a_major, b_major)))
+    assert plain.stream_k_ctas == 0
+    if sk.stream_k_ctas:
+        assert sk.est_us < 0.95 * plain.est_us and sk.tile_cfg & F.FP8_TILE_STREAMK
+    else:
+        assert (sk.tile_cfg, sk.tiles, sk.units) == (plain.tile_cfg, plain.tiles, plain.units)
+    if (m, n, k) == (2048, 6912, 1536):
+        assert sk.stream_k_ctas == 0
+    forced = F.fp8_mm_plan(with_ws(F, args(F, m, n, k, a_major, b_major, tile_cfg=2 | F.FP8_TILE_STREAMK)))
+    assert forced.stream_k_ctas > 0
+
+
+def test_stream_k_forced_and_hybrid(fp8):
+    F = fp8
+    p = F.fp8_mm_plan(with_ws(F, args(F, 4096, 4096, 384, tile_cfg=1 | F.FP8_TILE_STREAMK)))
+    # 1024 tiles of 128x128: five whole waves of 148 data-parallel, 284 tiles' k-blocks stream-K
+    assert p.tile_cfg == 1 | F.FP8_TILE_STREAMK and p.dp_tiles == 5 * 148 and p.stream_k_ctas == 148
+    import ctypes
+    info = F.MmPlanInfo()
+    a = with_ws(F, args(F, 256, 256, 1024, tile_cfg=1 | F.FP8_TILE_STREAMK), nbytes=0)
+    a.workspace = None
+    assert F._lib.fp8_mm_plan(ctypes.byref(a), None, 148, ctypes.byref(info)) == F.FP8_ERR_WORKSPACE
+    bad = args(F, 256, 256, 1024, tile_cfg=3 | F.FP8_TILE_STREAMK)      # pair tiles have no stream-K
+    assert F._lib.fp8_mm_plan(ctypes.byref(bad), None, 148, ctypes.byref(info)) == F.FP8_ERR_INVALID_ARG
+    mis = with_ws(F, args(F, 256, 256, 1024))
+    mis.workspace = WS + 8                                              # not 16-byte aligned
+    assert F._lib.fp8_mm_plan(ctypes.byref(mis), None, 148, ctypes.byref(info)) == F.FP8_ERR_WORKSPACE

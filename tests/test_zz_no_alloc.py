@@ -5,10 +5,11 @@ manager it does not control, such as a plugin in a serving runtime with a fixed
 device-memory budget -- so they have no workspace to hand to fp8_dbias.  This
 entry point runs the same kernel with its scratch in a fixed 1 MiB array inside
 the library.  The test calls it through the C ABI twice in a row and checks each
-result against fp8_dbias (with a workspace) on the same input, within the bias
-gradient tolerance the other tests use: max(1 bf16 ulp, 2e-6 sum|g|).  It also
-checks that a request beyond the fixed scratch is refused.  This file is
-collected last so a stopped run has already run everything else.
+result against fp8_dbias (with a workspace) on the same input, and against the
+CPU oracle's column sums, within the bias gradient tolerance the other tests
+use: max(1 bf16 ulp, 2e-6 sum|g|).  It also checks that a request beyond the
+fixed scratch is refused.  This file is collected last so a stopped run has
+already run everything else.
 """
 import ctypes
 
@@ -16,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -36,6 +38,15 @@ def check_close(got, want, g):
     assert np.all(np.abs(got - want) <= tol), np.max(np.abs(got - want) / tol)
 
 
+def check_oracle(got, g_np, dtype, M, N, sg=1.0):
+    """got (bf16 device tensor) vs the oracle's fixed-order fp32 column sums."""
+    want, _, sa = oracle.dbias(g_np, dtype, M, N, sg)
+    gv = oracle.bf16_to_f32(got.cpu().view(torch.int16).numpy().view(np.uint16)).astype(np.float64)
+    ov = oracle.bf16_to_f32(want).astype(np.float64)
+    tol = np.maximum(oracle.bf16_ulp(ov), 2e-6 * sa)
+    assert np.all(np.abs(gv - ov) <= tol), np.max(np.abs(gv - ov) / tol)
+
+
 def test_dbias_noalloc_matches_workspace_entry_point():
     import fp8_delayed_scaling_03_b200 as F
     lib = F._lib
@@ -50,6 +61,8 @@ def test_dbias_noalloc_matches_workspace_entry_point():
         assert lib.fp8_dbias_noalloc(g.data_ptr(), F.FP8_DT_BF16, M, N, N, None, out.data_ptr(), stream) == 0
         torch.cuda.synchronize()
         check_close(out, ref, g)
+        if i == 0:
+            check_oracle(out, g.cpu().view(torch.int16).numpy().view(np.uint16), oracle.DT_BF16, M, N)
     # fp8 g with its scale (dequantized before the sum), two calls in a row
     M, N = 3000, 700
     codes = torch.randint(0, 0x5C, (M, 704), dtype=torch.int32).to(torch.uint8)
@@ -67,6 +80,7 @@ def test_dbias_noalloc_matches_workspace_entry_point():
         torch.cuda.synchronize()
         deq = g8.cpu().view(torch.float8_e5m2).double() / 37.5
         check_close(out, ref, deq)
+        check_oracle(out, np.ascontiguousarray(codes.numpy()), oracle.DT_E5M2, M, N, 37.5)
     # beyond the fixed scratch: refused, nothing enqueued
     big_n = 1 << 20
     assert F.fp8_dbias_workspace_bytes(2048, big_n) > (1 << 20)

@@ -104,6 +104,17 @@ def normal_device(shape, std: float, seed: int, device, dtype=torch.bfloat16) ->
     return (torch.randn(*shape, generator=g, dtype=torch.float32, device=device) * std).to(dtype)
 
 
+def normal_with_outliers_device(shape, std: float, seed: int, mask_seed: int, device, p: float = 1e-3,
+                                factor: float = 50.0, dtype=torch.bfloat16) -> torch.Tensor:
+    """normal_with_outliers drawn by seeded generators on `device` (for large
+    benchmark inputs)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    v = torch.randn(*shape, generator=g, dtype=torch.float32, device=device) * std
+    gm = torch.Generator(device=device).manual_seed(mask_seed)
+    mask = torch.rand(*shape, generator=gm, device=device) < p
+    return torch.where(mask, v * factor, v).to(dtype)
+
+
 # Benchmark workload: the linears of the pages' 12L/dim1024/B4xT512 model
 # (configuration 2), forward and backward, with a bf16 bias and its gradient.
 BENCH_LAYERS = 12

@@ -172,7 +172,7 @@ int validate_mm(const MmCall& c) {
   if (c.m > 0 && c.n > 0 && (!c.d || c.ldd < c.n || !aligned(c.d, 2))) return FP8_ERR_INVALID_ARG;
   const int base_cfg = c.tile_cfg & ~FP8_TILE_STREAMK;
   if (base_cfg < FP8_TILE_AUTO || base_cfg > FP8_TILE_SPLITK_128x128) return FP8_ERR_INVALID_ARG;
-  if ((c.tile_cfg & FP8_TILE_STREAMK) && base_cfg != FP8_TILE_128x128 && base_cfg != FP8_TILE_128x256)
+  if ((c.tile_cfg & FP8_TILE_STREAMK) && (base_cfg < FP8_TILE_128x128 || base_cfg > FP8_TILE_PAIR_256x256))
     return FP8_ERR_INVALID_ARG;
   if (c.ws_bytes && (!c.ws || !aligned(c.ws, 16))) return FP8_ERR_WORKSPACE;
   if (c.bias) {
@@ -310,9 +310,11 @@ TilePlan pick_tile(const MmCall* calls, int n, int sms, int64_t sk_slots = 0, in
         have = true;
       }
     }
-    // stream-K (single-CTA tiles, unbatched)
-    if (o.cfg == kGemmPair256 || batched || sk_slots <= 0) continue;
-    const int64_t P = std::min<int64_t>(sms, kSkMaxCtas);
+    // stream-K (unbatched; a pair tile's two CTAs keep one partial slot each)
+    if (batched || sk_slots <= 0) continue;
+    const bool pair = o.cfg == kGemmPair256;
+    const int64_t P = pair ? std::min<int64_t>(sms / 2, kSkMaxCtas / 2) : std::min<int64_t>(sms, kSkMaxCtas);
+    const int64_t unit_slots = pair ? sk_slots / 2 : sk_slots;
     const int64_t D = tiles >= 2 * P ? (tiles / P - 1) * P : 0;
     const int64_t u0 = D < cnt[0] ? (cnt[0] - D) * kb[0] : 0;
     const int64_t u1 = (tiles - std::max(D, cnt[0])) * kb[1];
@@ -322,7 +324,7 @@ TilePlan pick_tile(const MmCall* calls, int n, int sms, int64_t sk_slots = 0, in
     // at most kSkMaxParts partials): ceil((kb - 1) / floor(U / ctas)) <= 6
     const int64_t kbmax = std::max(kb[0], kb[1]);
     const int64_t min_units = std::max<int64_t>(kSkMinUnits, (kbmax - 1 + kSkMaxParts - 1) / kSkMaxParts);
-    int64_t ctas = std::min({P, sk_slots, std::max<int64_t>(force_sk ? 1 : 0, U / min_units)});
+    int64_t ctas = std::min({P, unit_slots, std::max<int64_t>(force_sk ? 1 : 0, U / min_units)});
     while (ctas > 1 && (kbmax - 1 + U / ctas - 1) / (U / ctas) > kSkMaxParts) --ctas;
     if (ctas < (force_sk ? 1 : 2)) continue;
     const int64_t nparts = U / ctas > 0 ? (kbmax - 1 + U / ctas - 1) / (U / ctas) : 0;
@@ -432,17 +434,26 @@ int plan_launch(const MmCall* calls, int n, int sms, TilePlan* plan, int* split)
   for (int i = 0; i < n; ++i) batched = batched || calls[i].batch > 1;
   const int64_t slots = batched ? 0 : sk_slots_available(calls, n);
   *split = 1;
+  // every pair of a stream-K launch on pair tiles must be resident at once
+  auto pairs_resident = [&](const TilePlan& pl) {
+    if (pl.cfg != kGemmPair256 || pl.sk_ctas == 0) return true;
+    int dev = 0;
+    const int64_t need = pl.dp_tiles > 0 ? std::min<int64_t>(sms / 2, kSkMaxCtas / 2) : pl.sk_ctas;
+    return cudaGetDevice(&dev) == cudaSuccess && gemm_pair_capacity(dev) >= need;
+  };
   if (force_sk) {
     if (batched) return FP8_ERR_INVALID_ARG;
-    if (slots < 1) return FP8_ERR_WORKSPACE;
+    if (slots < (req_cfg == kGemmPair256 ? 2 : 1)) return FP8_ERR_WORKSPACE;
     *plan = pick_tile(calls, n, sms, slots, req_cfg, true);
-    return plan->sk_ctas > 0 ? FP8_OK : FP8_ERR_WORKSPACE;
+    if (plan->sk_ctas == 0) return FP8_ERR_WORKSPACE;
+    return pairs_resident(*plan) ? FP8_OK : FP8_ERR_UNSUPPORTED;
   }
   if (req_cfg != FP8_TILE_AUTO) {
     *plan = TilePlan{};
     plan->cfg = req_cfg;
   } else {
     *plan = pick_tile(calls, n, sms, slots);
+    if (!pairs_resident(*plan)) *plan = pick_tile(calls, n, sms, 0);
   }
   int& cfg = plan->cfg;
   // Split-K (single-problem launches): few 128 x 128 tiles and a long K leave
@@ -914,7 +925,9 @@ int fp8_mm_plan(const fp8_mm_args* a, const fp8_mm_args* b, int num_sms, fp8_mm_
   const int64_t cap = cfg == kGemmPair256 ? num_sms / 2 : num_sms;
   out->tile_cfg = plan.sk_ctas ? (cfg | FP8_TILE_STREAMK) : cfg;
   out->tiles = tiles;
-  out->units = plan.sk_ctas ? static_cast<int>(std::max<int64_t>(plan.sk_ctas, std::min<int64_t>(plan.dp_tiles, std::min(num_sms, kSkMaxCtas))))
+  const int64_t sk_cap = cfg == kGemmPair256 ? std::min<int64_t>(num_sms / 2, kSkMaxCtas / 2)
+                                             : std::min<int64_t>(num_sms, kSkMaxCtas);
+  out->units = plan.sk_ctas ? static_cast<int>(plan.dp_tiles > 0 ? sk_cap : plan.sk_ctas)
                             : static_cast<int>(std::max<int64_t>(1, std::min(tiles, cap)));
   out->est_us = req_cfg != FP8_TILE_AUTO && !force_sk ? 0.0 : plan.est_us;
   out->stream_k_ctas = plan.sk_ctas;

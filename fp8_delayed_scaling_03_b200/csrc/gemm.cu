@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain, 1);
     if constexpr (kSplit) mbar_init(pbar, rank == 0 ? 1u : static_cast<uint32_t>(kEpiWarps));
-    if constexpr (!kPair && !kSplit)
+    if constexpr (!kSplit)
       for (int i = 0; i < kEpiWarps; ++i) mbar_init(&skbar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -498,6 +498,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float4* const sk_part = reinterpret_cast<float4*>(p.sk_part);
     uint8_t* const sk_stage = sA + ew * kSkStageBytes;
     uint32_t sk_phase = 0;
+    // the slot (and flag block) of a work unit's CTA of this rank: a pair tile
+    // keeps one partial per CTA, its 128-row half
+    auto sk_slot = [&](int u) { return kPair ? 2 * u + static_cast<int>(prank) : u; };
     auto sk_block = [&](int slot, int st) {
       return sk_part + ((static_cast<int64_t>(slot) * kEpiWarps + ew) * kSteps + st) * (kSkBlock / 16);
     };
@@ -543,7 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = w.nparts >= 1 && w.nparts <= kSkMaxParts;
         if (!ok && lane == 0 && p.status) atomicExch(p.status, kDevTimeout);  // outside the planner's bound: give up
         for (int q = 0; q < w.nparts && ok; ++q)
-          ok = flag_wait_warp(p.sk_flag + static_cast<int64_t>(w.part0 + q) * kEpiWarps + ew, p.status, abort_flag);
+          ok = flag_wait_warp(p.sk_flag + static_cast<int64_t>(sk_slot(w.part0 + q)) * kEpiWarps + ew, p.status,
+                              abort_flag);
         if (!ok) {
           *abort_flag = 1;
           break;
@@ -562,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             mbar_arrive_expect_tx(&skbar[ew], static_cast<uint32_t>(w.nparts * nst * kSkBlock));
             for (int q = 0; q < w.nparts; ++q)
-              bulk_copy_g2s(sk_stage + q * nst * kSkBlock, sk_block(w.part0 + q, st),
+              bulk_copy_g2s(sk_stage + q * nst * kSkBlock, sk_block(sk_slot(w.part0 + q), st),
                             static_cast<uint32_t>(nst * kSkBlock), &skbar[ew]);
           }
           if (!mbar_wait(&skbar[ew], sk_phase, p.status, abort_flag)) break;
@@ -612,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (w.kind != kFull) {
           if (w.kind == kPartial) {  // this part's accumulator goes to the CTA's slot
-            float4* dst = sk_block(unit, st) + lane;
+            float4* dst = sk_block(sk_slot(unit), st) + lane;
             #pragma unroll
             for (int j = 0; j < 32; j += 4)
               __stcg(dst + (j / 4) * 32, make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
@@ -672,11 +676,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (w.kind == kPartial) {  // this warp's share of the partial is written: raise its flag
-        warp_release_flag(p.sk_flag + static_cast<int64_t>(unit) * kEpiWarps + ew, 1u);
+        warp_release_flag(p.sk_flag + static_cast<int64_t>(sk_slot(unit)) * kEpiWarps + ew, 1u);
       } else if (w.kind == kOwner) {  // every lane has read the partials: clear their flags
         __syncwarp();
         if (lane == 0)
-          for (int q = 0; q < w.nparts; ++q) p.sk_flag[static_cast<int64_t>(w.part0 + q) * kEpiWarps + ew] = 0u;
+          for (int q = 0; q < w.nparts; ++q) p.sk_flag[static_cast<int64_t>(sk_slot(w.part0 + q)) * kEpiWarps + ew] = 0u;
       }
       if (kSplit && rank != 0) {  // partial parked: one bulk copy into rank 0's region
         fence_proxy_async_smem();  // this thread's parked bytes, visible to the copy engine
@@ -707,6 +711,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
+
+// Pairs (clusters of two 256x256-tile CTAs) that can be resident at once
+// (cached per device; 0 on failure).
+int pair_capacity_impl(int dev) {
+  using C = Cfg<256, true>;
+  static int cache[64] = {};
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  if (cudaFuncSetAttribute(fp8_gemm_kernel<256, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmem) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.gridDim = dim3(2 * (num_sms(dev) / 2));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<256, true, false>, &cfg) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cache[dev] = clusters;
+  return clusters;
+}
+
+int pair_capacity(int dev) { return pair_capacity_impl(dev); }
 
 template <int BN, bool kPair>
 cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t s) {
@@ -743,16 +775,16 @@ cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t 
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   // persistent grid: no more pairs than can be resident at once
-  static int max_pairs[64] = {};
-  if (dev < 64 && max_pairs[dev] == 0) {
-    cfg.gridDim = dim3(2 * (sms / 2));
-    int clusters = 0;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<BN, kPair, false>, &cfg);
-    if (e != cudaSuccess) return e;
-    max_pairs[dev] = clusters > 0 ? clusters : 1;
+  const int cap = pair_capacity(dev);
+  if (cap <= 0) return cudaErrorInvalidConfiguration;
+  int pairs = p.total_tiles < cap ? p.total_tiles : cap;
+  // stream-K: the planner's pair count (its whole-tile waves use sms / 2
+  // pairs, at most 80); every pair must be resident at once
+  if (p.sk_ctas > 0) {
+    const int sk_pairs = sms / 2 < 80 ? sms / 2 : 80;
+    pairs = p.dp_tiles > 0 ? sk_pairs : p.sk_ctas;
+    if (pairs > cap) return cudaErrorInvalidConfiguration;
   }
-  const int cap = dev < 64 ? max_pairs[dev] : 1;
-  const int pairs = p.total_tiles < cap ? p.total_tiles : cap;
   cfg.gridDim = dim3(2 * pairs);
   return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BN, kPair, false>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
 }
@@ -834,6 +866,8 @@ cudaError_t launch_fill(const FillParams& p, cudaStream_t s) {
   const int64_t blocks = std::min<int64_t>(cap, std::max<int64_t>(1, (total + 255) / 256));
   return launch_pdl(fill_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
 }
+
+int gemm_pair_capacity(int dev) { return pair_capacity(dev); }
 
 int gemm_split_factor(int tiles, int k_blocks, int sms, bool forced) {
   int dev = 0;

@@ -191,6 +191,8 @@ enum : int { kGemm128 = 1, kGemm256 = 2, kGemmPair256 = 3, kGemmSplit128 = 4 };
 // S with every rank given >= 4 k-blocks and all tiles' clusters resident in
 // one wave; forced: the largest S <= min(3, k_blocks) fitting one wave, else 2.
 int gemm_split_factor(int tiles, int k_blocks, int sms, bool forced);
+// CTA pairs (256x256 tiles) that can be resident at once on the device.
+int gemm_pair_capacity(int device);
 // maps[0..2]: A, B, D of pr[0]; maps[3..5]: those of pr[1] (zeroed if unused).
 cudaError_t launch_gemm(const CUtensorMap* maps, const GemmParams& p, int cfg, cudaStream_t s);
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s);

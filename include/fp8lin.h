@@ -71,10 +71,11 @@ typedef enum { FP8_K_MAJOR = 0, FP8_MN_MAJOR = 1 } fp8_major;
  * [r kb/S, (r+1) kb/S) and rank 0 adds the partial fp32 accumulators in rank
  * order before the epilogue; fp8_mm only -- a two-GEMM launch falls back to
  * 128x128).
- * Stream-K (FP8_TILE_STREAMK, or'ed with FP8_TILE_128x128 or
- * FP8_TILE_128x256; needs a workspace): one CTA per SM; whole waves of tiles
- * run data-parallel and the k-blocks of the remaining tiles are split evenly
- * over the CTAs, so that no SM idles while others finish a last partial wave.
+ * Stream-K (FP8_TILE_STREAMK, or'ed with FP8_TILE_128x128, FP8_TILE_128x256
+ * or FP8_TILE_PAIR_256x256; needs a workspace): one CTA (pair) per SM (pair
+ * of SMs); whole waves of tiles run data-parallel and the k-blocks of the
+ * remaining tiles are split evenly over the CTAs (pairs), so that no SM idles
+ * while others finish a last partial wave.
  * A tile cut between CTAs is finished by the CTA holding its first k-block,
  * which adds the others' fp32 partial accumulators (stored in the workspace)
  * in CTA order: the result is deterministic for a given GPU.

@@ -361,7 +361,7 @@ def test_mm_batched_large_sampled(fp8, batch, m, n, k, a_major, b_major):
 # ---------------------------------------------------------------- stream-K
 
 SK = 8                         # FP8_TILE_STREAMK
-SK_TILES = [1 | SK, 2 | SK]    # 128x128 and 128x256 tiles with stream-K forced
+SK_TILES = [1 | SK, 2 | SK, 3 | SK]    # 128x128, 128x256 and 256x256 pair tiles with stream-K forced
 SK_FLAG_BYTES = 160 * 8 * 4    # the workspace's zero-at-rest flag block
 
 

@@ -126,8 +126,11 @@ def test_stream_k_forced_and_hybrid(fp8):
     a = with_ws(F, args(F, 256, 256, 1024, tile_cfg=1 | F.FP8_TILE_STREAMK), nbytes=0)
     a.workspace = None
     assert F._lib.fp8_mm_plan(ctypes.byref(a), None, 148, ctypes.byref(info)) == F.FP8_ERR_WORKSPACE
-    bad = args(F, 256, 256, 1024, tile_cfg=3 | F.FP8_TILE_STREAMK)      # pair tiles have no stream-K
+    bad = args(F, 256, 256, 1024, tile_cfg=4 | F.FP8_TILE_STREAMK)      # split-K has no stream-K
     assert F._lib.fp8_mm_plan(ctypes.byref(bad), None, 148, ctypes.byref(info)) == F.FP8_ERR_INVALID_ARG
+    pair = F.fp8_mm_plan(with_ws(F, args(F, 4096, 11008, 4096, tile_cfg=3 | F.FP8_TILE_STREAMK)))
+    # 688 pair tiles on 74 pairs: eight whole waves, the rest stream-K over the 74 pairs
+    assert pair.dp_tiles == 8 * 74 and pair.stream_k_ctas == 74 and pair.units == 74
     mis = with_ws(F, args(F, 256, 256, 1024))
     mis.workspace = WS + 8                                              # not 16-byte aligned
     assert F._lib.fp8_mm_plan(ctypes.byref(mis), None, 148, ctypes.byref(info)) == F.FP8_ERR_WORKSPACE

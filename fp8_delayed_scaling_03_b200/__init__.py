@@ -80,8 +80,7 @@ class LinearFwdArgs(ctypes.Structure):
                 ("x8", _P), ("ldx8", _I64),
                 ("w8", _P), ("ldw8", _I64),
                 ("sx_out", _P), ("sw_out", _P), ("amax_x_out", _P), ("amax_w_out", _P),
-                ("y", _P), ("ldy", _I64),
-                ("workspace", _P), ("workspace_bytes", _SZ)]
+                ("y", _P), ("ldy", _I64)]
 
 
 class LinearBwdArgs(ctypes.Structure):
@@ -385,12 +384,11 @@ class ForwardResult:
 
 def linear_forward(x, w, ring_x: ScaleRing | None, ring_w: ScaleRing | None, bias=None, bias_scale=None,
                    fmt_x=FP8_E4M3, fmt_w=FP8_E4M3, x_scale_in=None, w_scale_in=None, hist_len=16,
-                   y=None, x8=None, w8=None, scales=None, workspace=None) -> ForwardResult:
+                   y=None, x8=None, w8=None, scales=None) -> ForwardResult:
     """y = x w^T + bias through fp8_linear_forward.  x/w may be bf16/fp16/fp32
     or fp8 codes (torch.float8_* or uint8 with their fmt, plus *_scale_in).
     scales: optional 4-element fp32 device buffer receiving sx, sw, amax_x,
-    amax_w (allocated here when None).  workspace: optional zero-filled
-    stream-K workspace of the GEMM (mm_workspace(M, N, K))."""
+    amax_w (allocated here when None)."""
     M, K = x.shape
     N = w.shape[0]
     dev = x.device
@@ -415,7 +413,7 @@ def linear_forward(x, w, ring_x: ScaleRing | None, ring_w: ScaleRing | None, bia
         _ptr(ring_x.buf) if ring_x is not None else None, _ptr(ring_w.buf) if ring_w is not None else None,
         _ptr(x8), _ld(x8), _ptr(w8), _ld(w8),
         _ptr(sc[0:1]), _ptr(sc[1:2]), _ptr(sc[2:3]), _ptr(sc[3:4]),
-        _ptr(y), _ld(y), _ptr(workspace), _nbytes(workspace))
+        _ptr(y), _ld(y))
     fp8_linear_forward(args, dev)
     return ForwardResult(y, x8, w8, sc[0:1], sc[1:2], sc[2:3], sc[3:4])
 
@@ -445,7 +443,6 @@ def linear_backward(g, fwd: ForwardResult, ring_g: ScaleRing | None, fmt_g=FP8_E
     dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if (need_dw and dw is None) else dw
     dbias = torch.empty(N, dtype=torch.bfloat16, device=dev) if (need_dbias and dbias is None) else dbias
     if need_dbias and workspace is None:
-        # the bias-gradient scratch and the dX + dW launch's stream-K scratch
         workspace = torch.zeros(max(16, fp8_linear_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
     sc = torch.empty(2, dtype=torch.float32, device=dev)
     H = ring_g.H if ring_g is not None else 16

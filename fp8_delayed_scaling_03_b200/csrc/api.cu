@@ -404,6 +404,7 @@ int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) 
   pr->scale_b = c.scale_b;
   pr->bias = c.bias;
   pr->bias_kind = !c.bias ? 0 : (c.bias_dtype == FP8_DT_BF16 ? 1 : (c.bias_dtype == FP8_DT_E4M3 ? 2 : 3));
+  pr->bias_vec = c.bias && aligned(c.bias, 16) ? 1 : 0;
   pr->bias_scale = c.bias_scale;
   pr->d = c.d;
   pr->ldd = c.ldd;
@@ -411,9 +412,6 @@ int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) 
   return FP8_OK;
 }
 
-// Enqueue one launch running n (1 or 2) validated GEMMs over one persistent
-// tile schedule.  side: writes folded into the launch; fin: rings whose
-// quantize deferred its finalize to this launch.
 // Stream-K slots the calls' workspace holds (0: no usable workspace).  A
 // two-GEMM launch shares calls[0]'s workspace.
 int64_t sk_slots_available(const MmCall* calls, int n) {
@@ -452,8 +450,10 @@ int plan_launch(const MmCall* calls, int n, int sms, TilePlan* plan, int* split)
     *plan = TilePlan{};
     plan->cfg = req_cfg;
   } else {
-    *plan = pick_tile(calls, n, sms, slots);
-    if (!pairs_resident(*plan)) *plan = pick_tile(calls, n, sms, 0);
+    // AUTO stays data-parallel: measured on a B200, the stream-K plans the
+    // cost model chose were slower inside the benchmark steps (the fixup's
+    // flag and copy latency is serialized at the end of the launch)
+    *plan = pick_tile(calls, n, sms, 0);
   }
   int& cfg = plan->cfg;
   // Split-K (single-problem launches): few 128 x 128 tiles and a long K leave
@@ -479,27 +479,6 @@ int plan_launch(const MmCall* calls, int n, int sms, TilePlan* plan, int* split)
     }
   }
   return FP8_OK;
-}
-
-// Two GEMMs (the backward's dX and dW) in one launch save a launch's fixed
-// cost (a few us), which matters for short launches; long ones run as two
-// launches, each with its own tile choice and an operand set that stays in L2
-// (measured on a B200 at M = 4096 with a 4096 x 11008 weight: one launch
-// 283 us, two 255 us).
-constexpr double kFuseMaxUs = 50.0;
-
-bool fuse_pair(const MmCall& dx, const MmCall& dw) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return true;
-  const int sms = num_sms(dev);
-  if (sms <= 0) return true;
-  const MmCall both[2] = {dx, dw};
-  TilePlan pb, px, pw;
-  int split = 1;
-  if (plan_launch(both, 2, sms, &pb, &split) || plan_launch(&dx, 1, sms, &px, &split) ||
-      plan_launch(&dw, 1, sms, &pw, &split))
-    return true;
-  return pb.est_us < kFuseMaxUs && pb.est_us <= px.est_us + pw.est_us;
 }
 
 // Enqueue one launch running n (1 or 2) validated GEMMs over one persistent
@@ -714,9 +693,6 @@ size_t linear_dbias_bytes(int64_t M, int64_t N) {
   return dbias_counter_bytes(N) + dbias_partial_bytes(std::max(Rd, Rc), N);
 }
 
-// Offset of the stream-K part in the backward workspace.
-size_t linear_sk_offset(int64_t M, int64_t N) { return (linear_dbias_bytes(M, N) + 255) & ~size_t(255); }
-
 // ring NULL selects current scaling, which reduces the amax into *amax_out
 // (required then).
 int validate_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld_in, int fmt,
@@ -854,9 +830,7 @@ int fp8_mm_pair(const fp8_mm_args* a, const fp8_mm_args* b, fp8_stream_t stream)
   if ((s = validate_mm(c[1]))) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool ga = c[0].m > 0 && c[0].n > 0 && c[0].k > 0, gb = c[1].m > 0 && c[1].n > 0 && c[1].k > 0;
-  // one launch, unless both are long enough that two launches run faster
-  // (forced tile configurations always share one launch)
-  if (ga && gb && (c[0].tile_cfg != FP8_TILE_AUTO || fuse_pair(c[0], c[1]))) return run_mm_group(c, 2, nullptr, st);
+  if (ga && gb) return run_mm_group(c, 2, nullptr, st);
   if ((s = run_mm_any(c[0], st))) return s;
   return run_mm_any(c[1], st);
 }
@@ -915,7 +889,7 @@ int fp8_mm_plan(const fp8_mm_args* a, const fp8_mm_args* b, int num_sms, fp8_mm_
   } else if (req_cfg != FP8_TILE_AUTO) {
     plan.cfg = req_cfg;
   } else {
-    plan = pick_tile(c, n, num_sms, slots);
+    plan = pick_tile(c, n, num_sms, 0);
   }
   const int cfg = plan.cfg;
   const int64_t tm = cfg == kGemmPair256 ? 256 : 128;
@@ -973,9 +947,8 @@ int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg, con
 }
 
 size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  if (M <= 0 || N <= 0) return 0;
-  // the bias-gradient part, then the stream-K part of the dX + dW launch
-  return linear_sk_offset(M, N) + std::max(sk_bytes_for(M, K, N), sk_bytes_for(N, K, M));
+  (void)K;
+  return linear_dbias_bytes(M, N);
 }
 
 int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
@@ -1011,8 +984,6 @@ int fp8_linear_forward(const fp8_linear_fwd_args* a, fp8_stream_t stream) {
   MmCall c{M, N, K, x8, a->fmt_x, FP8_K_MAJOR, xq ? a->ldx : a->ldx8, w8, a->fmt_w, FP8_K_MAJOR,
            wq ? a->ldw : a->ldw8, xq ? a->x_scale_in : a->sx_out, wq ? a->w_scale_in : a->sw_out,
            a->bias, a->bias_dtype, a->bias_scale, a->y, a->ldy, FP8_TILE_AUTO};
-  c.ws = a->workspace;
-  c.ws_bytes = a->workspace_bytes;
   if ((s = validate_mm(c))) return s;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1093,12 +1064,6 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   // dW[N,K] = G8^T . X8: A(i=n, m) = G8[m, n] MN-major, B(j=k, m) = X8[m, k] MN-major.
   MmCall cdw{N, K, M, g8, a->fmt_g, FP8_MN_MAJOR, ldg8, a->x8, a->fmt_x, FP8_MN_MAJOR, a->ldx8,
              sg, a->sx, nullptr, 0, nullptr, a->dw, a->lddw, FP8_TILE_AUTO};
-  // the stream-K part of the workspace, when the caller gave the whole size
-  const size_t sk_off = linear_sk_offset(M, N);
-  if (a->workspace && aligned(a->workspace, 16) && a->workspace_bytes > sk_off) {
-    cdx.ws = cdw.ws = static_cast<uint8_t*>(a->workspace) + sk_off;
-    cdx.ws_bytes = cdw.ws_bytes = a->workspace_bytes - sk_off;
-  }
   if (a->need_dx && (s = validate_mm(cdx))) return s;
   if (a->need_dw && (s = validate_mm(cdw))) return s;
   const size_t ws_need = a->need_dbias ? linear_dbias_bytes(M, N) : 0;
@@ -1140,14 +1105,10 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
       return s;
     }
   }
-  if (dx_gemm && dw_gemm && fuse_pair(cdx, cdw)) {  // one launch for both (they share the G8 operand)
+  if (dx_gemm && dw_gemm) {  // one launch for both (they share the G8 operand)
     const MmCall both[2] = {cdx, cdw};
     if ((s = run_mm_group(both, 2, side_pending ? &side : nullptr, st, fin, nfin, dbf.partial ? &dbf : nullptr)))
       return s;
-    side_pending = false;
-  } else if (dx_gemm && dw_gemm) {  // two launches; the first completes the deferred steps
-    if ((s = run_mm(cdx, side_pending ? &side : nullptr, st, fin, nfin, dbf.partial ? &dbf : nullptr))) return s;
-    if ((s = run_mm(cdw, nullptr, st))) return s;
     side_pending = false;
   } else if (dx_gemm || dw_gemm) {
     if ((s = run_mm(dx_gemm ? cdx : cdw, side_pending ? &side : nullptr, st, fin, nfin,

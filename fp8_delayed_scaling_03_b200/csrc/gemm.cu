@@ -155,15 +155,17 @@ __device__ __forceinline__ int sk_cta_of(const GemmParams& p, int64_t u) {
   return static_cast<int>(((u + 1) * p.sk_ctas + p.sk_total - 1) / p.sk_total) - 1;
 }
 
+template <bool kSk>
 __device__ __forceinline__ void sched_init(const GemmParams& p, int unit, Sched& s) {
   s.slot = unit;
   s.u = s.ue = 0;
-  if (unit < p.sk_ctas) {
+  if (kSk && unit < p.sk_ctas) {
     s.u = sk_begin(p, unit);
     s.ue = sk_begin(p, unit + 1);
   }
 }
 
+template <bool kSk>
 __device__ __forceinline__ bool sched_next(const GemmParams& p, int unit, int units, Sched& s, Work& w) {
   while (s.slot < p.nslots) {
     const int t = slot_tile(p, s.slot);
@@ -177,7 +179,7 @@ __device__ __forceinline__ bool sched_next(const GemmParams& p, int unit, int un
     w.nparts = 0;
     return true;
   }
-  if (s.u >= s.ue) return false;
+  if (!kSk || s.u >= s.ue) return false;
   // stream-K unit -> (tile, k-block); problem 0's stream-K tiles come first
   int t, kbt;
   int64_t ut;  // the tile's first unit
@@ -233,6 +235,47 @@ __device__ __forceinline__ float bias_value(const void* bias, int bias_kind, int
   return f.x * binv;
 }
 
+// The bias of the 32 columns [col0, col0 + 32) of an epilogue step, the same
+// for every lane: 16-byte loads of one address per warp (one L1 transaction,
+// broadcast), issued before the step's accumulator read so that their latency
+// hides behind it -- a per-lane value broadcast by 32 shuffles cost ~0.3 us
+// per step on a B200.  Needs a 16-byte aligned bias and col0 + 32 <= n.
+__device__ __forceinline__ void bias32_load(const void* bias, int kind, int col0, uint4 (&q)[4]) {
+  if (kind == 1) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(bias) + col0);
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = __ldg(src + i);
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(bias) + col0);
+    q[0] = __ldg(src);
+    q[1] = __ldg(src + 1);
+    q[2] = q[3] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+// The 32 values bias32_load fetched, as bias_value computes each one.
+__device__ __forceinline__ void bias32_values(const uint4 (&q)[4], int kind, float binv, float (&b)[32]) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(q);
+  if (kind == 1) {
+    #pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      b[2 * i] = __uint_as_float(w[i] << 16);
+      b[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 lo = kind == 2 ? dec_e4m3x2(static_cast<uint16_t>(w[i] & 0xFFFFu))
+                                  : dec_e5m2x2(static_cast<uint16_t>(w[i] & 0xFFFFu));
+      const float2 hi = kind == 2 ? dec_e4m3x2(static_cast<uint16_t>(w[i] >> 16))
+                                  : dec_e5m2x2(static_cast<uint16_t>(w[i] >> 16));
+      b[4 * i] = lo.x * binv;
+      b[4 * i + 1] = lo.y * binv;
+      b[4 * i + 2] = hi.x * binv;
+      b[4 * i + 3] = hi.y * binv;
+    }
+  }
+}
+
 // dbias[c] = bf16(fixed-order sum of the R partials of column c) for the
 // columns c = 32 * (blockIdx.x + k * gridDim.x) + lane: one warp per CTA,
 // 32 consecutive columns (coalesced rows of partials) at a time.
@@ -242,7 +285,9 @@ __device__ __forceinline__ void dbias_finish_warp(const DbiasFinish& f, int lane
     static_cast<__nv_bfloat16*>(f.dbias)[c] = __float2bfloat16_rn(sum_partials(f.partial + c, f.cols, f.R));
 }
 
-template <int BN, bool kPair, bool kSplit>
+// kSk: the stream-K build (its work items, partial slots and fixup); the
+// data-parallel build carries none of that code.
+template <int BN, bool kPair, bool kSplit, bool kSk>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
                     const __grid_constant__ CUtensorMap td0, const __grid_constant__ CUtensorMap ta1,
@@ -348,9 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool dep_done = false;
       int issued = 0;  // k-blocks loaded so far; the first kStages find their stage free
       Sched sc;
-      sched_init(p, unit, sc);
+      sched_init<kSk>(p, unit, sc);
       Work w;
-      while (!*abort_flag && sched_next(p, unit, units, sc, w)) {
+      while (!*abort_flag && sched_next<kSk>(p, unit, units, sc, w)) {
         const int t = w.t;
         int tb = first_tb, tm = first_tm, tn = first_tn;
         const int pi = t == first_t ? first_pi : tile_coords(p, t, tb, tm, tn);
@@ -403,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       Sched sc;
-      sched_init(p, unit, sc);
+      sched_init<kSk>(p, unit, sc);
       Work w;
-      while (!*abort_flag && sched_next(p, unit, units, sc, w)) {
+      while (!*abort_flag && sched_next<kSk>(p, unit, units, sc, w)) {
         const int t = w.t;
         const int pi = t >= p.tiles0 ? 1 : 0;
         const int k_blocks = FP8_PR(k_blocks);
@@ -505,9 +550,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       return sk_part + ((static_cast<int64_t>(slot) * kEpiWarps + ew) * kSteps + st) * (kSkBlock / 16);
     };
     Sched sc;
-    sched_init(p, unit, sc);
+    sched_init<kSk>(p, unit, sc);
     Work w;
-    while (!*abort_flag && sched_next(p, unit, units, sc, w)) {
+    while (!*abort_flag && sched_next<kSk>(p, unit, units, sc, w)) {
       const int t = w.t;
       int tb, tm, tn;
       const int pi = tile_coords(p, t, tb, tm, tn);
@@ -515,6 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // BEFORE the wait for the accumulator, so that no parameter read and no
       // global-memory latency sits between the TMEM read and the store.
       const int qm = FP8_PR(m), qn = FP8_PR(n), bias_kind = FP8_PR(bias_kind);
+      const bool bias_vec = bias_kind && FP8_PR(bias_vec);
       const bool tma_store = FP8_PR(tma_store) != 0;
       const bool have_k = kSplit ? (static_cast<int>(rank) + 1) * FP8_PR(k_blocks) / nsplit >
                                        static_cast<int>(rank) * FP8_PR(k_blocks) / nsplit
@@ -542,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // owner: the later parts' partials are in their slots; they are staged
       // `spr` steps at a time in this warp's share of the (now idle) operand ring
       int spr = kSteps;
-      if (w.kind == kOwner) {
+      if (kSk && w.kind == kOwner) {
         bool ok = w.nparts >= 1 && w.nparts <= kSkMaxParts;
         if (!ok && lane == 0 && p.status) atomicExch(p.status, kDevTimeout);  // outside the planner's bound: give up
         for (int q = 0; q < w.nparts && ok; ++q)
@@ -559,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       #pragma unroll 1
       for (int st = 0; st < kSteps; ++st) {
         const int col0 = col_half + st * kEpiCols;
-        if (w.kind == kOwner && st % spr == 0) {  // stage the partials of steps [st, st + spr)
+        if (kSk && w.kind == kOwner && st % spr == 0) {  // stage the partials of steps [st, st + spr)
           const int nst = min(spr, kSteps - st);
           fence_proxy_async_smem();  // this warp's reads of the previous round come first
           __syncwarp();
@@ -573,6 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           sk_phase ^= 1u;
         }
         uint32_t r[32];
+        // whole 32-column step with an aligned bias: its 32 values by broadcast loads
+        const bool step_bias_vec = bias_vec && col0 + kEpiCols <= qn;
+        uint4 bq[4];
+        if (step_bias_vec && st < live_steps) bias32_load(bias, bias_kind, col0, bq);
         if (st < live_steps) {
           if (have_k) {
             __syncwarp();  // tcgen05.ld is .sync.aligned
@@ -614,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (w.kind != kFull) {
+        if (kSk && w.kind != kFull) {
           if (w.kind == kPartial) {  // this part's accumulator goes to the CTA's slot
             float4* dst = sk_block(sk_slot(unit), st) + lane;
             #pragma unroll
@@ -641,7 +691,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // One uniform branch per step, none per element: a shuffle under a
         // per-element condition costs a reconvergence point each.
         float v[32];
-        if (bias_kind) {
+        if (step_bias_vec) {
+          float b[32];
+          bias32_values(bq, bias_kind, pi ? binv1 : binv0, b);
+          #pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * tinv + b[j];
+        } else if (bias_kind) {
           const float bst = pick(bl, st);
           #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * tinv + __shfl_sync(0xFFFFFFFFu, bst, j);
@@ -675,9 +730,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (col0 + j < qn) drow[col0 + j] = __float2bfloat16_rn(v[j]);
         }
       }
-      if (w.kind == kPartial) {  // this warp's share of the partial is written: raise its flag
+      if (kSk && w.kind == kPartial) {  // this warp's share of the partial is written: raise its flag
         warp_release_flag(p.sk_flag + static_cast<int64_t>(sk_slot(unit)) * kEpiWarps + ew, 1u);
-      } else if (w.kind == kOwner) {  // every lane has read the partials: clear their flags
+      } else if (kSk && w.kind == kOwner) {  // every lane has read the partials: clear their flags
         __syncwarp();
         if (lane == 0)
           for (int q = 0; q < w.nparts; ++q) p.sk_flag[static_cast<int64_t>(sk_slot(w.part0 + q)) * kEpiWarps + ew] = 0u;
@@ -718,7 +773,7 @@ int pair_capacity_impl(int dev) {
   using C = Cfg<256, true>;
   static int cache[64] = {};
   if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
-  if (cudaFuncSetAttribute(fp8_gemm_kernel<256, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(fp8_gemm_kernel<256, true, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmem) != cudaSuccess)
     return 0;
   cudaLaunchConfig_t cfg = {};
@@ -733,7 +788,7 @@ int pair_capacity_impl(int dev) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<256, true, false>, &cfg) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<256, true, false, false>, &cfg) != cudaSuccess) return 0;
   if (dev >= 0 && dev < 64) cache[dev] = clusters;
   return clusters;
 }
@@ -745,11 +800,14 @@ cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t 
   using C = Cfg<BN, kPair>;
   int dev = 0;
   cudaGetDevice(&dev);
+  // the stream-K build for launches with stream-K ranges, else the plain one
+  auto kernel = p.sk_ctas > 0 ? fp8_gemm_kernel<BN, kPair, false, true> : fp8_gemm_kernel<BN, kPair, false, false>;
   static bool configured[64] = {};
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
+    for (auto k : {fp8_gemm_kernel<BN, kPair, false, false>, fp8_gemm_kernel<BN, kPair, false, true>}) {
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+      if (e != cudaSuccess) return e;
+    }
     configured[dev] = true;
   }
   const int sms = num_sms(dev);
@@ -758,7 +816,7 @@ cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t 
     // planner's CTA count), the k-block ranges the first sk_ctas of them
     int grid = p.total_tiles < sms ? p.total_tiles : sms;
     if (p.sk_ctas > 0) grid = p.dp_tiles > 0 ? (sms < 160 ? sms : 160) : p.sk_ctas;
-    return launch_pdl(fp8_gemm_kernel<BN, kPair, false>, dim3(grid), dim3(kThreads), C::kSmem, s, mp[0], mp[1], mp[2], mp[3],
+    return launch_pdl(kernel, dim3(grid), dim3(kThreads), C::kSmem, s, mp[0], mp[1], mp[2], mp[3],
                       mp[4], mp[5], p);
   }
   cudaLaunchConfig_t cfg = {};
@@ -786,7 +844,7 @@ cudaError_t launch_cfg(const CUtensorMap* mp, const GemmParams& p, cudaStream_t 
     if (pairs > cap) return cudaErrorInvalidConfiguration;
   }
   cfg.gridDim = dim3(2 * pairs);
-  return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BN, kPair, false>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
+  return cudaLaunchKernelEx(&cfg, kernel, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
 }
 
 // Largest number of clusters of `split` CTAs of the split-K kernel that can be
@@ -796,7 +854,7 @@ int split_clusters(int dev, int split) {
   if (split < 2 || split > kMaxSplit) return 0;
   if (dev < 64 && cache[dev][split]) return cache[dev][split];
   using C = Cfg<128, false>;
-  cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<128, false, true>,
+  cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<128, false, true, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
@@ -811,7 +869,7 @@ int split_clusters(int dev, int split) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<128, false, true>, &cfg) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, fp8_gemm_kernel<128, false, true, false>, &cfg) != cudaSuccess) return 0;
   if (dev < 64) cache[dev][split] = clusters;
   return clusters;
 }
@@ -836,7 +894,7 @@ cudaError_t launch_split(const CUtensorMap* mp, const GemmParams& p, cudaStream_
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<128, false, true>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
+  return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<128, false, true, false>, mp[0], mp[1], mp[2], mp[3], mp[4], mp[5], p);
 }
 
 // The output of an empty contraction: every accumulator is zero, so each

@@ -80,9 +80,11 @@ typedef enum { FP8_K_MAJOR = 0, FP8_MN_MAJOR = 1 } fp8_major;
  * which adds the others' fp32 partial accumulators (stored in the workspace)
  * in CTA order: the result is deterministic for a given GPU.
  * FP8_TILE_AUTO chooses per shape with a cost model fitted to B200 timings --
- * split-K when the output has few tiles and K is long, stream-K when a
- * workspace is given and it pays.  Results do not depend on the choice beyond
- * the fp32 summation order. */
+ * split-K when the output has few tiles and K is long; never stream-K, whose
+ * fixup latency (flags, then the partials' copies, serialized at the end of
+ * the launch) made every stream-K choice of the model slower inside the
+ * benchmark steps on a B200.  Results do not depend on the choice beyond the
+ * fp32 summation order. */
 typedef enum {
   FP8_TILE_AUTO = 0, FP8_TILE_128x128 = 1, FP8_TILE_128x256 = 2, FP8_TILE_PAIR_256x256 = 3,
   FP8_TILE_SPLITK_128x128 = 4, FP8_TILE_STREAMK = 8
@@ -221,12 +223,12 @@ typedef struct fp8_mm_args {
   const void* bias; int bias_dtype; const float* bias_scale;
   void* d; int64_t ldd;
   int tile_cfg;   /* FP8_TILE_AUTO (0, chosen per shape) or one of fp8_tile_cfg */
-  /* Optional stream-K workspace (NULL / 0: none; results are the same, only
-   * the schedule differs): >= fp8_mm_workspace_bytes(m, n, k) bytes, 256-byte
-   * aligned, ZERO-FILLED before its first use; every call leaves its flags at
-   * zero again, so it may be reused by later calls of the same sizes that are
-   * ordered after this one (same stream).  A forced FP8_TILE_STREAMK without
-   * it returns FP8_ERR_WORKSPACE. */
+  /* Stream-K workspace, used only with FP8_TILE_STREAMK (NULL / 0 otherwise):
+   * >= fp8_mm_workspace_bytes(m, n, k) bytes, 16-byte aligned, ZERO-FILLED
+   * before its first use; every call leaves its flags at zero again, so it
+   * may be reused by later calls of the same sizes that are ordered after
+   * this one (same stream).  FP8_TILE_STREAMK without it returns
+   * FP8_ERR_WORKSPACE. */
   void* workspace; size_t workspace_bytes;
 } fp8_mm_args;
 FP8LIN_API int fp8_mm(const fp8_mm_args* args, fp8_stream_t stream);
@@ -255,13 +257,9 @@ FP8LIN_API int fp8_mm_batched(const fp8_mm_args* args, int64_t batch, int64_t st
 
 /* Two independent GEMMs (the backward's dX and dW) in ONE launch over one
  * persistent tile schedule.  Same results as two fp8_mm calls; the tile
- * configuration (a->tile_cfg, or chosen for the pair when AUTO) and the
- * stream-K workspace (a->workspace, >= fp8_mm_workspace_bytes of either
- * problem) are shared.  With FP8_TILE_AUTO, two GEMMs long enough that the
- * launch's fixed cost no longer matters (the cost model's estimate of the
- * shared launch is 50 us or more, or above the two separate launches) run
- * as two launches instead: each gets its own tile choice and operand set in
- * L2 (at M = 4096 with a 4096 x 11008 weight on a B200: 255 us vs 283 us). */
+ * configuration (a->tile_cfg, or chosen for the pair when AUTO) and, for
+ * FP8_TILE_STREAMK, the workspace (a->workspace, >= fp8_mm_workspace_bytes of
+ * either problem) are shared. */
 FP8LIN_API int fp8_mm_pair(const fp8_mm_args* a, const fp8_mm_args* b, fp8_stream_t stream);
 
 /* The tile configuration fp8_mm (b == NULL) or fp8_mm_pair (b != NULL) would
@@ -354,8 +352,6 @@ typedef struct fp8_linear_fwd_args {
   uint8_t* w8; int64_t ldw8;
   float* sx_out; float* sw_out; float* amax_x_out; float* amax_w_out;
   void* y; int64_t ldy;
-  void* workspace; size_t workspace_bytes;   /* optional stream-K workspace of the GEMM, as
-                                                fp8_mm_args (size fp8_mm_workspace_bytes(M, N, K)) */
 } fp8_linear_fwd_args;
 FP8LIN_API int fp8_linear_forward(const fp8_linear_fwd_args* args, fp8_stream_t stream);
 
@@ -369,12 +365,8 @@ FP8LIN_API int fp8_linear_forward(const fp8_linear_fwd_args* args, fp8_stream_t 
  *                                           only when the bias needs a grad)
  * sx, sw, x8, w8 are the FORWARD's snapshots and quantized operands: the
  * backward reuses the forward's scales.  Outputs are bf16 whatever the input
- * dtypes.  dX and dW share one launch as fp8_mm_pair decides with
- * FP8_TILE_AUTO.  workspace: fp8_linear_workspace_bytes(M, N, K) bytes, zero-filled
- * before first use, reusable by later calls of the same sizes on the same
- * stream: the bias-gradient scratch (as fp8_dbias; required when need_dbias,
- * which needs at least that part), then the stream-K scratch of the dX + dW
- * launch (used only when the whole size is given).  Up to 4 launches. */
+ * dtypes.  workspace: as fp8_dbias, needed only when need_dbias (size from
+ * fp8_linear_workspace_bytes).  Up to 4 launches. */
 typedef struct fp8_linear_bwd_args {
   int64_t M, N, K;
   const void* g; int g_dtype; int64_t ldg; const float* g_scale_in;
@@ -391,12 +383,11 @@ typedef struct fp8_linear_bwd_args {
 } fp8_linear_bwd_args;
 FP8LIN_API int fp8_linear_backward(const fp8_linear_bwd_args* args, fp8_stream_t stream);
 
-/* Workspace bytes of fp8_linear_backward (0 when M or N is 0): the bias
- * gradient's part -- at least fp8_dbias_workspace_bytes(M, N), since the
- * column-sum quantize of the backward may split g's rows more finely than
- * fp8_dbias does -- followed by the stream-K part of the dX + dW launch.
- * Zero-fill it once before first use; every call leaves it ready for the next
- * call of the same sizes. */
+/* Workspace bytes fp8_linear_backward needs for need_dbias (0 when M or N is
+ * 0).  At least fp8_dbias_workspace_bytes(M, N): the column-sum quantize of
+ * the backward may split g's rows more finely than fp8_dbias does.  Zero-fill
+ * it once before first use, like fp8_dbias's workspace; every call leaves it
+ * ready for the next call of the same sizes.  K does not enter. */
 FP8LIN_API size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------ status

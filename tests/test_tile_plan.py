@@ -88,32 +88,27 @@ def test_workspace_bytes(fp8):
     assert F.fp8_mm_workspace_bytes(0, 10, 10) == 0 and F.fp8_mm_workspace_bytes(10, 10, 0) == 0
     assert F.fp8_mm_workspace_bytes(64, 192, 128) == flags + 2 * slot     # two 128 x 128 x 128 blocks
     assert F.fp8_mm_workspace_bytes(2048, 1536, 6912) == flags + 160 * slot
-    lin = F.fp8_linear_workspace_bytes(2048, 1536, 6912)
-    assert lin >= F.fp8_dbias_workspace_bytes(2048, 1536) + flags + 160 * slot
+    # the linear backward's workspace is its bias-gradient scratch only
+    assert F.fp8_linear_workspace_bytes(2048, 1536, 6912) >= F.fp8_dbias_workspace_bytes(2048, 1536)
 
 
 @pytest.mark.parametrize("m,n,k,a_major,b_major", [
     (2048, 1536, 6912, 0, 1),     # dX with contraction 6912: 96 tiles of 128x256 on 148 SMs
     (2048, 1536, 6912, 0, 0),     # forward with K = 6912
     (512, 1536, 6912, 0, 1),
-    (2048, 6912, 1536, 0, 0),     # 432 tiles = 2.92 waves: already balanced
+    (4096, 11008, 4096, 0, 0),
 ])
-def test_stream_k_costed(fp8, m, n, k, a_major, b_major):
-    """With a workspace the planner also costs stream-K; AUTO takes it only
-    for a clear gain over every data-parallel plan, and never where the
-    data-parallel waves are already even (2048 x 6912 x 1536)."""
+def test_auto_never_stream_k(fp8, m, n, k, a_major, b_major):
+    """AUTO stays data-parallel even with a workspace (measured on a B200: the
+    stream-K plans the cost model picked were slower inside the benchmark
+    steps); forced stream-K still plans its ranges."""
     F = fp8
     plain = F.fp8_mm_plan(args(F, m, n, k, a_major, b_major))
-    sk = F.fp8_mm_plan(with_ws(F, args(F, m, n, k, a_major, b_major)))
-    assert plain.stream_k_ctas == 0
-    if sk.stream_k_ctas:
-        assert sk.est_us < 0.95 * plain.est_us and sk.tile_cfg & F.FP8_TILE_STREAMK
-    else:
-        assert (sk.tile_cfg, sk.tiles, sk.units) == (plain.tile_cfg, plain.tiles, plain.units)
-    if (m, n, k) == (2048, 6912, 1536):
-        assert sk.stream_k_ctas == 0
+    ws = F.fp8_mm_plan(with_ws(F, args(F, m, n, k, a_major, b_major)))
+    assert plain.stream_k_ctas == 0 and ws.stream_k_ctas == 0
+    assert (ws.tile_cfg, ws.tiles, ws.units, ws.est_us) == (plain.tile_cfg, plain.tiles, plain.units, plain.est_us)
     forced = F.fp8_mm_plan(with_ws(F, args(F, m, n, k, a_major, b_major, tile_cfg=2 | F.FP8_TILE_STREAMK)))
-    assert forced.stream_k_ctas > 0
+    assert forced.stream_k_ctas > 0 and forced.tile_cfg == 2 | F.FP8_TILE_STREAMK
 
 
 def test_stream_k_forced_and_hybrid(fp8):

@@ -404,7 +404,6 @@ int build_problem(const MmCall& c, int cfg, GemmProblem* pr, CUtensorMap* maps) 
   pr->scale_b = c.scale_b;
   pr->bias = c.bias;
   pr->bias_kind = !c.bias ? 0 : (c.bias_dtype == FP8_DT_BF16 ? 1 : (c.bias_dtype == FP8_DT_E4M3 ? 2 : 3));
-  pr->bias_vec = c.bias && aligned(c.bias, 16) ? 1 : 0;
   pr->bias_scale = c.bias_scale;
   pr->d = c.d;
   pr->ldd = c.ldd;

@@ -235,47 +235,6 @@ __device__ __forceinline__ float bias_value(const void* bias, int bias_kind, int
   return f.x * binv;
 }
 
-// The bias of the 32 columns [col0, col0 + 32) of an epilogue step, the same
-// for every lane: 16-byte loads of one address per warp (one L1 transaction,
-// broadcast), issued before the step's accumulator read so that their latency
-// hides behind it -- a per-lane value broadcast by 32 shuffles cost ~0.3 us
-// per step on a B200.  Needs a 16-byte aligned bias and col0 + 32 <= n.
-__device__ __forceinline__ void bias32_load(const void* bias, int kind, int col0, uint4 (&q)[4]) {
-  if (kind == 1) {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(bias) + col0);
-    #pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = __ldg(src + i);
-  } else {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(bias) + col0);
-    q[0] = __ldg(src);
-    q[1] = __ldg(src + 1);
-    q[2] = q[3] = make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-// The 32 values bias32_load fetched, as bias_value computes each one.
-__device__ __forceinline__ void bias32_values(const uint4 (&q)[4], int kind, float binv, float (&b)[32]) {
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(q);
-  if (kind == 1) {
-    #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      b[2 * i] = __uint_as_float(w[i] << 16);
-      b[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  } else {
-    #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float2 lo = kind == 2 ? dec_e4m3x2(static_cast<uint16_t>(w[i] & 0xFFFFu))
-                                  : dec_e5m2x2(static_cast<uint16_t>(w[i] & 0xFFFFu));
-      const float2 hi = kind == 2 ? dec_e4m3x2(static_cast<uint16_t>(w[i] >> 16))
-                                  : dec_e5m2x2(static_cast<uint16_t>(w[i] >> 16));
-      b[4 * i] = lo.x * binv;
-      b[4 * i + 1] = lo.y * binv;
-      b[4 * i + 2] = hi.x * binv;
-      b[4 * i + 3] = hi.y * binv;
-    }
-  }
-}
-
 // dbias[c] = bf16(fixed-order sum of the R partials of column c) for the
 // columns c = 32 * (blockIdx.x + k * gridDim.x) + lane: one warp per CTA,
 // 32 consecutive columns (coalesced rows of partials) at a time.
@@ -560,7 +519,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // BEFORE the wait for the accumulator, so that no parameter read and no
       // global-memory latency sits between the TMEM read and the store.
       const int qm = FP8_PR(m), qn = FP8_PR(n), bias_kind = FP8_PR(bias_kind);
-      const bool bias_vec = bias_kind && FP8_PR(bias_vec);
       const bool tma_store = FP8_PR(tma_store) != 0;
       const bool have_k = kSplit ? (static_cast<int>(rank) + 1) * FP8_PR(k_blocks) / nsplit >
                                        static_cast<int>(rank) * FP8_PR(k_blocks) / nsplit
@@ -619,10 +577,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           sk_phase ^= 1u;
         }
         uint32_t r[32];
-        // whole 32-column step with an aligned bias: its 32 values by broadcast loads
-        const bool step_bias_vec = bias_vec && col0 + kEpiCols <= qn;
-        uint4 bq[4];
-        if (step_bias_vec && st < live_steps) bias32_load(bias, bias_kind, col0, bq);
         if (st < live_steps) {
           if (have_k) {
             __syncwarp();  // tcgen05.ld is .sync.aligned
@@ -691,12 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // One uniform branch per step, none per element: a shuffle under a
         // per-element condition costs a reconvergence point each.
         float v[32];
-        if (step_bias_vec) {
-          float b[32];
-          bias32_values(bq, bias_kind, pi ? binv1 : binv0, b);
-          #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * tinv + b[j];
-        } else if (bias_kind) {
+        if (bias_kind) {
           const float bst = pick(bl, st);
           #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * tinv + __shfl_sync(0xFFFFFFFFu, bst, j);

@@ -100,7 +100,6 @@ struct GemmProblem {
   const float* scale_b;
   const void* bias;
   int bias_kind;              // 0 none, 1 bf16, 2 e4m3, 3 e5m2
-  int bias_vec;               // bias base 16-byte aligned: 32 values per 16-byte loads
   const float* bias_scale;
   void* d;
   int64_t ldd;

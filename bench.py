@@ -340,13 +340,16 @@ def time_kernels(F, lins, stream, reps=5):
         g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(reps):
-                g.replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        res_ms[cls] = e0.elapsed_time(e1) / reps
+        runs = []
+        for _ in range(3):  # median of three timed runs of `reps` replays
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            runs.append(e0.elapsed_time(e1) / reps)
+        res_ms[cls] = statistics.median(runs)
         del g
     # per-shape GEMM times: one graph per distinct GEMM launch of the step, 12 launches each
     shapes = {}
@@ -493,6 +496,13 @@ def time_target_shapes(F, device, stream, fp8_peak, hbm_gbs):
                 gemm.append(rec)
             del sets
     quant = []
+    # this box's device-to-device copy rate (read + write bytes), for context:
+    # the fractions above and below use the measured peak of the pool
+    src = torch.ones(1 << 28, dtype=torch.float32, device=device)
+    dst = torch.empty_like(src)
+    copy_us = _graph_us(stream, [lambda: torch.mul(src, 1.0, out=dst)], reps=5)
+    box_copy_gbs = round(2 * 4 * src.numel() / copy_us / 1e3, 1)
+    del src, dst
     ring = torch.empty(F.fp8_ring_bytes(wl.HIST_LEN) // 4, dtype=torch.float32, device=device)
     F.fp8_ring_init(ring, wl.HIST_LEN)
     for rows, cols in ((4096, 4096), (4096, 11008), (2048, 6912)):
@@ -518,7 +528,7 @@ def time_target_shapes(F, device, stream, fp8_peak, hbm_gbs):
                       "ring_step_deferred": {"us": round(dus, 2), "gbs": round(dgbs, 1),
                                              "frac_hbm": round(dgbs / hbm_gbs, 3)}})
         del sets, qargs
-    return gemm, quant
+    return gemm, quant, box_copy_gbs
 
 
 # --------------------------------------------------------------------------- GEMM traffic (ncu summary)
@@ -893,14 +903,17 @@ def main(argv=None):
             raise F.Fp8Error(F.fp8_get_device_status(), "device status after the other workloads")
         line["steps_other_workloads"] = others
 
-        tg, tq = time_target_shapes(F, device, stream, fp8_peak, pk["hbm_gbs"])
+        tg, tq, box_copy = time_target_shapes(F, device, stream, fp8_peak, pk["hbm_gbs"])
         line["targets"] = {
             "gemm": tg, "quantize": tq, "fp8_peak_tflops": fp8_peak, "hbm_gbs": pk["hbm_gbs"],
+            "box_copy_gbs": box_copy,
             "note": "separate fp8_mm launches per operation (dX, dW in the fused backward's in-place "
                     "transposed layouts); warm = the same operands back to back, cold = operand sets cycled so "
                     "each pass streams more than L2; frac_roofline = achieved / min(peak, AI x HBM BW) cold, "
                     "achieved / peak warm; quantize standalone (in-kernel ring finalize) and with the ring step "
-                    "deferred to the following GEMM (as fp8_linear_forward/backward launch it), cold"}
+                    "deferred to the following GEMM (as fp8_linear_forward/backward launch it), cold; "
+                    "box_copy_gbs = this box's rate for an elementwise 1 GiB -> 1 GiB fp32 copy kernel (read + write bytes), context "
+                    "for the HBM fractions, which use the pool's measured peak"}
 
         # ---- end to end through the C ABI with host buffers
         host_in = [[t.cpu().pin_memory() for t in L.inputs()] for L in lins]

@@ -325,7 +325,7 @@ def fp8_version() -> str:
 
 class ScaleRing:
     """Delayed-scaling state of one tensor: a device buffer laid out as
-    [hist (H fp32) | scale | ticket | step | scratch]."""
+    [hist (H fp32) | scale | step | ticket | scratch]."""
 
     def __init__(self, hist_len: int = 16, device="cuda", seed_amax: float | None = None, fmt: int = FP8_E4M3,
                  buf: torch.Tensor | None = None):
@@ -352,7 +352,7 @@ class ScaleRing:
 
     @property
     def step(self):
-        return int(self.buf[self.H + 2 : self.H + 3].view(torch.int32).item())
+        return int(self.buf[self.H + 1 : self.H + 2].view(torch.int32).item())
 
     def words(self):
         return self.buf.view(torch.int32)

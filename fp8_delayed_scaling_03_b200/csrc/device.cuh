@@ -440,6 +440,12 @@ __device__ __forceinline__ float next_scale(float s, float m, float fp8_max) {
 __device__ __forceinline__ void red_max_u32(uint32_t* p, uint32_t v) {
   asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// 64-bit relaxed fetch-add at gpu scope.
+__device__ __forceinline__ uint64_t atom_add_relaxed_u64(void* p, uint64_t v) {
+  uint64_t old;
+  asm volatile("atom.relaxed.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
 // fetch-add with acquire-release semantics at gpu scope: everything this thread
 // did before is visible to whoever acquires a later value of the counter, and
 // everything released by earlier incrementers is visible to this thread.

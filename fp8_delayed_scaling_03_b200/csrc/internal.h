@@ -12,11 +12,14 @@ namespace fp8lin {
 enum : int { kE4M3 = 0, kE5M2 = 1 };
 enum : int { kBF16 = 0, kFP16 = 1, kFP32 = 2, kDtE4M3 = 3, kDtE5M2 = 4 };
 
-// Ring word offsets (in 32-bit words) for history length H.
-inline int ring_scale(int H) { return H; }
-inline int ring_ticket(int H) { return H + 1; }
-inline int ring_step(int H) { return H + 2; }
-inline int ring_scratch(int H) { return H + 3; }
+// Ring word offsets (in 32-bit words) for history length H:
+// [hist (H) | scale | step | ticket | scratch].  With H even (and the ring
+// 8-byte aligned) ticket and scratch form one aligned 8-byte word, which the
+// in-kernel finalize updates with one 64-bit atomic per block.
+__host__ __device__ constexpr int ring_scale(int H) { return H; }
+__host__ __device__ constexpr int ring_step(int H) { return H + 1; }
+__host__ __device__ constexpr int ring_ticket(int H) { return H + 2; }
+__host__ __device__ constexpr int ring_scratch(int H) { return H + 3; }
 
 struct QuantizeParams {
   const void* in;
@@ -25,7 +28,7 @@ struct QuantizeParams {
   int64_t ld_out;
   int64_t chunks_per_row;     // ceil(cols / 16)
   int64_t total_chunks;
-  float* ring;                // [hist | scale | ticket | step | scratch]
+  float* ring;                // [hist | scale | step | ticket | scratch]
   int H;
   float fp8_max;
   float* amax_out;

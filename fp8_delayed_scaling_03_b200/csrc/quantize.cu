@@ -13,19 +13,21 @@
 //      cvt.rn.satfinite.{e4m3,e5m2}x2, storing 16 fp8 codes per 16-byte store;
 //   3. warp max (redux.sync) -> block max -> one relaxed red.max on the ring's
 //      scratch word (non-negative floats order like their bit patterns);
-//   4. an acquire-release fetch-add on the ring's ticket: the block that draws
-//      the tensor's last ticket sees every block's max, folds the launch's
-//      amax into hist[step % H], reduces the window, and publishes
-//      fp8_max / max as the next scale (kept when the max is 0 or inf or the
-//      quotient overflows), then rezeroes ticket and scratch.  History and
-//      step are prefetched into shared memory at kernel start, so this tail is
-//      two dependent global round trips.
+//   4. a fetch-add on the ring's ticket: the block that draws the tensor's
+//      last ticket sees every block's max, folds the launch's amax into
+//      hist[step % H], reduces the window, and publishes fp8_max / max as the
+//      next scale (kept when the max is 0 or inf or the quotient overflows),
+//      then rezeroes ticket and scratch.  When ticket and scratch share an
+//      aligned 8-byte word (even H), the ticket is one relaxed 64-bit add whose
+//      return value already carries the max: one round trip, no fence.
+//      Otherwise an acquire-release add, then an exchange of the scratch word.
+//      History and step are prefetched into shared memory at kernel start.
 //   4'. with defer_finalize (the fused linear entry points, where a GEMM that
 //      reads the output always follows) step 4 is skipped: each block's max
 //      goes to the scratch word and the GEMM -- which starts reading only after
 //      this grid has completed -- does the finalize in one warp while its
-//      mainloop runs.  That takes the release fence, the ticket round trip and
-//      the last block's round trips (about 1.5 us) off every quantize launch.
+//      mainloop runs.  That takes the ticket round trip and the last block's
+//      ring update off every quantize launch.
 // The column-sum variant (quantize of g with the bias gradient) walks 2-D
 // tiles of 256 columns instead, so each thread also accumulates the column
 // sums of its 16 columns; per-tile partials meet in a workspace and the last
@@ -159,13 +161,26 @@ __device__ __forceinline__ void chunk_pos(const QuantizeParams& p, int64_t c, in
 __device__ __forceinline__ void ring_finalize(const QuantizeParams& p, uint32_t bits, uint32_t nblocks, float s,
                                               uint32_t step, const float* hist_s) {
   uint32_t* words = reinterpret_cast<uint32_t*>(p.ring);
-  uint32_t* ticket = words + p.H + 1;
-  uint32_t* scratch = words + p.H + 3;
+  uint32_t* ticket = words + ring_ticket(p.H);
+  uint32_t* scratch = words + ring_scratch(p.H);
   if (bits) red_max_u32(scratch, bits);
-  // The release orders the red above before the ticket; the block that draws
-  // the last ticket acquires every earlier block's red.
-  if (atom_add_acq_rel(ticket, 1u) != nblocks - 1) return;
-  const float a = __uint_as_float(atomicExch(scratch, 0u));
+  float a;
+  const bool paired = (reinterpret_cast<uintptr_t>(ticket) & 7u) == 0;
+  if (paired) {
+    // ticket (low half) and scratch (high half) are one 8-byte word.  The red
+    // above and this add both write bytes of it, so program order puts this
+    // block's max before its ticket in that word's coherence order; the add
+    // that draws the last ticket therefore returns every block's max in its
+    // high half.  No fence and no second round trip.
+    const uint64_t old = atom_add_relaxed_u64(ticket, 1ull);
+    if (static_cast<uint32_t>(old) != nblocks - 1) return;
+    a = __uint_as_float(static_cast<uint32_t>(old >> 32));
+  } else {
+    // The release orders the red above before the ticket; the block that draws
+    // the last ticket acquires every earlier block's red.
+    if (atom_add_acq_rel(ticket, 1u) != nblocks - 1) return;
+    a = __uint_as_float(atomicExch(scratch, 0u));
+  }
   const uint32_t slot = step % static_cast<uint32_t>(p.H);
   float m = a;
   if (p.H <= kHistCache) {
@@ -178,8 +193,9 @@ __device__ __forceinline__ void ring_finalize(const QuantizeParams& p, uint32_t 
   const float snew = next_scale(s, m, p.fp8_max);
   p.ring[slot] = a;
   p.ring[p.H] = snew;
-  words[p.H + 2] = step + 1;
-  atomicExch(ticket, 0u);
+  words[ring_step(p.H)] = step + 1;
+  if (paired) *reinterpret_cast<volatile unsigned long long*>(ticket) = 0ull;  // ticket and scratch
+  else atomicExch(ticket, 0u);
   if (p.amax_out) *p.amax_out = a;
 }
 
@@ -197,7 +213,7 @@ __device__ __forceinline__ float scale_of(const QuantizeParams& p) {
 __device__ __forceinline__ void ring_tail(const QuantizeParams& p, uint32_t bits, uint32_t nblocks, float s,
                                           uint32_t step, const float* hist_s) {
   if (p.defer_finalize) {
-    if (bits) red_max_u32(reinterpret_cast<uint32_t*>(p.ring) + p.H + 3, bits);
+    if (bits) red_max_u32(reinterpret_cast<uint32_t*>(p.ring) + ring_scratch(p.H), bits);
     return;
   }
   ring_finalize(p, bits, nblocks, s, step, hist_s);
@@ -251,14 +267,14 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_cons
   const uint32_t nblocks = second ? gridDim.x - pair.blocks0 : pair.blocks0;
 
   const float s = scale_of(p);
-  const bool ring_step = p.ring && !p.defer_finalize;  // this launch finalizes the ring
+  const bool do_step = p.ring && !p.defer_finalize;  // this launch finalizes the ring
   uint32_t step = 0;
   if (threadIdx.x == 0) {
-    if (ring_step) step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
+    if (do_step) step = reinterpret_cast<const uint32_t*>(p.ring)[ring_step(p.H)];
     if (bid == 0 && p.scale_out) *p.scale_out = s;
   }
   // Only the tensor's last block writes its ring, after every block read it.
-  if (ring_step && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
+  if (do_step && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
 
   float amax = 0.0f;
   const int64_t stride = static_cast<int64_t>(nblocks) * kThreads;
@@ -412,13 +428,13 @@ __global__ void __launch_bounds__(kThreads) quantize_colsum_kernel(const __grid_
   const uint32_t nblocks = gridDim.x * gridDim.y;
   const uint32_t bid = blockIdx.y * gridDim.x + blockIdx.x;
   const float s = scale_of(p);
-  const bool ring_step = p.ring && !p.defer_finalize;
+  const bool do_step = p.ring && !p.defer_finalize;
   uint32_t step = 0;
   if (threadIdx.x == 0) {
-    if (ring_step) step = reinterpret_cast<const uint32_t*>(p.ring)[p.H + 2];
+    if (do_step) step = reinterpret_cast<const uint32_t*>(p.ring)[ring_step(p.H)];
     if (bid == 0 && p.scale_out) *p.scale_out = s;
   }
-  if (ring_step && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
+  if (do_step && p.H <= kHistCache && threadIdx.x < p.H) hist_s[threadIdx.x] = p.ring[threadIdx.x];
 
   const int cl = threadIdx.x % kChunkLanes;
   const int rl = threadIdx.x / kChunkLanes;
@@ -488,10 +504,10 @@ __global__ void ring_set_kernel(float* ring, int H, float scale) {
   for (int i = threadIdx.x; i < H; i += blockDim.x) ring[i] = 0.0f;
   if (threadIdx.x == 0) {
     uint32_t* w = reinterpret_cast<uint32_t*>(ring);
-    ring[H] = scale;
-    w[H + 1] = 0u;
-    w[H + 2] = 0u;
-    w[H + 3] = 0u;
+    ring[ring_scale(H)] = scale;
+    w[ring_step(H)] = 0u;
+    w[ring_ticket(H)] = 0u;
+    w[ring_scratch(H)] = 0u;
   }
 }
 

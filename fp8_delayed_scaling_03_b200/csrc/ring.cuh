@@ -18,8 +18,8 @@ namespace fp8lin {
 __device__ __forceinline__ void ring_finalize_warp(const RingFinalize& f, int lane) {
   uint32_t* words = reinterpret_cast<uint32_t*>(f.ring);
   const int H = f.H;
-  const uint32_t step = words[H + 2];
-  const float a = __uint_as_float(words[H + 3]);
+  const uint32_t step = words[ring_step(H)];
+  const float a = __uint_as_float(words[ring_scratch(H)]);
   const float s = f.ring[H];
   const uint32_t slot = step % static_cast<uint32_t>(H);
   float m = a;
@@ -30,8 +30,8 @@ __device__ __forceinline__ void ring_finalize_warp(const RingFinalize& f, int la
   if (lane == 0) {
     f.ring[slot] = a;
     f.ring[H] = next_scale(s, m, f.fp8_max);
-    words[H + 2] = step + 1;
-    words[H + 3] = 0u;
+    words[ring_step(H)] = step + 1;
+    words[ring_scratch(H)] = 0u;
     if (f.amax_out) *f.amax_out = a;
   }
 }

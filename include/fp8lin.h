@@ -103,11 +103,13 @@ typedef enum {
 
 /* ------------------------------------------------------------------ rings
  * A scale ring is the delayed-scaling state of one tensor, one device buffer
- * of fp8_ring_bytes(H) bytes, 4-byte aligned, laid out as 32-bit words:
+ * of fp8_ring_bytes(H) bytes, 4-byte aligned (8-byte aligned with an even H
+ * lets the in-kernel finalize use one 64-bit atomic on ticket + scratch),
+ * laid out as 32-bit words:
  *   [0, H)   hist    fp32 amax history (slot step % H holds the newest)
  *   H        scale   fp32 scale the next quantize multiplies by
- *   H+1      ticket  u32 block counter of the in-kernel finalize (0 at rest)
- *   H+2      step    u32 number of quantizes folded so far
+ *   H+1      step    u32 number of quantizes folded so far
+ *   H+2      ticket  u32 block counter of the in-kernel finalize (0 at rest)
  *   H+3      scratch u32 bits of the running amax of a launch (0 at rest)
  * [tests/extension@2eeac02]: the ring packs history, scale and counter in one
  * buffer; the quantize kernel's last block folds the amax in and publishes

@@ -50,8 +50,8 @@ def oracle_ring_words(r: oracle.Ring) -> np.ndarray:
     w = np.zeros(r.H + 4, np.uint32)
     w[: r.H] = r.hist.view(np.uint32)
     w[r.H] = np.float32(r.scale).view(np.uint32)
-    w[r.H + 1] = 0
-    w[r.H + 2] = r.step
+    w[r.H + 1] = r.step
+    w[r.H + 2] = 0
     w[r.H + 3] = 0
     return w
 

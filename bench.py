@@ -197,6 +197,16 @@ class Linear:
                                    self.bias_ptr, self.bias_dtype, self.bias_scale_ptr, F.FP8_E4M3, F.FP8_E4M3, H,
                                    p(self.rings[0]), p(self.rings[1]), p(self.x8), ldk, p(self.w8), ldk,
                                    sc, sc + 4, sc + 12, sc + 16, p(self.y), N)
+        # The weight quantized ahead of the forward (its own launch, its ring
+        # stepping there), and the forward taking that pre-quantized weight
+        # with its snapshot as the scale: the same outputs and ring words.
+        self.qw = F.QuantizeArgs(p(self.w), F.FP8_DT_BF16, N, K, K, F.FP8_E4M3, p(self.rings[1]), H, p(self.w8), ldk,
+                                 sc + 16, sc + 4)
+        self.fwd_w8 = F.LinearFwdArgs(M, N, K, p(self.x), F.FP8_DT_BF16, K, None, p(self.w8), F.FP8_DT_E4M3, ldk,
+                                      sc + 4, self.bias_ptr, self.bias_dtype, self.bias_scale_ptr, F.FP8_E4M3,
+                                      F.FP8_E4M3, H, p(self.rings[0]), None, p(self.x8), ldk, None, 0,
+                                      sc, sc + 4, sc + 12, None, p(self.y), N)
+        self.w_ready = torch.cuda.Event()
         self.bwd = F.LinearBwdArgs(M, N, K, p(self.g), F.FP8_DT_BF16, N, None, F.FP8_E5M2, H, p(self.rings[2]),
                                    p(self.g8), ldn, sc + 8, sc + 20, p(self.x8), ldk, sc, F.FP8_E4M3,
                                    p(self.w8), ldk, sc + 4, F.FP8_E4M3, 1, 1, int(need_dbias), p(self.dx), K,
@@ -251,13 +261,37 @@ def step_flops(lins) -> int:
     return sum(6 * L.shape.M * L.shape.N * L.shape.K for L in lins)
 
 
-def run_step(F, lins, stream_handle):
-    """Forward over the linears in order, then backward in reverse, through the C ABI."""
-    fwd, bwd = F._lib.fp8_linear_forward, F._lib.fp8_linear_backward
-    for L in lins:
-        s = fwd(ctypes.byref(L.fwd), stream_handle)
-        if s:
-            raise F.Fp8Error(s, "fp8_linear_forward")
+def run_step(F, lins, stream, side=None):
+    """Forward over the linears in order, then backward in reverse, through the
+    C ABI.  With a side stream, the weights are quantized there first (one
+    fp8_quantize per weight, in forward order) while the main stream runs the
+    forward linears on the pre-quantized weights, each waiting only for its own
+    weight: the weight casts overlap the earlier linears' GEMMs, which leave
+    HBM mostly idle.  Weights do not depend on the activations, so this order
+    is the step's own dependency graph."""
+    lib = F._lib
+    fwd, bwd = lib.fp8_linear_forward, lib.fp8_linear_backward
+    h = stream.cuda_stream
+    if side is None:
+        for L in lins:
+            s = fwd(ctypes.byref(L.fwd), h)
+            if s:
+                raise F.Fp8Error(s, "fp8_linear_forward")
+    else:
+        start = torch.cuda.Event()
+        start.record(stream)
+        side.wait_event(start)
+        for L in lins:
+            s = lib.fp8_quantize_ex(ctypes.byref(L.qw), 0, side.cuda_stream)
+            if s:
+                raise F.Fp8Error(s, "fp8_quantize_ex (weight)")
+            L.w_ready.record(side)
+        for L in lins:
+            stream.wait_event(L.w_ready)
+            s = fwd(ctypes.byref(L.fwd_w8), h)
+            if s:
+                raise F.Fp8Error(s, "fp8_linear_forward")
+    stream_handle = h
     for L in reversed(lins):
         s = bwd(ctypes.byref(L.bwd), stream_handle)
         if s:
@@ -271,7 +305,7 @@ LAUNCHES_PER_LINEAR = 4
 
 # --------------------------------------------------------------------------- kernel-level timing
 
-def step_primitives(F, lins, h):
+def step_primitives(F, lins, h, split_w=False):
     """The step's kernel launches as (class, algorithmic work, label, call) in
     launch order, through the standalone entry points that do the same work as
     the fused fp8_linear_forward / fp8_linear_backward: quantize x+w, forward
@@ -293,7 +327,12 @@ def step_primitives(F, lins, h):
                             sc + 16, sc + 4)
         fwd = F.MmArgs(M, N, K, L.x8.data_ptr(), 0, 0, ldk, L.w8.data_ptr(), 0, 0, ldk, sc, sc + 4,
                        L.bias_ptr, L.bias_dtype, L.bias_scale_ptr, L.y.data_ptr(), N, 0)
-        out.append(("quantize", (M * K + N * K) * 3, None, call(lib.fp8_quantize_dual, qx, qw)))
+        if split_w:  # the weight in its own launch (the side-stream schedule), then x
+            out.append(("quantize", N * K * 3, None, (lambda qw=qw: lib.fp8_quantize_ex(ctypes.byref(qw), 0, h))))
+            out.append(("quantize", M * K * 3, None, (lambda qx=qx: lib.fp8_quantize_ex(ctypes.byref(qx), 0, h))))
+            keep.append((qx, qw))
+        else:
+            out.append(("quantize", (M * K + N * K) * 3, None, call(lib.fp8_quantize_dual, qx, qw)))
         out.append(("gemm", 2 * M * N * K, f"fwd {M}x{N}x{K}", call(lib.fp8_mm, fwd)))
     for L in reversed(lins):
         M, K, N = L.shape.M, L.shape.K, L.shape.N
@@ -318,14 +357,14 @@ def step_primitives(F, lins, h):
     return out, keep
 
 
-def time_kernels(F, lins, stream, reps=5):
+def time_kernels(F, lins, stream, reps=5, split_w=False):
     """Device time of each kernel class of the step: the class's launches (in
     step order, same buffers) captured as one CUDA graph and replayed between
     CUDA events on the launching stream, so host launch gaps are excluded.
     Returns (ms per step by class, work by class, launches by class, per-shape
     GEMM times)."""
     h = stream.cuda_stream
-    prims, keep = step_primitives(F, lins, h)
+    prims, keep = step_primitives(F, lins, h, split_w)
     res_ms, work, count = {}, {}, {}
     for cls in ("gemm", "quantize"):
         calls = [c for c in prims if c[0] == cls]
@@ -747,16 +786,16 @@ def graph_kernel_nodes(graph):
         return None
 
 
-def capture_step(F, lins, stream, warmup):
+def capture_step(F, lins, stream, warmup, side=None):
     """Eager step (first-launch set-up outside the capture), then the step
     captured as one CUDA graph (kept, so its kernel nodes can be counted) and
     replayed `warmup` times."""
     with torch.cuda.stream(stream):
-        run_step(F, lins, stream.cuda_stream)
+        run_step(F, lins, stream, side)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph(keep_graph=True)
     with torch.cuda.graph(graph, stream=stream):
-        run_step(F, lins, stream.cuda_stream)
+        run_step(F, lins, stream, side)
     for _ in range(warmup):
         graph.replay()
     torch.cuda.synchronize()
@@ -796,6 +835,10 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=wl.BENCH_LAYERS, help="layers of the dim1024 workload "
                     "(profiling runs only)")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, kernel timing, targets and cpu baseline")
+    ap.add_argument("--weights", default="fused", choices=["side", "fused"],
+                    help="side: weights quantized on a second stream ahead of the forward linears (pre-quantized "
+                         "weights), overlapping the earlier GEMMs; fused: x and w quantized in each linear's "
+                         "fp8_linear_forward")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     wl.BENCH_LAYERS = args.layers
@@ -815,9 +858,10 @@ def main(argv=None):
 
     lins = build_model(F, device, rank, args.workload)
     stream = torch.cuda.Stream(device)
+    side = torch.cuda.Stream(device) if args.weights == "side" else None
     torch.cuda.synchronize()
     flops_step = step_flops(lins)
-    graph = capture_step(F, lins, stream, args.warmup)
+    graph = capture_step(F, lins, stream, args.warmup, side)
 
     # ---- timed region
     if world > 1:
@@ -835,6 +879,9 @@ def main(argv=None):
     clocks = clk.report()
     cfg = config_dict(args.workload)
     cfg["working_set_bytes"] = working_set_bytes(lins)
+    cfg["weights"] = ("quantized on a second stream ahead of the forward linears, which take them pre-quantized "
+                      "(each waits for its own weight only)" if side is not None else
+                      "quantized with x inside each fp8_linear_forward")
 
     kernels_per_step = graph_kernel_nodes(graph)
     cfg["kernels_per_step"] = kernels_per_step if kernels_per_step is not None else \
@@ -849,7 +896,7 @@ def main(argv=None):
         pk, pk_kind = peaks()
         fp8_peak, peak_key = fp8_peak_for(pk, clocks)
         # ---- kernel-level timing and roofline of the dominant kernel (the GEMM class)
-        tot, work, count, shapes = time_kernels(F, lins, stream)
+        tot, work, count, shapes = time_kernels(F, lins, stream, split_w=side is not None)
         gemm_tflops = work["gemm"] / (tot["gemm"] / 1e3) / 1e12
         traffic = gemm_traffic_per_launch(args.workload)
         line["roofline"] = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
@@ -872,9 +919,9 @@ def main(argv=None):
             "step_minus_gemm_class_ms": max(step_ms - tot["gemm"], 0.0),
             "quantize": {"achieved_gbs": q_gbs, "peak_gbs": pk["hbm_gbs"], "frac": q_gbs / pk["hbm_gbs"],
                          "bytes_per_elem": 3,
-                         "note": "bf16 in + fp8 out; x+w in one launch, g (with its bias-gradient partials when "
-                                 "the bias needs a gradient) in one launch; standalone class graph, each launch "
-                                 "finalizing its ring"},
+                         "note": "bf16 in + fp8 out; x and w in one launch (fused weights) or in two (weights on "
+                                 "the side stream), g (with its bias-gradient partials when the bias needs a "
+                                 "gradient) in one launch; standalone class graph, each launch finalizing its ring"},
             "gemm_by_shape": shapes}
 
         # ---- the other workloads' steps, timed the same way
@@ -883,13 +930,13 @@ def main(argv=None):
             if wname == args.workload:
                 continue
             olins = build_model(F, device, rank, wname)
-            og = capture_step(F, olins, stream, args.warmup)
+            og = capture_step(F, olins, stream, args.warmup, side)
             oreps = max(5, args.steps // 2)
             if world > 1:
                 dist.barrier()
             oms = reduce_max(time_graph_ms(og, stream, oreps), world, device)
             ofl = step_flops(olins)
-            ot, owork, ocount, _ = time_kernels(F, olins, stream)
+            ot, owork, ocount, _ = time_kernels(F, olins, stream, split_w=side is not None)
             otf = owork["gemm"] / (ot["gemm"] / 1e3) / 1e12
             others[wname] = {"workload": WORKLOADS[wname][0],
                              "value": aggregate_throughput(ofl * oreps, world, oms / 1e3) / 1e12, "unit": UNIT,

@@ -419,8 +419,9 @@ def time_kernels(F, lins, stream, reps=5, split_w=False):
 # --------------------------------------------------------------------------- target shapes, per operation
 
 def _graph_us(stream, fns, reps=3):
-    """Mean device time of one call of `fns` (cycled) inside a CUDA graph of
-    len(fns) * 4 calls, replayed `reps` times between CUDA events."""
+    """Device time of one call of `fns` (cycled) inside a CUDA graph of
+    len(fns) * 4 calls: `reps` replays between CUDA events, the median of three
+    such runs."""
     g = torch.cuda.CUDAGraph()
     n = len(fns) * 4
     with torch.cuda.graph(g, stream=stream):
@@ -429,14 +430,17 @@ def _graph_us(stream, fns, reps=3):
     g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
+    runs = []
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        runs.append(e0.elapsed_time(e1) * 1e3 / (reps * n))
     del g
-    return e0.elapsed_time(e1) * 1e3 / (reps * n)
+    return statistics.median(runs)
 
 
 def _sets_for(bytes_per_set, floor=320 << 20, cap=12):

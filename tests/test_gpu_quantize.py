@@ -188,3 +188,54 @@ def test_quantize_dbias_entry(fp8, rows, cols):
         ov = oracle.bf16_to_f32(want).astype(np.float64)
         assert np.all(np.abs(gv - ov) <= np.maximum(oracle.bf16_ulp(ov), 2e-6 * sa))
     assert fp8.fp8_get_device_status() == 0
+
+
+@pytest.mark.parametrize("H,offset", [(1, 0), (3, 0), (5, 0), (16, 4), (6, 4), (16, 0), (2, 0)])
+def test_ring_finalize_paths(fp8, H, offset):
+    """Both forms of the last-block finalize against the oracle over several
+    multi-block steps: with an even H and an 8-byte aligned ring, ticket and
+    scratch share one 8-byte word (one 64-bit atomic per block); an odd H or a
+    ring only 4-byte aligned (offset 4 bytes) takes the two-word protocol.
+    Codes, amax, snapshot and every ring word bit for bit; also through the
+    column-sum quantize (fp8_quantize_dbias) and the dual launch."""
+    words = fp8.fp8_ring_bytes(H) // 4
+    k = offset // 4
+
+    def ring_at(tag):
+        base = torch.zeros(words + 2, dtype=torch.float32, device="cuda")
+        r = fp8.ScaleRing(H, buf=base[k:k + words])
+        fp8.fp8_ring_init(r.buf, H)
+        assert (r.buf.data_ptr() % 8 == 0) == (offset == 0)
+        return r
+
+    ring, oring = ring_at(0), oracle.Ring(H)
+    for step in range(H + 3):  # wraps the history at least once
+        x = wl.normal((1536, 1000), 0.5 * (1.3 ** (step % 7)), 7100 + step)
+        check_step(fp8, x, fp8.FP8_E4M3 if step % 2 == 0 else fp8.FP8_E5M2, ring, oring)
+    # column-sum quantize (the bias-gradient path) on the same kind of ring
+    rg, org = ring_at(1), oracle.Ring(H)
+    rows, cols = 700, 600
+    ws = torch.zeros(max(16, fp8.fp8_dbias_workspace_bytes(rows, cols)), dtype=torch.uint8, device="cuda")
+    for step in range(3):
+        g = wl.normal((rows, cols), 1e-3 * (1 + step), 7200 + step)
+        gd, out = g.cuda(), fp8_buffer(rows, cols)
+        db = torch.empty(cols, dtype=torch.bfloat16, device="cuda")
+        fp8.fp8_quantize_dbias(fp8.quantize_args(gd, 1, rg.buf, H, out), db, ws)
+        torch.cuda.synchronize()
+        q, _, _ = oracle.quantize(bits(g), oracle.DT_BF16, 1, org)
+        assert_codes_equal(host_rows(out), q, 1)
+        assert np.array_equal(ring_words(rg), oracle_ring_words(org))
+    # dual launch: two rings of this kind in one grid
+    r1, r2, o1, o2 = ring_at(2), ring_at(3), oracle.Ring(H), oracle.Ring(H)
+    for step in range(3):
+        x = wl.normal((1024, 640), 1.0 + step, 7300 + step)
+        w = wl.normal((512, 640), 0.05, 7350 + step)
+        xd, wd = x.cuda(), w.cuda()
+        x8, w8 = fp8_buffer(1024, 640), fp8_buffer(512, 640)
+        fp8.fp8_quantize_dual(fp8.quantize_args(xd, 0, r1.buf, H, x8), fp8.quantize_args(wd, 0, r2.buf, H, w8))
+        torch.cuda.synchronize()
+        oracle.quantize(bits(x), dt_code(x), 0, o1)
+        oracle.quantize(bits(w), dt_code(w), 0, o2)
+        assert np.array_equal(ring_words(r1), oracle_ring_words(o1))
+        assert np.array_equal(ring_words(r2), oracle_ring_words(o2))
+    assert fp8.fp8_get_device_status() == 0

@@ -464,3 +464,25 @@ def test_mm_pair_stream_k(fp8, tile):
     gemm_dw, _, sab = oracle.gemm_acc(gs, 1, 1, ldg, xs, 0, 1, ldx, N, K, M)
     want, _ = oracle.epilogue(gemm_dw, 3.0, 0.25)
     assert_gemm_close(dw.cpu().view(torch.int16).numpy().view(np.uint16), want, sab, 3.0, 0.25, "pair sk dw")
+
+
+@pytest.mark.parametrize("a_major,b_major", LAYOUTS)
+def test_mm_nan_codes_propagate(fp8, a_major, b_major):
+    """NaN codes in the operands (E4M3 0x7F/0xFF in A, E5M2 0x7E in B): every
+    output whose dot product contains one is NaN, all others are finite and
+    match the oracle."""
+    rng = np.random.default_rng(77 + 2 * a_major + b_major)
+    m, n, k = 300, 260, 200
+    A = codes_like_tensor(rng, 0, (m, k), 60.0)
+    B = codes_like_tensor(rng, 1, (n, k), 3000.0)
+    A[11, 3], A[250, 199] = 0x7F, 0xFF
+    B[100, 0] = 0x7E
+    _, y, _ = run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=0, fmt_b=1, a_codes=A, b_codes=B)
+    yf = oracle.bf16_to_f32(y)
+    nan_rows, nan_cols = {11, 250}, {100}
+    for i in range(m):
+        for_rows = np.isnan(yf[i])
+        if i in nan_rows:
+            assert for_rows.all()
+        else:
+            assert np.array_equal(np.where(for_rows)[0], np.array(sorted(nan_cols)))

@@ -205,7 +205,10 @@ static int fmt_shift(int fmt) { return fmt == ORC_E4M3 ? 9 : 16; }
  *   acc_f32[i*J+j]: products accumulated in fp32, k = 0,1,...,Kc-1;
  *   exact[i*J+j]  : the exact dot (int128), rounded once to double (optional);
  *   sumabs[i*J+j] : sum_k |A(i,k) B(j,k)| in double (optional).
- * Any NaN operand makes all three NaN. */
+ * Non-finite operands follow IEEE fp32 arithmetic (the pages state fp32
+ * accumulation and nothing on special values): a NaN operand, an inf x 0
+ * product or products of both infinite signs make the output NaN, other
+ * infinite products make it +-inf; then all three outputs hold that value. */
 void orc_gemm(int64_t I, int64_t J, int64_t Kc,
               const uint8_t* a, int fmt_a, int64_t a_si, int64_t a_sk,
               const uint8_t* b, int fmt_b, int64_t b_sj, int64_t b_sk,
@@ -221,20 +224,20 @@ void orc_gemm(int64_t I, int64_t J, int64_t Kc,
       float acc = 0.0f;
       __int128 ex = 0;
       double sa = 0.0;
-      int nan = 0;
+      int finite = 1;
       for (int64_t k = 0; k < Kc; ++k) {
         double va = ta[a[i * a_si + k * a_sk]];
         double vb = tb[b[j * b_sj + k * b_sk]];
-        if (isnan(va) || isnan(vb) || isinf(va) || isinf(vb)) { nan = 1; break; }
-        float p = (float)(va * vb);  /* exact: at most 8 significant bits */
-        acc = acc + p;
+        float p = (float)(va * vb);  /* exact for finite operands (at most 8 significant bits) */
+        acc = acc + p;               /* IEEE fp32: inf and NaN propagate as fp32 arithmetic does */
+        if (!isfinite(va) || !isfinite(vb)) { finite = 0; continue; }
         if (exact) ex += (__int128)(int64_t)(va * ua) * (__int128)(int64_t)(vb * ub);
         if (sumabs) sa += fabs(va * vb);
       }
-      if (nan) {
-        acc_f32[i * J + j] = NAN;
-        if (exact) exact[i * J + j] = NAN;
-        if (sumabs) sumabs[i * J + j] = NAN;
+      if (!finite) {  /* acc is +-inf or NaN: the exact sum is that value too */
+        acc_f32[i * J + j] = acc;
+        if (exact) exact[i * J + j] = acc;
+        if (sumabs) sumabs[i * J + j] = fabs(acc);
         continue;
       }
       acc_f32[i * J + j] = acc;
@@ -247,8 +250,9 @@ void orc_gemm(int64_t I, int64_t J, int64_t Kc,
 /* The same dot products for a list of n (i, j) output coordinates only, for
  * sampled checks of shapes whose full product is too slow on the CPU.  Each
  * point is the loop of orc_gemm for that (i, j): fp32 accumulation with k
- * ascending, sum |a_k b_k| in double, and a NaN or infinite operand makes
- * both results NaN. */
+ * ascending, sum |a_k b_k| in double; with a NaN or infinite operand the
+ * accumulator is whatever IEEE fp32 arithmetic makes of it (NaN, or +-inf)
+ * and so is the sum of magnitudes. */
 void orc_gemm_points(int64_t n, const int64_t* ii, const int64_t* jj, int64_t Kc,
                      const uint8_t* a, int fmt_a, int64_t a_si, int64_t a_sk,
                      const uint8_t* b, int fmt_b, int64_t b_sj, int64_t b_sk,
@@ -261,17 +265,17 @@ void orc_gemm_points(int64_t n, const int64_t* ii, const int64_t* jj, int64_t Kc
     int64_t i = ii[t], j = jj[t];
     float acc = 0.0f;
     double sa = 0.0;
-    int nan = 0;
+    int finite = 1;
     for (int64_t k = 0; k < Kc; ++k) {
       double va = ta[a[i * a_si + k * a_sk]];
       double vb = tb[b[j * b_sj + k * b_sk]];
-      if (isnan(va) || isnan(vb) || isinf(va) || isinf(vb)) { nan = 1; break; }
       float p = (float)(va * vb);
       acc = acc + p;
+      if (!isfinite(va) || !isfinite(vb)) { finite = 0; continue; }
       sa += fabs(va * vb);
     }
-    acc_f32[t] = nan ? NAN : acc;
-    sumabs[t] = nan ? NAN : sa;
+    acc_f32[t] = acc;
+    sumabs[t] = finite ? sa : fabs(acc);
   }
 }
 

@@ -75,14 +75,19 @@ def assert_gemm_close(y_gpu_bits: np.ndarray, y_orc_bits: np.ndarray, sumabs: np
     g = oracle.bf16_to_f32(y_gpu_bits).astype(np.float64)
     o = oracle.bf16_to_f32(y_orc_bits).astype(np.float64)
     tol = oracle.gemm_tolerance(y_orc_bits, sumabs, sa, sb)
+    # non-finite oracle outputs (IEEE fp32 accumulation of NaN / inf operands)
+    # must be matched exactly: NaN by NaN, an infinity by the same infinity
     both_nan = np.isnan(g) & np.isnan(o)
-    err = np.where(both_nan, 0.0, np.abs(g - o))
-    bad = ~((err <= tol) | both_nan)  # a NaN output's tolerance is NaN too
+    same_inf = np.isinf(o) & (g == o)
+    exact = both_nan | same_inf
+    with np.errstate(invalid="ignore"):
+        err = np.where(exact, 0.0, np.abs(g - o))
+    bad = ~((err <= tol) | exact)  # a non-finite output's tolerance is non-finite too
     if bad.any():
         idx = np.argwhere(bad)[:6]
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside tolerance; first "
                              f"{[(tuple(i), g[tuple(i)], o[tuple(i)], tol[tuple(i)]) for i in idx]}")
-    live = ~both_nan
+    live = ~exact
     return float(np.max(err[live] / tol[live])) if live.any() else 0.0
 
 

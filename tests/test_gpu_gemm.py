@@ -486,3 +486,29 @@ def test_mm_nan_codes_propagate(fp8, a_major, b_major):
             assert for_rows.all()
         else:
             assert np.array_equal(np.where(for_rows)[0], np.array(sorted(nan_cols)))
+
+
+@pytest.mark.parametrize("a_major,b_major", LAYOUTS)
+def test_mm_inf_codes_follow_ieee(fp8, a_major, b_major):
+    """E5M2 infinities in A against E4M3 B: outputs are what IEEE fp32
+    accumulation gives, as in the oracle -- +-inf for one infinite product,
+    NaN for inf x 0 and for products of both infinite signs -- and bf16 +-inf
+    / NaN after the epilogue; all other outputs finite and within tolerance."""
+    rng = np.random.default_rng(91 + 2 * a_major + b_major)
+    m, n, k = 260, 200, 150
+    A = codes_like_tensor(rng, 1, (m, k), 3000.0)
+    B = codes_like_tensor(rng, 0, (n, k), 60.0)
+    B[B == 0x80] = 0x08
+    B[B == 0x00] = 0x08
+    A[5, 10] = 0x7C                      # row 5: +-inf by the sign of B(j, 10)
+    A[77, 149] = 0xFC                    # row 77: -+inf
+    A[130, 3] = 0x7C
+    B[60, 3] = 0x00                      # (130, 60): inf x 0 = NaN; rest of row 130 inf
+    A[200, 20], A[200, 21] = 0x7C, 0xFC
+    B[:, 20] = B[:, 21] = 0x38           # row 200: +inf - inf = NaN everywhere
+    _, y, want = run_case(fp8, rng, m, n, k, a_major, b_major, fmt_a=1, fmt_b=0, a_codes=A, b_codes=B)
+    yf, wf = oracle.bf16_to_f32(y), oracle.bf16_to_f32(want)
+    assert np.isinf(yf[5]).all() and np.isinf(yf[77]).all() and np.isnan(yf[200]).all()
+    assert np.isnan(yf[130, 60]) and np.isinf(yf[130, :60]).all()
+    assert np.array_equal(np.isnan(yf), np.isnan(wf)) and np.array_equal(yf[np.isinf(wf)], wf[np.isinf(wf)])
+    assert np.isfinite(np.delete(yf, [5, 77, 130, 200], axis=0)).all()

@@ -96,24 +96,62 @@ def test_gemm_points_exact_rational():
         assert abs(Fraction(float(sab[t])) - sa) <= Kc * Fraction(2) ** -53 * sa
 
 
-@pytest.mark.parametrize("code", (0x7C, 0xFC, 0x7E, 0xFF))
-def test_gemm_points_nonfinite_operand(code):
-    """An E5M2 inf (0x7C, 0xFC) or NaN (0x7E, 0xFF) operand makes the points
-    that read it NaN in both outputs, exactly where the full routine gives
-    NaN; the other points are unaffected."""
+def ieee_dot_f32(av, bv):
+    """sum_k a_k b_k with numpy float32 arithmetic in k order (IEEE: inf and NaN
+    propagate, inf * 0 and inf - inf are NaN)."""
+    acc = np.float32(0.0)
+    with np.errstate(invalid="ignore", over="ignore"):
+        for x, y in zip(av, bv):
+            acc = np.float32(acc + np.float32(np.float64(x) * np.float64(y)))
+    return acc
+
+
+@pytest.mark.parametrize("case", ["nan", "pinf", "ninf", "inf_times_zero", "both_infs"])
+def test_gemm_nonfinite_operands_follow_ieee_fp32(case):
+    """Non-finite fp8 operands (E5M2 +-inf 0x7C/0xFC, NaN 0x7E; E4M3 NaN 0x7F):
+    the full GEMM and the sampled points give what IEEE fp32 arithmetic gives
+    (numpy float32, k order) -- NaN, +-inf -- at the outputs that read them,
+    with the sum of magnitudes non-finite there too; every other output is
+    unchanged and finite."""
     rng = np.random.default_rng(103)
     I, J, Kc = 6, 5, 40
     a = rand_codes(rng, E5M2, (I, Kc))
     b = rand_codes(rng, E4M3, (J, Kc))
-    a[2, 17] = code
-    acc, _, sab = oracle.gemm_acc(a, E5M2, Kc, 1, b, E4M3, Kc, 1, I, J, Kc)
+    b[b == 0x80] = 0x08  # no zero operands except the planted one
+    b[b == 0x00] = 0x08
+    if case == "nan":
+        a[2, 17] = 0x7E
+    elif case == "pinf":
+        a[2, 17] = 0x7C
+    elif case == "ninf":
+        a[2, 17] = 0xFC
+    elif case == "inf_times_zero":
+        a[2, 17] = 0x7C
+        b[3, 17] = 0x00          # (2, 3): inf * 0
+    else:
+        a[2, 17], a[2, 30] = 0x7C, 0xFC
+        b[:, 17] = b[:, 30] = 0x38  # 1.0: the two infinite products have opposite signs
+    acc, ex, sab = oracle.gemm_acc(a, E5M2, Kc, 1, b, E4M3, Kc, 1, I, J, Kc, exact=True)
     ii = np.repeat(np.arange(I), J)
     jj = np.tile(np.arange(J), I)
     pacc, psab = oracle.gemm_acc_points(ii, jj, a, E5M2, Kc, 1, b, E4M3, Kc, 1, Kc)
-    nan_rows = ii == 2
-    assert np.all(np.isnan(pacc[nan_rows])) and np.all(np.isnan(psab[nan_rows]))
-    assert np.all(np.isnan(acc[2])) and np.all(np.isnan(sab[2]))
-    assert np.array_equal(pacc[~nan_rows], acc[ii[~nan_rows], jj[~nan_rows]])
+    da, db = oracle.decode(E5M2, a), oracle.decode(E4M3, b)
+    for i in range(I):
+        for j in range(J):
+            want = ieee_dot_f32(da[i], db[j])
+            got = acc[i, j]
+            if i == 2:
+                assert not np.isfinite(want)
+                assert (np.isnan(want) and np.isnan(got)) or want == got, (case, i, j, got, want)
+                assert not np.isfinite(sab[i, j]) and not np.isfinite(ex[i, j])
+            else:
+                assert np.isfinite(got) and np.isfinite(sab[i, j])
+    if case == "inf_times_zero":
+        assert np.isnan(acc[2, 3]) and np.isinf(acc[2, 0])
+    if case == "both_infs":
+        assert np.all(np.isnan(acc[2]))
+    assert np.array_equal(pacc, acc[ii, jj], equal_nan=True)
+    assert np.array_equal(np.isfinite(psab), np.isfinite(sab[ii, jj]))
 
 
 def test_mutant_points_with_swapped_strides_is_caught():

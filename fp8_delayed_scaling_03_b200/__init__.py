@@ -119,6 +119,7 @@ _SIGS = {
     "fp8_linear_backward": (_I, [ctypes.POINTER(LinearBwdArgs), _P]),
     "fp8_linear_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "fp8_get_device_status": (_I, []),
+    "fp8_wait_selftest": (_I, [_P, ctypes.c_uint64, _P, _P]),
     "fp8_status_string": (ctypes.c_char_p, [_I]),
     "fp8_version": (ctypes.c_char_p, []),
 }
@@ -311,6 +312,13 @@ def fp8_linear_workspace_bytes(M: int, N: int, K: int) -> int:
 
 def fp8_get_device_status() -> int:
     return _lib.fp8_get_device_status()
+
+
+def fp8_wait_selftest(flag: torch.Tensor, limit_ns: int, results: torch.Tensor) -> None:
+    """Runs the bounded-wait diagnostic kernel: results[0] / results[1] = 1
+    where the flag wait / the mbarrier wait was satisfied, 0 where it ran out
+    (which fp8_get_device_status then reports as FP8_ERR_DEVICE_TIMEOUT)."""
+    _check(_lib.fp8_wait_selftest(_ptr(flag), limit_ns, _ptr(results), _stream(flag.device)), "fp8_wait_selftest")
 
 
 def fp8_status_string(status: int) -> str:

@@ -1132,6 +1132,19 @@ int fp8_linear_backward(const fp8_linear_bwd_args* a, fp8_stream_t stream) {
   return FP8_OK;
 }
 
+int fp8_wait_selftest(const void* flag, uint64_t limit_ns, int* results, fp8_stream_t stream) {
+  if (!flag || !results || !aligned(flag, 4) || !aligned(results, 4)) return FP8_ERR_INVALID_ARG;
+  if (limit_ns == 0 || limit_ns > 2000000000ull) return FP8_ERR_INVALID_ARG;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int* status = status_ptr(dev);
+  if (!status) return cuda_fail(cudaGetLastError());
+  e = launch_wait_selftest(static_cast<const uint32_t*>(flag), status, results, limit_ns,
+                           reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP8_OK : cuda_fail(e);
+}
+
 int fp8_get_device_status(void) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FP8_ERR_CUDA;

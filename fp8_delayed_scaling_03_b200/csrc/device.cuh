@@ -89,7 +89,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // abort may be NULL.  kCluster: acquire at cluster scope (see above).
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
-                                          volatile int* abort) {
+                                          volatile int* abort, uint64_t limit_ns = FP8LIN_WAIT_LIMIT_NS) {
   const uint32_t a = smem_u32(bar);
   auto probe = [&]() { return kCluster ? mbar_try_wait_acq_cluster(a, parity) : mbar_try_wait(a, parity); };
   #pragma unroll 1
@@ -102,7 +102,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     for (int i = 0; i < 256; ++i)
       if (probe()) return true;
     if (abort && *abort) return false;
-    if (globaltimer_ns() - t0 > FP8LIN_WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       if (status) atomicExch(status, kDevTimeout);
       if (abort) *abort = 1;
       return false;
@@ -372,7 +372,8 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
 // semantics, so each lane's later loads see the guarded data.  Bounded like
 // mbar_wait: after FP8LIN_WAIT_LIMIT_NS a timeout is recorded in *status and
 // false returned (also as soon as *abort is set).
-__device__ __forceinline__ bool flag_wait_warp(const uint32_t* f, int* status, volatile int* abort) {
+__device__ __forceinline__ bool flag_wait_warp(const uint32_t* f, int* status, volatile int* abort,
+                                               uint64_t limit_ns = FP8LIN_WAIT_LIMIT_NS) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0 && !ld_acquire_u32(f)) {
     ok = 0;
@@ -383,7 +384,7 @@ __device__ __forceinline__ bool flag_wait_warp(const uint32_t* f, int* status, v
       for (int i = 0; i < 64 && !ok; ++i) ok = ld_acquire_u32(f) != 0;
       if (ok) break;
       if (abort && *abort) break;
-      if (globaltimer_ns() - t0 > FP8LIN_WAIT_LIMIT_NS) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         if (status) atomicExch(status, kDevTimeout);
         if (abort) *abort = 1;
         break;

@@ -200,6 +200,8 @@ int gemm_pair_capacity(int device);
 cudaError_t launch_gemm(const CUtensorMap* maps, const GemmParams& p, int cfg, cudaStream_t s);
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s);
 cudaError_t launch_fill(const FillParams& p, cudaStream_t s);
+cudaError_t launch_wait_selftest(const uint32_t* flag, int* status, int* results, uint64_t limit_ns,
+                                 cudaStream_t s);
 
 // Column-sum geometry (R row splits of rows_per_split rows over 256-column
 // tiles) shared by the size queries and the launchers: dbias_geometry for the

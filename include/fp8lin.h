@@ -398,6 +398,17 @@ FP8LIN_API size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * reads that word (synchronizing the device) and clears it; FP8_OK if clear. */
 FP8LIN_API int fp8_get_device_status(void);
 
+/* The bounded waits themselves, exercised on purpose (a diagnostic, not a
+ * step of the path): one tiny kernel waits, with a time limit of limit_ns
+ * nanoseconds (1 ns .. 2 s), on the 32-bit device word *flag becoming
+ * non-zero (the stream-K flag protocol) and on an mbarrier that nothing ever
+ * arrives on (the GEMM pipeline protocol).  results (device, 2 ints): 1 where
+ * the wait was satisfied, 0 where it ran out.  A wait that runs out records
+ * FP8_ERR_DEVICE_TIMEOUT for fp8_get_device_status; the kernel then returns,
+ * and the context stays usable.  flag and results 4-byte aligned, else
+ * FP8_ERR_INVALID_ARG. */
+FP8LIN_API int fp8_wait_selftest(const void* flag, uint64_t limit_ns, int* results, fp8_stream_t stream);
+
 /* Static description of a status code (for FP8_ERR_CUDA: the last CUDA error
  * this library saw, on the calling host thread). */
 FP8LIN_API const char* fp8_status_string(int status);

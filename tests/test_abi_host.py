@@ -253,3 +253,14 @@ def test_fused_entry_points_validation(fp8):
     zero = fp8.MmArgs(m=0, n=128, k=128, a=A, lda=128, b=A + 0x10000, ldb=128, scale_a=A + 0x20000,
                       scale_b=A + 0x20010, d=A + 0x30000, ldd=128)
     assert f.fp8_mm_pair(ctypes.byref(zero), ctypes.byref(zero), None) == E.FP8_OK
+
+
+def test_wait_selftest_validation(fp8):
+    """Arguments are checked before anything is launched (no GPU needed)."""
+    f = fp8._lib.fp8_wait_selftest
+    assert f(None, 1000, 0x1000, None) == fp8.FP8_ERR_INVALID_ARG
+    assert f(0x1000, 1000, None, None) == fp8.FP8_ERR_INVALID_ARG
+    assert f(0x1002, 1000, 0x1000, None) == fp8.FP8_ERR_INVALID_ARG     # flag not 4-byte aligned
+    assert f(0x1000, 1000, 0x1001, None) == fp8.FP8_ERR_INVALID_ARG     # results not 4-byte aligned
+    assert f(0x1000, 0, 0x1000, None) == fp8.FP8_ERR_INVALID_ARG        # no limit
+    assert f(0x1000, 2_000_000_001, 0x1000, None) == fp8.FP8_ERR_INVALID_ARG  # above 2 s

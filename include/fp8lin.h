@@ -93,7 +93,7 @@ typedef enum {
 typedef enum {
   FP8_OK = 0,
   FP8_ERR_INVALID_ARG = -1,    /* NULL required pointer, bad enum, ld < cols, ... */
-  FP8_ERR_UNSUPPORTED = -2,    /* valid request this build does not implement   */
+  FP8_ERR_UNSUPPORTED = -2,    /* valid request this library does not implement */
   FP8_ERR_MISALIGNED = -3,     /* fp8 ld % 16 != 0 or base not 16-byte aligned  */
   FP8_ERR_CUDA = -4,           /* a CUDA call failed (see fp8_status_string)    */
   FP8_ERR_DEVICE_TIMEOUT = -5, /* a kernel gave up on a bounded wait            */

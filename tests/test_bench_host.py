@@ -141,3 +141,41 @@ def test_e2e_harness_orders_copies_and_kernels(monkeypatch):
         r = records[ops[k][2]]
         copies_out = [j for j, o in enumerate(ops[:k]) if o[0] == "s3" and o[1] == "copy"]
         assert all(j < r for j in copies_out)
+
+
+def test_fp8_peak_denominator_choice():
+    """Burst bf16 x 2 while the timed region held the maximum clock with no
+    power-cap reason; the sustained figure under the cap or a lowered clock."""
+    import bench
+    pk = {"bf16_tflops": 1644.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6551.0}
+    assert bench.fp8_peak_for(pk, {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}) == (3288.0, "bf16_tflops")
+    assert bench.fp8_peak_for(pk, {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}) == \
+        (2800.0, "bf16_tflops_sustained")
+    assert bench.fp8_peak_for(pk, {"sm_mhz": 1500, "sm_max_mhz": 1965, "reasons": []})[1] == "bf16_tflops_sustained"
+    burst_only = {"bf16_tflops": 1644.0}
+    assert bench.fp8_peak_for(burst_only, {"sm_mhz": 1500, "sm_max_mhz": 1965, "reasons": []}) == \
+        (3288.0, "bf16_tflops")
+
+
+def test_gemm_compulsory_bytes_and_operand_sets():
+    import bench
+    M, N, K = 2048, 6912, 1536
+    assert bench.gemm_min_bytes("fwd", M, N, K) == M * K + N * K + 2 * M * N
+    assert bench.gemm_min_bytes("fwd", M, N, K, bias_bytes=N) == M * K + N * K + 2 * M * N + N
+    assert bench.gemm_min_bytes("dX", M, N, K) == M * N + N * K + 2 * M * K
+    assert bench.gemm_min_bytes("dW", M, N, K) == M * N + M * K + 2 * N * K
+    for per in (1, 10 << 20, 100 << 20, 1 << 30):
+        n = bench._sets_for(per)
+        assert 2 <= n <= 12 and (n * per >= (320 << 20) or n == 12)
+
+
+def test_traffic_summary_is_tied_to_the_gemm_source(monkeypatch):
+    """roofline.traffic comes from the committed ncu summary only while
+    gemm.cu still has the hash recorded there."""
+    import bench
+    got = bench.gemm_traffic_per_launch("c4")
+    if got is not None:
+        assert got > 0
+        monkeypatch.setattr(bench, "gemm_source_sha", lambda: "0000000000000000")
+        assert bench.gemm_traffic_per_launch("c4") is None
+    assert bench.gemm_traffic_per_launch("no-such-workload") is None

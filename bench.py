@@ -571,7 +571,32 @@ def time_target_shapes(F, device, stream, fp8_peak, hbm_gbs):
                       "ring_step_deferred": {"us": round(dus, 2), "gbs": round(dgbs, 1),
                                              "frac_hbm": round(dgbs / hbm_gbs, 3)}})
         del sets, qargs
-    return gemm, quant, box_copy_gbs
+    # the bias gradient: the backward's fused g quantize + column sums
+    # (fp8_quantize_dbias, E5M2, ring finalize and sums in the launch) and the
+    # standalone column sum of a bf16 g (fp8_dbias), cold
+    dbias = []
+    for rows, cols in ((4096, 11008), (2048, 6912), (2048, 4096)):
+        nsets = _sets_for(rows * cols * 3)
+        gs = [torch.randn(rows, cols, device=device).mul_(1e-3).to(torch.bfloat16) for _ in range(nsets)]
+        outs = [torch.empty(rows, cols, dtype=torch.uint8, device=device) for _ in range(nsets)]
+        db = torch.empty(cols, dtype=torch.bfloat16, device=device)
+        ws = torch.zeros(max(16, F.fp8_dbias_workspace_bytes(rows, cols)), dtype=torch.uint8, device=device)
+        qargs = [F.QuantizeArgs(g.data_ptr(), 0, rows, cols, cols, F.FP8_E5M2, ring.data_ptr(), wl.HIST_LEN,
+                                o.data_ptr(), cols, None, None) for g, o in zip(gs, outs)]
+        qfns = [(lambda a=a: F._lib.fp8_quantize_dbias(ctypes.byref(a), db.data_ptr(), ws.data_ptr(), ws.numel(), h))
+                for a in qargs]
+        qus = _graph_us(stream, qfns)
+        dfns = [(lambda g=g: F._lib.fp8_dbias(g.data_ptr(), 0, rows, cols, cols, None, db.data_ptr(), ws.data_ptr(),
+                                               ws.numel(), h)) for g in gs]
+        dus = _graph_us(stream, dfns)
+        q_gbs, d_gbs = rows * cols * 3 / qus / 1e3, rows * cols * 2 / dus / 1e3
+        dbias.append({"shape": f"{rows}x{cols} bf16",
+                      "quantize_dbias": {"us": round(qus, 2), "gbs": round(q_gbs, 1),
+                                         "frac_hbm": round(q_gbs / hbm_gbs, 3), "bytes_per_elem": 3},
+                      "dbias_only": {"us": round(dus, 2), "gbs": round(d_gbs, 1),
+                                     "frac_hbm": round(d_gbs / hbm_gbs, 3), "bytes_per_elem": 2}})
+        del gs, outs, qargs
+    return gemm, quant, box_copy_gbs, dbias
 
 
 # --------------------------------------------------------------------------- GEMM traffic (ncu summary)
@@ -954,9 +979,9 @@ def main(argv=None):
             raise F.Fp8Error(F.fp8_get_device_status(), "device status after the other workloads")
         line["steps_other_workloads"] = others
 
-        tg, tq, box_copy = time_target_shapes(F, device, stream, fp8_peak, pk["hbm_gbs"])
+        tg, tq, box_copy, tdb = time_target_shapes(F, device, stream, fp8_peak, pk["hbm_gbs"])
         line["targets"] = {
-            "gemm": tg, "quantize": tq, "fp8_peak_tflops": fp8_peak, "hbm_gbs": pk["hbm_gbs"],
+            "gemm": tg, "quantize": tq, "dbias": tdb, "fp8_peak_tflops": fp8_peak, "hbm_gbs": pk["hbm_gbs"],
             "box_copy_gbs": box_copy,
             "note": "separate fp8_mm launches per operation (dX, dW in the fused backward's in-place "
                     "transposed layouts); warm = the same operands back to back, cold = operand sets cycled so "

@@ -244,11 +244,12 @@ void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
 }
 
 // The column-sum quantize whose sums a GEMM launch finishes (the linear
-// backward): about 592 blocks, at least 32 rows each.  Measured on a B200 in
-// the dim1024 training step (g of 2048 x 1024 and 2048 x 4096): 2% faster
-// than the dbias kernel's geometry; 16-row or 1184-block splits were slower.
+// backward): about 444 blocks (one resident wave: three per SM), at least 32
+// rows each.  Measured on a B200 in the dim1024 and production steps: 592
+// blocks (1.33 waves) were 0.7 % slower in the dim1024 step; 16-row or
+// 1184-block splits were slower with the kernel's earlier form.
 void colsum_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
-  split_geometry(M, N, 592, 32, R, rows_per_split);
+  split_geometry(M, N, 444, 32, R, rows_per_split);
 }
 
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s) {

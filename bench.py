@@ -566,10 +566,20 @@ def time_target_shapes(F, device, stream, fp8_peak, hbm_gbs):
         dus = _graph_us(stream, dfns)
         F.fp8_ring_finalize(ring, wl.HIST_LEN, F.FP8_E4M3)
         dgbs = per_set / dus / 1e3
+        # current (dynamic) scaling: an amax pass, then the cast with fp8_max / amax
+        # (algorithmic bytes as above; the amax pass reads the input a second time)
+        am = torch.zeros(1, dtype=torch.float32, device=device)
+        yfns = [(lambda x=x, o=o: F._lib.fp8_quantize(x.data_ptr(), 0, rows, cols, cols, 0, None, 0, o.data_ptr(),
+                                                      cols, am.data_ptr(), None, h)) for x, o in sets]
+        yus = _graph_us(stream, yfns)
+        ygbs = per_set / yus / 1e3
         quant.append({"shape": f"{rows}x{cols} bf16->e4m3", "us": round(us, 2), "gbs": round(gbs, 1),
                       "frac_hbm": round(gbs / hbm_gbs, 3),
                       "ring_step_deferred": {"us": round(dus, 2), "gbs": round(dgbs, 1),
-                                             "frac_hbm": round(dgbs / hbm_gbs, 3)}})
+                                             "frac_hbm": round(dgbs / hbm_gbs, 3)},
+                      "current_scaling": {"us": round(yus, 2), "gbs": round(ygbs, 1),
+                                          "frac_hbm": round(ygbs / hbm_gbs, 3),
+                                          "min_bytes_with_second_read": per_set + rows * cols * 2}})
         del sets, qargs
     # the bias gradient: the backward's fused g quantize + column sums
     # (fp8_quantize_dbias, E5M2, ring finalize and sums in the launch) and the

@@ -670,8 +670,7 @@ int run_quantize_dbias(const fp8_quantize_args& g, void* dbias, void* workspace,
   cp.q.defer_finalize = defer && g.ring ? 1 : 0;
   int s = amax_pass(g.in_dtype, &cp.q, nullptr, st);
   if (s) return s;
-  if (defer) colsum_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
-  else dbias_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
+  colsum_geometry(g.rows, g.cols, &cp.R, &cp.rows_per_split);
   cp.counters = static_cast<unsigned*>(workspace);
   cp.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dbias_counter_bytes(g.cols));
   cp.dbias = dbias;
@@ -910,13 +909,9 @@ int fp8_mm_plan(const fp8_mm_args* a, const fp8_mm_args* b, int num_sms, fp8_mm_
 
 size_t fp8_mm_workspace_bytes(int64_t m, int64_t n, int64_t k) { return sk_bytes_for(m, n, k); }
 
-size_t fp8_dbias_workspace_bytes(int64_t M, int64_t N) {
-  if (M <= 0 || N <= 0) return 0;
-  int R;
-  int64_t rps;
-  dbias_geometry(M, N, &R, &rps);
-  return dbias_counter_bytes(N) + dbias_partial_bytes(R, N);
-}
+// One size for fp8_dbias and the column-sum quantize (standalone or in the
+// linear backward): the larger of the two geometries' partials.
+size_t fp8_dbias_workspace_bytes(int64_t M, int64_t N) { return linear_dbias_bytes(M, N); }
 
 int fp8_dbias(const void* g, int g_dtype, int64_t M, int64_t N, int64_t ldg, const float* g_scale, void* dbias,
               void* workspace, size_t workspace_bytes, fp8_stream_t stream) {

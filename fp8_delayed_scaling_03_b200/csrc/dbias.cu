@@ -221,10 +221,13 @@ __global__ void __launch_bounds__(kRowLanes * 32) dbias_kernel(const DbiasParams
 namespace {
 
 // Row splits of an [M, N] column sum over 256-column tiles: about `blocks`
-// (col tile, row split) blocks in total, each split at least min_rows rows.
-void split_geometry(int64_t M, int64_t N, int64_t blocks, int64_t min_rows, int* R, int64_t* rows_per_split) {
+// (col tile, row split) blocks in total (at most `blocks` with at_most, the
+// row splits rounded down instead of up), each split at least min_rows rows.
+void split_geometry(int64_t M, int64_t N, int64_t blocks, int64_t min_rows, bool at_most, int* R,
+                    int64_t* rows_per_split) {
   const int64_t col_tiles = (N + kCols - 1) / kCols;
-  int64_t r = (blocks + col_tiles - 1) / (col_tiles > 0 ? col_tiles : 1);
+  const int64_t ct = col_tiles > 0 ? col_tiles : 1;
+  int64_t r = at_most ? blocks / ct : (blocks + ct - 1) / ct;
   const int64_t rmax = (M + min_rows - 1) / min_rows;
   if (r > rmax) r = rmax;
   if (r < 1) r = 1;
@@ -238,18 +241,22 @@ void split_geometry(int64_t M, int64_t N, int64_t blocks, int64_t min_rows, int*
 
 }  // namespace
 
-// The dbias kernel: about 296 blocks (two per SM of a B200), at least 64 rows each.
+// The dbias kernel: at most 444 blocks (three per SM of a B200; its 48
+// registers would allow five), at least 64 rows each.  Measured on a B200
+// (bf16 g): 0.75 / 0.50 / 0.32 of HBM at 4096x11008 / 2048x6912 / 2048x4096
+// against 0.72 / 0.40 / 0.28 with about 296 blocks; at most 592 or 740
+// blocks of >= 32 rows were slower than 444 on every shape.
 void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
-  split_geometry(M, N, 296, 64, R, rows_per_split);
+  split_geometry(M, N, 444, 64, true, R, rows_per_split);
 }
 
-// The column-sum quantize whose sums a GEMM launch finishes (the linear
-// backward): about 444 blocks (one resident wave: three per SM), at least 32
-// rows each.  Measured on a B200 in the dim1024 and production steps: 592
+// The column-sum quantize (standalone, or in the linear backward where a GEMM
+// launch finishes its sums): at most 444 blocks (one resident wave: three per SM), at least
+// 32 rows each.  Measured on a B200 in the dim1024 and production steps: 592
 // blocks (1.33 waves) were 0.7 % slower in the dim1024 step; 16-row or
 // 1184-block splits were slower with the kernel's earlier form.
 void colsum_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split) {
-  split_geometry(M, N, 444, 32, R, rows_per_split);
+  split_geometry(M, N, 444, 32, true, R, rows_per_split);
 }
 
 cudaError_t launch_dbias(const DbiasParams& p, cudaStream_t s) {

@@ -205,10 +205,10 @@ cudaError_t launch_wait_selftest(const uint32_t* flag, int* status, int* results
 
 // Column-sum geometry (R row splits of rows_per_split rows over 256-column
 // tiles) shared by the size queries and the launchers: dbias_geometry for the
-// dbias kernel and the standalone column-sum quantize, colsum_geometry for
-// the column-sum quantize of the linear backward (its sums finished by the
-// GEMM launch).  Workspaces hold the per-tile counters first (16-byte
-// rounded), then the R x N fp32 partials.
+// dbias kernel, colsum_geometry for the column-sum quantize (standalone, or
+// in the linear backward with its sums finished by the GEMM launch).
+// Workspaces hold the per-tile counters first (16-byte rounded), then R x N
+// fp32 partials for the larger R of the two, so one workspace serves both.
 constexpr int kDbiasColsPerTile = 256;
 void dbias_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split);
 void colsum_geometry(int64_t M, int64_t N, int* R, int64_t* rows_per_split);

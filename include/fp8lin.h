@@ -386,10 +386,11 @@ typedef struct fp8_linear_bwd_args {
 FP8LIN_API int fp8_linear_backward(const fp8_linear_bwd_args* args, fp8_stream_t stream);
 
 /* Workspace bytes fp8_linear_backward needs for need_dbias (0 when M or N is
- * 0).  At least fp8_dbias_workspace_bytes(M, N): the column-sum quantize of
- * the backward may split g's rows more finely than fp8_dbias does.  Zero-fill
- * it once before first use, like fp8_dbias's workspace; every call leaves it
- * ready for the next call of the same sizes.  K does not enter. */
+ * 0).  Equal to fp8_dbias_workspace_bytes(M, N): one size covers the row
+ * splits of fp8_dbias and of the column-sum quantize (fp8_quantize_dbias and
+ * the backward's g).  Zero-fill it once before first use, like fp8_dbias's
+ * workspace; every call leaves it ready for the next call of the same sizes.
+ * K does not enter. */
 FP8LIN_API size_t fp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------ status

@@ -151,9 +151,10 @@ def test_dbias_workspace_rules(fp8):
     assert fp8.fp8_dbias_workspace_bytes(0, 10) == 0
     need = fp8.fp8_dbias_workspace_bytes(2048, 1024)
     assert need > 0 and need % 16 == 0
-    # the linear backward's column sums may split rows more finely than fp8_dbias
+    # fp8_dbias and the column-sum quantize (standalone or in the linear
+    # backward) share one workspace size
     lin = fp8.fp8_linear_workspace_bytes(2048, 1024, 4096)
-    assert lin >= need and lin % 16 == 0
+    assert lin == need
     assert fp8.fp8_linear_workspace_bytes(0, 1024, 4096) == 0
     f = fp8._lib.fp8_dbias
     assert f(A, E.FP8_DT_BF16, 2048, 1024, 1024, None, A + 0x100, None, 0, None) == E.FP8_ERR_WORKSPACE
@@ -209,23 +210,32 @@ def test_linear_backward_validation(fp8):
     assert bwd(fp8, sg_out=None) == E.FP8_ERR_INVALID_ARG
     assert bwd(fp8, N=0, need_dx=0) == E.FP8_OK  # g and dW empty: nothing enqueued
     assert bwd(fp8, M=0, need_dw=0, g=None) == E.FP8_OK
-    # the backward's column sums need fp8_linear_workspace_bytes, which can
-    # exceed what fp8_dbias needs; a workspace sized for fp8_dbias is refused
+    # one workspace size serves fp8_dbias, fp8_quantize_dbias and the
+    # backward's column sums; one byte short of it is refused
     M, N, K = 2048, 1024, 1024
     lin, dbw = fp8.fp8_linear_workspace_bytes(M, N, K), fp8.fp8_dbias_workspace_bytes(M, N)
-    assert lin > dbw
+    assert lin == dbw
     big = dict(M=M, N=N, K=K, ldg=N, ldg8=N, ldx8=K, ldw8=K, lddx=K, lddw=K, need_dbias=1, dbias=A + 0xA0000,
                workspace=A + 0x100000)
-    assert bwd(fp8, workspace_bytes=dbw, **big) == E.FP8_ERR_WORKSPACE
+    assert bwd(fp8, workspace_bytes=lin - 1, **big) == E.FP8_ERR_WORKSPACE
     assert bwd(fp8, workspace_bytes=lin, workspace=A + 0x100008, **{k: v for k, v in big.items()
                                                                    if k != "workspace"}) == E.FP8_ERR_WORKSPACE
+
+
+def test_colsum_split_stays_in_one_wave(fp8):
+    # the column-sum quantize runs at most 444 blocks (three per SM on 148
+    # SMs): 43 column tiles of 11008 columns get 10 row splits, not 11 (473
+    # blocks would spill into a second wave); 27 tiles of 6912 get 16, not 17
+    for M, N, tiles, R in ((4096, 11008, 43, 10), (2048, 6912, 27, 16), (4096, 4096, 16, 27)):
+        counters = (tiles * 4 + 15) // 16 * 16
+        assert fp8.fp8_dbias_workspace_bytes(M, N) == counters + R * N * 4, (M, N)
 
 
 def test_linear_workspace_covers_dbias(fp8):
     for M in (1, 3, 64, 100, 512, 2048, 4096, 65536):
         for N in (1, 100, 192, 1024, 1536, 4096, 6912, 11008):
             lin, dbw = fp8.fp8_linear_workspace_bytes(M, N, 64), fp8.fp8_dbias_workspace_bytes(M, N)
-            assert lin >= dbw > 0 and lin % 16 == 0
+            assert lin == dbw > 0 and lin % 16 == 0
 
 
 def test_fused_entry_points_validation(fp8):

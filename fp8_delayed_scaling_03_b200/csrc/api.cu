@@ -621,16 +621,20 @@ QuantizeParams make_qparams(const void* in, int in_dtype, int64_t rows, int64_t 
 // max |x| into it in one launch.
 int amax_pass(int in_dtype, QuantizeParams* a, QuantizeParams* b, cudaStream_t st) {
   const QuantizeParams* d[2] = {nullptr, nullptr};
+  SideWrites zero;
+  std::memset(&zero, 0, sizeof(zero));
   int n = 0;
   for (QuantizeParams* q : {a, b}) {
     if (!q || q->ring) continue;
     q->dyn_amax = q->amax_out;
-    cudaError_t e = cudaMemsetAsync(q->amax_out, 0, sizeof(float), st);
-    if (e != cudaSuccess) return cuda_fail(e);
+    zero.zero_dst[n] = q->amax_out;
     d[n++] = q;
   }
   if (n == 0) return FP8_OK;
-  cudaError_t e = launch_amax(in_dtype, d[0], d[1], st);
+  // The amax words start at zero: a one-thread kernel (not a memset, so the
+  // amax grid stays a programmatic dependent and prefetches while it runs).
+  cudaError_t e = launch_side_writes(zero, st);
+  if (e == cudaSuccess) e = launch_amax(in_dtype, d[0], d[1], st);
   return e == cudaSuccess ? FP8_OK : cuda_fail(e);
 }
 

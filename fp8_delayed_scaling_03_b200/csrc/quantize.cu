@@ -236,16 +236,13 @@ __device__ __forceinline__ uint32_t block_max_bits(float amax, uint32_t* warp_ma
 // chunks per thread per iteration (plus as many prefetched): 64 bytes of input
 constexpr int unroll_for(int bytes) { return bytes == 2 ? 2 : 1; }
 
-template <typename T, int FMT>
-__global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_constant__ QuantizePair pair) {
-  __shared__ uint32_t warp_max[kThreads / 32];
-  __shared__ float hist_s[kHistCache];
-  constexpr int U = unroll_for(sizeof(T));
-  // Before the dependency wait: the blocks that become resident first (one
-  // per SM fits beside a GEMM CTA still running) prefetch the contiguous
-  // inputs into L2, each a 1/pf_blocks slice of every tensor, so the DRAM
-  // latency overlaps the previous kernel's tail.  Safe whatever that kernel
-  // writes: a prefetch only warms L2, the loads below come after the wait.
+// Before the dependency wait: the blocks that become resident first (one per
+// SM fits beside a GEMM CTA still running) prefetch the contiguous inputs into
+// L2, each a 1/pf_blocks slice of every tensor, so the DRAM latency overlaps
+// the previous kernel's tail.  Safe whatever that kernel writes: a prefetch
+// only warms L2, the loads come after the wait.
+template <typename T>
+__device__ __forceinline__ void prefetch_inputs(const QuantizePair& pair) {
   if (threadIdx.x == 0 && blockIdx.x < static_cast<unsigned>(pair.pf_blocks)) {
     const int ntensors = pair.blocks0 < static_cast<int>(gridDim.x) ? 2 : 1;
     for (int i = 0; i < ntensors; ++i) {
@@ -262,6 +259,14 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_cons
         prefetch_l2_bulk(static_cast<const uint8_t*>(q.in) + off, static_cast<uint32_t>(min(span, bytes - off)));
     }
   }
+}
+
+template <typename T, int FMT>
+__global__ void __launch_bounds__(kThreads, 4) quantize_kernel(const __grid_constant__ QuantizePair pair) {
+  __shared__ uint32_t warp_max[kThreads / 32];
+  __shared__ float hist_s[kHistCache];
+  constexpr int U = unroll_for(sizeof(T));
+  prefetch_inputs<T>(pair);
   pdl_wait();
   pdl_trigger();
   const bool second = blockIdx.x >= pair.blocks0;
@@ -361,6 +366,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const __grid_constant__ QuantizePair pair) {
   __shared__ uint32_t warp_max[kThreads / 32];
   constexpr int U = unroll_for(sizeof(T));
+  prefetch_inputs<T>(pair);
   pdl_wait();
   pdl_trigger();
   const bool second = blockIdx.x >= pair.blocks0;

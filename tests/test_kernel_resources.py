@@ -71,13 +71,14 @@ def gemm_builds(kernels):
 
 def test_spills(gemm, quant):
     """No GEMM build spills.  The flat quantize and amax builds for 2-byte
-    inputs keep one 8-byte stack slot at their 64-register cap (quantize: 12
-    bytes stored, 16 loaded; amax: 16 in all), no more."""
+    inputs (both prefetch their input into L2 before the dependency wait)
+    keep a small stack slot at their 64-register cap, at most 28 bytes of
+    spill traffic (12 stored, 16 loaded), no more."""
     for name, res in gemm.items():
         assert res["spill"] == 0, (name, res)
     for name, res in quant.items():
         two_byte = "__half" in name or "bfloat16" in name
-        allowed = 28 if two_byte and "15quantize_kernelI" in name else 16 if two_byte and "11amax_kernelI" in name else 0
+        allowed = 28 if two_byte and ("15quantize_kernelI" in name or "11amax_kernelI" in name) else 0
         assert res["spill"] <= allowed, (name, res)
 
 

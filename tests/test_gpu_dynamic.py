@@ -86,7 +86,9 @@ def test_dual_dynamic_and_delayed(fp8):
     x = wl.normal((700, 520), 9.0, 1460)
     w = wl.normal((520, 520), 0.1, 1461)
     x8, w8 = fp8_buffer(700, 520), fp8_buffer(520, 520)
-    sc = torch.zeros(4, device="cuda")
+    # -1.0 (0xBF800000) is above every finite |x| as raw bits: both amax words
+    # must be cleared before the reduction, or they keep it
+    sc = torch.full((4,), -1.0, device="cuda")
     xd, wd = x.cuda(), w.cuda()
     fp8.fp8_quantize_dual(fp8.quantize_args(xd, 1, None, 0, x8, sc[0:1], sc[1:2]),
                           fp8.quantize_args(wd, 1, None, 0, w8, sc[2:3], sc[3:4]))

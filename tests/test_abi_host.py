@@ -231,6 +231,20 @@ def test_colsum_split_stays_in_one_wave(fp8):
         assert fp8.fp8_dbias_workspace_bytes(M, N) == counters + R * N * 4, (M, N)
 
 
+def test_bias_gradient_split_bounds(fp8):
+    # for any shape, the row splits R behind the workspace size keep every
+    # column-sum grid (col tiles x R) within one wave of 444 blocks unless a
+    # single split per tile already exceeds it, and never split below 32 rows
+    for M in (1, 31, 32, 33, 100, 512, 2048, 3000, 4096, 65536):
+        for N in (1, 255, 256, 257, 1024, 6912, 11008, 120000):
+            tiles = -(-N // 256)
+            counters = (tiles * 4 + 15) // 16 * 16
+            part = fp8.fp8_dbias_workspace_bytes(M, N) - counters   # R x N fp32, 16-byte rounded
+            r16 = lambda r: (r * N * 4 + 15) // 16 * 16  # noqa: E731
+            bound = min(max(1, 444 // tiles), -(-M // 32))
+            assert r16(1) <= part <= r16(bound), (M, N, part, bound)
+
+
 def test_linear_workspace_covers_dbias(fp8):
     for M in (1, 3, 64, 100, 512, 2048, 4096, 65536):
         for N in (1, 100, 192, 1024, 1536, 4096, 6912, 11008):

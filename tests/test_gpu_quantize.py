@@ -165,7 +165,8 @@ def test_quantize_dual_matches_two_launches(fp8, dtype):
         assert np.array_equal(ring_words(r2), oracle_ring_words(o2))
 
 
-@pytest.mark.parametrize("rows,cols", [(2048, 1024), (300, 100), (4096, 4096), (1, 7), (77, 1534)])
+@pytest.mark.parametrize("rows,cols", [(2048, 1024), (300, 100), (4096, 4096), (1, 7), (77, 1534), (3, 120000),
+                                       (300, 113920)])
 def test_quantize_dbias_entry(fp8, rows, cols):
     """fp8_quantize_dbias: codes and ring bit-exact, dbias within
     max(1 bf16 ulp, 2e-6 sum|g|) of the oracle's column sums."""
@@ -187,6 +188,43 @@ def test_quantize_dbias_entry(fp8, rows, cols):
         gv = oracle.bf16_to_f32(bits(db.cpu())).astype(np.float64)
         ov = oracle.bf16_to_f32(want).astype(np.float64)
         assert np.all(np.abs(gv - ov) <= np.maximum(oracle.bf16_ulp(ov), 2e-6 * sa))
+    assert fp8.fp8_get_device_status() == 0
+
+
+def dbias_close(db, want, sa, what):
+    gv = oracle.bf16_to_f32(bits(db.cpu())).astype(np.float64)
+    ov = oracle.bf16_to_f32(want).astype(np.float64)
+    assert np.all(np.abs(gv - ov) <= np.maximum(oracle.bf16_ulp(ov), 2e-6 * sa)), what
+
+
+@pytest.mark.parametrize("rows,cols", [(2048, 1024), (77, 1534), (1, 300), (1000, 11008), (3, 120000),
+                                       (300, 113920)])
+def test_dbias_entry(fp8, rows, cols):
+    """fp8_dbias against the oracle's column sums, within max(1 bf16 ulp,
+    2e-6 sum|g|): bf16 and fp32 g, and E4M3 codes with a scale (dequantized
+    before the sum); shapes from one row split to many, and with more than
+    444 column tiles (one split per tile), each call twice on one workspace
+    (the tile counters back at zero between calls)."""
+    ws = torch.zeros(max(16, fp8.fp8_dbias_workspace_bytes(rows, cols)), dtype=torch.uint8, device="cuda")
+    for dtype in (torch.bfloat16, torch.float32):
+        g = wl.normal((rows, cols), 1e-3, 990 + rows, dtype=dtype)
+        gd = g.cuda()
+        want, _, sa = oracle.dbias(bits(g) if dtype == torch.bfloat16 else g.numpy().view(np.uint32),
+                                   dt_code(g), rows, cols)
+        for _ in range(2):
+            db = torch.empty(cols, dtype=torch.bfloat16, device="cuda")
+            fp8.fp8_dbias(gd, db, ws)
+            torch.cuda.synchronize()
+            dbias_close(db, want, sa, (rows, cols, dtype))
+    gen = torch.Generator().manual_seed(rows + cols)
+    codes = (torch.randint(0, 0x7E, (rows, cols), generator=gen, dtype=torch.int32) |
+             (torch.randint(0, 2, (rows, cols), generator=gen, dtype=torch.int32) << 7)).to(torch.uint8)  # no NaN
+    sg = torch.tensor([19.25], device="cuda")
+    db = torch.empty(cols, dtype=torch.bfloat16, device="cuda")
+    fp8.fp8_dbias(codes.cuda(), db, ws, g_scale=sg, g_fmt=fp8.FP8_E4M3)
+    torch.cuda.synchronize()
+    want, _, sa = oracle.dbias(codes.numpy(), oracle.DT_E4M3, rows, cols, 19.25)
+    dbias_close(db, want, sa, (rows, cols, "e4m3"))
     assert fp8.fp8_get_device_status() == 0
 
 

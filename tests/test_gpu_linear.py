@@ -369,6 +369,51 @@ def test_backward_fused_colsum_dtypes(fp8, dtype, M, N, K):
     assert fp8.fp8_get_device_status() == 0
 
 
+@pytest.mark.parametrize("need_dx,need_dw", [(True, False), (False, True)])
+@pytest.mark.parametrize("need_dbias", [False, True])
+def test_backward_need_masks(fp8, need_dx, need_dw, need_dbias):
+    """dX alone or dW alone: the backward's one GEMM launch (instead of the
+    dX + dW pair) also completes the g ring's step and, with the bias
+    gradient, the column sums.  Over two steps g8, the snapshot, amax and
+    every ring word are bit-exact, the requested gradient is within the GEMM
+    tolerance in full, and the buffer of the gradient not requested is left
+    as it was."""
+    rng = np.random.default_rng(7 + int(need_dx) + 2 * int(need_dbias))
+    M, N, K = 700, 520, 384
+    rx, rw, rg = fp8.ScaleRing(16), fp8.ScaleRing(16), fp8.ScaleRing(16)
+    org = oracle.Ring(16)
+    x = wl.normal((M, K), 1.0, 41)
+    w = wl.normal((N, K), 0.05, 42)
+    f = fp8.linear_forward(x.cuda(), w.cuda(), rx, rw)
+    torch.cuda.synchronize()
+    x8, w8 = host_rows(f.x8), host_rows(f.w8)
+    dx = torch.full((M, K), 7.0, dtype=torch.bfloat16, device="cuda")
+    dw = torch.full((N, K), 7.0, dtype=torch.bfloat16, device="cuda")
+    for step in range(2):
+        g = wl.normal((M, N), 1e-3 * (1 + 2 * step), 43 + step)
+        b = fp8.linear_backward(g.cuda(), f, rg, need_dx=need_dx, need_dw=need_dw, need_dbias=need_dbias,
+                                dx=dx, dw=dw)
+        torch.cuda.synchronize()
+        gb = bits(g)
+        g8o, ag, sg = oracle.quantize(gb, oracle.DT_BF16, E5, org, ld_out=(N + 15) // 16 * 16)
+        assert b.sg.item() == sg and b.amax_g.item() == ag
+        g8c = np.ascontiguousarray(g8o[:, :N])
+        assert_codes_equal(host_rows(b.g8), g8c, E5)
+        assert np.array_equal(ring_words(rg), oracle_ring_words(org))
+        what = f"step {step} need_dx={need_dx} need_dw={need_dw} need_dbias={need_dbias}"
+        if need_dx:
+            gemm_check(dx, g8c, 0, E5, w8, E4, M, K, N, sg, f.sw.item(), "dx", True, rng, what=what + " dx")
+        else:
+            assert bool((dx == 7.0).all()), what
+        if need_dw:
+            gemm_check(dw, g8c, 0, E5, x8, E4, N, K, M, sg, f.sx.item(), "dw", True, rng, what=what + " dw")
+        else:
+            assert bool((dw == 7.0).all()), what
+        if need_dbias:
+            dbias_check(b.dbias, gb, M, N)
+    assert fp8.fp8_get_device_status() == 0
+
+
 def test_backward_prequantized_g_dbias(fp8):
     """A pre-quantized g (E5M2 codes with its scale) skips its quantize
     (sg = g_scale_in, amax_g = 0, ring untouched) and dbias dequantizes each

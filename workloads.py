@@ -45,11 +45,6 @@ def log_uniform(lo: float, hi: float, seed: int) -> float:
     return math.exp(math.log(lo) + u * (math.log(hi) - math.log(lo)))
 
 
-def bits16(t: torch.Tensor):
-    """bf16/fp16 CPU tensor -> numpy uint16 bit patterns (no copy of values)."""
-    return t.contiguous().view(torch.int16).numpy().view("uint16")
-
-
 @dataclass(frozen=True)
 class LinearShape:
     name: str
@@ -120,8 +115,3 @@ def normal_with_outliers_device(shape, std: float, seed: int, mask_seed: int, de
 BENCH_LAYERS = 12
 BENCH_LAYER = C2_LAYER
 BENCH_BIAS_STD = 0.01
-
-
-def bench_flops_per_step(layers: int = BENCH_LAYERS) -> int:
-    """fwd + dX + dW: 3 GEMMs of 2*M*N*K flops per linear."""
-    return layers * sum(6 * s.M * s.N * s.K for s in BENCH_LAYER)

@@ -989,10 +989,13 @@ def main(argv=None):
             raise F.Fp8Error(F.fp8_get_device_status(), "device status after the other workloads")
         line["steps_other_workloads"] = others
 
-        tg, tq, box_copy, tdb = time_target_shapes(F, device, stream, fp8_peak, pk["hbm_gbs"])
+        # the per-operation launches run right after the steps above: their
+        # SM clock (and any power-cap reason) is sampled and reported with them
+        with ClockSampler(local) as tclk:
+            tg, tq, box_copy, tdb = time_target_shapes(F, device, stream, fp8_peak, pk["hbm_gbs"])
         line["targets"] = {
             "gemm": tg, "quantize": tq, "dbias": tdb, "fp8_peak_tflops": fp8_peak, "hbm_gbs": pk["hbm_gbs"],
-            "box_copy_gbs": box_copy,
+            "box_copy_gbs": box_copy, "clocks": tclk.report(),
             "note": "separate fp8_mm launches per operation (dX, dW in the fused backward's in-place "
                     "transposed layouts); warm = the same operands back to back, cold = operand sets cycled so "
                     "each pass streams more than L2; frac_roofline = achieved / min(peak, AI x HBM BW) cold, "

@@ -179,3 +179,42 @@ def test_traffic_summary_is_tied_to_the_gemm_source(monkeypatch):
         monkeypatch.setattr(bench, "gemm_source_sha", lambda: "0000000000000000")
         assert bench.gemm_traffic_per_launch("c4") is None
     assert bench.gemm_traffic_per_launch("no-such-workload") is None
+
+
+def test_clock_sampler_against_fake_nvml(monkeypatch):
+    """The sampler reads the SM clock and the clock-event reason bits through
+    NVML in a thread (reads only) and reports their median and the union of
+    the reasons by name; without NVML it reports that instead of clocks."""
+    import sys
+    import time
+    import types
+
+    import bench
+
+    clocks = iter([1965, 1965, 1800, 1965, 1700] + [1965] * 10000)
+    reasons = iter([0, 0x4, 0, 0x4 | 0x40, 0] + [0] * 10000)
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByPciBusId=lambda bus: "h",
+        nvmlDeviceGetHandleByIndex=lambda i: "h",
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: next(clocks),
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: next(reasons))
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    props = types.SimpleNamespace(pci_domain_id=0, pci_bus_id=0x1b, pci_device_id=0)
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda i: props)
+    with bench.ClockSampler(0) as clk:
+        t0 = time.time()
+        while len(clk.samples) < 5 and time.time() - t0 < 5:
+            time.sleep(0.01)
+    r = clk.report()
+    assert r["sm_max_mhz"] == 1965 and r["samples"] >= 5
+    assert "sw_power_cap" in r["reasons"] and "hw_thermal_slowdown" in r["reasons"]
+    assert set(r["reasons"]) <= set(bench.ClockSampler.REASONS.values())
+
+    def broken():
+        raise RuntimeError("no NVML here")
+    monkeypatch.setattr(fake, "nvmlInit", broken)
+    r = bench.ClockSampler(0).report()
+    assert r["sm_mhz"] is None and r["reasons"] == [] and "no NVML" in r["error"]
